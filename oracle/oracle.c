@@ -1,0 +1,205 @@
+/*
+ * ORACLE -- test infrastructure only.  Nothing in the product path may call,
+ * link or load this file; only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg do.  It shares no code with the GPU path.
+ *
+ * What it computes: single-token paged-KV decode attention, the problem stated
+ * in "spec(BACKEND-ROCM): the ROCm head_dim=128 decode arm, the ROCm half of
+ * #382" (vllm.cpp PR #564, section "The gap it specs": bf16 decode attention
+ * over a paged KV cache for GQA models) and in "perf(rocke): prepare saved
+ * paged decode bindings once" (rocm-libraries PR #13700, section "Summary":
+ * one-token split-KV attention, optional LSE output).  The pages print no
+ * formula; their statement that a warp-strided online softmax differs from the
+ * sequential kernel only by reduction order (PR #564, section "It is a mirror
+ * of merged work, not new design") means the result is ordinary softmax
+ * attention, and PR #13700 ("Testing Summary") checks against an independent
+ * FP32 reference.  So the oracle is that definition, written out in double:
+ *
+ *   for every sequence b and query head h, with kv head kh = h / (Hq/Hkv):
+ *     token t (0 <= t < L_b) lives in physical block block_tables[b][t / bs],
+ *       slot t % bs:   k_t = K[phys, kh, slot, :],  v_t = V[phys, kh, slot, :]
+ *     s_t   = scale * sum_d q[b,h,d] * k_t[d]
+ *     M     = max_t s_t,  Z = sum_t exp(s_t - M)
+ *     out   = sum_t exp(s_t - M) * v_t / Z
+ *     lse   = M + ln Z                    (natural log, includes `scale`)
+ *   L_b = 0 gives out = 0 and lse = -inf.
+ *
+ * Exact two-pass softmax: no splits, no online rescaling.  bf16 inputs are
+ * widened exactly to double.  Strides are in elements; every dimension may be
+ * strided.  Work is spread over (b, kh) pairs with pthreads, which changes no
+ * arithmetic order inside a pair.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+static double bf16_to_double(uint16_t bits) {
+  uint32_t w = (uint32_t)bits << 16;
+  float f;
+  memcpy(&f, &w, 4);
+  return (double)f;
+}
+
+typedef struct {
+  const uint16_t *q;
+  const uint16_t *k;
+  const uint16_t *v;
+  const int32_t *tables;
+  const int32_t *lens;
+  int64_t B, Hq, Hkv, D, bs, table_width;
+  int64_t q_str[3];   /* b, h, d */
+  int64_t kv_str[4];  /* block, kv head, slot, d (same for K and V) */
+  double scale;
+  double *out;        /* [B, Hq, D] contiguous */
+  double *lse;        /* [B, Hq] */
+} problem;
+
+/* One query head of one sequence: the definition above, term by term. */
+static void attend_one(const problem *p, int64_t b, int64_t h, double *s, double *o, double *lse) {
+  const int64_t g = p->Hq / p->Hkv;
+  const int64_t kh = h / g;
+  const int64_t L = p->lens[b];
+  const uint16_t *qrow = p->q + b * p->q_str[0] + h * p->q_str[1];
+  for (int64_t d = 0; d < p->D; ++d) o[d] = 0.0;
+  if (L <= 0) {
+    *lse = -INFINITY;
+    return;
+  }
+  /* scores */
+  for (int64_t t = 0; t < L; ++t) {
+    int64_t phys = p->tables[b * p->table_width + t / p->bs];
+    int64_t slot = t % p->bs;
+    const uint16_t *krow = p->k + phys * p->kv_str[0] + kh * p->kv_str[1] + slot * p->kv_str[2];
+    double acc = 0.0;
+    for (int64_t d = 0; d < p->D; ++d)
+      acc += bf16_to_double(qrow[d * p->q_str[2]]) * bf16_to_double(krow[d * p->kv_str[3]]);
+    s[t] = p->scale * acc;
+  }
+  /* exact softmax */
+  double M = s[0];
+  for (int64_t t = 1; t < L; ++t)
+    if (s[t] > M) M = s[t];
+  double Z = 0.0;
+  for (int64_t t = 0; t < L; ++t) {
+    s[t] = exp(s[t] - M);
+    Z += s[t];
+  }
+  /* weighted sum of values */
+  for (int64_t t = 0; t < L; ++t) {
+    int64_t phys = p->tables[b * p->table_width + t / p->bs];
+    int64_t slot = t % p->bs;
+    const uint16_t *vrow = p->v + phys * p->kv_str[0] + kh * p->kv_str[1] + slot * p->kv_str[2];
+    double w = s[t] / Z;
+    for (int64_t d = 0; d < p->D; ++d) o[d] += w * bf16_to_double(vrow[d * p->kv_str[3]]);
+  }
+  *lse = M + log(Z);
+}
+
+typedef struct {
+  const problem *p;
+  const int32_t *pairs; /* NULL: all (b, h); else npairs (b, h) pairs */
+  int64_t npairs;
+  int64_t max_len;
+  int nthreads, tid;
+} job;
+
+static void *worker(void *arg) {
+  job *j = (job *)arg;
+  const problem *p = j->p;
+  double *s = (double *)malloc(sizeof(double) * (size_t)(j->max_len > 0 ? j->max_len : 1));
+  if (!s) return (void *)1;
+  if (j->pairs) {
+    for (int64_t i = j->tid; i < j->npairs; i += j->nthreads) {
+      int64_t b = j->pairs[2 * i], h = j->pairs[2 * i + 1];
+      attend_one(p, b, h, s, p->out + i * p->D, p->lse + i);
+    }
+  } else {
+    const int64_t g = p->Hq / p->Hkv;
+    for (int64_t u = j->tid; u < p->B * p->Hkv; u += j->nthreads) {
+      int64_t b = u / p->Hkv, kh = u % p->Hkv;
+      for (int64_t h = kh * g; h < (kh + 1) * g; ++h)
+        attend_one(p, b, h, s, p->out + (b * p->Hq + h) * p->D, p->lse + b * p->Hq + h);
+    }
+  }
+  free(s);
+  return NULL;
+}
+
+static int run(const problem *p, const int32_t *pairs, int64_t npairs, int nthreads) {
+  int64_t max_len = 0;
+  for (int64_t b = 0; b < p->B; ++b)
+    if (p->lens[b] > max_len) max_len = p->lens[b];
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 512) nthreads = 512;
+  pthread_t th[512];
+  job jobs[512];
+  for (int t = 0; t < nthreads; ++t) {
+    jobs[t].p = p;
+    jobs[t].pairs = pairs;
+    jobs[t].npairs = npairs;
+    jobs[t].max_len = max_len;
+    jobs[t].nthreads = nthreads;
+    jobs[t].tid = t;
+  }
+  for (int t = 1; t < nthreads; ++t) pthread_create(&th[t], NULL, worker, &jobs[t]);
+  int rc = worker(&jobs[0]) != NULL;
+  for (int t = 1; t < nthreads; ++t) {
+    void *r = NULL;
+    pthread_join(th[t], &r);
+    rc |= r != NULL;
+  }
+  return rc;
+}
+
+static int fill(problem *p, const uint16_t *q, const int64_t *q_str, const uint16_t *k,
+                const uint16_t *v, const int64_t *kv_str, const int32_t *tables,
+                int64_t table_width, const int32_t *lens, int64_t B, int64_t Hq, int64_t Hkv,
+                int64_t D, int64_t bs, double scale, double *out, double *lse) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || bs <= 0) return 2;
+  p->q = q;
+  p->k = k;
+  p->v = v;
+  p->tables = tables;
+  p->lens = lens;
+  p->B = B;
+  p->Hq = Hq;
+  p->Hkv = Hkv;
+  p->D = D;
+  p->bs = bs;
+  p->table_width = table_width;
+  memcpy(p->q_str, q_str, sizeof(p->q_str));
+  memcpy(p->kv_str, kv_str, sizeof(p->kv_str));
+  p->scale = scale;
+  p->out = out;
+  p->lse = lse;
+  return 0;
+}
+
+/* Every (b, h): out [B, Hq, D] and lse [B, Hq], double.  Returns 0 on success. */
+int oracle_decode(const uint16_t *q, const int64_t *q_str, const uint16_t *k_cache,
+                  const uint16_t *v_cache, const int64_t *kv_str, const int32_t *block_tables,
+                  int64_t table_width, const int32_t *seq_lens, int64_t B, int64_t Hq, int64_t Hkv,
+                  int64_t D, int64_t bs, double scale, double *out, double *lse, int nthreads) {
+  problem p;
+  int rc = fill(&p, q, q_str, k_cache, v_cache, kv_str, block_tables, table_width, seq_lens, B,
+                Hq, Hkv, D, bs, scale, out, lse);
+  return rc ? rc : run(&p, NULL, 0, nthreads);
+}
+
+/* Selected (b, h) pairs only: out [npairs, D], lse [npairs]. */
+int oracle_decode_pairs(const uint16_t *q, const int64_t *q_str, const uint16_t *k_cache,
+                        const uint16_t *v_cache, const int64_t *kv_str,
+                        const int32_t *block_tables, int64_t table_width, const int32_t *seq_lens,
+                        int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t bs, double scale,
+                        const int32_t *pairs, int64_t npairs, double *out, double *lse,
+                        int nthreads) {
+  problem p;
+  int rc = fill(&p, q, q_str, k_cache, v_cache, kv_str, block_tables, table_width, seq_lens, B,
+                Hq, Hkv, D, bs, scale, out, lse);
+  for (int64_t i = 0; !rc && i < npairs; ++i)
+    if (pairs[2 * i] < 0 || pairs[2 * i] >= B || pairs[2 * i + 1] < 0 || pairs[2 * i + 1] >= Hq)
+      rc = 2;
+  return rc ? rc : run(&p, pairs, npairs, nthreads);
+}
