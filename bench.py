@@ -1,0 +1,362 @@
+#!/usr/bin/env python
+"""Benchmark: paged single-token decode attention on B200.
+
+One step = one full pass of the hot path (partition kernel + split-reduce kernel)
+over one decode batch.  Default workload: the Llama-8B-shaped decode batch
+(B=32, Hq/Hkv=32/8, D=128, block_size 16, seq_lens ~ U{512..4096}, synthetic bf16
+~N(0,1), tables over a 4096-block pool).  --workload picks another named one.
+
+Prints one JSON line (rank 0).  `value` is achieved algorithmic HBM GB/s of the
+whole step (all ranks' bytes / max-over-ranks device time); `us_per_call` is the
+mean device time per step.  Timing: W warm-up steps, then K timed steps, each
+bracketed by CUDA events on the launching stream, with a 256 MiB L2-flush write
+between steps outside the events; barrier + synchronize around the timed region.
+
+--impl reference times the CPU oracle (the reference arm of this path) on the
+host cores instead; it never touches the GPU.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--workload", default="llama8b")
+    ap.add_argument("--num-splits", type=int, default=None, help="override the workload's partition count")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline time budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (short profiling runs)")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_config(w, plan):
+    import synth  # noqa: F401
+    cfg = {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.D,
+           "block_size": w.block_size, "max_blocks_per_seq": w.max_blocks_per_seq,
+           "kv_tokens": w.kv_tokens(), "seq_len_min": int(w.seq_lens.min()), "seq_len_max": int(w.seq_lens.max()),
+           "recipe": w.recipe, "lse": w.want_lse, "seed": w.seed}
+    if plan is not None:
+        cfg.update({"num_splits": plan["num_splits"], "partition_tokens": plan["partition_tokens"],
+                    "heads_per_tile": plan["heads_per_tile"], "ctas": plan["ctas"]})
+    cfg["l2"] = f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write outside the timed events)"
+    return cfg
+
+
+def partition_bytes(w, S):
+    """Algorithmic bytes of one partition-kernel launch: K/V pages, q, live table
+    entries, seq_lens; plus out/lse when it writes them itself (S == 1)."""
+    L = w.seq_lens.astype(np.int64)
+    b = int((4 * L * w.Hkv * w.D).sum()) + 2 * w.B * w.Hq * w.D
+    b += int(4 * ((L + w.block_size - 1) // w.block_size).sum()) + 4 * w.B
+    if S == 1:
+        b += 2 * w.B * w.Hq * w.D + (4 * w.B * w.Hq if w.want_lse else 0)
+    return b
+
+
+def cpu_baseline(w, budget_s, runs_max=50):
+    """Time the oracle as it stands on this host's cores on a bounded sample."""
+    import oracle
+    threads = oracle.default_threads()
+    bytes_per = w.algorithmic_bytes()
+    times = []
+    t_all = time.perf_counter()
+    while True:
+        t0 = time.perf_counter()
+        oracle.decode_workload(w, nthreads=threads)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() - t_all > budget_s or len(times) >= runs_max:
+            break
+    med = statistics.median(times)
+    return {"value": round(bytes_per / med / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"whole {w.name} batch, {len(times)} run(s), median {med * 1e6:.0f} us/call "
+                      f"(double precision, {threads} threads)",
+            "us_per_call": round(med * 1e6, 1)}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running (reads only)."""
+
+    def __init__(self, index, period=0.002):
+        self.index, self.period = index, period
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return self
+        names = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+                 "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                    get = getattr(self._nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                        self._nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                    r = get(self._h)
+                    for n, bit in names.items():
+                        if r & bit:
+                            self.reasons.add(n)
+                except Exception:
+                    pass
+                time.sleep(self.period)
+
+        self._t = threading.Thread(target=run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def traffic_from_profiles(workload, kernel_sha):
+    """ncu dram bytes per launch recorded under profiles/, if taken on this kernel source."""
+    path = os.path.join(ROOT, "profiles", f"partition_kernel_{workload}.md")
+    try:
+        txt = open(path).read()
+    except OSError:
+        return None
+    vals = dict(line.split(":", 1) for line in txt.splitlines() if line.startswith(("source_sha256:", "dram_bytes_per_launch:")))
+    if vals.get("source_sha256", "").strip() != kernel_sha:
+        return None
+    try:
+        return int(vals["dram_bytes_per_launch"].strip())
+    except (KeyError, ValueError):
+        return None
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for f in ("pad_partition.cu", "pad_device.cuh", "pad_internal.h"):
+        with open(os.path.join(ROOT, "paged_kv_attention_partition_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def run_reference(args, rank, world):
+    import synth
+    metric = "decode attention µs/call and achieved HBM GB/s vs B200 peak (1 GPU)"
+    if rank != 0:
+        return
+    w = synth.config(args.workload)
+    cb = cpu_baseline(w, args.cpu_seconds)
+    us = cb["us_per_call"]
+    line = {"impl": "reference", "metric": metric, "value": cb["value"], "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1e3, 4), "us_per_call": us,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded generator, no dataset)", "config": workload_config(w, None),
+            "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+            "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    import paged_kv_attention_partition_b200 as pad
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    # weak scaling: every rank decodes its own batch of the same shape
+    base = synth.config(args.workload)
+    w = synth.config(args.workload, seed=base.seed + 1000 * rank) if rank else base
+    splits = w.num_splits if args.num_splits is None else args.num_splits
+    plan = pad.pad_decode_plan(w.B, w.Hq, w.Hkv, w.D, w.block_size, w.max_blocks_per_seq, num_splits=splits,
+                               device=local)
+    S = plan["num_splits"]
+
+    def dev_bf16(a):
+        return torch.from_numpy(a).view(torch.bfloat16).to(dev)
+
+    q, k, v = dev_bf16(w.q), dev_bf16(w.k_cache), dev_bf16(w.v_cache)
+    tables = torch.from_numpy(w.block_tables).to(dev)
+    lens = torch.from_numpy(w.seq_lens).to(dev)
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev) if w.want_lse else None
+    ws = torch.empty(max(plan["workspace_bytes"], 256) // 4 + 64, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+
+    def step_phased(ev):
+        pad.pad_decode_partition(q, k, v, tables, lens, w.scale, splits, out, lse, ws, stream)
+        ev[1].record(stream)
+        pad.pad_decode_reduce(q, k, v, tables, lens, w.scale, splits, out, lse, ws, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.fill_(1.0)
+            step_phased([None, torch.cuda.Event(enable_timing=True)])
+            pad.pad_decode(q, k, v, tables, lens, w.scale, num_splits=splits, out=out, lse=lse, stream=stream)
+    stream.synchronize()
+
+    # ---- timed region: exactly K steps, device events per phase ------------
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        with torch.cuda.stream(stream):
+            for i in range(args.steps):
+                flush.fill_(float(i))
+                ev = events[i]
+                ev[0].record(stream)
+                step_phased(ev)
+                ev[2].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    step_ms = [e[0].elapsed_time(e[2]) for e in events]
+    part_ms = [e[0].elapsed_time(e[1]) for e in events]
+    red_ms = [e[1].elapsed_time(e[2]) for e in events]
+    total_ms = sum(step_ms)
+    my_bytes = w.algorithmic_bytes() * args.steps
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        bt = torch.tensor([float(my_bytes)], device=dev, dtype=torch.float64)
+        dist.all_reduce(bt, op=dist.ReduceOp.SUM)
+        all_bytes = float(bt.item())
+    else:
+        all_bytes = float(my_bytes)
+    value = all_bytes / (total_ms / 1e3) / 1e9
+
+    # ---- end to end through the public one-call API, host buffers -----------
+    # Per step: pinned host -> device copy of the step's inputs (q, block table,
+    # seq_lens; the KV cache stays resident in HBM as in a decode loop), the call,
+    # device -> host copy of out and lse.
+    hq = torch.from_numpy(w.q).view(torch.bfloat16).pin_memory()
+    ht = torch.from_numpy(w.block_tables).pin_memory()
+    hl = torch.from_numpy(w.seq_lens).pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory() if lse is not None else None
+    h2d = hq.numel() * 2 + ht.numel() * 4 + hl.numel() * 4
+    d2h = hout.numel() * 2 + (hlse.numel() * 4 if hlse is not None else 0)
+    e2e_steps = 0 if args.no_e2e else max(10, args.steps // 2)
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(e2e_steps)]
+    with torch.cuda.stream(stream):
+        for i in range(-3 if e2e_steps else 0, e2e_steps):
+            flush.fill_(float(i))
+            if i >= 0:
+                e2e_ev[i][0].record(stream)
+            q.copy_(hq, non_blocking=True)
+            tables.copy_(ht, non_blocking=True)
+            lens.copy_(hl, non_blocking=True)
+            pad.pad_decode(q, k, v, tables, lens, w.scale, num_splits=splits, out=out, lse=lse, stream=stream)
+            hout.copy_(out, non_blocking=True)
+            if hlse is not None:
+                hlse.copy_(lse, non_blocking=True)
+            if i >= 0:
+                e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(e[0].elapsed_time(e[1]) for e in e2e_ev) if e2e_steps else float("nan")
+    if world > 1 and e2e_steps:
+        t = torch.tensor([e2e_ms / e2e_steps * args.steps], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    else:
+        e2e_total = e2e_ms / max(e2e_steps, 1) * args.steps
+    e2e_value = all_bytes / (e2e_total / 1e3) / 1e9
+
+    errs = pad.pad_check_device_errors(stream)
+    if errs:
+        raise SystemExit(f"device error word {errs:#x}")
+
+    if rank == 0:
+        peak, peak_kind = measured_peaks()
+        p_bytes = partition_bytes(w, S)
+        p_ms = statistics.mean(part_ms)
+        achieved = p_bytes / (p_ms / 1e3) / 1e9
+        sha = kernel_source_sha()
+        traffic = traffic_from_profiles(w.name, sha)
+        kname = f"partition_kernel<{w.D},{plan['heads_per_tile'] // 8}>"
+        line = {
+            "metric": "decode attention µs/call and achieved HBM GB/s vs B200 peak (1 GPU)",
+            "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 5), "us_per_call": round(total_ms / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded counter-based generator; no dataset)",
+            "config": workload_config(w, plan),
+            "hbm_frac_of_peak": round(value / peak, 4),
+            "phases_us": {"partition": round(p_ms * 1e3, 2), "reduce": round(statistics.mean(red_ms) * 1e3, 2)},
+            "roofline": {"kernel": kname, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                         "peak_kind": f"{peak_kind} copy bandwidth", "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "algorithmic_bytes_per_launch": p_bytes, "traffic": traffic, "source_sha": sha},
+            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "us_per_call": round(e2e_total / args.steps * 1e3, 2), "api": "pad_decode"},
+            "gpu_launches": args.steps * (2 if plan["reduce"] else 1),
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            cb = cpu_baseline(w, args.cpu_seconds)
+            line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,196 @@
+/*
+ * pad.h -- C ABI of the paged-KV single-token decode attention library (libpad).
+ *
+ * The operation: for every sequence b of a decode batch, one query token per
+ * query head attends over the L_b tokens of that sequence held in a paged KV
+ * cache, the pages being named by the sequence's row of a block table.  This is
+ * the problem of "spec(BACKEND-ROCM): the ROCm head_dim=128 decode arm, the ROCm
+ * half of #382" (vllm.cpp PR #564, section "The gap it specs": bf16 paged decode
+ * attention for head_dim 128 GQA models, one K/V read serving a GQA group) and of
+ * "perf(rocke): prepare saved paged decode bindings once" (rocm-libraries PR
+ * #13700, section "Summary": one-token split-KV attention with an optional
+ * log-sum-exp output; section "Runnable saved-binding HIP-event comparison":
+ * batch, heads, kv-heads, head-dim, seqlen-q = 1, seqlen-k, kv-block-size).
+ *
+ * Math (natural log; `scale` multiplies q.k before the softmax):
+ *   kh = h / (Hq / Hkv)                      consecutive query heads share a KV head
+ *   token t < L_b sits in block block_tables[b][t / bs], slot t % bs
+ *   s_t = scale * <q[b,h,:], K[block, kh, slot, :]>
+ *   out[b,h,:] = sum_t softmax(s)_t * V[block, kh, slot, :]     (bf16, RNE once)
+ *   lse[b,h]   = log(sum_t exp(s_t))                             (fp32)
+ *   L_b = 0 gives out = 0 and lse = -inf.
+ *
+ * How it runs on the device: a partition kernel splits each sequence's tokens
+ * into partitions of P tokens (P a multiple of bs); each CTA streams one
+ * partition's K/V pages for one KV head through shared memory once, serves all
+ * query heads of the GQA group from that read, and keeps a running max/sum
+ * (online softmax) in fp32.  With more than one partition a reduce kernel merges
+ * the partial outputs weighted by their log-sum-exp.
+ *
+ * Conventions for every entry point:
+ *  - All tensor data pointers are DEVICE pointers owned by the caller.  The
+ *    library never frees them and keeps no reference after the call returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  Outputs are valid once the stream has completed the work; inputs
+ *    must stay alive and unmodified until then.
+ *  - On any validation failure the call returns before launching anything and
+ *    writes nothing: `out` and `lse` are left untouched.
+ *  - Device-resident data that cannot be checked without a synchronisation
+ *    (block ids, seq_lens) must be valid: 0 <= block id < num_blocks for every
+ *    live page, 0 <= seq_lens[b] <= max_blocks_per_seq * block_size.  The kernels
+ *    check both anyway; a violation is never dereferenced (the page is skipped,
+ *    the length clamped), and sets a sticky per-device error word reported by
+ *    pad_check_device_errors().
+ */
+#ifndef PAD_H
+#define PAD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PAD_ABI_VERSION 1
+
+typedef enum pad_status {
+  PAD_OK = 0,
+  PAD_ERR_INVALID_ARG = 1,  /* bad dtype, shape, stride, alignment or scalar */
+  PAD_ERR_UNSUPPORTED = 2,  /* valid problem outside the compiled envelope */
+  PAD_ERR_WORKSPACE = 3,    /* split scratch could not be obtained (e.g. growth under capture) */
+  PAD_ERR_CUDA = 4,         /* a CUDA runtime call failed; see pad_last_error() */
+  PAD_ERR_DEVICE_CHECK = 5  /* a kernel saw an invalid block id or sequence length */
+} pad_status;
+
+typedef enum pad_dtype { PAD_BF16 = 0, PAD_F32 = 1, PAD_I32 = 2 } pad_dtype;
+
+/* A strided tensor view.  `stride` is in ELEMENTS.  Unused trailing dims are
+ * ignored.  `dtype` holds a pad_dtype value. */
+typedef struct pad_tensor {
+  void *data;
+  int32_t dtype;
+  int32_t ndim;
+  int64_t shape[4];
+  int64_t stride[4];
+} pad_tensor;
+
+/* Launch plan chosen for one problem shape. */
+typedef struct pad_plan {
+  int32_t num_splits;        /* effective number of partitions per sequence (S) */
+  int32_t partition_tokens;  /* P, tokens per partition, a multiple of block_size */
+  int32_t heads_per_tile;    /* query heads handled per CTA, padded (8, 16 or 32) */
+  int32_t head_tiles;        /* CTAs per (sequence, KV head, partition): ceil(group / heads_per_tile) */
+  int32_t warps_per_cta;     /* warps in the partition kernel's CTA */
+  int32_t stage_tokens;      /* tokens per shared-memory pipeline stage */
+  int32_t stages;            /* pipeline depth */
+  int32_t ctas;              /* partition-kernel CTAs launched (B * Hkv * head_tiles * S) */
+  int32_t reduce;            /* 1 when the split-reduce kernel runs (S > 1) */
+  int64_t workspace_bytes;   /* split scratch the call needs (0 when S == 1) */
+} pad_plan;
+
+/*
+ * pad_decode -- paged single-token decode attention.
+ *
+ *  q             bf16 [B, Hq, D], stride[2] == 1, every row 16-byte aligned.
+ *  k_cache       bf16 [num_blocks, Hkv, block_size, D], stride[3] == 1; dims 0-2
+ *                may have any non-negative strides whose byte size is a multiple
+ *                of 16 (so both [blocks, Hkv, bs, D] "HND" and a permuted view of a
+ *                [blocks, bs, Hkv, D] "NHD" cache are accepted).  Base 16-byte aligned.
+ *  v_cache       bf16, same shape as k_cache, its own strides, same rules.
+ *  block_tables  int32 [B, max_blocks_per_seq], stride[1] == 1.  Entries past
+ *                ceil(L_b / block_size) are never read.
+ *  seq_lens      int32 [B], contiguous.
+ *  scale         finite; multiplies q.k before the softmax (commonly 1/sqrt(D)).
+ *  num_splits    0 = let the library choose; S >= 1 asks for partitions of
+ *                P = round_up(ceil(C / S), block_size) tokens, C =
+ *                max_blocks_per_seq * block_size (the effective S = ceil(C / P) is
+ *                reported by pad_decode_plan).  S == 1 skips the reduce kernel.
+ *  out           bf16 [B, Hq, D], stride[2] == 1, rows 16-byte aligned.  Must not
+ *                overlap any input.
+ *  lse           NULL = no log-sum-exp output (nothing else is written); else
+ *                fp32 [B, Hq], any strides.  A non-NULL lse whose shape is wrong
+ *                is an error, never silently dropped.
+ *  stream        cudaStream_t.
+ *
+ * Supported envelope: D in {64, 128, 256}; Hq / Hkv <= 256; block_size a power of
+ * two in [1, 256].  Split scratch is owned by the library, kept per (device,
+ * stream) and grown on demand; growing it while `stream` is being captured into a
+ * CUDA graph returns PAD_ERR_WORKSPACE (call once outside capture first).
+ */
+pad_status pad_decode(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
+                      const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
+                      int32_t num_splits, pad_tensor *out, pad_tensor *lse, void *stream);
+
+/*
+ * pad_decode_partition / pad_decode_reduce -- the two passes of pad_decode run
+ * one at a time, with split scratch supplied by the caller instead of the
+ * library ("perf(rocke): prepare saved paged decode bindings once", section
+ * "Summary": a split-KV pass, then a reduce pass that reads the partials and
+ * writes the output and, when requested, the LSE).
+ *
+ * Arguments are those of pad_decode plus `workspace`: DEVICE memory owned by the
+ * caller, 256-byte aligned, of at least pad_decode_plan(...).workspace_bytes
+ * bytes (it may be NULL when that is 0).  Both calls must see the same arguments
+ * and the same workspace, in order on one stream (or with the caller ordering
+ * them).  The workspace holds, for every (b, query head, partition), the fp32
+ * output normalised by its own softmax sum ([B, Hq, S, D]) and, after it at the
+ * next 256-byte boundary, the partition's fp32 natural-log LSE ([B, Hq, S]);
+ * partitions past ceil(L_b / P) are neither written nor read.
+ *
+ * pad_decode_partition with S == 1 writes `out`/`lse` directly and touches no
+ * workspace; pad_decode_reduce then returns PAD_OK without launching.  The
+ * workspace must not be shared by calls that may run concurrently.
+ */
+pad_status pad_decode_partition(const pad_tensor *q, const pad_tensor *k_cache,
+                                const pad_tensor *v_cache, const pad_tensor *block_tables,
+                                const pad_tensor *seq_lens, float scale, int32_t num_splits,
+                                pad_tensor *out, pad_tensor *lse, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+pad_status pad_decode_reduce(const pad_tensor *q, const pad_tensor *k_cache,
+                             const pad_tensor *v_cache, const pad_tensor *block_tables,
+                             const pad_tensor *seq_lens, float scale, int32_t num_splits,
+                             pad_tensor *out, pad_tensor *lse, void *workspace,
+                             size_t workspace_bytes, void *stream);
+
+/*
+ * pad_decode_plan -- the launch geometry pad_decode would use for this shape
+ * (the per-shape heuristic when num_splits == 0).  Pure host computation; no
+ * launch.  `device` < 0 means the current device (its SM count feeds the
+ * heuristic).  Returns PAD_ERR_INVALID_ARG / PAD_ERR_UNSUPPORTED exactly when
+ * pad_decode would for the same shape.
+ */
+pad_status pad_decode_plan(int64_t batch, int64_t num_q_heads, int64_t num_kv_heads,
+                           int64_t head_dim, int64_t block_size, int64_t max_blocks_per_seq,
+                           int32_t num_splits, int32_t device, pad_plan *plan);
+
+/* Static string for a status code. */
+const char *pad_status_string(pad_status status);
+
+/* Message for the last failure on the calling thread ("" if none). */
+const char *pad_last_error(void);
+
+/*
+ * pad_check_device_errors -- synchronises `stream`, then reads and clears the
+ * current device's sticky error word.  Returns PAD_ERR_DEVICE_CHECK if any kernel
+ * since the last check saw an invalid block id (bit 0x1) or sequence length
+ * (bit 0x2); the bits are stored in *bits when bits != NULL.
+ */
+pad_status pad_check_device_errors(void *stream, uint32_t *bits);
+
+/*
+ * pad_release_workspace -- frees the split scratch held for `device` (< 0: all
+ * devices) after synchronising that device.  Safe to call at any time outside
+ * stream capture; later calls re-grow scratch on demand.
+ */
+pad_status pad_release_workspace(int32_t device);
+
+/* PAD_ABI_VERSION of the loaded library. */
+int32_t pad_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAD_H */

@@ -1,0 +1,229 @@
+"""Paged-KV single-token decode attention for B200 (sm_100a).
+
+A thin Python binding over the C ABI in ``include/pad.h`` (``libpad.so``): it
+turns torch tensors into ``pad_tensor`` descriptors and calls the library.  All
+arithmetic runs in the library's CUDA kernels; there is no Python or CPU
+fallback, and the import fails loudly if ``libpad.so`` has not been built
+(``python -m paged_kv_attention_partition_b200._build``).
+
+Functions carry the C names: ``pad_decode``, ``pad_decode_plan``,
+``pad_check_device_errors``, ``pad_release_workspace``, ``pad_status_string``,
+``pad_last_error``, ``pad_abi_version``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple, Union
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpad.so")
+
+PAD_OK, PAD_ERR_INVALID_ARG, PAD_ERR_UNSUPPORTED, PAD_ERR_WORKSPACE, PAD_ERR_CUDA, PAD_ERR_DEVICE_CHECK = range(6)
+PAD_BF16, PAD_F32, PAD_I32 = 0, 1, 2
+_DTYPES = {torch.bfloat16: PAD_BF16, torch.float32: PAD_F32, torch.int32: PAD_I32}
+
+
+class PadTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+class PadPlan(ctypes.Structure):
+    _fields_ = [("num_splits", ctypes.c_int32), ("partition_tokens", ctypes.c_int32),
+                ("heads_per_tile", ctypes.c_int32), ("head_tiles", ctypes.c_int32),
+                ("warps_per_cta", ctypes.c_int32), ("stage_tokens", ctypes.c_int32),
+                ("stages", ctypes.c_int32), ("ctas", ctypes.c_int32), ("reduce", ctypes.c_int32),
+                ("workspace_bytes", ctypes.c_int64)]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+class PadError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{_status_name(status)}: {message}")
+        self.status = status
+
+
+def _status_name(st: int) -> str:
+    return ("PAD_OK", "PAD_ERR_INVALID_ARG", "PAD_ERR_UNSUPPORTED", "PAD_ERR_WORKSPACE",
+            "PAD_ERR_CUDA", "PAD_ERR_DEVICE_CHECK")[st] if 0 <= st < 6 else f"status {st}"
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libpad.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m paged_kv_attention_partition_b200._build`")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(PadTensor)
+    lib.pad_decode.argtypes = [P, P, P, P, P, ctypes.c_float, ctypes.c_int32, P, P, ctypes.c_void_p]
+    lib.pad_decode.restype = ctypes.c_int
+    for name in ("pad_decode_partition", "pad_decode_reduce"):
+        fn = getattr(lib, name)
+        fn.argtypes = [P, P, P, P, P, ctypes.c_float, ctypes.c_int32, P, P, ctypes.c_void_p, ctypes.c_size_t,
+                       ctypes.c_void_p]
+        fn.restype = ctypes.c_int
+    lib.pad_decode_plan.argtypes = [ctypes.c_int64] * 6 + [ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(PadPlan)]
+    lib.pad_decode_plan.restype = ctypes.c_int
+    lib.pad_status_string.argtypes = [ctypes.c_int]
+    lib.pad_status_string.restype = ctypes.c_char_p
+    lib.pad_last_error.argtypes = []
+    lib.pad_last_error.restype = ctypes.c_char_p
+    lib.pad_check_device_errors.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]
+    lib.pad_check_device_errors.restype = ctypes.c_int
+    lib.pad_release_workspace.argtypes = [ctypes.c_int32]
+    lib.pad_release_workspace.restype = ctypes.c_int
+    lib.pad_abi_version.argtypes = []
+    lib.pad_abi_version.restype = ctypes.c_int32
+    _lib = lib
+    return lib
+
+
+def pad_last_error() -> str:
+    return load_library().pad_last_error().decode()
+
+
+def pad_status_string(status: int) -> str:
+    return load_library().pad_status_string(status).decode()
+
+
+def pad_abi_version() -> int:
+    return load_library().pad_abi_version()
+
+
+def _raise(st: int):
+    if st != PAD_OK:
+        raise PadError(st, pad_last_error())
+
+
+def describe(t: torch.Tensor) -> PadTensor:
+    """pad_tensor descriptor of a torch tensor (pointer, dtype, shape, element strides)."""
+    if t.dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    if t.dim() > 4:
+        raise ValueError("at most 4 dims")
+    d = PadTensor()
+    d.data = t.data_ptr()
+    d.dtype = _DTYPES[t.dtype]
+    d.ndim = t.dim()
+    for i in range(t.dim()):
+        d.shape[i] = t.shape[i]
+        d.stride[i] = t.stride(i)
+    return d
+
+
+def _stream_handle(stream, device) -> int:
+    if stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def pad_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
+               seq_lens: torch.Tensor, scale: float, num_splits: int = 0, out: Optional[torch.Tensor] = None,
+               lse: Union[None, bool, torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Paged single-token decode attention (see ``pad_decode`` in include/pad.h).
+
+    q [B, Hq, D] bf16; k_cache/v_cache [num_blocks, Hkv, block_size, D] bf16 (any
+    16-byte-multiple strides on dims 0-2, e.g. ``nhd.transpose(1, 2)``);
+    block_tables [B, W] int32; seq_lens [B] int32.  ``lse=True`` allocates the
+    fp32 [B, Hq] log-sum-exp output, a tensor receives it, None skips it.
+    Returns (out, lse).  Asynchronous on ``stream`` (default: torch's current)."""
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("q must be a CUDA tensor")
+    for name, t in (("k_cache", k_cache), ("v_cache", v_cache), ("block_tables", block_tables),
+                    ("seq_lens", seq_lens)):
+        if t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, q on {dev}")
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    if lse is True:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+    elif lse is False:
+        lse = None
+    for name, t in (("out", out), ("lse", lse)):
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, q on {dev}")
+    lib = load_library()
+    dq, dk, dv, dt, dl, do = (describe(t) for t in (q, k_cache, v_cache, block_tables, seq_lens, out))
+    dlse = describe(lse) if lse is not None else None
+    with torch.cuda.device(dev):
+        st = lib.pad_decode(ctypes.byref(dq), ctypes.byref(dk), ctypes.byref(dv), ctypes.byref(dt),
+                            ctypes.byref(dl), float(scale), int(num_splits), ctypes.byref(do),
+                            ctypes.byref(dlse) if dlse is not None else None, _stream_handle(stream, dev))
+    _raise(st)
+    return out, lse
+
+
+def _phase(fn_name, q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, workspace, stream):
+    dev = q.device
+    if workspace is not None and (workspace.device != dev or not workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous tensor on q's device")
+    descs = [describe(t) for t in (q, k_cache, v_cache, block_tables, seq_lens, out)]
+    dlse = describe(lse) if lse is not None else None
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    with torch.cuda.device(dev):
+        st = getattr(load_library(), fn_name)(
+            *(ctypes.byref(d) for d in descs[:5]), float(scale), int(num_splits), ctypes.byref(descs[5]),
+            ctypes.byref(dlse) if dlse is not None else None, ws_ptr, ws_bytes, _stream_handle(stream, dev))
+    _raise(st)
+
+
+def pad_decode_partition(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, workspace,
+                         stream=None) -> None:
+    """First pass only (see include/pad.h); ``workspace`` is a caller-owned device
+    tensor of at least ``pad_decode_plan(...)["workspace_bytes"]`` bytes."""
+    _phase("pad_decode_partition", q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse,
+           workspace, stream)
+
+
+def pad_decode_reduce(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, workspace,
+                      stream=None) -> None:
+    """Second pass only: merges the partitions pad_decode_partition left in ``workspace``."""
+    _phase("pad_decode_reduce", q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse,
+           workspace, stream)
+
+
+def pad_decode_plan(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, block_size: int,
+                    max_blocks_per_seq: int, num_splits: int = 0, device: int = -1) -> dict:
+    """Launch geometry pad_decode would use for this shape (no launch)."""
+    plan = PadPlan()
+    st = load_library().pad_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, block_size,
+                                        max_blocks_per_seq, num_splits, device, ctypes.byref(plan))
+    _raise(st)
+    return plan.as_dict()
+
+
+def pad_check_device_errors(stream=None, device=None) -> int:
+    """Synchronise, then read and clear the device's sticky error word.  Returns
+    the bits: 0 = clean, 0x1 = an out-of-range block id, 0x2 = an out-of-range
+    sequence length.  Raises PadError only when the check itself fails."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    bits = ctypes.c_uint32(0)
+    with torch.cuda.device(dev):
+        st = load_library().pad_check_device_errors(_stream_handle(stream, dev), ctypes.byref(bits))
+    if st not in (PAD_OK, PAD_ERR_DEVICE_CHECK):
+        _raise(st)
+    return bits.value
+
+
+def pad_release_workspace(device: int = -1) -> None:
+    """Free the library's split scratch for one device (all when < 0)."""
+    _raise(load_library().pad_release_workspace(device))
+
+
+__all__ = ["pad_decode", "pad_decode_partition", "pad_decode_reduce", "pad_decode_plan", "pad_check_device_errors", "pad_release_workspace",
+           "pad_status_string", "pad_last_error", "pad_abi_version", "describe", "load_library",
+           "PadError", "PadTensor", "PadPlan"]

@@ -1,0 +1,500 @@
+// Host side of libpad: argument validation, the per-shape launch plan, the
+// library-owned split scratch, and the two launches.  Declared in include/pad.h.
+#include "pad.h"
+
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <map>
+#include <mutex>
+#include <string>
+#include <utility>
+
+#include "pad_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+pad_status fail(pad_status st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+pad_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(PAD_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int ilog2(int64_t x) {
+  int r = 0;
+  while ((1ll << r) < x) ++r;
+  return r;
+}
+
+// ---- shape checks (no data access) ----------------------------------------
+
+struct Shape {
+  int64_t B, Hq, Hkv, D, bs, W, g;
+};
+
+pad_status check_shape(const Shape &s, int32_t num_splits) {
+  if (s.B < 0 || s.Hq <= 0 || s.Hkv <= 0 || s.D <= 0 || s.bs <= 0 || s.W <= 0)
+    return fail(PAD_ERR_INVALID_ARG, "sizes must be positive (B >= 0): B=%lld Hq=%lld Hkv=%lld D=%lld bs=%lld W=%lld",
+                (long long)s.B, (long long)s.Hq, (long long)s.Hkv, (long long)s.D, (long long)s.bs,
+                (long long)s.W);
+  if (s.Hq % s.Hkv != 0)
+    return fail(PAD_ERR_INVALID_ARG, "num_q_heads (%lld) must be a multiple of num_kv_heads (%lld)",
+                (long long)s.Hq, (long long)s.Hkv);
+  if (num_splits < 0) return fail(PAD_ERR_INVALID_ARG, "num_splits must be >= 0 (got %d)", num_splits);
+  if (s.D != 64 && s.D != 128 && s.D != 256)
+    return fail(PAD_ERR_UNSUPPORTED, "head_dim %lld not supported (64, 128, 256)", (long long)s.D);
+  if (!is_pow2(s.bs) || s.bs > 256)
+    return fail(PAD_ERR_UNSUPPORTED, "block_size %lld must be a power of two in [1, 256]", (long long)s.bs);
+  if (s.g > 256)
+    return fail(PAD_ERR_UNSUPPORTED, "GQA group %lld exceeds 256 query heads per KV head", (long long)s.g);
+  if (s.W * s.bs > (int64_t)1 << 30)
+    return fail(PAD_ERR_UNSUPPORTED, "table capacity %lld tokens too large", (long long)(s.W * s.bs));
+  return PAD_OK;
+}
+
+int sm_count(int device) {
+  static int cache[64] = {0};
+  if (device < 0 || device >= 64) return 148;
+  if (cache[device] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = 148;
+    }
+    cache[device] = n;
+  }
+  return cache[device];
+}
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// Per-shape launch plan.  The lengths live on the device, so the plan sees only
+// the table capacity C = W * bs.  Partitions are whole pages.  With num_splits==0:
+// the partition is the smallest size that keeps the split scratch traffic (2 * g
+// * D * 4 bytes written and read back per partition) under ~1/16 of the K/V bytes
+// it streams (4 * D * P), and at least 256 tokens, so that many CTAs keep every
+// SM busy and the longest CTA stays short even on ragged batches.
+void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan) {
+  const int64_t C = s.W * s.bs;
+  int hpt = s.g <= 8 ? 8 : (s.g <= 16 ? 16 : 32);
+  if (hpt > pad::max_heads_per_tile((int)s.D)) hpt = pad::max_heads_per_tile((int)s.D);
+  const int64_t HT = (s.g + hpt - 1) / hpt;
+  int64_t P;
+  if (num_splits >= 1) {
+    P = round_up((C + num_splits - 1) / num_splits, s.bs);
+  } else {
+    int64_t p_min = 32 * s.g;
+    if (p_min < 256) p_min = 256;
+    P = round_up(p_min, 64);
+    P = round_up(P, s.bs);
+    // never more than ~64 waves of CTAs at two per SM
+    const int64_t units = s.B * s.Hkv * HT;
+    const int64_t max_ctas = (int64_t)sm_count(device < 0 ? 0 : device) * 2 * 64;
+    while (units > 0 && units * ((C + P - 1) / P) > max_ctas && P < C) P *= 2;
+  }
+  if (P > round_up(C, s.bs)) P = round_up(C, s.bs);
+  if (P < s.bs) P = s.bs;
+  const int64_t S = (C + P - 1) / P;
+  plan->num_splits = (int32_t)S;
+  plan->partition_tokens = (int32_t)P;
+  plan->heads_per_tile = hpt;
+  plan->head_tiles = (int32_t)HT;
+  plan->warps_per_cta = pad::kWarps;
+  plan->stage_tokens = pad::kStageTokens;
+  plan->stages = pad::stages_for((int)s.D);
+  plan->ctas = (int64_t)(s.B * s.Hkv * HT * S) > 0x7fffffffll ? 0x7fffffff : (int32_t)(s.B * s.Hkv * HT * S);
+  plan->reduce = S > 1 ? 1 : 0;
+  plan->workspace_bytes = S > 1 ? (int64_t)(round_up(s.B * s.Hq * S * s.D * 4, 256) + round_up(s.B * s.Hq * S * 4, 256)) : 0;
+}
+
+// ---- tensor descriptor checks -----------------------------------------------
+
+pad_status check_tensor(const pad_tensor *t, const char *name, pad_dtype dt, int ndim) {
+  if (t == nullptr) return fail(PAD_ERR_INVALID_ARG, "%s is NULL", name);
+  if (t->data == nullptr) return fail(PAD_ERR_INVALID_ARG, "%s.data is NULL", name);
+  if (t->dtype != dt) return fail(PAD_ERR_INVALID_ARG, "%s has dtype %d, expected %d", name, t->dtype, (int)dt);
+  if (t->ndim != ndim) return fail(PAD_ERR_INVALID_ARG, "%s has %d dims, expected %d", name, t->ndim, ndim);
+  for (int i = 0; i < ndim; ++i) {
+    if (t->shape[i] < 0) return fail(PAD_ERR_INVALID_ARG, "%s.shape[%d] < 0", name, i);
+    if (t->stride[i] < 0) return fail(PAD_ERR_INVALID_ARG, "%s.stride[%d] < 0", name, i);
+  }
+  return PAD_OK;
+}
+
+// rows of 16-bit elements along the last dim must be contiguous and 16-byte aligned
+pad_status check_rows16(const pad_tensor *t, const char *name) {
+  const int last = t->ndim - 1;
+  if (t->stride[last] != 1) return fail(PAD_ERR_INVALID_ARG, "%s: last dim must be contiguous", name);
+  if (reinterpret_cast<uintptr_t>(t->data) % 16 != 0)
+    return fail(PAD_ERR_INVALID_ARG, "%s: data must be 16-byte aligned", name);
+  for (int i = 0; i < last; ++i)
+    if ((t->stride[i] * 2) % 16 != 0 && t->shape[i] > 1)
+      return fail(PAD_ERR_INVALID_ARG, "%s: stride[%d]=%lld is not a multiple of 16 bytes", name, i,
+                  (long long)t->stride[i]);
+  return PAD_OK;
+}
+
+pad_status check_device_ptr(const void *p, int device, const char *name) {
+  cudaPointerAttributes a;
+  cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(PAD_ERR_INVALID_ARG, "%s: not a CUDA pointer (%s)", name, cudaGetErrorString(e));
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+    return fail(PAD_ERR_INVALID_ARG, "%s: must be device memory", name);
+  if (a.type == cudaMemoryTypeDevice && a.device != device)
+    return fail(PAD_ERR_INVALID_ARG, "%s: lives on device %d, current device is %d", name, a.device, device);
+  return PAD_OK;
+}
+
+// ---- library-owned split scratch, one buffer per (device, stream) -----------
+
+struct Workspace {
+  void *ptr = nullptr;
+  size_t bytes = 0;
+};
+std::mutex g_ws_mu;
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+
+pad_status get_workspace(int device, cudaStream_t stream, size_t bytes, void **out) {
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  Workspace &w = g_ws[{device, stream}];
+  if (w.bytes >= bytes) {
+    *out = w.ptr;
+    return PAD_OK;
+  }
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(stream, &cs);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+  if (cs != cudaStreamCaptureStatusNone)
+    return fail(PAD_ERR_WORKSPACE,
+                "split scratch must grow to %zu bytes while the stream is being captured; "
+                "run one call with this shape outside capture first", bytes);
+  if (w.ptr != nullptr) {
+    // queued work on this stream may still read the old buffer
+    e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    cudaFree(w.ptr);
+    w.ptr = nullptr;
+    w.bytes = 0;
+  }
+  size_t want = bytes + bytes / 4;  // headroom for nearby shapes
+  e = cudaMalloc(&w.ptr, want);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    e = cudaMalloc(&w.ptr, bytes);
+    want = bytes;
+  }
+  if (e != cudaSuccess) {
+    w.ptr = nullptr;
+    return fail(PAD_ERR_WORKSPACE, "cudaMalloc(%zu) for split scratch failed: %s", bytes, cudaGetErrorString(e));
+  }
+  w.bytes = want;
+  *out = w.ptr;
+  return PAD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t pad_abi_version(void) { return PAD_ABI_VERSION; }
+
+const char *pad_status_string(pad_status st) {
+  switch (st) {
+    case PAD_OK: return "PAD_OK";
+    case PAD_ERR_INVALID_ARG: return "PAD_ERR_INVALID_ARG";
+    case PAD_ERR_UNSUPPORTED: return "PAD_ERR_UNSUPPORTED";
+    case PAD_ERR_WORKSPACE: return "PAD_ERR_WORKSPACE";
+    case PAD_ERR_CUDA: return "PAD_ERR_CUDA";
+    case PAD_ERR_DEVICE_CHECK: return "PAD_ERR_DEVICE_CHECK";
+  }
+  return "PAD_ERR_UNKNOWN";
+}
+
+const char *pad_last_error(void) { return g_last_error.c_str(); }
+
+pad_status pad_decode_plan(int64_t batch, int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
+                           int64_t block_size, int64_t max_blocks_per_seq, int32_t num_splits,
+                           int32_t device, pad_plan *plan) {
+  if (plan == nullptr) return fail(PAD_ERR_INVALID_ARG, "plan is NULL");
+  Shape s{batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+          num_kv_heads > 0 ? num_q_heads / num_kv_heads : 0};
+  pad_status st = check_shape(s, num_splits);
+  if (st != PAD_OK) return st;
+  if (device < 0) {
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess) {
+      cudaGetLastError();
+      d = -1;
+    }
+    device = d;
+  }
+  make_plan(s, num_splits, device, plan);
+  if ((int64_t)plan->ctas > 0x7fffffffll / 2)
+    return fail(PAD_ERR_UNSUPPORTED, "too many CTAs for one launch");
+  return PAD_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Everything one call needs after validation: kernel parameters and the plan.
+struct Prepared {
+  pad::PartitionParams p;
+  pad_plan plan;
+  int D;
+  int device;
+};
+
+pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
+                   const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale, int32_t num_splits,
+                   const pad_tensor *out, const pad_tensor *lse, Prepared *pr, bool *empty) {
+  pad_status st;
+  *empty = false;
+  if ((st = check_tensor(q, "q", PAD_BF16, 3)) != PAD_OK) return st;
+  if ((st = check_tensor(k_cache, "k_cache", PAD_BF16, 4)) != PAD_OK) return st;
+  if ((st = check_tensor(v_cache, "v_cache", PAD_BF16, 4)) != PAD_OK) return st;
+  if ((st = check_tensor(block_tables, "block_tables", PAD_I32, 2)) != PAD_OK) return st;
+  if ((st = check_tensor(seq_lens, "seq_lens", PAD_I32, 1)) != PAD_OK) return st;
+  if ((st = check_tensor(out, "out", PAD_BF16, 3)) != PAD_OK) return st;
+  if (lse != nullptr && (st = check_tensor(lse, "lse", PAD_F32, 2)) != PAD_OK) return st;
+
+  const int64_t B = q->shape[0], Hq = q->shape[1], D = q->shape[2];
+  const int64_t NB = k_cache->shape[0], Hkv = k_cache->shape[1], bs = k_cache->shape[2];
+  for (int i = 0; i < 4; ++i)
+    if (v_cache->shape[i] != k_cache->shape[i])
+      return fail(PAD_ERR_INVALID_ARG, "v_cache.shape[%d]=%lld differs from k_cache", i, (long long)v_cache->shape[i]);
+  if (k_cache->shape[3] != D)
+    return fail(PAD_ERR_INVALID_ARG, "k_cache head_dim %lld != q head_dim %lld", (long long)k_cache->shape[3], (long long)D);
+  if (block_tables->shape[0] != B)
+    return fail(PAD_ERR_INVALID_ARG, "block_tables has %lld rows, batch is %lld", (long long)block_tables->shape[0], (long long)B);
+  if (block_tables->stride[1] != 1 && block_tables->shape[1] > 1)
+    return fail(PAD_ERR_INVALID_ARG, "block_tables rows must be contiguous");
+  if (seq_lens->shape[0] != B)
+    return fail(PAD_ERR_INVALID_ARG, "seq_lens has %lld entries, batch is %lld", (long long)seq_lens->shape[0], (long long)B);
+  if (seq_lens->stride[0] != 1 && B > 1) return fail(PAD_ERR_INVALID_ARG, "seq_lens must be contiguous");
+  if (out->shape[0] != B || out->shape[1] != Hq || out->shape[2] != D)
+    return fail(PAD_ERR_INVALID_ARG, "out shape must equal q shape [%lld, %lld, %lld]", (long long)B, (long long)Hq, (long long)D);
+  if (lse != nullptr && (lse->shape[0] != B || lse->shape[1] != Hq))
+    return fail(PAD_ERR_INVALID_ARG, "lse shape must be [B, Hq] = [%lld, %lld]", (long long)B, (long long)Hq);
+  if (!isfinite(scale)) return fail(PAD_ERR_INVALID_ARG, "scale must be finite");
+  if (NB <= 0 || NB > 0x7fffffffll) return fail(PAD_ERR_INVALID_ARG, "num_blocks %lld out of range", (long long)NB);
+  if ((st = check_rows16(q, "q")) != PAD_OK) return st;
+  if ((st = check_rows16(k_cache, "k_cache")) != PAD_OK) return st;
+  if ((st = check_rows16(v_cache, "v_cache")) != PAD_OK) return st;
+  if ((st = check_rows16(out, "out")) != PAD_OK) return st;
+  if (reinterpret_cast<uintptr_t>(block_tables->data) % 4 || reinterpret_cast<uintptr_t>(seq_lens->data) % 4 ||
+      (lse != nullptr && reinterpret_cast<uintptr_t>(lse->data) % 4))
+    return fail(PAD_ERR_INVALID_ARG, "int32/fp32 tensors must be 4-byte aligned");
+
+  Shape s{B, Hq, Hkv, D, bs, block_tables->shape[1], Hkv > 0 ? Hq / Hkv : 0};
+  if ((st = check_shape(s, num_splits)) != PAD_OK) return st;
+  if (B == 0) {
+    *empty = true;
+    return PAD_OK;
+  }
+
+  int device = 0;
+  cudaError_t e = cudaGetDevice(&device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if ((st = check_device_ptr(q->data, device, "q")) != PAD_OK) return st;
+  if ((st = check_device_ptr(k_cache->data, device, "k_cache")) != PAD_OK) return st;
+  if ((st = check_device_ptr(v_cache->data, device, "v_cache")) != PAD_OK) return st;
+  if ((st = check_device_ptr(block_tables->data, device, "block_tables")) != PAD_OK) return st;
+  if ((st = check_device_ptr(seq_lens->data, device, "seq_lens")) != PAD_OK) return st;
+  if ((st = check_device_ptr(out->data, device, "out")) != PAD_OK) return st;
+  if (lse != nullptr && (st = check_device_ptr(lse->data, device, "lse")) != PAD_OK) return st;
+
+  make_plan(s, num_splits, device, &pr->plan);
+  if ((int64_t)B * Hkv * pr->plan.head_tiles * pr->plan.num_splits > 0x7fffffffll)
+    return fail(PAD_ERR_UNSUPPORTED, "too many CTAs for one launch");
+
+  uint32_t *err = nullptr;
+  if ((e = pad::device_error_word(device, &err)) != cudaSuccess) return cuda_fail(e, "error word");
+
+  pad::PartitionParams &p = pr->p;
+  p = pad::PartitionParams{};
+  p.q = static_cast<const uint16_t *>(q->data);
+  p.q_sb = q->stride[0];
+  p.q_sh = q->stride[1];
+  p.k = static_cast<const uint16_t *>(k_cache->data);
+  p.v = static_cast<const uint16_t *>(v_cache->data);
+  p.k_sblk = k_cache->stride[0];
+  p.k_sh = k_cache->stride[1];
+  p.k_ss = k_cache->stride[2];
+  p.v_sblk = v_cache->stride[0];
+  p.v_sh = v_cache->stride[1];
+  p.v_ss = v_cache->stride[2];
+  p.tables = static_cast<const int32_t *>(block_tables->data);
+  p.table_stride = block_tables->stride[0];
+  p.max_blocks = (int32_t)block_tables->shape[1];
+  p.num_blocks = (int32_t)NB;
+  p.seq_lens = static_cast<const int32_t *>(seq_lens->data);
+  p.B = (int32_t)B;
+  p.Hq = (int32_t)Hq;
+  p.Hkv = (int32_t)Hkv;
+  p.g = (int32_t)(Hq / Hkv);
+  p.HT = pr->plan.head_tiles;
+  p.bs_log2 = ilog2(bs);
+  p.P = pr->plan.partition_tokens;
+  p.S = pr->plan.num_splits;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.out = static_cast<uint16_t *>(out->data);
+  p.o_sb = out->stride[0];
+  p.o_sh = out->stride[1];
+  p.lse = lse != nullptr ? static_cast<float *>(lse->data) : nullptr;
+  p.lse_sb = lse != nullptr ? lse->stride[0] : 0;
+  p.lse_sh = lse != nullptr ? lse->stride[1] : 0;
+  p.err = err;
+  pr->D = (int)D;
+  pr->device = device;
+  return PAD_OK;
+}
+
+void bind_workspace(Prepared &pr, void *ws) {
+  const int64_t opart = round_up((int64_t)pr.p.B * pr.p.Hq * pr.plan.num_splits * pr.D * 4, 256);
+  pr.p.o_part = static_cast<float *>(ws);
+  pr.p.lse_part = reinterpret_cast<float *>(static_cast<char *>(ws) + opart);
+}
+
+pad_status check_caller_workspace(const Prepared &pr, void *ws, size_t bytes) {
+  if (ws == nullptr) return fail(PAD_ERR_INVALID_ARG, "workspace is NULL but %lld bytes are needed", (long long)pr.plan.workspace_bytes);
+  if (bytes < (size_t)pr.plan.workspace_bytes)
+    return fail(PAD_ERR_INVALID_ARG, "workspace has %zu bytes, %lld needed", bytes, (long long)pr.plan.workspace_bytes);
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return fail(PAD_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  return check_device_ptr(ws, pr.device, "workspace");
+}
+
+pad_status run_partition(const Prepared &pr, cudaStream_t stream) {
+  cudaError_t e = pad::launch_partition(pr.p, pr.D, pr.plan.heads_per_tile, stream);
+  return e == cudaSuccess ? PAD_OK : cuda_fail(e, "partition kernel launch");
+}
+
+pad_status run_reduce(const Prepared &pr, cudaStream_t stream) {
+  pad::ReduceParams r{};
+  r.o_part = pr.p.o_part;
+  r.lse_part = pr.p.lse_part;
+  r.seq_lens = pr.p.seq_lens;
+  r.B = pr.p.B;
+  r.Hq = pr.p.Hq;
+  r.D = pr.D;
+  r.S = pr.p.S;
+  r.P = pr.p.P;
+  r.capacity = pr.p.max_blocks << pr.p.bs_log2;
+  r.out = pr.p.out;
+  r.o_sb = pr.p.o_sb;
+  r.o_sh = pr.p.o_sh;
+  r.lse = pr.p.lse;
+  r.lse_sb = pr.p.lse_sb;
+  r.lse_sh = pr.p.lse_sh;
+  cudaError_t e = pad::launch_reduce(r, stream);
+  return e == cudaSuccess ? PAD_OK : cuda_fail(e, "reduce kernel launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+pad_status pad_decode(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
+                      const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
+                      int32_t num_splits, pad_tensor *out, pad_tensor *lse, void *stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  Prepared pr;
+  bool empty = false;
+  pad_status st = prepare(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, &pr, &empty);
+  if (st != PAD_OK || empty) return st;
+  if (pr.plan.reduce) {
+    void *ws = nullptr;
+    if ((st = get_workspace(pr.device, stream, (size_t)pr.plan.workspace_bytes, &ws)) != PAD_OK) return st;
+    bind_workspace(pr, ws);
+  }
+  if ((st = run_partition(pr, stream)) != PAD_OK) return st;
+  return pr.plan.reduce ? run_reduce(pr, stream) : PAD_OK;
+}
+
+pad_status pad_decode_partition(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
+                                const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
+                                int32_t num_splits, pad_tensor *out, pad_tensor *lse, void *workspace,
+                                size_t workspace_bytes, void *stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  Prepared pr;
+  bool empty = false;
+  pad_status st = prepare(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, &pr, &empty);
+  if (st != PAD_OK || empty) return st;
+  if (pr.plan.reduce) {
+    if ((st = check_caller_workspace(pr, workspace, workspace_bytes)) != PAD_OK) return st;
+    bind_workspace(pr, workspace);
+  }
+  return run_partition(pr, stream);
+}
+
+pad_status pad_decode_reduce(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
+                             const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
+                             int32_t num_splits, pad_tensor *out, pad_tensor *lse, void *workspace,
+                             size_t workspace_bytes, void *stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  Prepared pr;
+  bool empty = false;
+  pad_status st = prepare(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, &pr, &empty);
+  if (st != PAD_OK || empty || !pr.plan.reduce) return st;
+  if ((st = check_caller_workspace(pr, workspace, workspace_bytes)) != PAD_OK) return st;
+  bind_workspace(pr, workspace);
+  return run_reduce(pr, stream);
+}
+
+pad_status pad_check_device_errors(void *stream_, uint32_t *bits) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int device = 0;
+  if ((e = cudaGetDevice(&device)) != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  uint32_t *word = nullptr;
+  if ((e = pad::device_error_word(device, &word)) != cudaSuccess) return cuda_fail(e, "error word");
+  uint32_t v = 0;
+  if ((e = cudaMemcpy(&v, word, 4, cudaMemcpyDeviceToHost)) != cudaSuccess) return cuda_fail(e, "read error word");
+  const uint32_t zero = 0;
+  if ((e = cudaMemcpy(word, &zero, 4, cudaMemcpyHostToDevice)) != cudaSuccess) return cuda_fail(e, "clear error word");
+  if (bits != nullptr) *bits = v;
+  if (v != 0)
+    return fail(PAD_ERR_DEVICE_CHECK, "kernel saw %s%s", (v & pad::kErrBlockId) ? "an out-of-range block id " : "",
+                (v & pad::kErrSeqLen) ? "an out-of-range sequence length" : "");
+  return PAD_OK;
+}
+
+pad_status pad_release_workspace(int32_t device) {
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  int cur = 0;
+  cudaError_t e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  for (auto it = g_ws.begin(); it != g_ws.end();) {
+    if (device >= 0 && it->first.first != device) {
+      ++it;
+      continue;
+    }
+    if ((e = cudaSetDevice(it->first.first)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    if (it->second.ptr != nullptr) cudaFree(it->second.ptr);
+    it = g_ws.erase(it);
+  }
+  if ((e = cudaSetDevice(cur)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  return PAD_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,167 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/pad.h declares, plans shapes, and rejects bad arguments before touching
+the device (no compute call is made here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import paged_kv_attention_partition_b200 as pad
+from paged_kv_attention_partition_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return pad.load_library()
+
+
+def declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w \*]*?\b(pad_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert {"pad_decode", "pad_decode_plan", "pad_status_string", "pad_last_error",
+            "pad_check_device_errors", "pad_release_workspace", "pad_abi_version"} <= set(names)
+    out = subprocess.run(["nm", "-D", "--defined-only", pad.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (\w+)$", out, flags=re.M))
+    missing = [n for n in names if n not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    for n in names:
+        getattr(lib, n)
+
+
+def test_library_is_built_for_sm100a():
+    cmd = _build.compile_command("x.so")
+    assert "arch=compute_100a,code=sm_100a" in " ".join(cmd)
+
+
+def test_status_strings(lib):
+    assert pad.pad_status_string(0) == "PAD_OK"
+    assert pad.pad_status_string(5) == "PAD_ERR_DEVICE_CHECK"
+    assert pad.pad_abi_version() == 1
+
+
+def test_plan_follows_the_partition_rule(lib):
+    # explicit splits: P = round_up(ceil(C / S), bs), S_eff = ceil(C / P)
+    p = pad.pad_decode_plan(64, 40, 8, 128, 16, 512, num_splits=16, device=0)
+    assert (p["num_splits"], p["partition_tokens"], p["reduce"]) == (16, 512, 1)
+    assert p["ctas"] == 64 * 8 * 16 and p["head_tiles"] == 1 and p["heads_per_tile"] == 8
+    assert p["workspace_bytes"] >= 64 * 40 * 16 * (128 + 1) * 4
+    p = pad.pad_decode_plan(16, 16, 4, 256, 16, 2048, num_splits=32, device=0)
+    assert (p["num_splits"], p["partition_tokens"]) == (32, 1024)
+    p = pad.pad_decode_plan(1, 4, 1, 128, 16, 16, num_splits=1, device=0)
+    assert (p["num_splits"], p["reduce"], p["workspace_bytes"]) == (1, 0, 0)
+    p = pad.pad_decode_plan(2, 4, 1, 128, 16, 4, num_splits=7, device=0)  # C=64, P=16
+    assert (p["num_splits"], p["partition_tokens"]) == (4, 16)
+    p = pad.pad_decode_plan(2, 4, 1, 128, 1, 100, num_splits=3, device=0)  # bs=1: P=34, S=3
+    assert (p["num_splits"], p["partition_tokens"]) == (3, 34)
+
+
+def test_heuristic_plans(lib):
+    for shape in [(32, 32, 8, 128, 16, 256), (256, 32, 1, 128, 32, 1024), (64, 40, 8, 128, 16, 512),
+                  (16, 16, 4, 256, 16, 2048), (1, 4, 1, 128, 16, 16), (3, 64, 1, 128, 16, 4)]:
+        p = pad.pad_decode_plan(*shape, num_splits=0, device=0)
+        B, Hq, Hkv, D, bs, W = shape
+        g = Hq // Hkv
+        C = W * bs
+        assert p["partition_tokens"] % bs == 0 and p["partition_tokens"] <= max(C, bs)
+        assert p["num_splits"] == -(-C // p["partition_tokens"])
+        assert p["heads_per_tile"] * p["head_tiles"] >= g
+        # scratch traffic per partition stays small against its K/V bytes
+        if p["num_splits"] > 1:
+            assert 2 * g / p["partition_tokens"] <= 1 / 16 + 1e-9
+    # group 20 at D=256 runs as two 16-head tiles
+    p = pad.pad_decode_plan(2, 20, 1, 256, 16, 10, num_splits=1, device=0)
+    assert (p["heads_per_tile"], p["head_tiles"]) == (16, 2)
+
+
+def _fake(dtype, shape, strides=None, addr=0x100000):
+    t = pad.PadTensor()
+    t.data = addr
+    t.dtype = dtype
+    t.ndim = len(shape)
+    if strides is None:
+        strides, acc = [], 1
+        for s in reversed(shape):
+            strides.insert(0, acc)
+            acc *= s
+    for i, (s, st) in enumerate(zip(shape, strides)):
+        t.shape[i] = s
+        t.stride[i] = st
+    return t
+
+
+def _call(lib, q, k, v, t, l, out, lse=None, scale=0.1, splits=0):
+    r = lambda x: ctypes.byref(x) if x is not None else None
+    return lib.pad_decode(r(q), r(k), r(v), r(t), r(l), scale, splits, r(out), r(lse), None)
+
+
+GOOD = dict(
+    q=(pad.PAD_BF16, (2, 8, 128)), k=(pad.PAD_BF16, (10, 2, 16, 128)), v=(pad.PAD_BF16, (10, 2, 16, 128)),
+    t=(pad.PAD_I32, (2, 5)), l=(pad.PAD_I32, (2,)), out=(pad.PAD_BF16, (2, 8, 128)), lse=(pad.PAD_F32, (2, 8)))
+
+
+def _args(**override):
+    spec = {**GOOD, **override}
+    return {k: (_fake(*v) if v is not None else None) for k, v in spec.items()}
+
+
+@pytest.mark.parametrize("override,status", [
+    (dict(q=(pad.PAD_F32, (2, 8, 128))), pad.PAD_ERR_INVALID_ARG),          # wrong dtype
+    (dict(v=(pad.PAD_BF16, (10, 1, 16, 128))), pad.PAD_ERR_INVALID_ARG),    # K/V shapes differ
+    (dict(q=(pad.PAD_BF16, (2, 7, 128)), out=(pad.PAD_BF16, (2, 7, 128)), lse=(pad.PAD_F32, (2, 7))),
+     pad.PAD_ERR_INVALID_ARG),                                               # Hq % Hkv != 0
+    (dict(lse=(pad.PAD_F32, (2, 9))), pad.PAD_ERR_INVALID_ARG),             # lse shape mismatch
+    (dict(out=(pad.PAD_BF16, (2, 8, 64))), pad.PAD_ERR_INVALID_ARG),        # out shape mismatch
+    (dict(t=(pad.PAD_I32, (3, 5))), pad.PAD_ERR_INVALID_ARG),               # table rows != B
+    (dict(l=(pad.PAD_I32, (3,))), pad.PAD_ERR_INVALID_ARG),                 # seq_lens != B
+    (dict(q=(pad.PAD_BF16, (2, 8, 96)), k=(pad.PAD_BF16, (10, 2, 16, 96)), v=(pad.PAD_BF16, (10, 2, 16, 96)),
+          out=(pad.PAD_BF16, (2, 8, 96))), pad.PAD_ERR_UNSUPPORTED),        # head_dim 96
+    (dict(k=(pad.PAD_BF16, (10, 2, 12, 128)), v=(pad.PAD_BF16, (10, 2, 12, 128))), pad.PAD_ERR_UNSUPPORTED),  # bs 12
+])
+def test_validation_rejects_before_any_launch(lib, override, status):
+    a = _args(**override)
+    assert _call(lib, a["q"], a["k"], a["v"], a["t"], a["l"], a["out"], a["lse"]) == status
+    assert pad.pad_last_error()
+
+
+def test_validation_scalars_and_alignment(lib):
+    a = _args()
+    assert _call(lib, a["q"], a["k"], a["v"], a["t"], a["l"], a["out"], a["lse"], scale=float("nan")) == pad.PAD_ERR_INVALID_ARG
+    assert _call(lib, a["q"], a["k"], a["v"], a["t"], a["l"], a["out"], a["lse"], splits=-1) == pad.PAD_ERR_INVALID_ARG
+    a = _args()
+    a["k"].data = 0x100008  # not 16-byte aligned
+    assert _call(lib, a["q"], a["k"], a["v"], a["t"], a["l"], a["out"], a["lse"]) == pad.PAD_ERR_INVALID_ARG
+    a = _args()
+    a["k"].stride[2] = 132  # row stride of 264 bytes: not a multiple of 16
+    assert _call(lib, a["q"], a["k"], a["v"], a["t"], a["l"], a["out"], a["lse"]) == pad.PAD_ERR_INVALID_ARG
+    a = _args()
+    a["q"].stride[2] = 2  # head dim not contiguous
+    assert _call(lib, a["q"], a["k"], a["v"], a["t"], a["l"], a["out"], a["lse"]) == pad.PAD_ERR_INVALID_ARG
+    assert _call(lib, None, a["k"], a["v"], a["t"], a["l"], a["out"], a["lse"]) == pad.PAD_ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_no_op(lib):
+    a = _args(q=(pad.PAD_BF16, (0, 8, 128)), t=(pad.PAD_I32, (0, 5)), l=(pad.PAD_I32, (0,)),
+              out=(pad.PAD_BF16, (0, 8, 128)), lse=(pad.PAD_F32, (0, 8)))
+    assert _call(lib, a["q"], a["k"], a["v"], a["t"], a["l"], a["out"], a["lse"]) == pad.PAD_OK
+
+
+def test_binding_has_no_cpu_path():
+    import torch
+    import paged_kv_attention_partition_b200 as p
+    q = torch.zeros(1, 4, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        p.pad_decode(q, q, q, q, q, 0.1)
