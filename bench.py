@@ -345,8 +345,9 @@ def main():
             "roofline": {"kernel": kname, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "peak_kind": f"{peak_kind} copy bandwidth", "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "algorithmic_bytes_per_launch": p_bytes, "traffic": traffic, "source_sha": sha},
-            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "us_per_call": round(e2e_total / args.steps * 1e3, 2), "api": "pad_decode"},
+            "e2e": None if not e2e_steps else {
+                "value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "us_per_call": round(e2e_total / args.steps * 1e3, 2), "api": "pad_decode"},
             "gpu_launches": args.steps * (2 if plan["reduce"] else 1),
             "clocks": clocks.summary(),
         }
