@@ -155,6 +155,37 @@ pad_status pad_decode_reduce(const pad_tensor *q, const pad_tensor *k_cache,
                              size_t workspace_bytes, void *stream);
 
 /*
+ * pad_decode_static_scratch -- pad_decode for callers that cannot allocate device
+ * memory.  The source pages have no counterpart of this entry point.
+ *
+ * Some callers must not call cudaMalloc (or anything that allocates) when they
+ * decode: a runtime that plans all of its memory up front, a thread that may not
+ * take the allocator's locks or absorb the synchronisation an allocation or a
+ * free can cause, an embedding with no allocator to lend.  pad_decode grows
+ * scratch on demand and pad_decode_partition/pad_decode_reduce want the caller's
+ * scratch; this call uses neither.  Its split scratch is a fixed 32 MiB array
+ * compiled into the library, which every GPU that loads the library holds until
+ * the process exits.
+ *
+ * Arguments, results and validation are those of pad_decode.  It calls no
+ * allocating routine.  Shapes whose split scratch (pad_decode_plan(...)
+ * .workspace_bytes) exceeds 32 MiB are rejected with PAD_ERR_WORKSPACE before
+ * anything is launched.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture.  All calls on a device share the one array and it keeps
+ * the last call's contents (nothing in it needs to start zeroed).  Calls that may
+ * overlap on the GPU -- on different streams without ordering between them, or
+ * from different host threads -- race on the array and corrupt each other's
+ * results: serialise them.
+ */
+pad_status pad_decode_static_scratch(const pad_tensor *q, const pad_tensor *k_cache,
+                                     const pad_tensor *v_cache, const pad_tensor *block_tables,
+                                     const pad_tensor *seq_lens, float scale, int32_t num_splits,
+                                     pad_tensor *out, pad_tensor *lse, void *stream);
+
+/*
  * pad_decode_plan -- the launch geometry pad_decode would use for this shape
  * (the per-shape heuristic when num_splits == 0).  Pure host computation; no
  * launch.  `device` < 0 means the current device (its SM count feeds the

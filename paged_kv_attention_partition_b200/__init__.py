@@ -67,6 +67,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     P = ctypes.POINTER(PadTensor)
     lib.pad_decode.argtypes = [P, P, P, P, P, ctypes.c_float, ctypes.c_int32, P, P, ctypes.c_void_p]
     lib.pad_decode.restype = ctypes.c_int
+    lib.pad_decode_static_scratch.argtypes = lib.pad_decode.argtypes
+    lib.pad_decode_static_scratch.restype = ctypes.c_int
     for name in ("pad_decode_partition", "pad_decode_reduce"):
         fn = getattr(lib, name)
         fn.argtypes = [P, P, P, P, P, ctypes.c_float, ctypes.c_int32, P, P, ctypes.c_void_p, ctypes.c_size_t,
@@ -162,6 +164,30 @@ def pad_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, bl
         st = lib.pad_decode(ctypes.byref(dq), ctypes.byref(dk), ctypes.byref(dv), ctypes.byref(dt),
                             ctypes.byref(dl), float(scale), int(num_splits), ctypes.byref(do),
                             ctypes.byref(dlse) if dlse is not None else None, _stream_handle(stream, dev))
+    _raise(st)
+    return out, lse
+
+
+def pad_decode_static_scratch(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits=0, out=None,
+                              lse=None, stream=None):
+    """pad_decode for callers that cannot allocate device memory: the split
+    scratch is a fixed 32 MiB array inside the library (see include/pad.h).  The
+    output tensors are still the caller's; pass them in (``out``, ``lse``) to
+    keep the call itself allocation-free.  Calls sharing a device must not
+    overlap on the GPU.  Returns (out, lse)."""
+    dev = q.device
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    if lse is True:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+    elif lse is False:
+        lse = None
+    descs = [describe(t) for t in (q, k_cache, v_cache, block_tables, seq_lens, out)]
+    dlse = describe(lse) if lse is not None else None
+    with torch.cuda.device(dev):
+        st = load_library().pad_decode_static_scratch(
+            *(ctypes.byref(d) for d in descs[:5]), float(scale), int(num_splits), ctypes.byref(descs[5]),
+            ctypes.byref(dlse) if dlse is not None else None, _stream_handle(stream, dev))
     _raise(st)
     return out, lse
 

@@ -498,3 +498,9 @@ pad_status pad_release_workspace(int32_t device) {
 }
 
 }  // extern "C"
+
+namespace pad {
+// Lets other translation units of the library report a failure through
+// pad_last_error().
+void set_last_error(const char *msg) { g_last_error = msg; }
+}  // namespace pad

@@ -68,3 +68,7 @@ cudaError_t launch_reduce(const ReduceParams &p, cudaStream_t s);
 cudaError_t device_error_word(int device, uint32_t **ptr);
 
 }  // namespace pad
+
+namespace pad {
+void set_last_error(const char *msg);
+}  // namespace pad
