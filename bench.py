@@ -71,17 +71,6 @@ def workload_config(w, plan):
     return cfg
 
 
-def partition_bytes(w, S):
-    """Algorithmic bytes of one partition-kernel launch: K/V pages, q, live table
-    entries, seq_lens; plus out/lse when it writes them itself (S == 1)."""
-    L = w.seq_lens.astype(np.int64)
-    b = int((4 * L * w.Hkv * w.D).sum()) + 2 * w.B * w.Hq * w.D
-    b += int(4 * ((L + w.block_size - 1) // w.block_size).sum()) + 4 * w.B
-    if S == 1:
-        b += 2 * w.B * w.Hq * w.D + (4 * w.B * w.Hq if w.want_lse else 0)
-    return b
-
-
 def cpu_baseline(w, budget_s, runs_max=50):
     """Time the oracle as it stands on this host's cores on a bounded sample."""
     import oracle
@@ -236,24 +225,24 @@ def main():
     lens = torch.from_numpy(w.seq_lens).to(dev)
     out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev) if w.want_lse else None
-    ws = torch.empty(max(plan["workspace_bytes"], 256) // 4 + 64, dtype=torch.float32, device=dev)
+    # caller-owned partials scratch (contents irrelevant)
+    ws = torch.empty(plan["workspace_bytes"] // 4 + 64, dtype=torch.float32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(dev)
 
-    def step_phased(ev):
-        pad.pad_decode_partition(q, k, v, tables, lens, w.scale, splits, out, lse, ws, stream)
-        ev[1].record(stream)
-        pad.pad_decode_reduce(q, k, v, tables, lens, w.scale, splits, out, lse, ws, stream)
+    def step():
+        # the whole hot path: one persistent launch (partition + fused reduce)
+        pad.pad_decode_with_workspace(q, k, v, tables, lens, w.scale, splits, out, lse, ws, stream)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             flush.fill_(1.0)
-            step_phased([None, torch.cuda.Event(enable_timing=True)])
+            step()
             pad.pad_decode(q, k, v, tables, lens, w.scale, num_splits=splits, out=out, lse=lse, stream=stream)
     stream.synchronize()
 
-    # ---- timed region: exactly K steps, device events per phase ------------
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    # ---- timed region: exactly K steps, device events around each launch ----
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -263,14 +252,13 @@ def main():
                 flush.fill_(float(i))
                 ev = events[i]
                 ev[0].record(stream)
-                step_phased(ev)
-                ev[2].record(stream)
+                step()
+                ev[1].record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    step_ms = [e[0].elapsed_time(e[2]) for e in events]
-    part_ms = [e[0].elapsed_time(e[1]) for e in events]
-    red_ms = [e[1].elapsed_time(e[2]) for e in events]
+    step_ms = [e[0].elapsed_time(e[1]) for e in events]
+    part_ms = step_ms  # the step is exactly one launch of the partition kernel
     total_ms = sum(step_ms)
     my_bytes = w.algorithmic_bytes() * args.steps
     if world > 1:
@@ -327,12 +315,14 @@ def main():
 
     if rank == 0:
         peak, peak_kind = measured_peaks()
-        p_bytes = partition_bytes(w, S)
+        # the only kernel of the step writes out/lse itself: its algorithmic bytes
+        # are the whole call's
+        p_bytes = w.algorithmic_bytes()
         p_ms = statistics.mean(part_ms)
         achieved = p_bytes / (p_ms / 1e3) / 1e9
         sha = kernel_source_sha()
         traffic = traffic_from_profiles(w.name, sha)
-        kname = f"partition_kernel<{w.D},{plan['heads_per_tile'] // 8}>"
+        kname = f"partition_kernel<{w.D},{plan['heads_per_tile']}>"
         line = {
             "metric": "decode attention µs/call and achieved HBM GB/s vs B200 peak (1 GPU)",
             "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -341,14 +331,14 @@ def main():
             "data": "synthetic (seeded counter-based generator; no dataset)",
             "config": workload_config(w, plan),
             "hbm_frac_of_peak": round(value / peak, 4),
-            "phases_us": {"partition": round(p_ms * 1e3, 2), "reduce": round(statistics.mean(red_ms) * 1e3, 2)},
+            "us_per_call_min_max": [round(min(step_ms) * 1e3, 2), round(max(step_ms) * 1e3, 2)],
             "roofline": {"kernel": kname, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "peak_kind": f"{peak_kind} copy bandwidth", "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "algorithmic_bytes_per_launch": p_bytes, "traffic": traffic, "source_sha": sha},
             "e2e": None if not e2e_steps else {
                 "value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "us_per_call": round(e2e_total / args.steps * 1e3, 2), "api": "pad_decode"},
-            "gpu_launches": args.steps * (2 if plan["reduce"] else 1),
+            "gpu_launches": args.steps,  # one persistent kernel per step
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -20,12 +20,14 @@
  *   lse[b,h]   = log(sum_t exp(s_t))                             (fp32)
  *   L_b = 0 gives out = 0 and lse = -inf.
  *
- * How it runs on the device: a partition kernel splits each sequence's tokens
- * into partitions of P tokens (P a multiple of bs); each CTA streams one
- * partition's K/V pages for one KV head through shared memory once, serves all
- * query heads of the GQA group from that read, and keeps a running max/sum
- * (online softmax) in fp32.  With more than one partition a reduce kernel merges
- * the partial outputs weighted by their log-sum-exp.
+ * How it runs on the device: each sequence's tokens are cut into partitions of P
+ * tokens (P a multiple of bs).  One persistent kernel claims (sequence, KV head,
+ * head tile, partition) units; for each it streams the partition's K/V pages
+ * for one KV head through shared memory once (TMA), serves all query heads of
+ * the GQA group from that read, and keeps a running max/sum (online softmax) in
+ * fp32.  When a sequence has more than one non-empty partition, the unit that
+ * finishes last merges the partial outputs weighted by their log-sum-exp (the
+ * split reduce, folded into the same launch).
  *
  * Conventions for every entry point:
  *  - All tensor data pointers are DEVICE pointers owned by the caller.  The
@@ -79,14 +81,16 @@ typedef struct pad_tensor {
 typedef struct pad_plan {
   int32_t num_splits;        /* effective number of partitions per sequence (S) */
   int32_t partition_tokens;  /* P, tokens per partition, a multiple of block_size */
-  int32_t heads_per_tile;    /* query heads handled per CTA, padded (8, 16 or 32) */
-  int32_t head_tiles;        /* CTAs per (sequence, KV head, partition): ceil(group / heads_per_tile) */
-  int32_t warps_per_cta;     /* warps in the partition kernel's CTA */
+  int32_t heads_per_tile;    /* query heads per work unit, padded (8, 16 or 32) */
+  int32_t head_tiles;        /* work units per (sequence, KV head, partition): ceil(group / heads_per_tile) */
+  int32_t warps_per_cta;     /* warps in the kernel's CTA (4 load-and-compute, 1 scheduler, 1 merger) */
   int32_t stage_tokens;      /* tokens per shared-memory pipeline stage */
   int32_t stages;            /* pipeline depth */
-  int32_t ctas;              /* partition-kernel CTAs launched (B * Hkv * head_tiles * S) */
-  int32_t reduce;            /* 1 when the split-reduce kernel runs (S > 1) */
-  int64_t workspace_bytes;   /* split scratch the call needs (0 when S == 1) */
+  int32_t ctas;              /* persistent CTAs launched (min(units, SM count)) */
+  int32_t reduce;            /* 1 when partitions may need merging (S > 1) */
+  int64_t workspace_bytes;   /* partial-output scratch (0 when S == 1) */
+  int64_t control_bytes;     /* claim word + merge counters (library-owned except for
+                                pad_decode_static_scratch) */
 } pad_plan;
 
 /*
@@ -105,7 +109,8 @@ typedef struct pad_plan {
  *  num_splits    0 = let the library choose; S >= 1 asks for partitions of
  *                P = round_up(ceil(C / S), block_size) tokens, C =
  *                max_blocks_per_seq * block_size (the effective S = ceil(C / P) is
- *                reported by pad_decode_plan).  S == 1 skips the reduce kernel.
+ *                reported by pad_decode_plan).  With S == 1 no partial is ever
+ *                written.
  *  out           bf16 [B, Hq, D], stride[2] == 1, rows 16-byte aligned.  Must not
  *                overlap any input.
  *  lse           NULL = no log-sum-exp output (nothing else is written); else
@@ -114,45 +119,39 @@ typedef struct pad_plan {
  *  stream        cudaStream_t.
  *
  * Supported envelope: D in {64, 128, 256}; Hq / Hkv <= 256; block_size a power of
- * two in [1, 256].  Split scratch is owned by the library, kept per (device,
- * stream) and grown on demand; growing it while `stream` is being captured into a
- * CUDA graph returns PAD_ERR_WORKSPACE (call once outside capture first).
+ * two in [1, 256].  Scratch (partials, and a control block of claim word and
+ * merge counters that every launch leaves zero) is owned by the library, kept
+ * per (device, stream) and grown on demand; growing it while `stream` is being
+ * captured into a CUDA graph returns PAD_ERR_WORKSPACE (call once outside
+ * capture first).
  */
 pad_status pad_decode(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
                       const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
                       int32_t num_splits, pad_tensor *out, pad_tensor *lse, void *stream);
 
 /*
- * pad_decode_partition / pad_decode_reduce -- the two passes of pad_decode run
- * one at a time, with split scratch supplied by the caller instead of the
- * library ("perf(rocke): prepare saved paged decode bindings once", section
- * "Summary": a split-KV pass, then a reduce pass that reads the partials and
- * writes the output and, when requested, the LSE).
+ * pad_decode_with_workspace -- pad_decode with its scratch supplied by the
+ * caller instead of the library ("perf(rocke): prepare saved paged decode
+ * bindings once", section "Technical Changes": a binding owns its private
+ * scratch, kept alive until the work queued on it completes).
  *
  * Arguments are those of pad_decode plus `workspace`: DEVICE memory owned by the
  * caller, 256-byte aligned, of at least pad_decode_plan(...).workspace_bytes
- * bytes (it may be NULL when that is 0).  Both calls must see the same arguments
- * and the same workspace, in order on one stream (or with the caller ordering
- * them).  The workspace holds, for every (b, query head, partition), the fp32
- * output normalised by its own softmax sum ([B, Hq, S, D]) and, after it at the
- * next 256-byte boundary, the partition's fp32 natural-log LSE ([B, Hq, S]);
- * partitions past ceil(L_b / P) are neither written nor read.
- *
- * pad_decode_partition with S == 1 writes `out`/`lse` directly and touches no
- * workspace; pad_decode_reduce then returns PAD_OK without launching.  The
- * workspace must not be shared by calls that may run concurrently.
+ * bytes (may be NULL when that is 0, i.e. S == 1); its initial contents do not
+ * matter.  It must not be shared by calls that may run concurrently.  Layout
+ * (offsets rounded up to 256 bytes): fp32 partial outputs [B, Hq, S, D], each
+ * normalised by its own softmax sum, then fp32 partial LSEs [B, Hq, S].  After
+ * a call, the partials of every (b, head) whose sequence had more than one
+ * non-empty partition are left in place; partitions past ceil(L_b / P) are
+ * neither written nor read.  The small control block (claim word and merge
+ * counters, control_bytes) stays library-owned per (device, stream), as for
+ * pad_decode: allocated zeroed on first use and kept zero by every launch.
  */
-pad_status pad_decode_partition(const pad_tensor *q, const pad_tensor *k_cache,
-                                const pad_tensor *v_cache, const pad_tensor *block_tables,
-                                const pad_tensor *seq_lens, float scale, int32_t num_splits,
-                                pad_tensor *out, pad_tensor *lse, void *workspace,
-                                size_t workspace_bytes, void *stream);
-
-pad_status pad_decode_reduce(const pad_tensor *q, const pad_tensor *k_cache,
-                             const pad_tensor *v_cache, const pad_tensor *block_tables,
-                             const pad_tensor *seq_lens, float scale, int32_t num_splits,
-                             pad_tensor *out, pad_tensor *lse, void *workspace,
-                             size_t workspace_bytes, void *stream);
+pad_status pad_decode_with_workspace(const pad_tensor *q, const pad_tensor *k_cache,
+                                     const pad_tensor *v_cache, const pad_tensor *block_tables,
+                                     const pad_tensor *seq_lens, float scale, int32_t num_splits,
+                                     pad_tensor *out, pad_tensor *lse, void *workspace,
+                                     size_t workspace_bytes, void *stream);
 
 /*
  * pad_decode_static_scratch -- pad_decode for callers that cannot allocate device
@@ -175,7 +174,9 @@ pad_status pad_decode_reduce(const pad_tensor *q, const pad_tensor *k_cache,
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call before
  * any stream capture.  All calls on a device share the one array and it keeps
- * the last call's contents (nothing in it needs to start zeroed).  Calls that may
+ * the last call's contents; each call clears, on `stream` before its launch
+ * (cudaMemsetAsync, which allocates nothing), the counter words that must start
+ * at zero.  Calls that may
  * overlap on the GPU -- on different streams without ordering between them, or
  * from different host threads -- race on the array and corrupt each other's
  * results: serialise them.

@@ -6,9 +6,10 @@ arithmetic runs in the library's CUDA kernels; there is no Python or CPU
 fallback, and the import fails loudly if ``libpad.so`` has not been built
 (``python -m paged_kv_attention_partition_b200._build``).
 
-Functions carry the C names: ``pad_decode``, ``pad_decode_plan``,
-``pad_check_device_errors``, ``pad_release_workspace``, ``pad_status_string``,
-``pad_last_error``, ``pad_abi_version``.
+Functions carry the C names: ``pad_decode``, ``pad_decode_with_workspace``,
+``pad_decode_static_scratch``, ``pad_decode_plan``, ``pad_check_device_errors``,
+``pad_release_workspace``, ``pad_status_string``, ``pad_last_error``,
+``pad_abi_version``.
 """
 from __future__ import annotations
 
@@ -36,7 +37,7 @@ class PadPlan(ctypes.Structure):
                 ("heads_per_tile", ctypes.c_int32), ("head_tiles", ctypes.c_int32),
                 ("warps_per_cta", ctypes.c_int32), ("stage_tokens", ctypes.c_int32),
                 ("stages", ctypes.c_int32), ("ctas", ctypes.c_int32), ("reduce", ctypes.c_int32),
-                ("workspace_bytes", ctypes.c_int64)]
+                ("workspace_bytes", ctypes.c_int64), ("control_bytes", ctypes.c_int64)]
 
     def as_dict(self) -> dict:
         return {name: getattr(self, name) for name, _ in self._fields_}
@@ -69,11 +70,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pad_decode.restype = ctypes.c_int
     lib.pad_decode_static_scratch.argtypes = lib.pad_decode.argtypes
     lib.pad_decode_static_scratch.restype = ctypes.c_int
-    for name in ("pad_decode_partition", "pad_decode_reduce"):
-        fn = getattr(lib, name)
-        fn.argtypes = [P, P, P, P, P, ctypes.c_float, ctypes.c_int32, P, P, ctypes.c_void_p, ctypes.c_size_t,
-                       ctypes.c_void_p]
-        fn.restype = ctypes.c_int
+    lib.pad_decode_with_workspace.argtypes = [P, P, P, P, P, ctypes.c_float, ctypes.c_int32, P, P, ctypes.c_void_p,
+                                              ctypes.c_size_t, ctypes.c_void_p]
+    lib.pad_decode_with_workspace.restype = ctypes.c_int
     lib.pad_decode_plan.argtypes = [ctypes.c_int64] * 6 + [ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(PadPlan)]
     lib.pad_decode_plan.restype = ctypes.c_int
     lib.pad_status_string.argtypes = [ctypes.c_int]
@@ -192,34 +191,25 @@ def pad_decode_static_scratch(q, k_cache, v_cache, block_tables, seq_lens, scale
     return out, lse
 
 
-def _phase(fn_name, q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, workspace, stream):
+def pad_decode_with_workspace(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, workspace,
+                              stream=None) -> None:
+    """pad_decode with caller-owned partials scratch (see include/pad.h):
+    ``workspace`` is a contiguous device tensor of at least
+    ``pad_decode_plan(...)["workspace_bytes"]`` bytes (any contents), or None
+    when that is 0."""
     dev = q.device
     if workspace is not None and (workspace.device != dev or not workspace.is_contiguous()):
         raise ValueError("workspace must be a contiguous tensor on q's device")
     descs = [describe(t) for t in (q, k_cache, v_cache, block_tables, seq_lens, out)]
     dlse = describe(lse) if lse is not None else None
-    ws_ptr = workspace.data_ptr() if workspace is not None else None
-    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     with torch.cuda.device(dev):
-        st = getattr(load_library(), fn_name)(
+        st = load_library().pad_decode_with_workspace(
             *(ctypes.byref(d) for d in descs[:5]), float(scale), int(num_splits), ctypes.byref(descs[5]),
-            ctypes.byref(dlse) if dlse is not None else None, ws_ptr, ws_bytes, _stream_handle(stream, dev))
+            ctypes.byref(dlse) if dlse is not None else None,
+            workspace.data_ptr() if workspace is not None else None,
+            workspace.numel() * workspace.element_size() if workspace is not None else 0,
+            _stream_handle(stream, dev))
     _raise(st)
-
-
-def pad_decode_partition(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, workspace,
-                         stream=None) -> None:
-    """First pass only (see include/pad.h); ``workspace`` is a caller-owned device
-    tensor of at least ``pad_decode_plan(...)["workspace_bytes"]`` bytes."""
-    _phase("pad_decode_partition", q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse,
-           workspace, stream)
-
-
-def pad_decode_reduce(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, workspace,
-                      stream=None) -> None:
-    """Second pass only: merges the partitions pad_decode_partition left in ``workspace``."""
-    _phase("pad_decode_reduce", q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse,
-           workspace, stream)
 
 
 def pad_decode_plan(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, block_size: int,
@@ -250,6 +240,7 @@ def pad_release_workspace(device: int = -1) -> None:
     _raise(load_library().pad_release_workspace(device))
 
 
-__all__ = ["pad_decode", "pad_decode_partition", "pad_decode_reduce", "pad_decode_plan", "pad_check_device_errors", "pad_release_workspace",
+__all__ = ["pad_decode", "pad_decode_with_workspace", "pad_decode_static_scratch", "pad_decode_plan",
+           "pad_check_device_errors", "pad_release_workspace",
            "pad_status_string", "pad_last_error", "pad_abi_version", "describe", "load_library",
            "PadError", "PadTensor", "PadPlan"]

@@ -1,11 +1,14 @@
-// Host side of libpad: argument validation, the per-shape launch plan, the
-// library-owned split scratch, and the two launches.  Declared in include/pad.h.
+// Host side of libpad: argument validation, the per-shape launch plan, TMA
+// tensor maps for the K/V caches, the split scratch, and the launch.  Declared
+// in include/pad.h.
 #include "pad.h"
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <string.h>
 
 #include <map>
 #include <mutex>
@@ -39,6 +42,8 @@ int ilog2(int64_t x) {
   while ((1ll << r) < x) ++r;
   return r;
 }
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
 // ---- shape checks (no data access) ----------------------------------------
 
@@ -80,14 +85,13 @@ int sm_count(int device) {
   return cache[device];
 }
 
-int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
-
 // Per-shape launch plan.  The lengths live on the device, so the plan sees only
-// the table capacity C = W * bs.  Partitions are whole pages.  With num_splits==0:
-// the partition is the smallest size that keeps the split scratch traffic (2 * g
-// * D * 4 bytes written and read back per partition) under ~1/16 of the K/V bytes
-// it streams (4 * D * P), and at least 256 tokens, so that many CTAs keep every
-// SM busy and the longest CTA stays short even on ragged batches.
+// the table capacity C = W * bs.  Partitions are whole pages.  With num_splits==0
+// the partition is the smallest size that keeps the split scratch (g * D * 4
+// bytes written per partition) under ~1/16 of the K/V bytes it streams (4 * D *
+// P), and at least 256 tokens: many small units keep every SM busy and bound the
+// tail of a ragged batch, while the fused reduce reads the partials back from L2.
+// The grid is one persistent CTA per SM (fewer when there are fewer units).
 void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan) {
   const int64_t C = s.W * s.bs;
   int hpt = s.g <= 8 ? 8 : (s.g <= 16 ? 16 : 32);
@@ -97,28 +101,26 @@ void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan) {
   if (num_splits >= 1) {
     P = round_up((C + num_splits - 1) / num_splits, s.bs);
   } else {
-    int64_t p_min = 32 * s.g;
+    int64_t p_min = 16 * s.g;
     if (p_min < 256) p_min = 256;
-    P = round_up(p_min, 64);
-    P = round_up(P, s.bs);
-    // never more than ~64 waves of CTAs at two per SM
-    const int64_t units = s.B * s.Hkv * HT;
-    const int64_t max_ctas = (int64_t)sm_count(device < 0 ? 0 : device) * 2 * 64;
-    while (units > 0 && units * ((C + P - 1) / P) > max_ctas && P < C) P *= 2;
+    P = round_up(round_up(p_min, 64), s.bs);
   }
   if (P > round_up(C, s.bs)) P = round_up(C, s.bs);
   if (P < s.bs) P = s.bs;
   const int64_t S = (C + P - 1) / P;
+  const int64_t units = s.B * s.Hkv * HT * S;
+  const int64_t sms = sm_count(device < 0 ? 0 : device);
   plan->num_splits = (int32_t)S;
   plan->partition_tokens = (int32_t)P;
   plan->heads_per_tile = hpt;
   plan->head_tiles = (int32_t)HT;
-  plan->warps_per_cta = pad::kWarps;
+  plan->warps_per_cta = pad::kWorkers + 2;
   plan->stage_tokens = pad::kStageTokens;
-  plan->stages = pad::stages_for((int)s.D);
-  plan->ctas = (int64_t)(s.B * s.Hkv * HT * S) > 0x7fffffffll ? 0x7fffffff : (int32_t)(s.B * s.Hkv * HT * S);
+  plan->stages = pad::partition_stages((int)s.D, hpt);
+  plan->ctas = (int32_t)(units < sms ? (units > 0 ? units : 1) : sms);
   plan->reduce = S > 1 ? 1 : 0;
-  plan->workspace_bytes = S > 1 ? (int64_t)(round_up(s.B * s.Hq * S * s.D * 4, 256) + round_up(s.B * s.Hq * S * 4, 256)) : 0;
+  plan->workspace_bytes = (int64_t)pad::workspace_layout(s.B, s.Hq, S, s.D).total;
+  plan->control_bytes = (int64_t)pad::control_layout(s.B, s.Hkv, HT, S).total;
 }
 
 // ---- tensor descriptor checks -----------------------------------------------
@@ -162,18 +164,24 @@ pad_status check_device_ptr(const void *p, int device, const char *name) {
   return PAD_OK;
 }
 
-// ---- library-owned split scratch, one buffer per (device, stream) -----------
+// ---- library-owned buffers, one of each kind per (device, stream) -----------
+//
+// Partials: split outputs, no initial contents needed.  Control: claim word and
+// merge counters, zero-filled when (re)allocated and left zero by every launch
+// that completes, so one buffer serves calls of any shape in stream order.
 
 struct Workspace {
   void *ptr = nullptr;
   size_t bytes = 0;
 };
 std::mutex g_ws_mu;
-std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;   // partials
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ctl;  // control blocks
 
-pad_status get_workspace(int device, cudaStream_t stream, size_t bytes, void **out) {
+pad_status get_buffer(std::map<std::pair<int, cudaStream_t>, Workspace> &pool, int device, cudaStream_t stream,
+                      size_t bytes, void **out) {
   std::lock_guard<std::mutex> lock(g_ws_mu);
-  Workspace &w = g_ws[{device, stream}];
+  Workspace &w = pool[{device, stream}];
   if (w.bytes >= bytes) {
     *out = w.ptr;
     return PAD_OK;
@@ -186,7 +194,7 @@ pad_status get_workspace(int device, cudaStream_t stream, size_t bytes, void **o
                 "split scratch must grow to %zu bytes while the stream is being captured; "
                 "run one call with this shape outside capture first", bytes);
   if (w.ptr != nullptr) {
-    // queued work on this stream may still read the old buffer
+    // queued work on this stream may still use the old buffer
     e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
     cudaFree(w.ptr);
@@ -204,61 +212,20 @@ pad_status get_workspace(int device, cudaStream_t stream, size_t bytes, void **o
     w.ptr = nullptr;
     return fail(PAD_ERR_WORKSPACE, "cudaMalloc(%zu) for split scratch failed: %s", bytes, cudaGetErrorString(e));
   }
+  e = cudaMemsetAsync(w.ptr, 0, want, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(library scratch)");
   w.bytes = want;
   *out = w.ptr;
   return PAD_OK;
 }
 
-}  // namespace
+// ---- one call: validate, plan, bind, launch ---------------------------------
 
-extern "C" {
-
-int32_t pad_abi_version(void) { return PAD_ABI_VERSION; }
-
-const char *pad_status_string(pad_status st) {
-  switch (st) {
-    case PAD_OK: return "PAD_OK";
-    case PAD_ERR_INVALID_ARG: return "PAD_ERR_INVALID_ARG";
-    case PAD_ERR_UNSUPPORTED: return "PAD_ERR_UNSUPPORTED";
-    case PAD_ERR_WORKSPACE: return "PAD_ERR_WORKSPACE";
-    case PAD_ERR_CUDA: return "PAD_ERR_CUDA";
-    case PAD_ERR_DEVICE_CHECK: return "PAD_ERR_DEVICE_CHECK";
-  }
-  return "PAD_ERR_UNKNOWN";
-}
-
-const char *pad_last_error(void) { return g_last_error.c_str(); }
-
-pad_status pad_decode_plan(int64_t batch, int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
-                           int64_t block_size, int64_t max_blocks_per_seq, int32_t num_splits,
-                           int32_t device, pad_plan *plan) {
-  if (plan == nullptr) return fail(PAD_ERR_INVALID_ARG, "plan is NULL");
-  Shape s{batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
-          num_kv_heads > 0 ? num_q_heads / num_kv_heads : 0};
-  pad_status st = check_shape(s, num_splits);
-  if (st != PAD_OK) return st;
-  if (device < 0) {
-    int d = 0;
-    if (cudaGetDevice(&d) != cudaSuccess) {
-      cudaGetLastError();
-      d = -1;
-    }
-    device = d;
-  }
-  make_plan(s, num_splits, device, plan);
-  if ((int64_t)plan->ctas > 0x7fffffffll / 2)
-    return fail(PAD_ERR_UNSUPPORTED, "too many CTAs for one launch");
-  return PAD_OK;
-}
-
-}  // extern "C"
-
-namespace {
-
-// Everything one call needs after validation: kernel parameters and the plan.
 struct Prepared {
   pad::PartitionParams p;
   pad_plan plan;
+  pad::WorkspaceLayout ws;
+  pad::ControlLayout cl;
   int D;
   int device;
 };
@@ -323,8 +290,10 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
   if (lse != nullptr && (st = check_device_ptr(lse->data, device, "lse")) != PAD_OK) return st;
 
   make_plan(s, num_splits, device, &pr->plan);
-  if ((int64_t)B * Hkv * pr->plan.head_tiles * pr->plan.num_splits > 0x7fffffffll)
-    return fail(PAD_ERR_UNSUPPORTED, "too many CTAs for one launch");
+  const int64_t units = B * Hkv * pr->plan.head_tiles * (int64_t)pr->plan.num_splits;
+  if (units > 0x7fffffffll) return fail(PAD_ERR_UNSUPPORTED, "too many work units (%lld) for one launch", (long long)units);
+  pr->ws = pad::workspace_layout(B, Hq, pr->plan.num_splits, D);
+  pr->cl = pad::control_layout(B, Hkv, pr->plan.head_tiles, pr->plan.num_splits);
 
   uint32_t *err = nullptr;
   if ((e = pad::device_error_word(device, &err)) != cudaSuccess) return cuda_fail(e, "error word");
@@ -355,6 +324,7 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
   p.bs_log2 = ilog2(bs);
   p.P = pr->plan.partition_tokens;
   p.S = pr->plan.num_splits;
+  p.n_units = (uint32_t)units;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.out = static_cast<uint16_t *>(out->data);
   p.o_sb = out->stride[0];
@@ -368,49 +338,89 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
   return PAD_OK;
 }
 
-void bind_workspace(Prepared &pr, void *ws) {
-  const int64_t opart = round_up((int64_t)pr.p.B * pr.p.Hq * pr.plan.num_splits * pr.D * 4, 256);
-  pr.p.o_part = static_cast<float *>(ws);
-  pr.p.lse_part = reinterpret_cast<float *>(static_cast<char *>(ws) + opart);
+void bind_buffers(Prepared &pr, void *partials, void *control) {
+  char *base = static_cast<char *>(partials);
+  pr.p.o_part = reinterpret_cast<float *>(base + pr.ws.o_part);
+  pr.p.lse_part = reinterpret_cast<float *>(base + pr.ws.lse_part);
+  char *cbase = static_cast<char *>(control);
+  pr.p.ctl = reinterpret_cast<uint32_t *>(cbase + pr.cl.ctl);
+  pr.p.counters = reinterpret_cast<uint32_t *>(cbase + pr.cl.counters);
 }
 
-pad_status check_caller_workspace(const Prepared &pr, void *ws, size_t bytes) {
-  if (ws == nullptr) return fail(PAD_ERR_INVALID_ARG, "workspace is NULL but %lld bytes are needed", (long long)pr.plan.workspace_bytes);
-  if (bytes < (size_t)pr.plan.workspace_bytes)
-    return fail(PAD_ERR_INVALID_ARG, "workspace has %zu bytes, %lld needed", bytes, (long long)pr.plan.workspace_bytes);
-  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return fail(PAD_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-  return check_device_ptr(ws, pr.device, "workspace");
+pad_status check_caller_buffer(const Prepared &pr, void *buf, size_t bytes, size_t need, const char *name) {
+  if (need == 0) return PAD_OK;
+  if (buf == nullptr) return fail(PAD_ERR_INVALID_ARG, "%s is NULL but %zu bytes are needed", name, need);
+  if (bytes < need) return fail(PAD_ERR_INVALID_ARG, "%s has %zu bytes, %zu needed", name, bytes, need);
+  if (reinterpret_cast<uintptr_t>(buf) % 256 != 0) return fail(PAD_ERR_INVALID_ARG, "%s must be 256-byte aligned", name);
+  return check_device_ptr(buf, pr.device, name);
 }
 
-pad_status run_partition(const Prepared &pr, cudaStream_t stream) {
-  cudaError_t e = pad::launch_partition(pr.p, pr.D, pr.plan.heads_per_tile, stream);
+pad_status run(const Prepared &pr, cudaStream_t stream) {
+  cudaError_t e = pad::launch_partition(pr.p, pr.D, pr.plan.heads_per_tile, pr.plan.ctas, stream);
   return e == cudaSuccess ? PAD_OK : cuda_fail(e, "partition kernel launch");
-}
-
-pad_status run_reduce(const Prepared &pr, cudaStream_t stream) {
-  pad::ReduceParams r{};
-  r.o_part = pr.p.o_part;
-  r.lse_part = pr.p.lse_part;
-  r.seq_lens = pr.p.seq_lens;
-  r.B = pr.p.B;
-  r.Hq = pr.p.Hq;
-  r.D = pr.D;
-  r.S = pr.p.S;
-  r.P = pr.p.P;
-  r.capacity = pr.p.max_blocks << pr.p.bs_log2;
-  r.out = pr.p.out;
-  r.o_sb = pr.p.o_sb;
-  r.o_sh = pr.p.o_sh;
-  r.lse = pr.p.lse;
-  r.lse_sb = pr.p.lse_sb;
-  r.lse_sh = pr.p.lse_sh;
-  cudaError_t e = pad::launch_reduce(r, stream);
-  return e == cudaSuccess ? PAD_OK : cuda_fail(e, "reduce kernel launch");
 }
 
 }  // namespace
 
+namespace pad {
+// Lets other translation units of the library report a failure through
+// pad_last_error().
+void set_last_error(const char *msg) { g_last_error = msg; }
+
+pad_status decode_with_buffers(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
+                               const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
+                               int32_t num_splits, pad_tensor *out, pad_tensor *lse, void *partials,
+                               size_t partials_bytes, void *control, size_t control_bytes, cudaStream_t stream) {
+  Prepared pr;
+  bool empty = false;
+  pad_status st = prepare(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, &pr, &empty);
+  if (st != PAD_OK || empty) return st;
+  if ((st = check_caller_buffer(pr, partials, partials_bytes, pr.ws.total, "partials buffer")) != PAD_OK) return st;
+  if ((st = check_caller_buffer(pr, control, control_bytes, pr.cl.total, "control buffer")) != PAD_OK) return st;
+  bind_buffers(pr, partials, control);
+  return run(pr, stream);
+}
+}  // namespace pad
+
 extern "C" {
+
+int32_t pad_abi_version(void) { return PAD_ABI_VERSION; }
+
+const char *pad_status_string(pad_status st) {
+  switch (st) {
+    case PAD_OK: return "PAD_OK";
+    case PAD_ERR_INVALID_ARG: return "PAD_ERR_INVALID_ARG";
+    case PAD_ERR_UNSUPPORTED: return "PAD_ERR_UNSUPPORTED";
+    case PAD_ERR_WORKSPACE: return "PAD_ERR_WORKSPACE";
+    case PAD_ERR_CUDA: return "PAD_ERR_CUDA";
+    case PAD_ERR_DEVICE_CHECK: return "PAD_ERR_DEVICE_CHECK";
+  }
+  return "PAD_ERR_UNKNOWN";
+}
+
+const char *pad_last_error(void) { return g_last_error.c_str(); }
+
+pad_status pad_decode_plan(int64_t batch, int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
+                           int64_t block_size, int64_t max_blocks_per_seq, int32_t num_splits, int32_t device,
+                           pad_plan *plan) {
+  if (plan == nullptr) return fail(PAD_ERR_INVALID_ARG, "plan is NULL");
+  Shape s{batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+          num_kv_heads > 0 ? num_q_heads / num_kv_heads : 0};
+  pad_status st = check_shape(s, num_splits);
+  if (st != PAD_OK) return st;
+  if (device < 0) {
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess) {
+      cudaGetLastError();
+      d = -1;
+    }
+    device = d;
+  }
+  make_plan(s, num_splits, device, plan);
+  if (batch * num_kv_heads * plan->head_tiles * (int64_t)plan->num_splits > 0x7fffffffll)
+    return fail(PAD_ERR_UNSUPPORTED, "too many work units for one launch");
+  return PAD_OK;
+}
 
 pad_status pad_decode(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
                       const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
@@ -420,43 +430,27 @@ pad_status pad_decode(const pad_tensor *q, const pad_tensor *k_cache, const pad_
   bool empty = false;
   pad_status st = prepare(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, &pr, &empty);
   if (st != PAD_OK || empty) return st;
-  if (pr.plan.reduce) {
-    void *ws = nullptr;
-    if ((st = get_workspace(pr.device, stream, (size_t)pr.plan.workspace_bytes, &ws)) != PAD_OK) return st;
-    bind_workspace(pr, ws);
-  }
-  if ((st = run_partition(pr, stream)) != PAD_OK) return st;
-  return pr.plan.reduce ? run_reduce(pr, stream) : PAD_OK;
+  void *ws = nullptr, *ctl = nullptr;
+  if (pr.ws.total > 0 && (st = get_buffer(g_ws, pr.device, stream, pr.ws.total, &ws)) != PAD_OK) return st;
+  if ((st = get_buffer(g_ctl, pr.device, stream, pr.cl.total, &ctl)) != PAD_OK) return st;
+  bind_buffers(pr, ws, ctl);
+  return run(pr, stream);
 }
 
-pad_status pad_decode_partition(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
-                                const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
-                                int32_t num_splits, pad_tensor *out, pad_tensor *lse, void *workspace,
-                                size_t workspace_bytes, void *stream_) {
+pad_status pad_decode_with_workspace(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
+                                     const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
+                                     int32_t num_splits, pad_tensor *out, pad_tensor *lse, void *workspace,
+                                     size_t workspace_bytes, void *stream_) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   Prepared pr;
   bool empty = false;
   pad_status st = prepare(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, &pr, &empty);
   if (st != PAD_OK || empty) return st;
-  if (pr.plan.reduce) {
-    if ((st = check_caller_workspace(pr, workspace, workspace_bytes)) != PAD_OK) return st;
-    bind_workspace(pr, workspace);
-  }
-  return run_partition(pr, stream);
-}
-
-pad_status pad_decode_reduce(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
-                             const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
-                             int32_t num_splits, pad_tensor *out, pad_tensor *lse, void *workspace,
-                             size_t workspace_bytes, void *stream_) {
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-  Prepared pr;
-  bool empty = false;
-  pad_status st = prepare(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, &pr, &empty);
-  if (st != PAD_OK || empty || !pr.plan.reduce) return st;
-  if ((st = check_caller_workspace(pr, workspace, workspace_bytes)) != PAD_OK) return st;
-  bind_workspace(pr, workspace);
-  return run_reduce(pr, stream);
+  if ((st = check_caller_buffer(pr, workspace, workspace_bytes, pr.ws.total, "workspace")) != PAD_OK) return st;
+  void *ctl = nullptr;
+  if ((st = get_buffer(g_ctl, pr.device, stream, pr.cl.total, &ctl)) != PAD_OK) return st;
+  bind_buffers(pr, workspace, ctl);
+  return run(pr, stream);
 }
 
 pad_status pad_check_device_errors(void *stream_, uint32_t *bits) {
@@ -472,9 +466,18 @@ pad_status pad_check_device_errors(void *stream_, uint32_t *bits) {
   const uint32_t zero = 0;
   if ((e = cudaMemcpy(word, &zero, 4, cudaMemcpyHostToDevice)) != cudaSuccess) return cuda_fail(e, "clear error word");
   if (bits != nullptr) *bits = v;
+  if (v & pad::kErrTimeout) {
+    // an aborted launch may have left claim/merge counters set: re-zero the
+    // library's own scratch on this device
+    std::lock_guard<std::mutex> lock(g_ws_mu);
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    for (auto &kv : g_ctl)
+      if (kv.first.first == device && kv.second.ptr != nullptr) cudaMemset(kv.second.ptr, 0, kv.second.bytes);
+  }
   if (v != 0)
-    return fail(PAD_ERR_DEVICE_CHECK, "kernel saw %s%s", (v & pad::kErrBlockId) ? "an out-of-range block id " : "",
-                (v & pad::kErrSeqLen) ? "an out-of-range sequence length" : "");
+    return fail(PAD_ERR_DEVICE_CHECK, "kernel saw %s%s%s", (v & pad::kErrBlockId) ? "an out-of-range block id; " : "",
+                (v & pad::kErrSeqLen) ? "an out-of-range sequence length; " : "",
+                (v & pad::kErrTimeout) ? "a wait that timed out (internal error)" : "");
   return PAD_OK;
 }
 
@@ -483,24 +486,20 @@ pad_status pad_release_workspace(int32_t device) {
   int cur = 0;
   cudaError_t e = cudaGetDevice(&cur);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  for (auto it = g_ws.begin(); it != g_ws.end();) {
-    if (device >= 0 && it->first.first != device) {
-      ++it;
-      continue;
+  for (auto *pool : {&g_ws, &g_ctl}) {
+    for (auto it = pool->begin(); it != pool->end();) {
+      if (device >= 0 && it->first.first != device) {
+        ++it;
+        continue;
+      }
+      if ((e = cudaSetDevice(it->first.first)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+      if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+      if (it->second.ptr != nullptr) cudaFree(it->second.ptr);
+      it = pool->erase(it);
     }
-    if ((e = cudaSetDevice(it->first.first)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
-    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-    if (it->second.ptr != nullptr) cudaFree(it->second.ptr);
-    it = g_ws.erase(it);
   }
   if ((e = cudaSetDevice(cur)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
   return PAD_OK;
 }
 
 }  // extern "C"
-
-namespace pad {
-// Lets other translation units of the library report a failure through
-// pad_last_error().
-void set_last_error(const char *msg) { g_last_error = msg; }
-}  // namespace pad

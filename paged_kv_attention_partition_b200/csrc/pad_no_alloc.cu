@@ -74,30 +74,41 @@ extern "C" pad_status pad_decode_static_scratch(const pad_tensor *q, const pad_t
                                                 const pad_tensor *v_cache, const pad_tensor *block_tables,
                                                 const pad_tensor *seq_lens, float scale, int32_t num_splits,
                                                 pad_tensor *out, pad_tensor *lse, void *stream) {
-  // Reject shapes whose split partials do not fit, before anything is launched.
+  // The array holds the control block (claim word, merge counters) first and the
+  // split partials after it.  Reject shapes that do not fit before launching.
+  size_t control = 0;
   if (q != nullptr && k_cache != nullptr && block_tables != nullptr && q->ndim == 3 && k_cache->ndim == 4 &&
       block_tables->ndim == 2) {
     pad_plan plan;
     if (pad_decode_plan(q->shape[0], q->shape[1], k_cache->shape[1], q->shape[2], k_cache->shape[2],
-                        block_tables->shape[1], num_splits, -1, &plan) == PAD_OK &&
-        (size_t)plan.workspace_bytes > pad::kStaticScratchBytes) {
-      char msg[256];
-      snprintf(msg, sizeof msg,
-               "this shape needs %lld bytes of split scratch; the static array holds %zu "
-               "(use fewer splits or pad_decode)",
-               (long long)plan.workspace_bytes, pad::kStaticScratchBytes);
-      pad::set_last_error(msg);
-      return PAD_ERR_WORKSPACE;
+                        block_tables->shape[1], num_splits, -1, &plan) == PAD_OK) {
+      control = (size_t)plan.control_bytes;
+      if (control + (size_t)plan.workspace_bytes > pad::kStaticScratchBytes) {
+        char msg[256];
+        snprintf(msg, sizeof msg,
+                 "this shape needs %lld bytes of split scratch; the static array holds %zu "
+                 "(use fewer splits or pad_decode)",
+                 (long long)(plan.control_bytes + plan.workspace_bytes), pad::kStaticScratchBytes);
+        pad::set_last_error(msg);
+        return PAD_ERR_WORKSPACE;
+      }
     }
   }
   void *scratch = nullptr;
   pad_status st = pad::static_scratch_address(&scratch);
   if (st != PAD_OK) return st;
-  // Nothing in the scratch has to start at zero: the split pass writes every
-  // partial the reduce pass reads.
-  st = pad_decode_partition(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, scratch,
-                            pad::kStaticScratchBytes, stream);
-  if (st != PAD_OK) return st;
-  return pad_decode_reduce(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, scratch,
-                           pad::kStaticScratchBytes, stream);
+  // The control block must start at zero.  A completed call leaves it zero, but
+  // the array outlives every call, so clear it on the stream first.
+  if (control > 0) {
+    cudaError_t e = cudaMemsetAsync(scratch, 0, control, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+      char msg[256];
+      snprintf(msg, sizeof msg, "cudaMemsetAsync(static scratch control block): %s", cudaGetErrorString(e));
+      pad::set_last_error(msg);
+      return PAD_ERR_CUDA;
+    }
+  }
+  return pad::decode_with_buffers(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse,
+                                  static_cast<char *>(scratch) + control, pad::kStaticScratchBytes - control,
+                                  scratch, control, static_cast<cudaStream_t>(stream));
 }

@@ -71,6 +71,21 @@ def test_tiny_workload_every_split_count(cuda_device):
         check_parity(to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, f"tiny/S={splits}")
 
 
+@pytest.mark.parametrize("Hq,Hkv,D", [(8, 2, 128), (32, 1, 128), (16, 4, 256)])
+@pytest.mark.parametrize("splits", [4, 2, 0])
+def test_many_short_units_per_cta(cuda_device, Hq, Hkv, D, splits):
+    # Capacity 256 tokens: S=4 gives one-stage (64-token) partitions, S=2
+    # two-stage ones with one-stage tails.  Hundreds of units share at most 148
+    # CTAs, so each CTA's load lookahead spans several units at once (the
+    # pipeline must not stall on a unit whose q rows are still waiting).
+    lens = np.random.default_rng(5).integers(0, 257, size=160).tolist()
+    w = _case(f"short_units_g{Hq // Hkv}_d{D}", 160, Hq, Hkv, D, 16, lens, seed=49, max_blocks_per_seq=16)
+    ref_out, ref_lse = oracle.decode_workload(w)
+    out, lse = DeviceWorkload(w, cuda_device).run(num_splits=splits)
+    check_parity(to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, f"short_units/S={splits}")
+    assert pad.pad_check_device_errors() == 0
+
+
 def test_block_table_permutation_is_bitwise_invariant(cuda_device):
     w = _case("perm", 2, 8, 2, 128, 16, [300, 77], seed=41, pool_blocks=60)
     out0, lse0 = DeviceWorkload(w, cuda_device).run(num_splits=3)
@@ -168,7 +183,8 @@ def test_plan_matches_launch_and_heuristic_shapes(cuda_device):
     p = pad.pad_decode_plan(16, 16, 4, 256, 16, 2048, num_splits=32)
     assert p["num_splits"] == 32 and p["partition_tokens"] == 1024
     p = pad.pad_decode_plan(1, 4, 1, 128, 16, 16, num_splits=1)
-    assert p["num_splits"] == 1 and p["reduce"] == 0 and p["workspace_bytes"] == 0
+    assert p["num_splits"] == 1 and p["reduce"] == 0 and p["workspace_bytes"] == 0 and p["ctas"] == 1
+    assert p["control_bytes"] == 256
     p = pad.pad_decode_plan(256, 32, 1, 128, 32, 1024, num_splits=0)
     assert p["partition_tokens"] % 32 == 0 and p["heads_per_tile"] == 32
 
@@ -226,37 +242,52 @@ def test_named_workload_full_size(cuda_device, name):
     torch.cuda.empty_cache()
 
 
+def _round256(x):
+    return -(-x // 256) * 256
+
+
 def test_partition_partials_match_oracle_on_subranges(cuda_device):
-    """The split pass alone: partition s of (b, h) must hold the attention over
+    """Caller-owned partials scratch: after the call, partition s of every (b, h)
+    whose sequence has several non-empty partitions holds the attention over
     tokens [s*P, min((s+1)*P, L_b)) (normalised by its own sum) and that range's
-    LSE; the reduce pass alone must then give the full result."""
+    LSE, and the merged output is the full result.  The scratch starts as
+    garbage (NaN) and is reused by a second call."""
     w = _case("phases", 3, 10, 2, 128, 16, [300, 45, 129], seed=48, max_blocks_per_seq=20)
     dw = DeviceWorkload(w, cuda_device)
     plan = pad.pad_decode_plan(w.B, w.Hq, w.Hkv, w.D, w.block_size, w.max_blocks_per_seq, num_splits=4)
-    S, P = plan["num_splits"], plan["partition_tokens"]
+    S, P, HT = plan["num_splits"], plan["partition_tokens"], plan["head_tiles"]
     assert S == 4 and P == 80
-    ws = torch.zeros(plan["workspace_bytes"] // 4, dtype=torch.float32, device=cuda_device)
-    out = torch.full((w.B, w.Hq, w.D), float("nan"), dtype=torch.bfloat16, device=cuda_device)
-    lse = torch.full((w.B, w.Hq), float("nan"), device=cuda_device)
-    pad.pad_decode_partition(dw.q, dw.k, dw.v, dw.tables, dw.lens, w.scale, 4, out, lse, ws)
-    torch.cuda.synchronize()
-    assert torch.isnan(out.float()).all() and torch.isnan(lse).all()  # the split pass writes scratch only
-    opart = ws[: w.B * w.Hq * S * w.D].view(w.B, w.Hq, S, w.D).cpu().numpy().astype(np.float64)
-    lse_off = -(-(w.B * w.Hq * S * w.D * 4) // 256) * 256 // 4
-    lpart = ws[lse_off: lse_off + w.B * w.Hq * S].view(w.B, w.Hq, S).cpu().numpy().astype(np.float64)
-    for b in range(w.B):
-        L = int(w.seq_lens[b])
-        for s in range(-(-L // P)):
-            a, e = s * P, min((s + 1) * P, L)
-            t = np.ascontiguousarray(w.block_tables[b:b + 1, a // 16: -(-e // 16)])
-            ro, rl = oracle.decode(np.ascontiguousarray(w.q[b:b + 1]), w.k_cache, w.v_cache, t,
-                                   np.asarray([e - a], np.int32), w.scale)
-            np.testing.assert_allclose(opart[b, :, s], ro[0], rtol=0, atol=1e-2)
-            np.testing.assert_allclose(lpart[b, :, s], rl[0], rtol=1e-4, atol=1e-4)
-    pad.pad_decode_reduce(dw.q, dw.k, dw.v, dw.tables, dw.lens, w.scale, 4, out, lse, ws)
-    torch.cuda.synchronize()
+    ws = torch.full((plan["workspace_bytes"] // 4,), float("nan"), dtype=torch.float32, device=cuda_device)
     ref_out, ref_lse = oracle.decode_workload(w)
-    check_parity(to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, "phases")
+    lse_off = _round256(w.B * w.Hq * S * w.D * 4) // 4
+    assert (lse_off + _round256(w.B * w.Hq * S * 4) // 4) * 4 == plan["workspace_bytes"]
+    assert plan["control_bytes"] == 256 + _round256(w.B * w.Hkv * HT * 4)
+    for call in range(2):
+        out = torch.full((w.B, w.Hq, w.D), float("nan"), dtype=torch.bfloat16, device=cuda_device)
+        lse = torch.full((w.B, w.Hq), float("nan"), device=cuda_device)
+        pad.pad_decode_with_workspace(dw.q, dw.k, dw.v, dw.tables, dw.lens, w.scale, 4, out, lse, ws)
+        torch.cuda.synchronize()
+        check_parity(to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, f"workspace call {call}")
+        opart = ws[: w.B * w.Hq * S * w.D].view(w.B, w.Hq, S, w.D).cpu().numpy().astype(np.float64)
+        lpart = ws[lse_off: lse_off + w.B * w.Hq * S].view(w.B, w.Hq, S).cpu().numpy().astype(np.float64)
+        for b in range(w.B):
+            L = int(w.seq_lens[b])
+            ns = -(-L // P)
+            if ns < 2:
+                continue
+            for s in range(ns):
+                a, e = s * P, min((s + 1) * P, L)
+                t = np.ascontiguousarray(w.block_tables[b:b + 1, a // 16: -(-e // 16)])
+                ro, rl = oracle.decode(np.ascontiguousarray(w.q[b:b + 1]), w.k_cache, w.v_cache, t,
+                                       np.asarray([e - a], np.int32), w.scale)
+                np.testing.assert_allclose(opart[b, :, s], ro[0], rtol=0, atol=1e-2)
+                np.testing.assert_allclose(lpart[b, :, s], rl[0], rtol=1e-4, atol=1e-4)
+    # a different shape on the same stream right after (the library's control
+    # block is reused and must have been left zero)
+    w2 = _case("phases2", 5, 8, 1, 64, 32, [1000, 3, 64, 65, 0], seed=49, max_blocks_per_seq=40)
+    out2, lse2 = DeviceWorkload(w2, cuda_device).run(num_splits=0)
+    r2o, r2l = oracle.decode_workload(w2)
+    check_parity(to_f64(out2), lse2.cpu().numpy(), r2o, r2l, "second shape")
     # too small a workspace is refused before launching
     with pytest.raises(pad.PadError):
-        pad.pad_decode_partition(dw.q, dw.k, dw.v, dw.tables, dw.lens, w.scale, 4, out, lse, ws[:16])
+        pad.pad_decode_with_workspace(dw.q, dw.k, dw.v, dw.tables, dw.lens, w.scale, 4, out, lse, ws[:16])
