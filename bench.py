@@ -231,7 +231,7 @@ def main():
     stream = torch.cuda.Stream(dev)
 
     def step():
-        # the whole hot path: one persistent launch (partition + fused reduce)
+        # the whole hot path: one launch (partition + fused reduce)
         pad.pad_decode_with_workspace(q, k, v, tables, lens, w.scale, splits, out, lse, ws, stream)
 
     with torch.cuda.stream(stream):
@@ -338,7 +338,7 @@ def main():
             "e2e": None if not e2e_steps else {
                 "value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "us_per_call": round(e2e_total / args.steps * 1e3, 2), "api": "pad_decode"},
-            "gpu_launches": args.steps,  # one persistent kernel per step
+            "gpu_launches": args.steps,  # one kernel launch per step
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

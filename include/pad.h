@@ -21,13 +21,13 @@
  *   L_b = 0 gives out = 0 and lse = -inf.
  *
  * How it runs on the device: each sequence's tokens are cut into partitions of P
- * tokens (P a multiple of bs).  One persistent kernel claims (sequence, KV head,
- * head tile, partition) units; for each it streams the partition's K/V pages
- * for one KV head through shared memory once (TMA), serves all query heads of
- * the GQA group from that read, and keeps a running max/sum (online softmax) in
- * fp32.  When a sequence has more than one non-empty partition, the unit that
- * finishes last merges the partial outputs weighted by their log-sum-exp (the
- * split reduce, folded into the same launch).
+ * tokens (P a multiple of bs).  One kernel launch runs a CTA per (sequence, KV
+ * head, head tile, partition) unit; each streams its partition's K/V pages for
+ * one KV head through shared memory once, serves all query heads of the GQA
+ * group from that read, and keeps a running max/sum (online softmax) in fp32.
+ * When a sequence has more than one non-empty partition, the unit that finishes
+ * last merges the partial outputs weighted by their log-sum-exp (the split
+ * reduce, folded into the same launch).
  *
  * Conventions for every entry point:
  *  - All tensor data pointers are DEVICE pointers owned by the caller.  The
@@ -83,14 +83,14 @@ typedef struct pad_plan {
   int32_t partition_tokens;  /* P, tokens per partition, a multiple of block_size */
   int32_t heads_per_tile;    /* query heads per work unit, padded (8, 16 or 32) */
   int32_t head_tiles;        /* work units per (sequence, KV head, partition): ceil(group / heads_per_tile) */
-  int32_t warps_per_cta;     /* warps in the kernel's CTA (4 load-and-compute, 1 scheduler, 1 merger) */
+  int32_t warps_per_cta;     /* warps per CTA (each loads and computes) */
   int32_t stage_tokens;      /* tokens per shared-memory pipeline stage */
   int32_t stages;            /* pipeline depth */
-  int32_t ctas;              /* persistent CTAs launched (min(units, SM count)) */
+  int32_t ctas;              /* CTAs launched: one per unit, B * Hkv * head_tiles * num_splits */
   int32_t reduce;            /* 1 when partitions may need merging (S > 1) */
   int64_t workspace_bytes;   /* partial-output scratch (0 when S == 1) */
-  int64_t control_bytes;     /* claim word + merge counters (library-owned except for
-                                pad_decode_static_scratch) */
+  int64_t control_bytes;     /* merge counters, 0 when S == 1 (library-owned except
+                                for pad_decode_static_scratch) */
 } pad_plan;
 
 /*
@@ -109,8 +109,8 @@ typedef struct pad_plan {
  *  num_splits    0 = let the library choose; S >= 1 asks for partitions of
  *                P = round_up(ceil(C / S), block_size) tokens, C =
  *                max_blocks_per_seq * block_size (the effective S = ceil(C / P) is
- *                reported by pad_decode_plan).  With S == 1 no partial is ever
- *                written.
+ *                reported by pad_decode_plan; at most 256).  With S == 1 no
+ *                partial is ever written.
  *  out           bf16 [B, Hq, D], stride[2] == 1, rows 16-byte aligned.  Must not
  *                overlap any input.
  *  lse           NULL = no log-sum-exp output (nothing else is written); else
@@ -119,11 +119,10 @@ typedef struct pad_plan {
  *  stream        cudaStream_t.
  *
  * Supported envelope: D in {64, 128, 256}; Hq / Hkv <= 256; block_size a power of
- * two in [1, 256].  Scratch (partials, and a control block of claim word and
- * merge counters that every launch leaves zero) is owned by the library, kept
- * per (device, stream) and grown on demand; growing it while `stream` is being
- * captured into a CUDA graph returns PAD_ERR_WORKSPACE (call once outside
- * capture first).
+ * two in [1, 256].  Scratch (partials, and a control block of merge counters
+ * that every launch leaves zero) is owned by the library, kept per (device,
+ * stream) and grown on demand; growing it while `stream` is being captured into
+ * a CUDA graph returns PAD_ERR_WORKSPACE (call once outside capture first).
  */
 pad_status pad_decode(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
                       const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
@@ -143,9 +142,9 @@ pad_status pad_decode(const pad_tensor *q, const pad_tensor *k_cache, const pad_
  * normalised by its own softmax sum, then fp32 partial LSEs [B, Hq, S].  After
  * a call, the partials of every (b, head) whose sequence had more than one
  * non-empty partition are left in place; partitions past ceil(L_b / P) are
- * neither written nor read.  The small control block (claim word and merge
- * counters, control_bytes) stays library-owned per (device, stream), as for
- * pad_decode: allocated zeroed on first use and kept zero by every launch.
+ * neither written nor read.  The small control block (merge counters,
+ * control_bytes) stays library-owned per (device, stream), as for pad_decode:
+ * allocated zeroed on first use and kept zero by every launch.
  */
 pad_status pad_decode_with_workspace(const pad_tensor *q, const pad_tensor *k_cache,
                                      const pad_tensor *v_cache, const pad_tensor *block_tables,
@@ -161,8 +160,8 @@ pad_status pad_decode_with_workspace(const pad_tensor *q, const pad_tensor *k_ca
  * decode: a runtime that plans all of its memory up front, a thread that may not
  * take the allocator's locks or absorb the synchronisation an allocation or a
  * free can cause, an embedding with no allocator to lend.  pad_decode grows
- * scratch on demand and pad_decode_partition/pad_decode_reduce want the caller's
- * scratch; this call uses neither.  Its split scratch is a fixed 32 MiB array
+ * scratch on demand and pad_decode_with_workspace wants the caller's scratch;
+ * this call uses neither.  Its split scratch is a fixed 32 MiB array
  * compiled into the library, which every GPU that loads the library holds until
  * the process exits.
  *
@@ -174,9 +173,9 @@ pad_status pad_decode_with_workspace(const pad_tensor *q, const pad_tensor *k_ca
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call before
  * any stream capture.  All calls on a device share the one array and it keeps
- * the last call's contents; each call clears, on `stream` before its launch
- * (cudaMemsetAsync, which allocates nothing), the counter words that must start
- * at zero.  Calls that may
+ * the last call's contents; each call clears, on `stream` after validating its
+ * arguments and before its launch (cudaMemsetAsync, which allocates nothing),
+ * the counter words that must start at zero.  Calls that may
  * overlap on the GPU -- on different streams without ordering between them, or
  * from different host threads -- race on the array and corrupt each other's
  * results: serialise them.
@@ -190,7 +189,8 @@ pad_status pad_decode_static_scratch(const pad_tensor *q, const pad_tensor *k_ca
  * pad_decode_plan -- the launch geometry pad_decode would use for this shape
  * (the per-shape heuristic when num_splits == 0).  Pure host computation; no
  * launch.  `device` < 0 means the current device (its SM count feeds the
- * heuristic).  Returns PAD_ERR_INVALID_ARG / PAD_ERR_UNSUPPORTED exactly when
+ * heuristic: a small batch gets shorter partitions, down to 64 tokens, so that
+ * it still fills the GPU).  Returns PAD_ERR_INVALID_ARG / PAD_ERR_UNSUPPORTED exactly when
  * pad_decode would for the same shape.
  */
 pad_status pad_decode_plan(int64_t batch, int64_t num_q_heads, int64_t num_kv_heads,

@@ -1,6 +1,5 @@
-// Host side of libpad: argument validation, the per-shape launch plan, TMA
-// tensor maps for the K/V caches, the split scratch, and the launch.  Declared
-// in include/pad.h.
+// Host side of libpad: argument validation, the per-shape launch plan, the
+// split scratch and merge counters, and the launch.  Declared in include/pad.h.
 #include "pad.h"
 
 #include <cuda.h>
@@ -87,11 +86,13 @@ int sm_count(int device) {
 
 // Per-shape launch plan.  The lengths live on the device, so the plan sees only
 // the table capacity C = W * bs.  Partitions are whole pages.  With num_splits==0
-// the partition is the smallest size that keeps the split scratch (g * D * 4
-// bytes written per partition) under ~1/16 of the K/V bytes it streams (4 * D *
-// P), and at least 256 tokens: many small units keep every SM busy and bound the
-// tail of a ragged batch, while the fused reduce reads the partials back from L2.
-// The grid is one persistent CTA per SM (fewer when there are fewer units).
+// the partition starts at 256 tokens (or 16 g, if larger: the split scratch a
+// partition writes, g * D * 4 bytes, stays under 1/16 of the K/V bytes it
+// streams, 4 * D * P) and is halved, down to max(64, 16 g), while the batch would
+// give fewer than two waves of CTAs on this device: many small units keep every
+// SM busy and bound the tail of a ragged batch, and the fused reduce reads the
+// partials back from L2.  At most kMaxSplits partitions per sequence.  One CTA
+// per unit; units past a sequence's length exit at once.
 void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan) {
   const int64_t C = s.W * s.bs;
   int hpt = s.g <= 8 ? 8 : (s.g <= 16 ? 16 : 32);
@@ -101,23 +102,27 @@ void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan) {
   if (num_splits >= 1) {
     P = round_up((C + num_splits - 1) / num_splits, s.bs);
   } else {
-    int64_t p_min = 16 * s.g;
-    if (p_min < 256) p_min = 256;
-    P = round_up(round_up(p_min, 64), s.bs);
+    const int64_t p_floor = round_up(16 * s.g > 64 ? 16 * s.g : 64, 64);
+    P = p_floor > 256 ? p_floor : 256;
+    const int64_t slots = (int64_t)sm_count(device < 0 ? 0 : device) *
+                          pad::ctas_per_sm_for((int)s.D, hpt);
+    const int64_t pairs = s.B * s.Hkv * HT;
+    while (P / 2 >= p_floor && P / 2 >= s.bs && pairs * ((C + P - 1) / P) < 2 * slots) P /= 2;
+    P = round_up(P, s.bs);
   }
   if (P > round_up(C, s.bs)) P = round_up(C, s.bs);
   if (P < s.bs) P = s.bs;
+  if ((C + P - 1) / P > pad::kMaxSplits) P = round_up((C + pad::kMaxSplits - 1) / pad::kMaxSplits, s.bs);
   const int64_t S = (C + P - 1) / P;
   const int64_t units = s.B * s.Hkv * HT * S;
-  const int64_t sms = sm_count(device < 0 ? 0 : device);
   plan->num_splits = (int32_t)S;
   plan->partition_tokens = (int32_t)P;
   plan->heads_per_tile = hpt;
   plan->head_tiles = (int32_t)HT;
-  plan->warps_per_cta = pad::kWorkers + 2;
+  plan->warps_per_cta = pad::kWarps;
   plan->stage_tokens = pad::kStageTokens;
   plan->stages = pad::partition_stages((int)s.D, hpt);
-  plan->ctas = (int32_t)(units < sms ? (units > 0 ? units : 1) : sms);
+  plan->ctas = (int32_t)(units > 0x7fffffffll ? 0x7fffffffll : units);
   plan->reduce = S > 1 ? 1 : 0;
   plan->workspace_bytes = (int64_t)pad::workspace_layout(s.B, s.Hq, S, s.D).total;
   plan->control_bytes = (int64_t)pad::control_layout(s.B, s.Hkv, HT, S).total;
@@ -166,9 +171,9 @@ pad_status check_device_ptr(const void *p, int device, const char *name) {
 
 // ---- library-owned buffers, one of each kind per (device, stream) -----------
 //
-// Partials: split outputs, no initial contents needed.  Control: claim word and
-// merge counters, zero-filled when (re)allocated and left zero by every launch
-// that completes, so one buffer serves calls of any shape in stream order.
+// Partials: split outputs, no initial contents needed.  Control: merge
+// counters, zero-filled when (re)allocated and left zero by every launch that
+// completes, so one buffer serves calls of any shape in stream order.
 
 struct Workspace {
   void *ptr = nullptr;
@@ -342,9 +347,8 @@ void bind_buffers(Prepared &pr, void *partials, void *control) {
   char *base = static_cast<char *>(partials);
   pr.p.o_part = reinterpret_cast<float *>(base + pr.ws.o_part);
   pr.p.lse_part = reinterpret_cast<float *>(base + pr.ws.lse_part);
-  char *cbase = static_cast<char *>(control);
-  pr.p.ctl = reinterpret_cast<uint32_t *>(cbase + pr.cl.ctl);
-  pr.p.counters = reinterpret_cast<uint32_t *>(cbase + pr.cl.counters);
+  pr.p.counters = pr.cl.total > 0 ? reinterpret_cast<uint32_t *>(static_cast<char *>(control) + pr.cl.counters)
+                                  : nullptr;
 }
 
 pad_status check_caller_buffer(const Prepared &pr, void *buf, size_t bytes, size_t need, const char *name) {
@@ -370,13 +374,18 @@ void set_last_error(const char *msg) { g_last_error = msg; }
 pad_status decode_with_buffers(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
                                const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
                                int32_t num_splits, pad_tensor *out, pad_tensor *lse, void *partials,
-                               size_t partials_bytes, void *control, size_t control_bytes, cudaStream_t stream) {
+                               size_t partials_bytes, void *control, size_t control_bytes, bool clear_control,
+                               cudaStream_t stream) {
   Prepared pr;
   bool empty = false;
   pad_status st = prepare(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, &pr, &empty);
   if (st != PAD_OK || empty) return st;
   if ((st = check_caller_buffer(pr, partials, partials_bytes, pr.ws.total, "partials buffer")) != PAD_OK) return st;
   if ((st = check_caller_buffer(pr, control, control_bytes, pr.cl.total, "control buffer")) != PAD_OK) return st;
+  if (clear_control && pr.cl.total > 0) {
+    cudaError_t e = cudaMemsetAsync(control, 0, pr.cl.total, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(control block)");
+  }
   bind_buffers(pr, partials, control);
   return run(pr, stream);
 }
@@ -432,7 +441,7 @@ pad_status pad_decode(const pad_tensor *q, const pad_tensor *k_cache, const pad_
   if (st != PAD_OK || empty) return st;
   void *ws = nullptr, *ctl = nullptr;
   if (pr.ws.total > 0 && (st = get_buffer(g_ws, pr.device, stream, pr.ws.total, &ws)) != PAD_OK) return st;
-  if ((st = get_buffer(g_ctl, pr.device, stream, pr.cl.total, &ctl)) != PAD_OK) return st;
+  if (pr.cl.total > 0 && (st = get_buffer(g_ctl, pr.device, stream, pr.cl.total, &ctl)) != PAD_OK) return st;
   bind_buffers(pr, ws, ctl);
   return run(pr, stream);
 }
@@ -448,7 +457,7 @@ pad_status pad_decode_with_workspace(const pad_tensor *q, const pad_tensor *k_ca
   if (st != PAD_OK || empty) return st;
   if ((st = check_caller_buffer(pr, workspace, workspace_bytes, pr.ws.total, "workspace")) != PAD_OK) return st;
   void *ctl = nullptr;
-  if ((st = get_buffer(g_ctl, pr.device, stream, pr.cl.total, &ctl)) != PAD_OK) return st;
+  if (pr.cl.total > 0 && (st = get_buffer(g_ctl, pr.device, stream, pr.cl.total, &ctl)) != PAD_OK) return st;
   bind_buffers(pr, workspace, ctl);
   return run(pr, stream);
 }
@@ -466,18 +475,9 @@ pad_status pad_check_device_errors(void *stream_, uint32_t *bits) {
   const uint32_t zero = 0;
   if ((e = cudaMemcpy(word, &zero, 4, cudaMemcpyHostToDevice)) != cudaSuccess) return cuda_fail(e, "clear error word");
   if (bits != nullptr) *bits = v;
-  if (v & pad::kErrTimeout) {
-    // an aborted launch may have left claim/merge counters set: re-zero the
-    // library's own scratch on this device
-    std::lock_guard<std::mutex> lock(g_ws_mu);
-    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-    for (auto &kv : g_ctl)
-      if (kv.first.first == device && kv.second.ptr != nullptr) cudaMemset(kv.second.ptr, 0, kv.second.bytes);
-  }
   if (v != 0)
-    return fail(PAD_ERR_DEVICE_CHECK, "kernel saw %s%s%s", (v & pad::kErrBlockId) ? "an out-of-range block id; " : "",
-                (v & pad::kErrSeqLen) ? "an out-of-range sequence length; " : "",
-                (v & pad::kErrTimeout) ? "a wait that timed out (internal error)" : "");
+    return fail(PAD_ERR_DEVICE_CHECK, "kernel saw %s%s", (v & pad::kErrBlockId) ? "an out-of-range block id; " : "",
+                (v & pad::kErrSeqLen) ? "an out-of-range sequence length" : "");
   return PAD_OK;
 }
 

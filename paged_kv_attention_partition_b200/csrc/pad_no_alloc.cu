@@ -7,9 +7,9 @@
 // pre-planned (a fixed arena carved up at start-up), a host thread that is not
 // allowed to take the allocator's locks or trigger the synchronisation cudaMalloc
 // and cudaFree may imply, or an embedding that has no allocator of its own to
-// hand the library.  pad_decode grows library-owned scratch on demand and the
-// two-pass entry points need the caller to supply scratch; this entry point needs
-// neither.
+// hand the library.  pad_decode grows library-owned scratch on demand and
+// pad_decode_with_workspace needs the caller to supply scratch; this entry point
+// needs neither.
 //
 // The scratch is one file-scope __device__ array of kStaticScratchBytes.  Every
 // GPU that loads the library holds it until the process exits, and every call on
@@ -74,8 +74,8 @@ extern "C" pad_status pad_decode_static_scratch(const pad_tensor *q, const pad_t
                                                 const pad_tensor *v_cache, const pad_tensor *block_tables,
                                                 const pad_tensor *seq_lens, float scale, int32_t num_splits,
                                                 pad_tensor *out, pad_tensor *lse, void *stream) {
-  // The array holds the control block (claim word, merge counters) first and the
-  // split partials after it.  Reject shapes that do not fit before launching.
+  // The array holds the control block (merge counters) first and the split
+  // partials after it.  Reject shapes that do not fit before launching.
   size_t control = 0;
   if (q != nullptr && k_cache != nullptr && block_tables != nullptr && q->ndim == 3 && k_cache->ndim == 4 &&
       block_tables->ndim == 2) {
@@ -98,17 +98,9 @@ extern "C" pad_status pad_decode_static_scratch(const pad_tensor *q, const pad_t
   pad_status st = pad::static_scratch_address(&scratch);
   if (st != PAD_OK) return st;
   // The control block must start at zero.  A completed call leaves it zero, but
-  // the array outlives every call, so clear it on the stream first.
-  if (control > 0) {
-    cudaError_t e = cudaMemsetAsync(scratch, 0, control, static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) {
-      char msg[256];
-      snprintf(msg, sizeof msg, "cudaMemsetAsync(static scratch control block): %s", cudaGetErrorString(e));
-      pad::set_last_error(msg);
-      return PAD_ERR_CUDA;
-    }
-  }
+  // the array outlives every call, so it is cleared on the stream after the
+  // arguments are validated and before the launch.
   return pad::decode_with_buffers(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse,
                                   static_cast<char *>(scratch) + control, pad::kStaticScratchBytes - control,
-                                  scratch, control, static_cast<cudaStream_t>(stream));
+                                  scratch, control, /*clear_control=*/true, static_cast<cudaStream_t>(stream));
 }

@@ -57,15 +57,18 @@ def test_plan_follows_the_partition_rule(lib):
     # explicit splits: P = round_up(ceil(C / S), bs), S_eff = ceil(C / P)
     p = pad.pad_decode_plan(64, 40, 8, 128, 16, 512, num_splits=16, device=0)
     assert (p["num_splits"], p["partition_tokens"], p["reduce"]) == (16, 512, 1)
-    # persistent grid: one CTA per SM (148 when no device answers)
-    assert p["ctas"] == 148 and p["head_tiles"] == 1 and p["heads_per_tile"] == 8
-    assert p["warps_per_cta"] == 6 and p["stage_tokens"] == 64 and p["stages"] >= 2
-    assert p["workspace_bytes"] >= 64 * 40 * 16 * (128 + 1) * 4 and p["control_bytes"] >= 256 + 64 * 8 * 4
+    # one CTA per (sequence, KV head, head tile, partition)
+    assert p["ctas"] == 64 * 8 * 16 and p["head_tiles"] == 1 and p["heads_per_tile"] == 8
+    assert p["warps_per_cta"] == 4 and p["stage_tokens"] == 64 and p["stages"] == 2
+    assert p["workspace_bytes"] >= 64 * 40 * 16 * (128 + 1) * 4 and p["control_bytes"] >= 64 * 8 * 4
     p = pad.pad_decode_plan(16, 16, 4, 256, 16, 2048, num_splits=32, device=0)
     assert (p["num_splits"], p["partition_tokens"]) == (32, 1024)
     p = pad.pad_decode_plan(1, 4, 1, 128, 16, 16, num_splits=1, device=0)
-    # one unit: one CTA; no partials, only the claim block
-    assert (p["num_splits"], p["reduce"], p["workspace_bytes"], p["ctas"], p["control_bytes"]) == (1, 0, 0, 1, 256)
+    # one unit: one CTA; no partials, no merge counters
+    assert (p["num_splits"], p["reduce"], p["workspace_bytes"], p["ctas"], p["control_bytes"]) == (1, 0, 0, 1, 0)
+    # at most 256 partitions per sequence
+    p = pad.pad_decode_plan(2, 4, 1, 128, 1, 4096, num_splits=4096, device=0)
+    assert (p["num_splits"], p["partition_tokens"]) == (256, 16)
     p = pad.pad_decode_plan(2, 4, 1, 128, 16, 4, num_splits=7, device=0)  # C=64, P=16
     assert (p["num_splits"], p["partition_tokens"]) == (4, 16)
     p = pad.pad_decode_plan(2, 4, 1, 128, 1, 100, num_splits=3, device=0)  # bs=1: P=34, S=3
@@ -82,10 +85,15 @@ def test_heuristic_plans(lib):
         assert p["partition_tokens"] % bs == 0 and p["partition_tokens"] <= max(C, bs)
         assert p["num_splits"] == -(-C // p["partition_tokens"])
         assert p["heads_per_tile"] * p["head_tiles"] >= g and p["heads_per_tile"] <= 32
-        # partitions of at least 256 tokens, and the partial each writes (g*D*4
+        # partitions of at least 64 tokens, and the partial each writes (g*D*4
         # bytes) at most 1/16 of the K/V bytes it streams (4*D*P)
         if p["num_splits"] > 1:
-            assert p["partition_tokens"] >= 256 and g / p["partition_tokens"] <= 1 / 16 + 1e-9
+            assert p["partition_tokens"] >= 64 and g / p["partition_tokens"] <= 1 / 16 + 1e-9
+    # large batches keep 256-token partitions; a small batch is cut finer (down to
+    # 64 tokens) until it fills about two waves of CTAs on 148 SMs
+    assert pad.pad_decode_plan(32, 32, 8, 128, 16, 256, num_splits=0, device=0)["partition_tokens"] == 256
+    assert pad.pad_decode_plan(1, 32, 8, 128, 16, 256, num_splits=0, device=0)["partition_tokens"] == 64
+    assert pad.pad_decode_plan(4, 32, 8, 128, 16, 256, num_splits=0, device=0)["partition_tokens"] == 128
     # group 20: one 32-head tile at D=128, two 16-head tiles at D=256; group 64: two tiles
     p = pad.pad_decode_plan(2, 20, 1, 128, 16, 10, num_splits=1, device=0)
     assert (p["heads_per_tile"], p["head_tiles"]) == (32, 1)
