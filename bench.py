@@ -1,16 +1,18 @@
 #!/usr/bin/env python
 """Benchmark: paged single-token decode attention on B200.
 
-One step = one full pass of the hot path (partition kernel + split-reduce kernel)
-over one decode batch.  Default workload: the Llama-8B-shaped decode batch
+One step = one full pass of the hot path (one launch: partition kernel with the
+split reduce folded in) over one decode batch.  Default workload: the Llama-8B-shaped decode batch
 (B=32, Hq/Hkv=32/8, D=128, block_size 16, seq_lens ~ U{512..4096}, synthetic bf16
 ~N(0,1), tables over a 4096-block pool).  --workload picks another named one.
 
 Prints one JSON line (rank 0).  `value` is achieved algorithmic HBM GB/s of the
 whole step (all ranks' bytes / max-over-ranks device time); `us_per_call` is the
 mean device time per step.  Timing: W warm-up steps, then K timed steps, each
-bracketed by CUDA events on the launching stream, with a 256 MiB L2-flush write
-between steps outside the events; barrier + synchronize around the timed region.
+bracketed by CUDA events on the launching stream, with an L2 flush between steps
+outside the events (a 256 MiB write, then a 256 MiB read so that the written
+lines are evicted too: every timed launch starts from a cold L2 holding no dirty
+data); barrier + synchronize around the timed region.
 
 --impl reference times the CPU oracle (the reference arm of this path) on the
 host cores instead; it never touches the GPU.
@@ -67,7 +69,8 @@ def workload_config(w, plan):
     if plan is not None:
         cfg.update({"num_splits": plan["num_splits"], "partition_tokens": plan["partition_tokens"],
                     "heads_per_tile": plan["heads_per_tile"], "ctas": plan["ctas"]})
-    cfg["l2"] = f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write outside the timed events)"
+    cfg["l2"] = (f"flushed between steps outside the timed events: {L2_FLUSH_BYTES >> 20} MiB write, "
+                 f"then {L2_FLUSH_BYTES >> 20} MiB read (cold, clean L2)")
     return cfg
 
 
@@ -228,7 +231,13 @@ def main():
     # caller-owned partials scratch (contents irrelevant)
     ws = torch.empty(plan["workspace_bytes"] // 4 + 64, dtype=torch.float32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_acc = torch.empty((), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(dev)
+
+    def flush_l2(i):
+        flush.fill_(float(i))
+        torch.sum(flush_rd, 0, out=flush_acc)
 
     def step():
         # the whole hot path: one launch (partition + fused reduce)
@@ -236,7 +245,7 @@ def main():
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            flush.fill_(1.0)
+            flush_l2(1)
             step()
             pad.pad_decode(q, k, v, tables, lens, w.scale, num_splits=splits, out=out, lse=lse, stream=stream)
     stream.synchronize()
@@ -249,7 +258,7 @@ def main():
     with ClockSampler(local) as clocks:
         with torch.cuda.stream(stream):
             for i in range(args.steps):
-                flush.fill_(float(i))
+                flush_l2(i)
                 ev = events[i]
                 ev[0].record(stream)
                 step()
@@ -287,7 +296,7 @@ def main():
     e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(e2e_steps)]
     with torch.cuda.stream(stream):
         for i in range(-3 if e2e_steps else 0, e2e_steps):
-            flush.fill_(float(i))
+            flush_l2(i)
             if i >= 0:
                 e2e_ev[i][0].record(stream)
             q.copy_(hq, non_blocking=True)

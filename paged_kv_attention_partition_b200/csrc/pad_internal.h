@@ -45,7 +45,7 @@ __host__ __device__ constexpr SmemPlan smem_plan_for(int D, int hpt) {
   s.stages = stages_for(D, hpt);
   s.stage_bytes = (size_t)kStageTokens * D * 2 * 2;  // K and V rows of one stage
   s.ring_bytes = (size_t)s.stages * s.stage_bytes;
-  s.warp_merge_bytes = (size_t)kWarps * hpt * (D + 2) * 4;
+  s.warp_merge_bytes = (size_t)kWarps * hpt * (D + 4 + 2) * 4;  // padded rows, then m and l
   s.split_merge_bytes = (size_t)hpt * (kMaxSplits + 1) * 4;
   size_t m = s.ring_bytes;
   if (s.warp_merge_bytes > m) m = s.warp_merge_bytes;

@@ -285,9 +285,11 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
   cp_async_wait<0>();
   __syncthreads();
 
-  // ---- merge the four warps' states through shared memory (the ring is free)
-  float *sm_o = reinterpret_cast<float *>(smem);  // [kWarps][HPT][D]
-  float *sm_m = sm_o + kWarps * HPT * D;           // [kWarps][HPT]
+  // ---- merge the four warps' states through shared memory (the ring is free);
+  // rows padded to D+4 floats so the fragment stores below are conflict free
+  constexpr int MROW = D + 4;
+  float *sm_o = reinterpret_cast<float *>(smem);  // [kWarps][HPT][MROW]
+  float *sm_m = sm_o + kWarps * HPT * MROW;        // [kWarps][HPT]
   float *sm_l = sm_m + kWarps * HPT;               // [kWarps][HPT]
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -304,11 +306,11 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
 #pragma unroll
     for (int mt = 0; mt < KT; ++mt) {
       const int d = mt * 16 + (lane >> 2);
-      float *o0 = sm_o + (warp * HPT + nt * 8 + (lane & 3) * 2) * D;
+      float *o0 = sm_o + (warp * HPT + nt * 8 + (lane & 3) * 2) * MROW;
       o0[d] = oacc[mt][nt][0];
-      o0[D + d] = oacc[mt][nt][1];
+      o0[MROW + d] = oacc[mt][nt][1];
       o0[d + 8] = oacc[mt][nt][2];
-      o0[D + d + 8] = oacc[mt][nt][3];
+      o0[MROW + d + 8] = oacc[mt][nt][3];
     }
   }
   __syncthreads();
@@ -327,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
       if (mw == -INFINITY) continue;  // warp saw no token of this partition
       const float f = fast_exp2(mw - m);
       l += f * sm_l[w * HPT + hl];
-      const float4 ow = *reinterpret_cast<const float4 *>(sm_o + (w * HPT + hl) * D + d);
+      const float4 ow = *reinterpret_cast<const float4 *>(sm_o + (w * HPT + hl) * MROW + d);
       o.x += f * ow.x;
       o.y += f * ow.y;
       o.z += f * ow.z;
@@ -350,11 +352,13 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
   }
   if (ns == 1) return;
 
-  // ---- split reduce: the CTA that finishes the set's last partition merges it
-  __threadfence();  // this thread's partial stores, before the count below
+  // ---- split reduce: the CTA that finishes the set's last partition merges it.
+  // The barrier orders every thread's partial stores before thread 0's fence,
+  // which publishes them (cumulatively) before the count.
   __syncthreads();
   if (tid == 0) {
     const uint32_t pair = ((uint32_t)b * p.Hkv + kvh) * p.HT + ht;
+    __threadfence();
     const uint32_t done = atomicAdd(p.counters + pair, 1u);
     const int last = done + 1 == (uint32_t)ns;
     if (last) {
