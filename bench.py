@@ -190,6 +190,36 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def rank_seed(base_seed, rank):
+    """Weak scaling: rank r decodes its own batch of the same shape, drawn with
+    seed base + 1000 r (rank 0 keeps the named workload's own seed)."""
+    return base_seed + 1000 * rank
+
+
+def max_over_ranks(x, device, world):
+    """The largest value of `x` over all ranks (the slowest rank's time)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def max_time_sum_bytes(total_ms, my_bytes, device, world):
+    """Whole-job aggregate: (max over ranks of the timed device time, sum over
+    ranks of the algorithmic bytes moved).  Every rank must call it."""
+    if world == 1:
+        return float(total_ms), float(my_bytes)
+    import torch
+    import torch.distributed as dist
+    t_max = max_over_ranks(total_ms, device, world)
+    bt = torch.tensor([float(my_bytes)], device=device, dtype=torch.float64)
+    dist.all_reduce(bt, op=dist.ReduceOp.SUM)
+    return t_max, float(bt.item())
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -214,7 +244,7 @@ def main():
 
     # weak scaling: every rank decodes its own batch of the same shape
     base = synth.config(args.workload)
-    w = synth.config(args.workload, seed=base.seed + 1000 * rank) if rank else base
+    w = synth.config(args.workload, seed=rank_seed(base.seed, rank)) if rank else base
     splits = w.num_splits if args.num_splits is None else args.num_splits
     plan = pad.pad_decode_plan(w.B, w.Hq, w.Hkv, w.D, w.block_size, w.max_blocks_per_seq, num_splits=splits,
                                device=local)
@@ -268,17 +298,7 @@ def main():
         dist.barrier()
     step_ms = [e[0].elapsed_time(e[1]) for e in events]
     part_ms = step_ms  # the step is exactly one launch of the partition kernel
-    total_ms = sum(step_ms)
-    my_bytes = w.algorithmic_bytes() * args.steps
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-        bt = torch.tensor([float(my_bytes)], device=dev, dtype=torch.float64)
-        dist.all_reduce(bt, op=dist.ReduceOp.SUM)
-        all_bytes = float(bt.item())
-    else:
-        all_bytes = float(my_bytes)
+    total_ms, all_bytes = max_time_sum_bytes(sum(step_ms), w.algorithmic_bytes() * args.steps, dev, world)
     value = all_bytes / (total_ms / 1e3) / 1e9
 
     # ---- end to end through the public one-call API, host buffers -----------
@@ -310,13 +330,9 @@ def main():
                 e2e_ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = sum(e[0].elapsed_time(e[1]) for e in e2e_ev) if e2e_steps else float("nan")
-    if world > 1 and e2e_steps:
-        t = torch.tensor([e2e_ms / e2e_steps * args.steps], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
-    else:
-        e2e_total = e2e_ms / max(e2e_steps, 1) * args.steps
-    e2e_value = all_bytes / (e2e_total / 1e3) / 1e9
+    # every rank takes the same collective steps, e2e leg or not
+    e2e_total = max_over_ranks(e2e_ms / max(e2e_steps, 1) * args.steps if e2e_steps else 0.0, dev, world)
+    e2e_value = all_bytes / (e2e_total / 1e3) / 1e9 if e2e_steps else float("nan")
 
     errs = pad.pad_check_device_errors(stream)
     if errs:
