@@ -103,7 +103,9 @@ typedef struct pad_plan {
  *                [blocks, bs, Hkv, D] "NHD" cache are accepted).  Base 16-byte aligned.
  *  v_cache       bf16, same shape as k_cache, its own strides, same rules.
  *  block_tables  int32 [B, max_blocks_per_seq], stride[1] == 1.  Entries past
- *                ceil(L_b / block_size) are never read.
+ *                ceil(L_b / block_size) may hold anything: their values are never
+ *                used (the kernel may read them, within the row, before it knows
+ *                L_b).
  *  seq_lens      int32 [B], contiguous.
  *  scale         finite; multiplies q.k before the softmax (commonly 1/sqrt(D)).
  *  num_splits    0 = let the library choose; S >= 1 asks for partitions of

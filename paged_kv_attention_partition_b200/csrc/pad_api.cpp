@@ -120,12 +120,60 @@ void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan) {
   plan->heads_per_tile = hpt;
   plan->head_tiles = (int32_t)HT;
   plan->warps_per_cta = pad::kWarps;
-  plan->stage_tokens = pad::kStageTokens;
+  plan->stage_tokens = pad::stage_tokens_for((int)s.D, hpt);
   plan->stages = pad::partition_stages((int)s.D, hpt);
   plan->ctas = (int32_t)(units > 0x7fffffffll ? 0x7fffffffll : units);
   plan->reduce = S > 1 ? 1 : 0;
   plan->workspace_bytes = (int64_t)pad::workspace_layout(s.B, s.Hq, S, s.D).total;
   plan->control_bytes = (int64_t)pad::control_layout(s.B, s.Hkv, HT, S).total;
+}
+
+// ---- TMA tensor maps of the K/V caches --------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against libcuda); null if the driver does not provide it.
+EncodeTiledFn tensor_map_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// A [num_blocks, Hkv, bs, D] bf16 cache as the 5-D tensor (64 head_dim
+// elements, slot, head_dim / 64, kv head, block) with boxes of (64, box_rows,
+// D / 64, 1, 1) and the 128-byte swizzle.  Byte strides of size-1 dimensions
+// are never used; a natural value stands in for them.
+pad_status encode_cache_map(CUtensorMap *map, const pad_tensor *t, int box_rows_, const char *name) {
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (enc == nullptr) return fail(PAD_ERR_CUDA, "the CUDA driver does not provide cuTensorMapEncodeTiled");
+  const int64_t NB = t->shape[0], Hkv = t->shape[1], bs = t->shape[2], D = t->shape[3];
+  auto stride_bytes = [&](int i, int64_t natural) -> cuuint64_t {
+    return (cuuint64_t)(t->shape[i] > 1 ? t->stride[i] * 2 : natural);
+  };
+  const cuuint64_t dims[5] = {64, (cuuint64_t)bs, (cuuint64_t)(D / 64), (cuuint64_t)Hkv, (cuuint64_t)NB};
+  const cuuint64_t strides[4] = {stride_bytes(2, D * 2), 128, stride_bytes(1, bs * D * 2),
+                                 stride_bytes(0, Hkv * bs * D * 2)};
+  const cuuint32_t box[5] = {64, (cuuint32_t)box_rows_, (cuuint32_t)(D / 64), 1, 1};
+  const cuuint32_t elem[5] = {1, 1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, t->data, dims, strides, box, elem,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(PAD_ERR_INVALID_ARG, "%s: strides/shape not expressible as a TMA tensor (cuTensorMapEncodeTiled %d)",
+                name, (int)r);
+  return PAD_OK;
 }
 
 // ---- tensor descriptor checks -----------------------------------------------
@@ -305,6 +353,9 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
 
   pad::PartitionParams &p = pr->p;
   p = pad::PartitionParams{};
+  const int rows = pad::box_rows((int)bs, (int)D, pr->plan.heads_per_tile);
+  if ((st = encode_cache_map(&p.tmk, k_cache, rows, "k_cache")) != PAD_OK) return st;
+  if ((st = encode_cache_map(&p.tmv, v_cache, rows, "v_cache")) != PAD_OK) return st;
   p.q = static_cast<const uint16_t *>(q->data);
   p.q_sb = q->stride[0];
   p.q_sh = q->stride[1];
@@ -475,9 +526,18 @@ pad_status pad_check_device_errors(void *stream_, uint32_t *bits) {
   const uint32_t zero = 0;
   if ((e = cudaMemcpy(word, &zero, 4, cudaMemcpyHostToDevice)) != cudaSuccess) return cuda_fail(e, "clear error word");
   if (bits != nullptr) *bits = v;
+  if (v & pad::kErrTimeout) {
+    // an abandoned launch may have left merge counters set: re-zero the
+    // library's own control blocks on this device
+    std::lock_guard<std::mutex> lock(g_ws_mu);
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    for (auto &kv : g_ctl)
+      if (kv.first.first == device && kv.second.ptr != nullptr) cudaMemset(kv.second.ptr, 0, kv.second.bytes);
+  }
   if (v != 0)
-    return fail(PAD_ERR_DEVICE_CHECK, "kernel saw %s%s", (v & pad::kErrBlockId) ? "an out-of-range block id; " : "",
-                (v & pad::kErrSeqLen) ? "an out-of-range sequence length" : "");
+    return fail(PAD_ERR_DEVICE_CHECK, "kernel saw %s%s%s", (v & pad::kErrBlockId) ? "an out-of-range block id; " : "",
+                (v & pad::kErrSeqLen) ? "an out-of-range sequence length; " : "",
+                (v & pad::kErrTimeout) ? "a stage whose copies never completed (internal error)" : "");
   return PAD_OK;
 }
 

@@ -1,6 +1,7 @@
 // Internal launch parameters shared by the host API and the kernel.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -12,45 +13,56 @@ namespace pad {
 enum : uint32_t {
   kErrBlockId = 0x1u,  // a live table entry outside [0, num_blocks)
   kErrSeqLen = 0x2u,   // seq_lens[b] < 0 or > table capacity
+  kErrTimeout = 0x4u,  // a bounded wait for a stage's copies gave up (internal error)
 };
 
-// Kernel geometry: one CTA of 4 warps per work unit; warp w computes tokens
-// 16w .. 16w+15 of every 64-token shared-memory stage, and all 128 threads load.
+// Kernel geometry: one CTA of 4 warps per work unit; one thread issues the
+// stage copies (TMA), all four warps compute.  The warps form kWarps / dsplit token groups of dsplit warps each: token group
+// tg computes tokens 16 tg .. 16 tg + 15 of every shared-memory stage (so a
+// stage holds 16 kWarps / dsplit tokens), and warp dh of the group keeps the
+// dh-th 1/dsplit of the head_dim rows of O^T (both warps of a group compute
+// the same scores).  Splitting head_dim halves the stage and the accumulator
+// where they would otherwise limit residency: at D = 256 (64 KB stages).
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
-constexpr int kStageTokens = 16 * kWarps;
 constexpr int kSmemBudget = 232448;  // 227 KiB per CTA
 constexpr int kMaxSplits = 256;      // partitions per sequence (bounds the merge's weight table)
 
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ constexpr int dsplit_for(int D, int hpt) { return D == 256 ? 2 : 1; }
+__host__ __device__ constexpr int stage_tokens_for(int D, int hpt) { return 16 * kWarps / dsplit_for(D, hpt); }
 
 // Pipeline depth and resident CTAs per SM of one (head_dim, heads-per-tile)
 // instantiation.  The ring is kept small so that several CTAs share each SM:
 // their loads, math and start/finish latencies overlap one another.
 __host__ __device__ constexpr int stages_for(int D, int hpt) { return D == 64 || (D == 128 && hpt == 32) ? 3 : 2; }
 __host__ __device__ constexpr int ctas_per_sm_for(int D, int hpt) {
-  return D == 64 ? (hpt == 32 ? 3 : 4) : D == 128 ? (hpt == 32 ? 2 : 3) : 1;
+  return D == 64 ? (hpt == 32 ? 3 : 4) : D == 128 ? (hpt == 32 ? 2 : 3) : (hpt == 16 ? 2 : 3);
 }
 
-// Shared memory of one CTA: the K/V ring, reused after the last stage for the
-// four warps' merge (O^T, m, l) and then for the split merge's weight table;
-// a 16-byte flag word at the end.
+// Shared memory of one CTA (from a 1024-byte aligned base): the K/V ring,
+// reused after the last stage for the token groups' merge (O^T, m, l) and then
+// for the split merge's weight table; then one mbarrier per stage and two flag
+// words.
 struct SmemPlan {
-  int stages;
-  size_t stage_bytes, ring_bytes, warp_merge_bytes, split_merge_bytes, total;
+  int stages, stage_tokens;
+  size_t stage_bytes, ring_bytes, warp_merge_bytes, split_merge_bytes, region_bytes, total;
 };
 
 __host__ __device__ constexpr SmemPlan smem_plan_for(int D, int hpt) {
   SmemPlan s{};
   s.stages = stages_for(D, hpt);
-  s.stage_bytes = (size_t)kStageTokens * D * 2 * 2;  // K and V rows of one stage
+  s.stage_tokens = stage_tokens_for(D, hpt);
+  s.stage_bytes = (size_t)s.stage_tokens * D * 2 * 2;  // K and V rows of one stage
   s.ring_bytes = (size_t)s.stages * s.stage_bytes;
-  s.warp_merge_bytes = (size_t)kWarps * hpt * (D + 4 + 2) * 4;  // padded rows, then m and l
+  s.warp_merge_bytes = (size_t)(kWarps / dsplit_for(D, hpt)) * hpt * (D + 4 + 2) * 4;  // padded rows, m, l
   s.split_merge_bytes = (size_t)hpt * (kMaxSplits + 1) * 4;
   size_t m = s.ring_bytes;
   if (s.warp_merge_bytes > m) m = s.warp_merge_bytes;
   if (s.split_merge_bytes > m) m = s.split_merge_bytes;
-  s.total = align_up(m, 16) + 16;
+  s.region_bytes = align_up(m, 128);
+  s.total = 1024 /* alignment slack */ + s.region_bytes + 128 /* barriers, flags */;
   return s;
 }
 
@@ -58,6 +70,10 @@ __host__ __device__ constexpr SmemPlan smem_plan_for(int D, int hpt) {
 inline int max_heads_per_tile(int D) { return D <= 128 ? 32 : 16; }
 
 struct PartitionParams {
+  // K and V caches as 5-D tiled tensors (64 head_dim elements, slot, head_dim
+  // / 64, kv head, block), one box = one page (or a stage's worth of a larger
+  // page) with the 128-byte swizzle.
+  CUtensorMap tmk, tmv;
   const uint16_t *q;
   int64_t q_sb, q_sh;  // element strides over (b, h); d is contiguous
   const uint16_t *k;
@@ -116,6 +132,11 @@ inline ControlLayout control_layout(int64_t B, int64_t Hkv, int64_t HT, int64_t 
 }
 
 cudaError_t launch_partition(const PartitionParams &p, int D, int heads_per_tile, int grid, cudaStream_t s);
+// Rows of one TMA box: a page, or a stage's worth of rows of a larger page.
+inline int box_rows(int block_size, int D, int hpt) {
+  const int st = stage_tokens_for(D, hpt);
+  return block_size < st ? block_size : st;
+}
 int partition_stages(int D, int heads_per_tile);
 cudaError_t device_error_word(int device, uint32_t **ptr);
 void set_last_error(const char *msg);

@@ -8,19 +8,25 @@
 // CTAs share each SM (the ring is sized for it), so one CTA's start -- table and
 // q latency -- and finish -- merge and stores -- overlap the others' streaming.
 //
-// The CTA streams its partition's K and V pages for one KV head from HBM into a
-// small shared-memory ring (16-byte cp.async per thread; rows XOR-swizzled so the
-// tensor-core operand loads are bank-conflict free; rows past L_b zero-filled
-// without a read).  Each thread's page ids for the next stage are loaded one
-// stage ahead, so the loads never wait on the block table.  Every query head of
+// One thread streams the partition's K and V pages for one KV head from HBM
+// into a small shared-memory ring with TMA: one tiled box per page (or per
+// stage's worth of rows of a larger page) for K and one for V, completing on the
+// stage's mbarrier.  The box is (64 head_dim elements, its rows, head_dim / 64)
+// with the 128-byte swizzle, so the tensor-core operand loads below are bank
+// conflict free; an out-of-range block id reads as zeros.  Every query head of
 // the GQA group is served from that one K/V read ("spec(BACKEND-ROCM): the ROCm
 // head_dim=128 decode arm", section "It is a mirror of merged work, not new
-// design": PagedAttnDecodeGqaBf16 fuses a GQA group over one K/V read).
+// design": PagedAttnDecodeGqaBf16 fuses a GQA group over one K/V read).  Pages
+// are whole, so the last page's slots past L_b arrive too: their scores are
+// masked and their V rows zeroed before use.
 //
-// Warp w computes tokens 16w .. 16w+15 of every 64-token stage and keeps its own
-// running max and sum per head (the warp-strided online softmax of the same
-// section; the four warps are merged at the end, so the sum is taken in another
-// order than a sequential kernel's).  Per 16-token tile and 8-head n-tile:
+// The warps form token groups: group tg computes tokens 16tg .. 16tg+15 of every
+// stage and keeps its own running max and sum per head (the warp-strided online
+// softmax of the same section; the groups are merged at the end, so the sum is
+// taken in another order than a sequential kernel's).  At head_dim 256 a group
+// is two warps that compute the same scores and each keep half of the head_dim
+// rows of O^T, which halves the stage and the accumulator.
+// Per 16-token tile and 8-head n-tile:
 //   S^T = K . Q^T                 (mma.m16n8k16 bf16, fp32 accumulate)
 //   P^T = exp2(S^T * scale*log2e - m)
 //   O^T += V^T . P^T              (P^T moved into the B-operand layout by movmatrix)
@@ -31,6 +37,9 @@
 // head tile) merges them by log-sum-exp while they are in L2:
 //   M = max_s lse_s,  w_s = exp(lse_s - M) / sum_s' exp(lse_s' - M),
 //   out = sum_s w_s o_s,  lse = M + log sum_s exp(lse_s - M).
+//
+// Every mbarrier wait is bounded in time: on expiry the CTA sets an error bit,
+// waits (bounded again) for the copies it issued, and returns.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -46,7 +55,23 @@ __device__ uint32_t g_err_word;
 
 namespace {
 constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kRescaleSlack = 8.f;                  // log2 units: weights stay below 256
+constexpr uint64_t kWaitLimitNs = 1000000000ull;      // no stage can legitimately take 1 s
+
+// Waits for the phase of `bar` with this parity; false (and the timeout bit)
+// after kWaitLimitNs.
+__device__ bool wait_stage(uint32_t bar, uint32_t parity, uint32_t *err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t start = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - start > kWaitLimitNs) {
+      atomicOr(err, kErrTimeout);
+      return false;
+    }
+  }
+  return true;
 }
+}  // namespace
 
 template <int D, int HPT>
 __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
@@ -54,20 +79,28 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
   constexpr SmemPlan SP = smem_plan_for(D, HPT);
   constexpr int NST = SP.stages;
   constexpr uint32_t STAGE_BYTES = (uint32_t)SP.stage_bytes;
+  constexpr int ST = SP.stage_tokens;      // tokens per stage
+  constexpr int ST_LOG2 = ST == 64 ? 6 : 5;
+  constexpr int DS = dsplit_for(D, HPT);   // warps sharing a token group (head_dim split)
+  constexpr int TG = kWarps / DS;          // token groups
   constexpr int NT = HPT / 8;              // 8-head n-tiles
-  constexpr int KT = D / 16;               // QK k-steps == PV m-tiles
+  constexpr int KT = D / 16;               // QK k-steps
+  constexpr int MT = KT / DS;              // PV m-tiles (16 head_dim rows each) per warp
   constexpr int CH = D / 8;                // 16-byte chunks per K/V row
+  constexpr int NH = D / 64;               // 128-byte column blocks per row
   constexpr int ROWB = D * 2;
-  constexpr int RPP = kThreads / CH;       // rows per loader pass
-  constexpr int NR = kStageTokens / RPP;   // rows each thread loads per stage
+  constexpr int IDW = (ST + 31) / 32;      // block ids per lane of warp 0 for one stage
   constexpr bool SPLIT_QK = NT <= 2;       // two QK accumulation chains when registers allow
-  static_assert(kStageTokens % RPP == 0, "loader shape");
-  static_assert(NST == 2 || NST == 3, "prologue handles 2 or 3 stages");
+  static_assert(ST == 16 * TG && (1 << ST_LOG2) == ST, "stage shape");
+  static_assert(NST >= 2 && NST <= 8, "at least one stage in flight during the math; barrier area");
   static_assert(SP.total <= (size_t)kSmemBudget, "shared-memory plan over budget");
-  extern __shared__ __align__(128) uint8_t smem[];
-  int *flag = reinterpret_cast<int *>(smem + SP.total - 16);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + SP.region_bytes);  // one per stage slot
+  int *flag = reinterpret_cast<int *>(smem + SP.region_bytes + 64);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tg = warp / DS, dh = warp % DS;  // token group, head_dim part
   uint32_t u = blockIdx.x;
   const int s = (int)(u % (uint32_t)p.S);
   u /= (uint32_t)p.S;
@@ -78,13 +111,41 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
   const int h0 = kvh * p.g + ht * HPT;  // this unit serves query heads h0 .. h0+gl-1
   const int gl = min(HPT, p.g - ht * HPT);
   const int capacity = p.max_blocks << p.bs_log2;
+  const int t0 = s * p.P;
+
+  // A box holds bsb rows: a whole page, or a stage's worth of a larger page.
+  const int bsb_log2 = min(p.bs_log2, ST_LOG2);
+  const int nbox = ST >> bsb_log2;  // boxes per stage
+  const uint32_t box_bytes = (uint32_t)ROWB << bsb_log2;
+  const int32_t *trow = p.tables + (int64_t)b * p.table_stride;
+
+  // Warp 0 fetches the block ids of the first NST stages while the length is
+  // still in flight (clamped to the table row; an id is used only for a stage
+  // that holds live tokens): lane j holds box j, j + 32, ... of a stage.
+  int ids[NST][IDW];
+  auto load_ids = [&](int (&dst)[IDW], int st) {
+    const int page0 = (t0 + st * ST) >> p.bs_log2;
+#pragma unroll
+    for (int w = 0; w < IDW; ++w) {
+      const int j = lane + 32 * w;
+      dst[w] = j < nbox ? __ldg(trow + min(page0 + j, p.max_blocks - 1)) : 0;
+    }
+  };
+  if (warp == 0) {
+#pragma unroll
+    for (int k = 0; k < NST; ++k) load_ids(ids[k], k);
+  }
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < NST; ++i) mbar_init(smem_addr(full + i), 1);
+    fence_mbar_init();
+  }
 
   int L = __ldg(p.seq_lens + b);
   if (L < 0 || L > capacity) {
     if (tid == 0 && s == 0 && kvh == 0 && ht == 0) atomicOr(p.err, kErrSeqLen);
     L = L < 0 ? 0 : capacity;
   }
-  const int t0 = s * p.P;
   const int t1 = min(t0 + p.P, L);
   if (t0 >= t1) {
     if (L == 0 && s == 0) {  // empty sequence: out = 0, lse = -inf
@@ -95,51 +156,58 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
     return;
   }
   const int ns = (L + p.P - 1) / p.P;  // non-empty partitions of sequence b
-  const int nstages = (t1 - t0 + kStageTokens - 1) / kStageTokens;
+  const int nstages = (t1 - t0 + ST - 1) / ST;
+  __syncthreads();  // the stage barriers are initialised
 
-  // ---- K/V loader: thread (lr, lc) copies 16-byte chunk lc of rows lr, lr+RPP,
-  // ... of a stage; row r, chunk c lands at r*ROWB + ((c ^ (r & 7)) * 16).
-  const int32_t *trow = p.tables + (int64_t)b * p.table_stride;
-  const int lc = tid % CH, lr = tid / CH;
-  const int64_t kh_k = (int64_t)kvh * p.k_sh + lc * 8, kh_v = (int64_t)kvh * p.v_sh + lc * 8;
-  int pid[NR];  // block ids of this thread's rows in the next stage to issue
-  auto load_ids = [&](int (&ids)[NR], int st) {
-    const int base = t0 + st * kStageTokens + lr;
-#pragma unroll
-    for (int i = 0; i < NR; ++i) {
-      const int t = base + i * RPP;
-      ids[i] = t < t1 ? __ldg(trow + (t >> p.bs_log2)) : 0;
-    }
-  };
-  auto issue = [&](const int (&ids)[NR], int st) {
+  // Stage st into ring slot st % NST (called by all of warp 0; lane 0 issues).
+  // Only boxes holding live tokens are copied.
+  auto issue = [&](const int (&sid)[IDW], int st) {
+    const int tb = t0 + st * ST;
+    const int nb = min(nbox, (t1 - tb + (1 << bsb_log2) - 1) >> bsb_log2);
     uint8_t *sK = smem + (st % NST) * STAGE_BYTES;
-    uint8_t *sV = sK + kStageTokens * ROWB;
-    const int base = t0 + st * kStageTokens;
+    uint8_t *sV = sK + ST * ROWB;
+    const uint32_t bar = smem_addr(full + st % NST);
+    const int slot0 = tb & ((1 << p.bs_log2) - 1);  // row of the box inside its page
+    if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)nb * box_bytes * 2);
 #pragma unroll
-    for (int i = 0; i < NR; ++i) {
-      const int r = lr + i * RPP;
-      const int t = base + r;
-      bool valid = t < t1;
-      const uint16_t *ks = p.k, *vs = p.v;
-      if (valid) {
-        const int phys = ids[i];
-        if ((unsigned)phys < (unsigned)p.num_blocks) {
-          const int slot = t & ((1 << p.bs_log2) - 1);
-          ks = p.k + (int64_t)phys * p.k_sblk + kh_k + (int64_t)slot * p.k_ss;
-          vs = p.v + (int64_t)phys * p.v_sblk + kh_v + (int64_t)slot * p.v_ss;
-        } else {
-          atomicOr(p.err, kErrBlockId);  // never dereferenced: the row reads as zero
-          valid = false;
+    for (int w = 0; w < IDW; ++w) {
+#pragma unroll 1
+      for (int jj = 0; jj < 32 && 32 * w + jj < nb; ++jj) {
+        const int j = 32 * w + jj;
+        const int id = __shfl_sync(0xffffffffu, sid[w], jj);
+        if (lane == 0) {
+          if ((unsigned)id >= (unsigned)p.num_blocks) atomicOr(p.err, kErrBlockId);  // the box reads as zeros
+          tma_load_5d(smem_addr(sK + j * box_bytes), &p.tmk, 0, slot0, 0, kvh, id, bar);
+          tma_load_5d(smem_addr(sV + j * box_bytes), &p.tmv, 0, slot0, 0, kvh, id, bar);
         }
       }
-      const uint32_t off = r * ROWB + ((lc ^ (r & 7)) << 4);
-      cp_async_16(smem_addr(sK + off), ks, valid);
-      cp_async_16(smem_addr(sV + off), vs, valid);
     }
   };
+  if (warp == 0) {
+#pragma unroll
+    for (int k = 0; k < NST - 1; ++k)
+      if (k < nstages) issue(ids[k], k);
+  }
+  int (&idn)[IDW] = ids[NST - 1];  // block ids of the next stage to issue
 
-  // Q^T fragments (B operand of S^T = K.Q^T), loaded first so their latency
-  // overlaps the block-table reads: lane holds head nt*8 + lane/4,
+  // Address of 16-byte chunk (column block h, chunk c7 of it) of row r in a K
+  // or V half-stage: rows grouped in boxes of 2^bsb_log2 rows, each box laid out
+  // [D/64][rows][128 B], and the TMA's 128-byte swizzle XORs the chunk index
+  // with bits 7-9 of the address.  rbase/rkey depend on the row only.
+  auto row_base = [&](int r, uint32_t &rbase, uint32_t &rkey) {
+    const int slot = r & ((1 << bsb_log2) - 1);
+    rbase = (uint32_t)((r - slot) * ROWB + slot * 128);
+    rkey = (uint32_t)((r - slot) * NH + slot);
+  };
+  auto chunk = [&](uint32_t rbase, uint32_t rkey, int h, int c7) -> uint32_t {
+    return rbase + ((uint32_t)h << (bsb_log2 + 7)) + ((((uint32_t)c7) ^ ((rkey + ((uint32_t)h << bsb_log2)) & 7u)) << 4);
+  };
+  // QK operand rows (ldmatrix of K) and PV operand rows (transposed ldmatrix of V)
+  uint32_t kb, kk_key, vb, vkey;
+  row_base(tg * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, kb, kk_key);
+  row_base(tg * 16 + (lane & 7) + ((lane >> 4) & 1) * 8, vb, vkey);
+
+  // Q^T fragments (B operand of S^T = K.Q^T): lane holds head nt*8 + lane/4,
   // dims 16kk + 2(lane%4) + {0,1} and + {8,9}.  Padded heads are zero.
   uint32_t qf[KT][NT][2];
 #pragma unroll
@@ -154,27 +222,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
     }
   }
 
-  // Prologue: the page ids of the first two stages are fetched together, then
-  // stages 0 .. NST-2 are issued; pid ends up holding stage NST-1's ids.
-  {
-    int pid2[NR];
-    load_ids(pid, 0);
-    if (nstages > 1) load_ids(pid2, 1);
-    issue(pid, 0);
-    cp_async_commit();
-    if constexpr (NST == 3) {
-      if (nstages > 1) {
-        issue(pid2, 1);
-        if (nstages > 2) load_ids(pid, 2);
-      }
-      cp_async_commit();
-    } else {
-#pragma unroll
-      for (int i = 0; i < NR; ++i) pid[i] = pid2[i];
-    }
-  }
-
-  float oacc[KT][NT][4];
+  float oacc[MT][NT][4];
   float m_run[NT][2], l_run[NT][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -184,27 +232,43 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
       l_run[nt][j] = 0.f;
     }
 #pragma unroll
-    for (int mt = 0; mt < KT; ++mt)
+    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
       for (int i = 0; i < 4; ++i) oacc[mt][nt][i] = 0.f;
   }
 
+  int st = 0;
+  bool aborted = false;
 #pragma unroll 1
-  for (int st = 0; st < nstages; ++st) {
+  for (; st < nstages; ++st) {
     const int nx = st + NST - 1;
-    if (nx < nstages) {
-      issue(pid, nx);                          // ids fetched one stage ago
-      if (nx + 1 < nstages) load_ids(pid, nx + 1);  // in flight during this stage's math
+    if (warp == 0 && nx < nstages) {
+      issue(idn, nx);                                 // ids fetched one stage ago
+      if (nx + 1 < nstages) load_ids(idn, nx + 1);   // in flight during this stage's math
     }
-    cp_async_commit();
-    cp_async_wait<NST - 1>();  // stage st has landed (this thread's copies)
-    __syncthreads();           // ... and every other thread's
+    const bool landed = wait_stage(smem_addr(full + st % NST), (st / NST) & 1, p.err);
 
-    const uint8_t *sK = smem + (st % NST) * STAGE_BYTES;
-    const uint8_t *sV = sK + kStageTokens * ROWB;
-    const int tbase = t0 + st * kStageTokens + warp * 16;
+    uint8_t *sK = smem + (st % NST) * STAGE_BYTES;
+    uint8_t *sV = sK + ST * ROWB;
+    const int tb = t0 + st * ST;
+    if (tb + ST > t1) {
+      // the last stage: V rows past t1 (slots past L_b, rows of boxes not
+      // copied) are zeroed so that their zero weights meet finite values
+#pragma unroll 1
+      for (int e = lane; e < 16 * CH; e += 32) {
+        const int r = tg * 16 + e / CH, c = e % CH;
+        if (tb + r >= t1) {
+          uint32_t rb, rk;
+          row_base(r, rb, rk);
+          *reinterpret_cast<uint4 *>(sV + chunk(rb, rk, c >> 3, c & 7)) = make_uint4(0, 0, 0, 0);
+        }
+      }
+      fence_proxy_async_smem();  // before the slot's next TMA write
+      __syncwarp();
+    }
+    const int tbase = tb + tg * 16;
     if (tbase < t1) {
-      // ---- S^T = K . Q^T over this warp's 16 tokens
+      // ---- S^T = K . Q^T over this token group's 16 tokens
       float sc[NT][4], sc2[NT][4];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
@@ -212,10 +276,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
         for (int i = 0; i < 4; ++i) sc[nt][i] = sc2[nt][i] = 0.f;
 #pragma unroll
       for (int kk = 0; kk < KT; ++kk) {
-        const int r = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int ch = kk * 2 + (lane >> 4);
         uint32_t a[4];
-        ldsm_x4(a, smem_addr(sK + r * ROWB + ((ch ^ (r & 7)) << 4)));
+        ldsm_x4(a, smem_addr(sK + chunk(kb, kk_key, kk >> 2, ((kk * 2) & 7) + (lane >> 4))));
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           if (SPLIT_QK && (kk & 1))
@@ -244,53 +306,72 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
           mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
           mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
         }
-        // row 0 of the tile is a live token, so the new maxima are finite
-        const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
-        const float al0 = fast_exp2(m_run[nt][0] - mn0), al1 = fast_exp2(m_run[nt][1] - mn1);
-        m_run[nt][0] = mn0;
-        m_run[nt][1] = mn1;
-        const float e0 = fast_exp2(s0 - mn0), e1 = fast_exp2(s1 - mn1);
-        const float e2 = fast_exp2(s2 - mn0), e3 = fast_exp2(s3 - mn1);
+        // Lazy rescale: a head's reference max moves only when a score passes
+        // it by more than kRescaleSlack (log2 units), so weights stay below
+        // 2^kRescaleSlack and the O^T rescale is skipped on almost every tile.
+        // Any reference point gives the same out and lse as long as l and O^T
+        // share it.  Row 0 of the tile is a live token, so mx0/mx1 are finite
+        // and the first tile always sets the reference.
+        if (__any_sync(0xffffffffu, mx0 > m_run[nt][0] + kRescaleSlack || mx1 > m_run[nt][1] + kRescaleSlack)) {
+          const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+          const float al0 = fast_exp2(m_run[nt][0] - mn0), al1 = fast_exp2(m_run[nt][1] - mn1);
+          m_run[nt][0] = mn0;
+          m_run[nt][1] = mn1;
+          l_run[nt][0] *= al0;
+          l_run[nt][1] *= al1;
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            oacc[mt][nt][0] *= al0;
+            oacc[mt][nt][1] *= al1;
+            oacc[mt][nt][2] *= al0;
+            oacc[mt][nt][3] *= al1;
+          }
+        }
+        const float e0 = fast_exp2(s0 - m_run[nt][0]), e1 = fast_exp2(s1 - m_run[nt][1]);
+        const float e2 = fast_exp2(s2 - m_run[nt][0]), e3 = fast_exp2(s3 - m_run[nt][1]);
         const uint32_t pA = pack_bf16x2(e0, e1);
         const uint32_t pB = pack_bf16x2(e2, e3);
         // The running sum takes the fp32 weights: summing the bf16-rounded ones
         // moves the LSE of a short sequence by up to 2^-9 (one weight's rounding).
-        l_run[nt][0] = l_run[nt][0] * al0 + e0 + e2;
-        l_run[nt][1] = l_run[nt][1] * al1 + e1 + e3;
-#pragma unroll
-        for (int mt = 0; mt < KT; ++mt) {
-          oacc[mt][nt][0] *= al0;
-          oacc[mt][nt][1] *= al1;
-          oacc[mt][nt][2] *= al0;
-          oacc[mt][nt][3] *= al1;
-        }
+        l_run[nt][0] += e0 + e2;
+        l_run[nt][1] += e1 + e3;
         pb[nt][0] = movmatrix_t(pA);
         pb[nt][1] = movmatrix_t(pB);
       }
 
-      // ---- O^T += V^T . P^T  (rows past t1 were zero-filled, their weights are 0)
+      // ---- O^T += V^T . P^T over this warp's head_dim rows (rows past t1 were
+      // zero-filled, their weights are 0)
 #pragma unroll
-      for (int mt = 0; mt < KT; ++mt) {
-        const int j = lane >> 3;
-        const int r = warp * 16 + (lane & 7) + (j >> 1) * 8;
-        const int ch = mt * 2 + (j & 1);
+      for (int mt = 0; mt < MT; ++mt) {
+        const int gm = dh * MT + mt;  // m-tile of head_dim rows
         uint32_t a[4];
-        ldsm_x4_t(a, smem_addr(sV + r * ROWB + ((ch ^ (r & 7)) << 4)));
+        ldsm_x4_t(a, smem_addr(sV + chunk(vb, vkey, gm >> 2, ((gm * 2) & 7) + ((lane >> 3) & 1))));
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) mma_16816(oacc[mt][nt], a, pb[nt][0], pb[nt][1]);
       }
     }
-    __syncthreads();  // every warp is done with slot st % NST before it is refilled
+    // every warp is done with slot st % NST before it is refilled; a stage
+    // whose copies never landed ends the loop for the whole CTA
+    if (__syncthreads_or(!landed)) {
+      aborted = true;
+      break;
+    }
   }
-  cp_async_wait<0>();
-  __syncthreads();
+  if (aborted) {
+    // leave no copy in flight: wait (bounded) for every stage issued after st
+    if (tid == 0)
+      for (int j = st; j < nstages && j < st + NST; ++j) wait_stage(smem_addr(full + j % NST), (j / NST) & 1, p.err);
+    __syncthreads();
+    return;
+  }
 
-  // ---- merge the four warps' states through shared memory (the ring is free);
-  // rows padded to D+4 floats so the fragment stores below are conflict free
+  // ---- merge the token groups' states through shared memory (the ring is
+  // free); rows padded to D+4 floats so the fragment stores are conflict free.
+  // The warps of a group hold identical (m, l); the first one stores them.
   constexpr int MROW = D + 4;
-  float *sm_o = reinterpret_cast<float *>(smem);  // [kWarps][HPT][MROW]
-  float *sm_m = sm_o + kWarps * HPT * MROW;        // [kWarps][HPT]
-  float *sm_l = sm_m + kWarps * HPT;               // [kWarps][HPT]
+  float *sm_o = reinterpret_cast<float *>(smem);  // [TG][HPT][MROW]
+  float *sm_m = sm_o + TG * HPT * MROW;            // [TG][HPT]
+  float *sm_l = sm_m + TG * HPT;                   // [TG][HPT]
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -298,15 +379,15 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
       float l = l_run[nt][j];
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-      if (lane < 4) {
-        sm_m[warp * HPT + nt * 8 + 2 * lane + j] = m_run[nt][j];
-        sm_l[warp * HPT + nt * 8 + 2 * lane + j] = l;
+      if (dh == 0 && lane < 4) {
+        sm_m[tg * HPT + nt * 8 + 2 * lane + j] = m_run[nt][j];
+        sm_l[tg * HPT + nt * 8 + 2 * lane + j] = l;
       }
     }
 #pragma unroll
-    for (int mt = 0; mt < KT; ++mt) {
-      const int d = mt * 16 + (lane >> 2);
-      float *o0 = sm_o + (warp * HPT + nt * 8 + (lane & 3) * 2) * MROW;
+    for (int mt = 0; mt < MT; ++mt) {
+      const int d = (dh * MT + mt) * 16 + (lane >> 2);
+      float *o0 = sm_o + (tg * HPT + nt * 8 + (lane & 3) * 2) * MROW;
       o0[d] = oacc[mt][nt][0];
       o0[MROW + d] = oacc[mt][nt][1];
       o0[d + 8] = oacc[mt][nt][2];
@@ -320,13 +401,13 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
     const int hl = i / D4, d = (i % D4) * 4;
     float m = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) m = fmaxf(m, sm_m[w * HPT + hl]);
+    for (int w = 0; w < TG; ++w) m = fmaxf(m, sm_m[w * HPT + hl]);
     float l = 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
+    for (int w = 0; w < TG; ++w) {
       const float mw = sm_m[w * HPT + hl];
-      if (mw == -INFINITY) continue;  // warp saw no token of this partition
+      if (mw == -INFINITY) continue;  // token group saw no token of this partition
       const float f = fast_exp2(mw - m);
       l += f * sm_l[w * HPT + hl];
       const float4 ow = *reinterpret_cast<const float4 *>(sm_o + (w * HPT + hl) * MROW + d);
