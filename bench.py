@@ -47,6 +47,10 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline time budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (short profiling runs)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="first B sequences of the workload (reduced profiling cases); default: the full batch")
+    ap.add_argument("--compact-pool", action="store_true",
+                    help="block pool = exactly the blocks the batch uses, no page shared (llama8b: no-alias variant)")
     return ap.parse_args()
 
 
@@ -65,7 +69,7 @@ def workload_config(w, plan):
     cfg = {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.D,
            "block_size": w.block_size, "max_blocks_per_seq": w.max_blocks_per_seq,
            "kv_tokens": w.kv_tokens(), "seq_len_min": int(w.seq_lens.min()), "seq_len_max": int(w.seq_lens.max()),
-           "recipe": w.recipe, "lse": w.want_lse, "seed": w.seed}
+           "recipe": w.recipe, "lse": w.want_lse, "seed": w.seed, "pool_blocks": w.num_blocks - 1}
     if plan is not None:
         cfg.update({"num_splits": plan["num_splits"], "partition_tokens": plan["partition_tokens"],
                     "heads_per_tile": plan["heads_per_tile"], "ctas": plan["ctas"]})
@@ -177,7 +181,7 @@ def run_reference(args, rank, world):
     metric = "decode attention µs/call and achieved HBM GB/s vs B200 peak (1 GPU)"
     if rank != 0:
         return
-    w = synth.config(args.workload)
+    w = synth.config(args.workload, batch=args.batch, compact_pool=args.compact_pool)
     cb = cpu_baseline(w, args.cpu_seconds)
     us = cb["us_per_call"]
     line = {"impl": "reference", "metric": metric, "value": cb["value"], "unit": "GB/s", "n_gpus": args.gpus,
@@ -243,8 +247,9 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     # weak scaling: every rank decodes its own batch of the same shape
-    base = synth.config(args.workload)
-    w = synth.config(args.workload, seed=rank_seed(base.seed, rank)) if rank else base
+    base = synth.config(args.workload, batch=args.batch, compact_pool=args.compact_pool)
+    w = synth.config(args.workload, seed=rank_seed(base.seed, rank), batch=args.batch,
+                     compact_pool=args.compact_pool) if rank else base
     splits = w.num_splits if args.num_splits is None else args.num_splits
     plan = pad.pad_decode_plan(w.B, w.Hq, w.Hkv, w.D, w.block_size, w.max_blocks_per_seq, num_splits=splits,
                                device=local)
@@ -346,7 +351,8 @@ def main():
         p_ms = statistics.mean(part_ms)
         achieved = p_bytes / (p_ms / 1e3) / 1e9
         sha = kernel_source_sha()
-        traffic = traffic_from_profiles(w.name, sha)
+        # the recorded ncu traffic is for the named workload at full size
+        traffic = traffic_from_profiles(w.name, sha) if args.batch is None and not args.compact_pool else None
         kname = f"partition_kernel<{w.D},{plan['heads_per_tile']}>"
         line = {
             "metric": "decode attention µs/call and achieved HBM GB/s vs B200 peak (1 GPU)",

@@ -253,35 +253,56 @@ def make_workload(
 CONFIG_NAMES = ("tiny", "llama8b", "qwen14b", "longctx_d256", "ragged_mqa")
 
 
-def config(name: str, seed: Optional[int] = None) -> Workload:
-    """The named decode workloads (seeds 0..4 by default)."""
+def config(name: str, seed: Optional[int] = None, batch: Optional[int] = None,
+           compact_pool: bool = False) -> Workload:
+    """The named decode workloads (seeds 0..4 by default).
+
+    `batch` keeps every other parameter and takes the first `batch` sequences
+    (lengths come from a counter-based stream, so they are a prefix of the full
+    batch's).  `compact_pool` makes the block pool exactly the blocks the batch
+    uses, drawn without replacement: no page is shared between sequences and the
+    device holds only what is read.  Both serve reduced profiling cases; the
+    llama8b workload with `compact_pool` is also its no-alias variant."""
     idx = CONFIG_NAMES.index(name)
     seed = idx if seed is None else seed
+
+    def pool(default):
+        return None if compact_pool else default
+
+    def nb(default):
+        return default if batch is None else int(batch)
+
     if name == "tiny":
         return make_workload(
-            name, 1, 4, 1, 128, 16, [256], seed=seed, pool_blocks=16, max_blocks_per_seq=16,
+            name, nb(1), 4, 1, 128, 16, [256] * nb(1), seed=seed, pool_blocks=pool(16 * nb(1)), max_blocks_per_seq=16,
             num_splits=1, recipe="B1 Hq4/Hkv1 D128 L256 bs16, N(0,1), table = permutation of 16 blocks, S=1")
     if name == "llama8b":
-        lens = uniform_int(32, 512, 4096, seed, S_LENS)
+        B = nb(32)
+        lens = uniform_int(B, 512, 4096, seed, S_LENS)
         return make_workload(
-            name, 32, 32, 8, 128, 16, lens, seed=seed, pool_blocks=4096, max_blocks_per_seq=256,
-            table_mode="cyclic", num_splits=0,
-            recipe="B32 Hq32/Hkv8 D128 bs16, L~U{512..4096}, N(0,1), cyclic over one permutation of a 4096-block pool")
+            name, B, 32, 8, 128, 16, lens, seed=seed, pool_blocks=pool(4096), max_blocks_per_seq=256,
+            table_mode="unique" if compact_pool else "cyclic", num_splits=0,
+            recipe=("B32 Hq32/Hkv8 D128 bs16, L~U{512..4096}, N(0,1), "
+                    + ("blocks without replacement (no aliasing)" if compact_pool
+                       else "cyclic over one permutation of a 4096-block pool")))
     if name == "qwen14b":
+        B = nb(64)
         return make_workload(
-            name, 64, 40, 8, 128, 16, [8192] * 64, seed=seed, pool_blocks=32768, max_blocks_per_seq=512,
+            name, B, 40, 8, 128, 16, [8192] * B, seed=seed, pool_blocks=pool(32768), max_blocks_per_seq=512,
             num_splits=16, want_lse=True,
             recipe="B64 Hq40/Hkv8 D128 L8192 bs16, N(0,1), permutation of a 32768-block pool, 512-token partitions, LSE on")
     if name == "longctx_d256":
+        B = nb(16)
         return make_workload(
-            name, 16, 16, 4, 256, 16, [32768] * 16, seed=seed, pool_blocks=32768, max_blocks_per_seq=2048,
+            name, B, 16, 4, 256, 16, [32768] * B, seed=seed, pool_blocks=pool(32768), max_blocks_per_seq=2048,
             v_dist=DIST_UNIFORM_PM1, num_splits=32,
             recipe="B16 Hq16/Hkv4 D256 L32768 bs16, K~N(0,1), V~U(-1,1), permutation of a 32768-block pool, 1024-token partitions")
     if name == "ragged_mqa":
-        u = uniform(256, seed, S_LENS)
+        B = nb(256)
+        u = uniform(B, seed, S_LENS)
         lens = np.clip(np.floor(np.exp(math.log(16) + u * (math.log(32768) - math.log(16)))), 16, 32768).astype(np.int32)
         return make_workload(
-            name, 256, 32, 1, 128, 32, lens, seed=seed, pool_blocks=300_000, max_blocks_per_seq=1024,
+            name, B, 32, 1, 128, 32, lens, seed=seed, pool_blocks=pool(300_000), max_blocks_per_seq=1024,
             num_splits=0,
             recipe="B256 Hq32/Hkv1 D128 bs32, L log-uniform [16,32768], N(0,1), without replacement from a 300000-block pool")
     raise KeyError(name)

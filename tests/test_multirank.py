@@ -84,6 +84,8 @@ def test_reference_arm_other_ranks_exit_quietly(capsys):
         steps = 1
         warmup = 0
         cpu_seconds = 1.0
+        batch = None
+        compact_pool = False
     # under torchrun only rank 0 runs and prints the reference line
     assert bench.run_reference(A(), 1, 2) is None
     assert capsys.readouterr().out == ""
