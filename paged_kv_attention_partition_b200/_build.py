@@ -14,7 +14,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpad.so")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
-SOURCES = ["pad_api.cpp", "pad_partition.cu", "pad_no_alloc.cu"]
+SOURCES = ["pad_api.cpp", "pad_partition.cu", "pad_umma.cu", "pad_no_alloc.cu"]
 
 
 def nvcc() -> str:

@@ -119,9 +119,10 @@ void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan) {
   plan->partition_tokens = (int32_t)P;
   plan->heads_per_tile = hpt;
   plan->head_tiles = (int32_t)HT;
-  plan->warps_per_cta = pad::kWarps;
-  plan->stage_tokens = pad::stage_tokens_for((int)s.D, hpt);
-  plan->stages = pad::partition_stages((int)s.D, hpt);
+  const bool umma = pad::umma_eligible((int)s.D, hpt, (int)s.bs);
+  plan->warps_per_cta = umma ? pad::kUmmaWarps : pad::kWarps;
+  plan->stage_tokens = umma ? pad::kUmmaStageTokens : pad::stage_tokens_for((int)s.D, hpt);
+  plan->stages = umma ? pad::umma_stages() : pad::partition_stages((int)s.D, hpt);
   plan->ctas = (int32_t)(units > 0x7fffffffll ? 0x7fffffffll : units);
   plan->reduce = S > 1 ? 1 : 0;
   plan->workspace_bytes = (int64_t)pad::workspace_layout(s.B, s.Hq, S, s.D).total;
@@ -173,6 +174,24 @@ pad_status encode_cache_map(CUtensorMap *map, const pad_tensor *t, int box_rows_
   if (r != CUDA_SUCCESS)
     return fail(PAD_ERR_INVALID_ARG, "%s: strides/shape not expressible as a TMA tensor (cuTensorMapEncodeTiled %d)",
                 name, (int)r);
+  return PAD_OK;
+}
+
+// q [B, Hq, D] as the 4-D tensor (64 head_dim elements, head, head_dim / 64, b)
+// with boxes of (64, heads, D / 64, 1) and the 128-byte swizzle.
+pad_status encode_q_map(CUtensorMap *map, const pad_tensor *q, int heads) {
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (enc == nullptr) return fail(PAD_ERR_CUDA, "the CUDA driver does not provide cuTensorMapEncodeTiled");
+  const int64_t B = q->shape[0], Hq = q->shape[1], D = q->shape[2];
+  const cuuint64_t dims[4] = {64, (cuuint64_t)Hq, (cuuint64_t)(D / 64), (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)(Hq > 1 ? q->stride[1] * 2 : D * 2), 128,
+                                 (cuuint64_t)(B > 1 ? q->stride[0] * 2 : Hq * D * 2)};
+  const cuuint32_t box[4] = {64, (cuuint32_t)heads, (cuuint32_t)(D / 64), 1};
+  const cuuint32_t elem[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, q->data, dims, strides, box, elem,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PAD_ERR_INVALID_ARG, "q: strides/shape not expressible as a TMA tensor (%d)", (int)r);
   return PAD_OK;
 }
 
@@ -277,6 +296,7 @@ pad_status get_buffer(std::map<std::pair<int, cudaStream_t>, Workspace> &pool, i
 struct Prepared {
   pad::PartitionParams p;
   pad_plan plan;
+  bool umma;  // the tcgen05 kernel runs this shape
   pad::WorkspaceLayout ws;
   pad::ControlLayout cl;
   int D;
@@ -353,9 +373,11 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
 
   pad::PartitionParams &p = pr->p;
   p = pad::PartitionParams{};
-  const int rows = pad::box_rows((int)bs, (int)D, pr->plan.heads_per_tile);
+  pr->umma = pad::umma_eligible((int)D, pr->plan.heads_per_tile, (int)bs);
+  const int rows = pr->umma ? 8 : pad::box_rows((int)bs, (int)D, pr->plan.heads_per_tile);
   if ((st = encode_cache_map(&p.tmk, k_cache, rows, "k_cache")) != PAD_OK) return st;
   if ((st = encode_cache_map(&p.tmv, v_cache, rows, "v_cache")) != PAD_OK) return st;
+  if (pr->umma && (st = encode_q_map(&p.tmq, q, pr->plan.heads_per_tile)) != PAD_OK) return st;
   p.q = static_cast<const uint16_t *>(q->data);
   p.q_sb = q->stride[0];
   p.q_sh = q->stride[1];
@@ -411,7 +433,8 @@ pad_status check_caller_buffer(const Prepared &pr, void *buf, size_t bytes, size
 }
 
 pad_status run(const Prepared &pr, cudaStream_t stream) {
-  cudaError_t e = pad::launch_partition(pr.p, pr.D, pr.plan.heads_per_tile, pr.plan.ctas, stream);
+  cudaError_t e = pr.umma ? pad::launch_umma(pr.p, pr.plan.ctas, stream)
+                          : pad::launch_partition(pr.p, pr.D, pr.plan.heads_per_tile, pr.plan.ctas, stream);
   return e == cudaSuccess ? PAD_OK : cuda_fail(e, "partition kernel launch");
 }
 

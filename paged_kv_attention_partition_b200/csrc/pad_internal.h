@@ -72,8 +72,11 @@ inline int max_heads_per_tile(int D) { return D <= 128 ? 32 : 16; }
 struct PartitionParams {
   // K and V caches as 5-D tiled tensors (64 head_dim elements, slot, head_dim
   // / 64, kv head, block), one box = one page (or a stage's worth of a larger
-  // page) with the 128-byte swizzle.
+  // page; 8 rows for the tcgen05 kernel) with the 128-byte swizzle.
   CUtensorMap tmk, tmv;
+  // q as a 4-D tiled tensor (64 head_dim elements, head, head_dim / 64, b), one
+  // box = a 32-head tile (tcgen05 kernel only).
+  CUtensorMap tmq;
   const uint16_t *q;
   int64_t q_sb, q_sh;  // element strides over (b, h); d is contiguous
   const uint16_t *k;
@@ -132,6 +135,14 @@ inline ControlLayout control_layout(int64_t B, int64_t Hkv, int64_t HT, int64_t 
 }
 
 cudaError_t launch_partition(const PartitionParams &p, int D, int heads_per_tile, int grid, cudaStream_t s);
+// The tcgen05 kernel (pad_umma.cu) takes 32-head tiles at head_dim 128 with
+// pages of at least 8 tokens (its K/V boxes are 8 rows of one page).
+inline bool umma_eligible(int D, int hpt, int block_size) { return D == 128 && hpt == 32 && block_size >= 8; }
+cudaError_t launch_umma(const PartitionParams &p, int grid, cudaStream_t s);
+int umma_stages();
+constexpr int kUmmaStageTokens = 128;
+constexpr int kUmmaWarps = 6;
+
 // Rows of one TMA box: a page, or a stage's worth of rows of a larger page.
 inline int box_rows(int block_size, int D, int hpt) {
   const int st = stage_tokens_for(D, hpt);

@@ -1,0 +1,104 @@
+// The split reduce folded into the partition launches ("perf(rocke): prepare
+// saved paged decode bindings once", section "Summary": split-KV attention
+// followed by a reduce pass), shared by the mma.sync and tcgen05 kernels.
+//
+// Every partition of a sequence with ns > 1 non-empty partitions writes its
+// partial output o_s (normalised by its own sum) and lse_s.  The CTA whose
+// count brings the (b, KV head, head tile) counter to ns merges the set:
+//   M = max_s lse_s,  w_s = exp(lse_s - M) / sum_s' exp(lse_s' - M),
+//   out = sum_s w_s o_s,  lse = M + log sum_s exp(lse_s - M).
+#pragma once
+
+#include <math.h>
+#include <stdint.h>
+
+#include "pad_device.cuh"
+#include "pad_internal.h"
+
+namespace pad {
+
+// Counts this partition; true (in every thread) for the CTA that completes
+// the set, which also resets the counter for the next launch.  The barrier
+// orders every thread's partial stores before thread 0's fence, which publishes
+// them (cumulatively) before the count.  Every thread of the CTA calls it.
+__device__ __forceinline__ bool claim_last_partition(const PartitionParams &p, int b, int kvh, int ht, int ns,
+                                                     int *flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t pair = ((uint32_t)b * p.Hkv + kvh) * p.HT + ht;
+    __threadfence();
+    const uint32_t done = atomicAdd(p.counters + pair, 1u);
+    const int last = done + 1 == (uint32_t)ns;
+    if (last) {
+      atomicExch(p.counters + pair, 0u);  // ready for the next launch
+      __threadfence();                    // the other partials' stores, before the loads below
+    }
+    *flag = last;
+  }
+  __syncthreads();
+  return *flag != 0;
+}
+
+// Merges the ns partials of query heads h0 .. h0+gl-1 of sequence b into bf16
+// out (+ lse).  `wt` is shared memory for gl * ns floats.  Every thread of the
+// CTA (NTHREADS of them) calls it.
+template <int D, int NTHREADS>
+__device__ void merge_partials(const PartitionParams &p, int b, int h0, int gl, int ns, float *wt) {
+  constexpr int D4 = D / 4, NW = NTHREADS / 32;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t row0 = ((int64_t)b * p.Hq + h0) * p.S;
+  for (int i = tid; i < gl * ns; i += NTHREADS) {
+    const int hl = i / ns, si = i % ns;
+    wt[hl * ns + si] = ld_cg_f32(p.lse_part + row0 + (int64_t)hl * p.S + si);
+  }
+  __syncthreads();
+  for (int hl = warp; hl < gl; hl += NW) {
+    float M = -INFINITY;
+    for (int si = lane; si < ns; si += 32) M = fmaxf(M, wt[hl * ns + si]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float sum = 0.f;
+    for (int si = lane; si < ns; si += 32) sum += __expf(wt[hl * ns + si] - M);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    const float inv = 1.f / sum;
+    __syncwarp();
+    for (int si = lane; si < ns; si += 32) wt[hl * ns + si] = __expf(wt[hl * ns + si] - M) * inv;
+    if (lane == 0 && p.lse != nullptr) p.lse[b * p.lse_sb + (int64_t)(h0 + hl) * p.lse_sh] = M + logf(sum);
+  }
+  __syncthreads();
+  for (int i = tid; i < gl * D4; i += NTHREADS) {
+    const int hl = i / D4, d = (i % D4) * 4;
+    const float *orow = p.o_part + (row0 + (int64_t)hl * p.S) * D + d;
+    const float *w = wt + hl * ns;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int si = 0;
+    for (; si + 8 <= ns; si += 8) {  // eight partials in flight per thread
+      float4 ov[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ov[j] = ld_cg_f4(orow + (int64_t)(si + j) * D);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float wj = w[si + j];
+        acc.x += wj * ov[j].x;
+        acc.y += wj * ov[j].y;
+        acc.z += wj * ov[j].z;
+        acc.w += wj * ov[j].w;
+      }
+    }
+    for (; si < ns; ++si) {
+      const float4 ov = ld_cg_f4(orow + (int64_t)si * D);
+      const float wj = w[si];
+      acc.x += wj * ov.x;
+      acc.y += wj * ov.y;
+      acc.z += wj * ov.z;
+      acc.w += wj * ov.w;
+    }
+    uint2 packed;
+    packed.x = pack_bf16x2(acc.x, acc.y);
+    packed.y = pack_bf16x2(acc.z, acc.w);
+    *reinterpret_cast<uint2 *>(p.out + b * p.o_sb + (int64_t)(h0 + hl) * p.o_sh + d) = packed;
+  }
+}
+
+}  // namespace pad

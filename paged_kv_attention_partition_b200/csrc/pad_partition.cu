@@ -48,6 +48,7 @@
 
 #include "pad_device.cuh"
 #include "pad_internal.h"
+#include "pad_merge.cuh"
 
 namespace pad {
 
@@ -432,80 +433,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
     }
   }
   if (ns == 1) return;
-
-  // ---- split reduce: the CTA that finishes the set's last partition merges it.
-  // The barrier orders every thread's partial stores before thread 0's fence,
-  // which publishes them (cumulatively) before the count.
-  __syncthreads();
-  if (tid == 0) {
-    const uint32_t pair = ((uint32_t)b * p.Hkv + kvh) * p.HT + ht;
-    __threadfence();
-    const uint32_t done = atomicAdd(p.counters + pair, 1u);
-    const int last = done + 1 == (uint32_t)ns;
-    if (last) {
-      atomicExch(p.counters + pair, 0u);  // ready for the next launch
-      __threadfence();                    // the other partials' stores, before the loads below
-    }
-    *flag = last;
-  }
-  __syncthreads();
-  if (!*flag) return;
-
-  // weights w[hl][s] = exp(lse_s - M) / sum, in shared memory (the ring is free)
-  float *wt = reinterpret_cast<float *>(smem);  // [HPT][ns]
-  const int64_t row0 = ((int64_t)b * p.Hq + h0) * p.S;
-  for (int i = tid; i < gl * ns; i += kThreads) {
-    const int hl = i / ns, si = i % ns;
-    wt[hl * ns + si] = ld_cg_f32(p.lse_part + row0 + (int64_t)hl * p.S + si);
-  }
-  __syncthreads();
-  for (int hl = warp; hl < gl; hl += kWarps) {
-    float M = -INFINITY;
-    for (int si = lane; si < ns; si += 32) M = fmaxf(M, wt[hl * ns + si]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float sum = 0.f;
-    for (int si = lane; si < ns; si += 32) sum += __expf(wt[hl * ns + si] - M);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    const float inv = 1.f / sum;
-    __syncwarp();
-    for (int si = lane; si < ns; si += 32) wt[hl * ns + si] = __expf(wt[hl * ns + si] - M) * inv;
-    if (lane == 0 && p.lse != nullptr) p.lse[b * p.lse_sb + (int64_t)(h0 + hl) * p.lse_sh] = M + logf(sum);
-  }
-  __syncthreads();
-  for (int i = tid; i < gl * D4; i += kThreads) {
-    const int hl = i / D4, d = (i % D4) * 4;
-    const float *orow = p.o_part + (row0 + (int64_t)hl * p.S) * D + d;
-    const float *w = wt + hl * ns;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    int si = 0;
-    for (; si + 4 <= ns; si += 4) {
-      float4 ov[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) ov[j] = ld_cg_f4(orow + (int64_t)(si + j) * D);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float wj = w[si + j];
-        acc.x += wj * ov[j].x;
-        acc.y += wj * ov[j].y;
-        acc.z += wj * ov[j].z;
-        acc.w += wj * ov[j].w;
-      }
-    }
-    for (; si < ns; ++si) {
-      const float4 ov = ld_cg_f4(orow + (int64_t)si * D);
-      const float wj = w[si];
-      acc.x += wj * ov.x;
-      acc.y += wj * ov.y;
-      acc.z += wj * ov.z;
-      acc.w += wj * ov.w;
-    }
-    uint2 packed;
-    packed.x = pack_bf16x2(acc.x, acc.y);
-    packed.y = pack_bf16x2(acc.z, acc.w);
-    *reinterpret_cast<uint2 *>(p.out + b * p.o_sb + (int64_t)(h0 + hl) * p.o_sh + d) = packed;
-  }
+  if (claim_last_partition(p, b, kvh, ht, ns, flag))
+    merge_partials<D, kThreads>(p, b, h0, gl, ns, reinterpret_cast<float *>(smem));  // the ring is free
 }
 
 int partition_stages(int D, int hpt) { return stages_for(D, hpt); }
