@@ -83,10 +83,12 @@ typedef struct pad_plan {
   int32_t partition_tokens;  /* P, tokens per partition, a multiple of block_size */
   int32_t heads_per_tile;    /* query heads per work unit, padded (8, 16 or 32) */
   int32_t head_tiles;        /* work units per (sequence, KV head, partition): ceil(group / heads_per_tile) */
-  int32_t warps_per_cta;     /* warps per CTA (each loads and computes) */
+  int32_t warps_per_cta;     /* warps per CTA: 4 (mma.sync kernel), 6 (tcgen05 kernel: 4 softmax,
+                                producer, MMA) */
   int32_t stage_tokens;      /* tokens per shared-memory pipeline stage */
   int32_t stages;            /* pipeline depth */
-  int32_t ctas;              /* CTAs launched: one per unit, B * Hkv * head_tiles * num_splits */
+  int32_t ctas;              /* CTAs launched: one per unit (B * Hkv * head_tiles * num_splits), or
+                                for the persistent tcgen05 kernel min(units, SM count) */
   int32_t reduce;            /* 1 when partitions may need merging (S > 1) */
   int64_t workspace_bytes;   /* partial-output scratch (0 when S == 1) */
   int64_t control_bytes;     /* merge counters, 0 when S == 1 (library-owned except
@@ -186,6 +188,22 @@ pad_status pad_decode_static_scratch(const pad_tensor *q, const pad_tensor *k_ca
                                      const pad_tensor *v_cache, const pad_tensor *block_tables,
                                      const pad_tensor *seq_lens, float scale, int32_t num_splits,
                                      pad_tensor *out, pad_tensor *lse, void *stream);
+
+/*
+ * pad_decode_tcgen05 -- pad_decode computed by the 5th-generation tensor-core
+ * kernel: S^T = K.Q^T and O^T += V^T.P^T as tcgen05.mma with the accumulators in
+ * tensor memory, K/V/q streamed by TMA in 8-token boxes, the softmax in four warps
+ * that own one token (one TMEM lane) each, one persistent CTA per SM walking the
+ * (sequence, KV head, partition) units.  Same arguments, results, scratch and
+ * errors as pad_decode.  It takes groups of 17..32 query heads per KV head at
+ * head_dim 128 with block_size >= 8 and returns PAD_ERR_UNSUPPORTED otherwise.
+ * pad_decode does not call it: on the workloads measured on B200 the mma.sync
+ * kernel behind pad_decode is faster (its chunk pipeline waits on page-copy
+ * latency with two 64 KB chunks in flight).
+ */
+pad_status pad_decode_tcgen05(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
+                              const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
+                              int32_t num_splits, pad_tensor *out, pad_tensor *lse, void *stream);
 
 /*
  * pad_decode_plan -- the launch geometry pad_decode would use for this shape

@@ -70,6 +70,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pad_decode.restype = ctypes.c_int
     lib.pad_decode_static_scratch.argtypes = lib.pad_decode.argtypes
     lib.pad_decode_static_scratch.restype = ctypes.c_int
+    lib.pad_decode_tcgen05.argtypes = lib.pad_decode.argtypes
+    lib.pad_decode_tcgen05.restype = ctypes.c_int
     lib.pad_decode_with_workspace.argtypes = [P, P, P, P, P, ctypes.c_float, ctypes.c_int32, P, P, ctypes.c_void_p,
                                               ctypes.c_size_t, ctypes.c_void_p]
     lib.pad_decode_with_workspace.restype = ctypes.c_int
@@ -191,6 +193,30 @@ def pad_decode_static_scratch(q, k_cache, v_cache, block_tables, seq_lens, scale
     return out, lse
 
 
+def pad_decode_tcgen05(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits=0, out=None, lse=None,
+                       stream=None):
+    """pad_decode on the 5th-generation tensor-core kernel (see
+    ``pad_decode_tcgen05`` in include/pad.h): groups of 17..32 query heads per KV
+    head at head_dim 128, block_size >= 8.  Returns (out, lse)."""
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("q must be a CUDA tensor")
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    if lse is True:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+    elif lse is False:
+        lse = None
+    descs = [describe(t) for t in (q, k_cache, v_cache, block_tables, seq_lens, out)]
+    dlse = describe(lse) if lse is not None else None
+    with torch.cuda.device(dev):
+        st = load_library().pad_decode_tcgen05(
+            *(ctypes.byref(d) for d in descs[:5]), float(scale), int(num_splits), ctypes.byref(descs[5]),
+            ctypes.byref(dlse) if dlse is not None else None, _stream_handle(stream, dev))
+    _raise(st)
+    return out, lse
+
+
 def pad_decode_with_workspace(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, workspace,
                               stream=None) -> None:
     """pad_decode with caller-owned partials scratch (see include/pad.h):
@@ -240,7 +266,7 @@ def pad_release_workspace(device: int = -1) -> None:
     _raise(load_library().pad_release_workspace(device))
 
 
-__all__ = ["pad_decode", "pad_decode_with_workspace", "pad_decode_static_scratch", "pad_decode_plan",
+__all__ = ["pad_decode", "pad_decode_with_workspace", "pad_decode_static_scratch", "pad_decode_tcgen05", "pad_decode_plan",
            "pad_check_device_errors", "pad_release_workspace",
            "pad_status_string", "pad_last_error", "pad_abi_version", "describe", "load_library",
            "PadError", "PadTensor", "PadPlan"]

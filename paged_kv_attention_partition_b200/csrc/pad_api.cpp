@@ -86,14 +86,17 @@ int sm_count(int device) {
 
 // Per-shape launch plan.  The lengths live on the device, so the plan sees only
 // the table capacity C = W * bs.  Partitions are whole pages.  With num_splits==0
-// the partition starts at 256 tokens (or 16 g, if larger: the split scratch a
-// partition writes, g * D * 4 bytes, stays under 1/16 of the K/V bytes it
-// streams, 4 * D * P) and is halved, down to max(64, 16 g), while the batch would
-// give fewer than two waves of CTAs on this device: many small units keep every
-// SM busy and bound the tail of a ragged batch, and the fused reduce reads the
-// partials back from L2.  At most kMaxSplits partitions per sequence.  One CTA
-// per unit; units past a sequence's length exit at once.
-void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan) {
+// the partition starts at max(512, 64 g) tokens, rounded up to a power of two
+// (a unit's fixed cost -- start, merge of the four warps, partial and count --
+// grows with the head group, so larger groups get longer partitions), and is
+// halved, down to max(64, 16 g) (the split scratch a partition writes, g * D *
+// 4 bytes, stays under 1/16 of the K/V bytes it streams, 4 * D * P), while the
+// batch would give fewer than two waves of CTAs on this device: a small batch
+// still fills every SM.  Measured on B200 this picks the best of 64..8192-token
+// partitions for the llama8b (512) and ragged_mqa (2048) batches.  At most
+// kMaxSplits partitions per sequence.  One CTA per unit; units past a
+// sequence's length exit at once.
+void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan, bool tcgen05 = false) {
   const int64_t C = s.W * s.bs;
   int hpt = s.g <= 8 ? 8 : (s.g <= 16 ? 16 : 32);
   if (hpt > pad::max_heads_per_tile((int)s.D)) hpt = pad::max_heads_per_tile((int)s.D);
@@ -103,7 +106,8 @@ void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan) {
     P = round_up((C + num_splits - 1) / num_splits, s.bs);
   } else {
     const int64_t p_floor = round_up(16 * s.g > 64 ? 16 * s.g : 64, 64);
-    P = p_floor > 256 ? p_floor : 256;
+    P = 512;
+    while (P < 64 * s.g) P *= 2;
     const int64_t slots = (int64_t)sm_count(device < 0 ? 0 : device) *
                           pad::ctas_per_sm_for((int)s.D, hpt);
     const int64_t pairs = s.B * s.Hkv * HT;
@@ -119,11 +123,13 @@ void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan) {
   plan->partition_tokens = (int32_t)P;
   plan->heads_per_tile = hpt;
   plan->head_tiles = (int32_t)HT;
-  const bool umma = pad::umma_eligible((int)s.D, hpt, (int)s.bs);
+  const bool umma = tcgen05 && pad::umma_eligible((int)s.D, hpt, (int)s.bs);
   plan->warps_per_cta = umma ? pad::kUmmaWarps : pad::kWarps;
   plan->stage_tokens = umma ? pad::kUmmaStageTokens : pad::stage_tokens_for((int)s.D, hpt);
   plan->stages = umma ? pad::umma_stages() : pad::partition_stages((int)s.D, hpt);
-  plan->ctas = (int32_t)(units > 0x7fffffffll ? 0x7fffffffll : units);
+  // one CTA per unit; the tcgen05 kernel is persistent: one CTA per SM walks the units
+  const int64_t sms = sm_count(device < 0 ? 0 : device);
+  plan->ctas = (int32_t)(umma ? (units < sms ? units : sms) : (units > 0x7fffffffll ? 0x7fffffffll : units));
   plan->reduce = S > 1 ? 1 : 0;
   plan->workspace_bytes = (int64_t)pad::workspace_layout(s.B, s.Hq, S, s.D).total;
   plan->control_bytes = (int64_t)pad::control_layout(s.B, s.Hkv, HT, S).total;
@@ -305,7 +311,8 @@ struct Prepared {
 
 pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
                    const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale, int32_t num_splits,
-                   const pad_tensor *out, const pad_tensor *lse, Prepared *pr, bool *empty) {
+                   const pad_tensor *out, const pad_tensor *lse, Prepared *pr, bool *empty,
+                   bool tcgen05 = false) {
   pad_status st;
   *empty = false;
   if ((st = check_tensor(q, "q", PAD_BF16, 3)) != PAD_OK) return st;
@@ -362,7 +369,12 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
   if ((st = check_device_ptr(out->data, device, "out")) != PAD_OK) return st;
   if (lse != nullptr && (st = check_device_ptr(lse->data, device, "lse")) != PAD_OK) return st;
 
-  make_plan(s, num_splits, device, &pr->plan);
+  if (tcgen05 && !pad::umma_eligible((int)D, s.g <= 8 ? 8 : (s.g <= 16 ? 16 : 32), (int)bs))
+    return fail(PAD_ERR_UNSUPPORTED,
+                "the tcgen05 kernel takes groups of 17..32 query heads per KV head at head_dim 128 with a block "
+                "size of at least 8 (got group %lld, head_dim %lld, block size %lld)",
+                (long long)s.g, (long long)D, (long long)bs);
+  make_plan(s, num_splits, device, &pr->plan, tcgen05);
   const int64_t units = B * Hkv * pr->plan.head_tiles * (int64_t)pr->plan.num_splits;
   if (units > 0x7fffffffll) return fail(PAD_ERR_UNSUPPORTED, "too many work units (%lld) for one launch", (long long)units);
   pr->ws = pad::workspace_layout(B, Hq, pr->plan.num_splits, D);
@@ -373,7 +385,7 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
 
   pad::PartitionParams &p = pr->p;
   p = pad::PartitionParams{};
-  pr->umma = pad::umma_eligible((int)D, pr->plan.heads_per_tile, (int)bs);
+  pr->umma = tcgen05;
   const int rows = pr->umma ? 8 : pad::box_rows((int)bs, (int)D, pr->plan.heads_per_tile);
   if ((st = encode_cache_map(&p.tmk, k_cache, rows, "k_cache")) != PAD_OK) return st;
   if ((st = encode_cache_map(&p.tmv, v_cache, rows, "v_cache")) != PAD_OK) return st;
@@ -512,6 +524,21 @@ pad_status pad_decode(const pad_tensor *q, const pad_tensor *k_cache, const pad_
   Prepared pr;
   bool empty = false;
   pad_status st = prepare(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, &pr, &empty);
+  if (st != PAD_OK || empty) return st;
+  void *ws = nullptr, *ctl = nullptr;
+  if (pr.ws.total > 0 && (st = get_buffer(g_ws, pr.device, stream, pr.ws.total, &ws)) != PAD_OK) return st;
+  if (pr.cl.total > 0 && (st = get_buffer(g_ctl, pr.device, stream, pr.cl.total, &ctl)) != PAD_OK) return st;
+  bind_buffers(pr, ws, ctl);
+  return run(pr, stream);
+}
+
+pad_status pad_decode_tcgen05(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
+                              const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
+                              int32_t num_splits, pad_tensor *out, pad_tensor *lse, void *stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  Prepared pr;
+  bool empty = false;
+  pad_status st = prepare(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, &pr, &empty, true);
   if (st != PAD_OK || empty) return st;
   void *ws = nullptr, *ctl = nullptr;
   if (pr.ws.total > 0 && (st = get_buffer(g_ws, pr.device, stream, pr.ws.total, &ws)) != PAD_OK) return st;

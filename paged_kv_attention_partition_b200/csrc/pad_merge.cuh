@@ -17,13 +17,24 @@
 
 namespace pad {
 
-// Counts this partition; true (in every thread) for the CTA that completes
-// the set, which also resets the counter for the next launch.  The barrier
-// orders every thread's partial stores before thread 0's fence, which publishes
-// them (cumulatively) before the count.  Every thread of the CTA calls it.
+// Barriers over the threads that take part: the whole CTA, or the 128 threads
+// of warps 0-3 (named barrier 1) while other warps of the CTA run on.
+struct CtaSync {
+  __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
+struct Warps0to3Sync {
+  __device__ __forceinline__ void operator()() const { asm volatile("bar.sync 1, 128;\n" ::: "memory"); }
+};
+
+// Counts this partition; true (in every participating thread) for the CTA that
+// completes the set, which also resets the counter for the next launch.  The
+// barrier orders every participant's partial stores before thread 0's fence,
+// which publishes them (cumulatively) before the count.  Every participating
+// thread calls it; thread 0 must be one of them.
+template <class Sync = CtaSync>
 __device__ __forceinline__ bool claim_last_partition(const PartitionParams &p, int b, int kvh, int ht, int ns,
-                                                     int *flag) {
-  __syncthreads();
+                                                     int *flag, Sync sync = Sync()) {
+  sync();
   if (threadIdx.x == 0) {
     const uint32_t pair = ((uint32_t)b * p.Hkv + kvh) * p.HT + ht;
     __threadfence();
@@ -35,15 +46,17 @@ __device__ __forceinline__ bool claim_last_partition(const PartitionParams &p, i
     }
     *flag = last;
   }
-  __syncthreads();
-  return *flag != 0;
+  sync();
+  const bool last = *flag != 0;
+  sync();  // every participant has read the flag before it is written again
+  return last;
 }
 
 // Merges the ns partials of query heads h0 .. h0+gl-1 of sequence b into bf16
-// out (+ lse).  `wt` is shared memory for gl * ns floats.  Every thread of the
-// CTA (NTHREADS of them) calls it.
-template <int D, int NTHREADS>
-__device__ void merge_partials(const PartitionParams &p, int b, int h0, int gl, int ns, float *wt) {
+// out (+ lse).  `wt` is shared memory for gl * ns floats.  The NTHREADS
+// participating threads (threadIdx.x 0 .. NTHREADS-1) call it.
+template <int D, int NTHREADS, class Sync = CtaSync>
+__device__ void merge_partials(const PartitionParams &p, int b, int h0, int gl, int ns, float *wt, Sync sync = Sync()) {
   constexpr int D4 = D / 4, NW = NTHREADS / 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t row0 = ((int64_t)b * p.Hq + h0) * p.S;
@@ -51,7 +64,7 @@ __device__ void merge_partials(const PartitionParams &p, int b, int h0, int gl, 
     const int hl = i / ns, si = i % ns;
     wt[hl * ns + si] = ld_cg_f32(p.lse_part + row0 + (int64_t)hl * p.S + si);
   }
-  __syncthreads();
+  sync();
   for (int hl = warp; hl < gl; hl += NW) {
     float M = -INFINITY;
     for (int si = lane; si < ns; si += 32) M = fmaxf(M, wt[hl * ns + si]);
@@ -66,7 +79,7 @@ __device__ void merge_partials(const PartitionParams &p, int b, int h0, int gl, 
     for (int si = lane; si < ns; si += 32) wt[hl * ns + si] = __expf(wt[hl * ns + si] - M) * inv;
     if (lane == 0 && p.lse != nullptr) p.lse[b * p.lse_sb + (int64_t)(h0 + hl) * p.lse_sh] = M + logf(sum);
   }
-  __syncthreads();
+  sync();
   for (int i = tid; i < gl * D4; i += NTHREADS) {
     const int hl = i / D4, d = (i % D4) * 4;
     const float *orow = p.o_part + (row0 + (int64_t)hl * p.S) * D + d;
@@ -99,6 +112,7 @@ __device__ void merge_partials(const PartitionParams &p, int b, int h0, int gl, 
     packed.y = pack_bf16x2(acc.z, acc.w);
     *reinterpret_cast<uint2 *>(p.out + b * p.o_sb + (int64_t)(h0 + hl) * p.o_sh + d) = packed;
   }
+  sync();  // `wt` is free again when the call returns
 }
 
 }  // namespace pad

@@ -26,9 +26,10 @@
 //                   swizzle) as the B operand of the PV product.  At the end
 //                   thread i owns head_dim row i of O^T.
 //
-// The chunk sequence is strictly ordered: QK(c) is issued after PV(c-1), so
-// the commit that signals S(c) also guarantees PV(c-1) finished -- the softmax
-// may then rescale O^T in TMEM and overwrite the single P^T buffer.
+// S^T and P^T are double buffered: the MMA thread issues QK(c+1) as soon as
+// chunk c+1 has landed, so the softmax warps find the next scores ready, and
+// PV(c) runs while the softmax works on chunk c+1.  A rescale of O^T waits for
+// PV(c-1); a P^T buffer is rewritten once PV(c-2) has read it.
 //
 // Output and split handling are those of partition_kernel: one non-empty
 // partition writes bf16 out (+ lse), otherwise fp32 partials and the last CTA of
@@ -56,7 +57,7 @@ constexpr int kBoxRows = 8;                      // tokens per TMA box
 constexpr uint32_t kBoxBytes = kBoxRows * kD * 2;          // 2 KB
 constexpr uint32_t kHalfBytes = kChunk * kD * 2;           // K (or V) of a chunk: 32 KB
 constexpr uint32_t kQBytes = kHeads * kD * 2;              // 8 KB
-constexpr uint32_t kPBytes = kChunk * 128;                 // P^T: 128 rows of 128 B
+constexpr uint32_t kPBytes = kChunk * 128;                 // one P^T buffer: 128 rows of 128 B
 constexpr int kSoftmaxWarps = 4;
 constexpr int kProducerWarp = 4, kMmaWarp = 5;
 constexpr int kUmmaThreads = 6 * 32;
@@ -193,62 +194,55 @@ __device__ __forceinline__ float warp_sum_scatter(float (&v)[32], int lane) {
 
 }  // namespace
 
-// Shared memory (1024-byte aligned base): Q 8 KB | K/V ring NST x (K 32 KB,
-// V 32 KB) | P^T 16 KB | reductions 1 KB | barriers and words.
+// One queued work unit.  nch > 0: chunks to stream; 0: an empty sequence (the
+// unit writes out = 0, lse = -inf); -1: no more units.
+struct UnitDesc {
+  int32_t b, kvh, ht, s, t0, t1, ns, nch;
+};
+constexpr int kQueue = 4;
+
+// Shared memory (1024-byte aligned base): q 2 x 8 KB | K/V ring NST x (K 32 KB,
+// V 32 KB) | P^T 2 x 16 KB | merge weights 32 KB | reductions 1 KB | queue,
+// barriers and words.  TMEM: S^T in two 32-column buffers, O^T after them.
 template <int NST>
 struct UmmaSmem {
   static constexpr uint32_t q = 0;
-  static constexpr uint32_t ring = kQBytes;
+  static constexpr uint32_t ring = 2 * kQBytes;
   static constexpr uint32_t pt = ring + NST * 2 * kHalfBytes;
-  static constexpr uint32_t red = pt + kPBytes;
-  static constexpr uint32_t bars = red + 1024;
-  static constexpr uint32_t total = bars + 256 + 1024 /* alignment slack */;
+  static constexpr uint32_t mw = pt + 2 * kPBytes;
+  static constexpr uint32_t red = mw + kHeads * kMaxSplits * 4;
+  static constexpr uint32_t queue = red + 1024;
+  static constexpr uint32_t bars = queue + kQueue * sizeof(UnitDesc);
+  static constexpr uint32_t total = bars + 512 + 1024 /* alignment slack */;
 };
 
+// Persistent: one CTA per SM walks the units blockIdx.x, blockIdx.x + G, ...
+// The producer warp finds the non-empty ones 32 at a time and queues them; the
+// MMA thread and the softmax warps consume the queue.  Chunk buffers, q
+// buffers, TMEM and barrier phases carry over from unit to unit, so the next
+// unit's copies stream while the current one finishes.
 template <int NST>
 __global__ void __launch_bounds__(kUmmaThreads, 1) umma_kernel(const __grid_constant__ PartitionParams p) {
   using SM = UmmaSmem<NST>;
+  static_assert(SM::total <= (uint32_t)kSmemBudget, "shared-memory plan over budget");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::bars);
-  // barriers: kv_full[NST] kv_empty[NST] q_full s_full p_full o_done mma_idle
+  UnitDesc *queue = reinterpret_cast<UnitDesc *>(smem + SM::queue);
+  // barriers: chunk ring, q buffers, S^T and P^T buffers (x2), O^T, unit queue
   const uint32_t kv_full0 = smem_addr(bars), kv_empty0 = smem_addr(bars + NST);
-  const uint32_t q_full = smem_addr(bars + 2 * NST), s_full = smem_addr(bars + 2 * NST + 1);
-  const uint32_t p_full = smem_addr(bars + 2 * NST + 2), o_done = smem_addr(bars + 2 * NST + 3);
-  const uint32_t mma_idle = smem_addr(bars + 2 * NST + 4);
-  uint32_t *words = reinterpret_cast<uint32_t *>(bars + 2 * NST + 8);  // [0] tmem base, [1] merge flag
+  const uint32_t q_full0 = smem_addr(bars + 2 * NST), q_empty0 = smem_addr(bars + 2 * NST + 2);
+  const uint32_t s_full0 = smem_addr(bars + 2 * NST + 4), s_free0 = smem_addr(bars + 2 * NST + 6);
+  const uint32_t p_full0 = smem_addr(bars + 2 * NST + 8), p_free0 = smem_addr(bars + 2 * NST + 10);
+  const uint32_t o_done = smem_addr(bars + 2 * NST + 12), o_free = smem_addr(bars + 2 * NST + 13);
+  const uint32_t uq_full0 = smem_addr(bars + 2 * NST + 14), uq_empty0 = smem_addr(bars + 2 * NST + 14 + kQueue);
+  const uint32_t mma_idle = smem_addr(bars + 2 * NST + 14 + 2 * kQueue);
+  uint32_t *words = reinterpret_cast<uint32_t *>(bars + 2 * NST + 15 + 2 * kQueue);  // [0] tmem, [1] flag
   volatile int *abort_flag = reinterpret_cast<volatile int *>(words + 2);
-  float *red = reinterpret_cast<float *>(smem + SM::red);  // [4][32] per-warp per-head values
+  float *red = reinterpret_cast<float *>(smem + SM::red);  // [4][32]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint32_t u = blockIdx.x;
-  const int s = (int)(u % (uint32_t)p.S);
-  u /= (uint32_t)p.S;
-  const int ht = (int)(u % (uint32_t)p.HT);
-  u /= (uint32_t)p.HT;
-  const int kvh = (int)(u % (uint32_t)p.Hkv);
-  const int b = (int)(u / (uint32_t)p.Hkv);
-  const int h0 = kvh * p.g + ht * kHeads;
-  const int gl = min(kHeads, p.g - ht * kHeads);
   const int capacity = p.max_blocks << p.bs_log2;
-  const int t0 = s * p.P;
-
-  int L = __ldg(p.seq_lens + b);
-  if (L < 0 || L > capacity) {
-    if (tid == 0 && s == 0 && kvh == 0 && ht == 0) atomicOr(p.err, kErrSeqLen);
-    L = L < 0 ? 0 : capacity;
-  }
-  const int t1 = min(t0 + p.P, L);
-  if (t0 >= t1) {
-    if (L == 0 && s == 0) {  // empty sequence: out = 0, lse = -inf
-      for (int i = tid; i < gl * kD; i += kUmmaThreads)
-        p.out[b * p.o_sb + (int64_t)(h0 + i / kD) * p.o_sh + (i % kD)] = 0;
-      if (p.lse != nullptr && tid < gl) p.lse[b * p.lse_sb + (int64_t)(h0 + tid) * p.lse_sh] = -INFINITY;
-    }
-    return;
-  }
-  const int ns = (L + p.P - 1) / p.P;
-  const int nchunks = (t1 - t0 + kChunk - 1) / kChunk;
 
   if (tid == 0) {
 #pragma unroll
@@ -256,222 +250,358 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_kernel(const __grid_cons
       mbar_init(kv_full0 + 8 * i, 1);
       mbar_init(kv_empty0 + 8 * i, 1);
     }
-    mbar_init(q_full, 1);
-    mbar_init(s_full, 1);
-    mbar_init(p_full, kSoftmaxWarps * 32);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(q_full0 + 8 * i, 1);
+      mbar_init(q_empty0 + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full0 + 8 * i, 1);                     // QK commit
+      mbar_init(s_free0 + 8 * i, kSoftmaxWarps * 32);    // every softmax thread has read S^T
+      mbar_init(p_full0 + 8 * i, kSoftmaxWarps * 32);    // every softmax thread has written its P^T row
+      mbar_init(p_free0 + 8 * i, 1);                     // PV commit
+    }
     mbar_init(o_done, 1);
+    mbar_init(o_free, kSoftmaxWarps * 32);
+    for (int i = 0; i < kQueue; ++i) {
+      mbar_init(uq_full0 + 8 * i, 1);
+      mbar_init(uq_empty0 + 8 * i, 1 + kSoftmaxWarps * 32);  // the MMA thread and every softmax thread
+    }
     mbar_init(mma_idle, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {  // 64 TMEM columns: S^T at +0, O^T at +32
-    tmem_alloc(smem_addr(words), 64);
+  if (warp == 0) {  // 128 TMEM columns: S^T buffers at +0 and +32, O^T at +64
+    tmem_alloc(smem_addr(words), 128);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = words[0];
-  const uint32_t tmem_s = tmem, tmem_o = tmem + 32;
+  const uint32_t tmem_o = tmem + 64;
 
   if (warp == kProducerWarp) {
-    // ---------------- TMA producer ----------------
-    const int32_t *trow = p.tables + (int64_t)b * p.table_stride;
-    if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, kQBytes);
-      tma_load_4d(smem_addr(smem + SM::q), &p.tmq, 0, h0, 0, b, q_full);
-    }
-    // lane j < 16 copies box j (tokens tb + 8j .. +7) of K and of V
-    int issued = 0;
-    for (int c = 0; c < nchunks; ++c) {
-      const int slot = c % NST;
-      if (c >= NST && !wait_bounded(kv_empty0 + 8 * slot, ((c / NST) - 1) & 1, p.err, abort_flag)) break;
-      const int tb = t0 + c * kChunk;
-      const int nbox = min(kChunk / kBoxRows, (t1 - tb + kBoxRows - 1) / kBoxRows);
-      const int tok = tb + kBoxRows * lane;
-      int id = 0;
-      if (lane < nbox) id = __ldg(trow + (tok >> p.bs_log2));
-      if (lane == 0) mbar_arrive_expect_tx(kv_full0 + 8 * slot, (uint32_t)nbox * kBoxBytes * 2);
-      __syncwarp();
-      if (lane < nbox) {
-        if ((unsigned)id >= (unsigned)p.num_blocks) atomicOr(p.err, kErrBlockId);  // reads as zeros
-        const int slot0 = tok & ((1 << p.bs_log2) - 1);
-        uint8_t *kdst = smem + SM::ring + slot * 2 * kHalfBytes + lane * kBoxBytes;
-        tma_load_5d(smem_addr(kdst), &p.tmk, 0, slot0, 0, kvh, id, kv_full0 + 8 * slot);
-        tma_load_5d(smem_addr(kdst + kHalfBytes), &p.tmv, 0, slot0, 0, kvh, id, kv_full0 + 8 * slot);
+    // ---------------- scheduler + TMA producer ----------------
+    const uint32_t G = gridDim.x;
+    int k = 0;      // units queued
+    int j = 0;      // units with chunks (q buffer use)
+    int g = 0;      // chunks issued
+    bool ok = true;
+    auto push = [&](const UnitDesc &d) -> bool {
+      const int qs = k % kQueue;
+      if (k >= kQueue && !wait_bounded(uq_empty0 + 8 * qs, ((k / kQueue) - 1) & 1, p.err, abort_flag)) return false;
+      if (lane == 0) {
+        queue[qs] = d;
+        mbar_arrive1(uq_full0 + 8 * qs);  // releases the entry
       }
-      issued = c + 1;
+      __syncwarp();
+      ++k;
+      return true;
+    };
+    for (uint32_t base = blockIdx.x; ok && base < p.n_units; base += 32 * G) {
+      // lane l looks at unit base + l G
+      const uint32_t uu = base + (uint32_t)lane * G;
+      UnitDesc d{};
+      bool live = false;
+      if (uu < p.n_units) {
+        uint32_t u = uu;
+        d.s = (int)(u % (uint32_t)p.S);
+        u /= (uint32_t)p.S;
+        d.ht = (int)(u % (uint32_t)p.HT);
+        u /= (uint32_t)p.HT;
+        d.kvh = (int)(u % (uint32_t)p.Hkv);
+        d.b = (int)(u / (uint32_t)p.Hkv);
+        int L = __ldg(p.seq_lens + d.b);
+        if (L < 0 || L > capacity) {
+          if (d.s == 0 && d.kvh == 0 && d.ht == 0) atomicOr(p.err, kErrSeqLen);
+          L = L < 0 ? 0 : capacity;
+        }
+        d.t0 = d.s * p.P;
+        d.t1 = min(d.t0 + p.P, L);
+        d.ns = (L + p.P - 1) / p.P;
+        d.nch = d.t0 < d.t1 ? (d.t1 - d.t0 + kChunk - 1) / kChunk : 0;
+        live = d.t0 < d.t1 || (L == 0 && d.s == 0);
+      }
+      uint32_t mask = __ballot_sync(0xffffffffu, live);
+      while (ok && mask) {
+        const int src = __ffs(mask) - 1;
+        mask &= mask - 1;
+        UnitDesc e;
+        e.b = __shfl_sync(0xffffffffu, d.b, src);
+        e.kvh = __shfl_sync(0xffffffffu, d.kvh, src);
+        e.ht = __shfl_sync(0xffffffffu, d.ht, src);
+        e.s = __shfl_sync(0xffffffffu, d.s, src);
+        e.t0 = __shfl_sync(0xffffffffu, d.t0, src);
+        e.t1 = __shfl_sync(0xffffffffu, d.t1, src);
+        e.ns = __shfl_sync(0xffffffffu, d.ns, src);
+        e.nch = __shfl_sync(0xffffffffu, d.nch, src);
+        if (!push(e)) {
+          ok = false;
+          break;
+        }
+        if (e.nch == 0) continue;
+        // q rows of the tile -> q buffer j % 2
+        const int h0 = e.kvh * p.g + e.ht * kHeads;
+        const int qs = j % 2;
+        if (j >= 2 && !wait_bounded(q_empty0 + 8 * qs, ((j / 2) - 1) & 1, p.err, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(q_full0 + 8 * qs, kQBytes);
+          tma_load_4d(smem_addr(smem + SM::q + qs * kQBytes), &p.tmq, 0, h0, 0, e.b, q_full0 + 8 * qs);
+        }
+        ++j;
+        // the unit's chunks: lane l < 16 copies box l (tokens tb + 8l .. +7) of K and of V
+        const int32_t *trow = p.tables + (int64_t)e.b * p.table_stride;
+        for (int c = 0; c < e.nch; ++c, ++g) {
+          const int slot = g % NST;
+          const int tb = e.t0 + c * kChunk;
+          const int nbox = min(kChunk / kBoxRows, (e.t1 - tb + kBoxRows - 1) / kBoxRows);
+          const int tok = tb + kBoxRows * lane;
+          const int id = lane < nbox ? __ldg(trow + (tok >> p.bs_log2)) : 0;
+          if (g >= NST && !wait_bounded(kv_empty0 + 8 * slot, ((g / NST) - 1) & 1, p.err, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) mbar_arrive_expect_tx(kv_full0 + 8 * slot, (uint32_t)nbox * kBoxBytes * 2);
+          __syncwarp();
+          if (lane < nbox) {
+            if ((unsigned)id >= (unsigned)p.num_blocks) atomicOr(p.err, kErrBlockId);  // reads as zeros
+            const int slot0 = tok & ((1 << p.bs_log2) - 1);
+            uint8_t *kdst = smem + SM::ring + slot * 2 * kHalfBytes + lane * kBoxBytes;
+            tma_load_5d(smem_addr(kdst), &p.tmk, 0, slot0, 0, e.kvh, id, kv_full0 + 8 * slot);
+            tma_load_5d(smem_addr(kdst + kHalfBytes), &p.tmv, 0, slot0, 0, e.kvh, id, kv_full0 + 8 * slot);
+          }
+        }
+      }
     }
-    // leave no copy in flight if the pipeline was abandoned
-    if (*abort_flag && lane == 0)
-      for (int c = max(0, issued - NST); c < issued; ++c)
+    if (ok) {
+      UnitDesc t{};
+      t.nch = -1;
+      push(t);
+    }
+    if (*abort_flag && lane == 0) {
+      // leave no copy in flight: the last NST chunks and the last two q tiles
+      for (int c = max(0, g - NST); c < g; ++c)
         wait_bounded(kv_full0 + 8 * (c % NST), (c / NST) & 1, p.err, abort_flag, true);
+      for (int x = max(0, j - 2); x < j; ++x) wait_bounded(q_full0 + 8 * (x % 2), (x / 2) & 1, p.err, abort_flag, true);
+    }
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issue (one thread) ----------------
+    // Per unit: QK of the first chunk, then for every chunk c: QK(c+1) into the
+    // other S^T buffer as soon as its copies landed, and PV(c) once the softmax
+    // has written P^T(c).  g counts chunks over all units (buffer = g % 2).
     if (lane == 0) {
       constexpr uint32_t IQK = umma_idesc(false, false), IPV = umma_idesc(true, true);
-      const uint32_t qb = smem_addr(smem + SM::q), pb = smem_addr(smem + SM::pt);
-      auto qk = [&](int c) {
-        const uint32_t kb = smem_addr(smem + SM::ring + (c % NST) * 2 * kHalfBytes);
+      int k = 0, j = 0, g = 0;
+      bool ok = true;
+      auto qk = [&](int gc, int qs) -> bool {
+        if (!wait_bounded(kv_full0 + 8 * (gc % NST), (gc / NST) & 1, p.err, abort_flag)) return false;
+        if (gc >= 2 && !wait_bounded(s_free0 + 8 * (gc & 1), ((gc >> 1) - 1) & 1, p.err, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t kb = smem_addr(smem + SM::ring + (gc % NST) * 2 * kHalfBytes);
+        const uint32_t qb = smem_addr(smem + SM::q + qs * kQBytes);
+        const uint32_t sd = tmem + (uint32_t)(gc & 1) * 32;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           // K: rows of 128 B in 8-row groups 2 KB apart, column block kk/4 at +1 KB
           const uint64_t a = smem_desc(kb + (kk >> 2) * 1024 + (kk & 3) * 32, 16, 2 * 1024);
           // Q: 32 heads x 128 B per column block (4 KB), 8-head groups 1 KB apart
           const uint64_t bq = smem_desc(qb + (kk >> 2) * 4096 + (kk & 3) * 32, 16, 1024);
-          umma_bf16(tmem_s, a, bq, IQK, kk > 0);
+          umma_bf16(sd, a, bq, IQK, kk > 0);
         }
+        umma_commit(s_full0 + 8 * (gc & 1));
+        return true;
       };
-      auto pv = [&](int c) {
-        const uint32_t vb = smem_addr(smem + SM::ring + (c % NST) * 2 * kHalfBytes + kHalfBytes);
+      auto pv = [&](int gc, bool first) -> bool {
+        if (!wait_bounded(p_full0 + 8 * (gc & 1), (gc >> 1) & 1, p.err, abort_flag)) return false;
+        // before a unit's first PV product overwrites O^T, the previous unit's
+        // epilogue has read it
+        if (first && j > 0 && !wait_bounded(o_free, (j - 1) & 1, p.err, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t vb = smem_addr(smem + SM::ring + (gc % NST) * 2 * kHalfBytes + kHalfBytes);
+        const uint32_t pb = smem_addr(smem + SM::pt + (gc & 1) * kPBytes);
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk) {
           // V^T (MN-major): 64-d column blocks 1 KB apart, 8-token groups 2 KB apart
           const uint64_t a = smem_desc(vb + kk * 2 * kBoxBytes, 1024, 2 * 1024);
           // P^T (MN-major): token rows of 128 B, 8-token groups 1 KB apart
           const uint64_t bp = smem_desc(pb + kk * 2 * 1024, 1024, 1024);
-          umma_bf16(tmem_o, a, bp, IPV, c > 0 || kk > 0);
+          umma_bf16(tmem_o, a, bp, IPV, !first || kk > 0);
         }
+        umma_commit(kv_empty0 + 8 * (gc % NST));  // the chunk's K and V are consumed
+        umma_commit(p_free0 + 8 * (gc & 1));       // P^T buffer free; O^T holds chunks ..gc
+        return true;
       };
-      bool ok = wait_bounded(q_full, 0, p.err, abort_flag);
-      int c = 0;
-      for (; ok && c < nchunks; ++c) {
-        if (!wait_bounded(kv_full0 + 8 * (c % NST), (c / NST) & 1, p.err, abort_flag)) break;
-        if (c > 0) {
-          // the softmax of chunk c-1 has read S and written P^T
-          if (!wait_bounded(p_full, (c - 1) & 1, p.err, abort_flag)) break;
-          tc_fence_after();
-          pv(c - 1);
-          umma_commit(kv_empty0 + 8 * ((c - 1) % NST));
+      while (ok) {
+        const int qe = k % kQueue;
+        if (!wait_bounded(uq_full0 + 8 * qe, (k / kQueue) & 1, p.err, abort_flag)) break;
+        const int nch = queue[qe].nch;
+        mbar_arrive1(uq_empty0 + 8 * qe);
+        ++k;
+        if (nch < 0) break;
+        if (nch == 0) continue;
+        const int qs = j % 2;
+        if (!wait_bounded(q_full0 + 8 * qs, (j / 2) & 1, p.err, abort_flag) || !qk(g, qs)) break;
+        for (int c = 0; ok && c < nch; ++c) {
+          const int gc = g + c;
+          if (c + 1 < nch) ok = qk(gc + 1, qs);
+          if (ok && c + 1 == nch) umma_commit(q_empty0 + 8 * qs);  // the tile's last QK read of q
+          if (ok) ok = pv(gc, c == 0);
         }
-        qk(c);
-        umma_commit(s_full);
-      }
-      if (c == nchunks && wait_bounded(p_full, (nchunks - 1) & 1, p.err, abort_flag)) {
-        tc_fence_after();
-        pv(nchunks - 1);
-        umma_commit(kv_empty0 + 8 * ((nchunks - 1) % NST));
+        if (!ok) break;
         umma_commit(o_done);
+        g += nch;
+        ++j;
       }
       umma_commit(mma_idle);  // every MMA issued above has completed when this arrives
     }
   } else {
-    // ---------------- softmax warps: thread i = token i of the chunk ----------------
+    // ---------------- softmax warps: thread i = token i of a chunk, then head_dim row i ----------------
     const int i = tid;  // 0..127 == TMEM lane
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    float mr[32], lp[32];
-#pragma unroll
-    for (int h = 0; h < 32; ++h) {
-      mr[h] = -INFINITY;
-      lp[h] = 0.f;
-    }
-    uint8_t *pt = smem + SM::pt;
-    bool ok = true;
-    for (int c = 0; c < nchunks; ++c) {
-      const bool landed = wait_bounded(s_full, c & 1, p.err, abort_flag);
-      uint32_t raw[32];
-      if (landed) {
-        tc_fence_after();
-        tmem_ld32(tmem_s + lane_off, raw);
-        tmem_wait_ld();
+    int k = 0, j = 0, g = 0;
+    while (true) {
+      const int qe = k % kQueue;
+      const bool got = wait_bounded(uq_full0 + 8 * qe, (k / kQueue) & 1, p.err, abort_flag);
+      if (!softmax_bar_and(got)) break;
+      const UnitDesc e = queue[qe];
+      mbar_arrive1(uq_empty0 + 8 * qe);
+      ++k;
+      if (e.nch < 0) break;
+      const int h0 = e.kvh * p.g + e.ht * kHeads;
+      const int gl = min(kHeads, p.g - e.ht * kHeads);
+      if (e.nch == 0) {  // empty sequence: out = 0, lse = -inf
+        for (int x = i; x < gl * kD; x += kSoftmaxWarps * 32)
+          p.out[e.b * p.o_sb + (int64_t)(h0 + x / kD) * p.o_sh + (x % kD)] = 0;
+        if (p.lse != nullptr && i < gl) p.lse[e.b * p.lse_sb + (int64_t)(h0 + i) * p.lse_sh] = -INFINITY;
+        continue;
       }
-      const int tb = t0 + c * kChunk;
-      const bool live = landed && tb + i < t1;
-      float sc[32], cm[32];
-#pragma unroll
-      for (int h = 0; h < 32; ++h) {
-        sc[h] = live ? __uint_as_float(raw[h]) * p.scale_log2 : -INFINITY;
-        cm[h] = sc[h];
-      }
-      // per-head maximum over the chunk's 128 tokens (token 0 of the chunk is live)
-      red[warp * 32 + lane] = warp_max_scatter(cm, lane);
-      if (!softmax_bar_and(landed)) {  // one decision for all 128 threads
-        ok = false;
-        break;
-      }
-      const float mh = fmaxf(fmaxf(red[lane], red[32 + lane]), fmaxf(red[64 + lane], red[96 + lane]));  // head = lane
-      bool grow = false;
+      float mr[32], lp[32];
 #pragma unroll
       for (int h = 0; h < 32; ++h) {
-        cm[h] = __shfl_sync(0xffffffffu, mh, h);
-        grow |= cm[h] > mr[h] + kSlack;
+        mr[h] = -INFINITY;
+        lp[h] = 0.f;
       }
-      softmax_bar();  // every warp has read `red` before its next use
-      if (grow) {  // the same decision in every thread: the values are identical
-        float al[32];
+      bool ok = true;
+      for (int c = 0; c < e.nch; ++c, ++g) {
+        // warp-uniform: tcgen05.ld is a warp-collective instruction
+        const bool landed = __all_sync(0xffffffffu, wait_bounded(s_full0 + 8 * (g & 1), (g >> 1) & 1, p.err, abort_flag));
+        uint32_t raw[32];
+        if (landed) {
+          tc_fence_after();
+          tmem_ld32(tmem + (uint32_t)(g & 1) * 32 + lane_off, raw);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive1(s_free0 + 8 * (g & 1));  // the next-but-one QK may overwrite this buffer
+        }
+        const int tb = e.t0 + c * kChunk;
+        const bool live = landed && tb + i < e.t1;
+        float sc[32], cm[32];
 #pragma unroll
         for (int h = 0; h < 32; ++h) {
-          const float mn = fmaxf(mr[h], cm[h]);
-          al[h] = fast_exp2(mr[h] - mn);
-          mr[h] = mn;
-          lp[h] *= al[h];
+          sc[h] = live ? __uint_as_float(raw[h]) * p.scale_log2 : -INFINITY;
+          cm[h] = sc[h];
         }
-        if (c > 0) {  // row i of O^T holds chunks 0..c-1 (PV(c-1) completed before S(c) was signalled)
-          uint32_t o[32];
-          tmem_ld32(tmem_o + lane_off, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < 32; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * al[h]);
-          tmem_st32(tmem_o + lane_off, o);
-          tmem_wait_st();
+        // per-head maximum over the chunk's 128 tokens (token 0 of the chunk is live)
+        red[warp * 32 + lane] = warp_max_scatter(cm, lane);
+        if (!softmax_bar_and(landed)) {  // one decision for all 128 threads
+          ok = false;
+          break;
         }
-      }
-      // weights, the fp32 running sums, and the P^T row of token i
-      uint32_t pk[16];
+        const float mh = fmaxf(fmaxf(red[lane], red[32 + lane]), fmaxf(red[64 + lane], red[96 + lane]));  // head = lane
+        bool grow = false;
 #pragma unroll
-      for (int h = 0; h < 32; h += 2) {
-        const float e0 = fast_exp2(sc[h] - mr[h]), e1 = fast_exp2(sc[h + 1] - mr[h + 1]);
-        lp[h] += e0;
-        lp[h + 1] += e1;
-        pk[h / 2] = pack_bf16x2(e0, e1);
-      }
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4)
-        *reinterpret_cast<uint4 *>(pt + i * 128 + ((q4 ^ (i & 7)) << 4)) =
-            make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-      if (!live) {
-        // V row of a token past t1 (a slot past L_b or a box not copied): zeros,
-        // after the chunk's copies have landed
-        wait_bounded(kv_full0 + 8 * (c % NST), (c / NST) & 1, p.err, abort_flag);
-        uint8_t *vrow = smem + SM::ring + (c % NST) * 2 * kHalfBytes + kHalfBytes + (i >> 3) * kBoxBytes + (i & 7) * 128;
-#pragma unroll
-        for (int q8 = 0; q8 < 8; ++q8) {
-          *reinterpret_cast<uint4 *>(vrow + q8 * 16) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4 *>(vrow + 1024 + q8 * 16) = make_uint4(0, 0, 0, 0);
+        for (int h = 0; h < 32; ++h) {
+          cm[h] = __shfl_sync(0xffffffffu, mh, h);
+          grow |= cm[h] > mr[h] + kSlack;
         }
+        softmax_bar();  // every warp has read `red` before its next use
+        if (grow) {  // the same decision in every thread: the values are identical
+          float al[32];
+#pragma unroll
+          for (int h = 0; h < 32; ++h) {
+            const float mn = fmaxf(mr[h], cm[h]);
+            al[h] = fast_exp2(mr[h] - mn);
+            mr[h] = mn;
+            lp[h] *= al[h];
+          }
+          // row i of O^T holds chunks 0..c-1 once PV(c-1) has completed
+          if (c > 0 &&
+              __all_sync(0xffffffffu, wait_bounded(p_free0 + 8 * ((g - 1) & 1), ((g - 1) >> 1) & 1, p.err, abort_flag))) {
+            tc_fence_after();
+            uint32_t o[32];
+            tmem_ld32(tmem_o + lane_off, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < 32; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * al[h]);
+            tmem_st32(tmem_o + lane_off, o);
+            tmem_wait_st();
+          }
+        }
+        // weights, the fp32 running sums, and the P^T row of token i (into the
+        // buffer PV(g-2) has finished reading)
+        if (g >= 2) wait_bounded(p_free0 + 8 * (g & 1), ((g >> 1) - 1) & 1, p.err, abort_flag);
+        uint8_t *pt = smem + SM::pt + (g & 1) * kPBytes;
+        uint32_t pk[16];
+#pragma unroll
+        for (int h = 0; h < 32; h += 2) {
+          const float e0 = fast_exp2(sc[h] - mr[h]), e1 = fast_exp2(sc[h + 1] - mr[h + 1]);
+          lp[h] += e0;
+          lp[h + 1] += e1;
+          pk[h / 2] = pack_bf16x2(e0, e1);
+        }
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          *reinterpret_cast<uint4 *>(pt + i * 128 + ((q4 ^ (i & 7)) << 4)) =
+              make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        if (!live) {
+          // V row of a token past t1 (a slot past L_b or a box not copied):
+          // zeros, after the chunk's copies have landed
+          wait_bounded(kv_full0 + 8 * (g % NST), (g / NST) & 1, p.err, abort_flag);
+          uint8_t *vrow = smem + SM::ring + (g % NST) * 2 * kHalfBytes + kHalfBytes + (i >> 3) * kBoxBytes + (i & 7) * 128;
+#pragma unroll
+          for (int q8 = 0; q8 < 8; ++q8) {
+            *reinterpret_cast<uint4 *>(vrow + q8 * 16) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(vrow + 1024 + q8 * 16) = make_uint4(0, 0, 0, 0);
+          }
+        }
+        fence_proxy_async_smem();  // P^T and zeroed rows, before the tensor core reads them
+        tc_fence_before();
+        mbar_arrive1(p_full0 + 8 * (g & 1));
       }
-      fence_proxy_async_smem();  // P^T and zeroed rows, before the tensor core reads them
-      tc_fence_before();
-      mbar_arrive1(p_full);
-    }
+      if (!ok) break;
 
-    // ---- epilogue: thread i = head_dim row i of O^T
-    const bool out_ready = ok && wait_bounded(o_done, 0, p.err, abort_flag);
-    if (softmax_bar_and(out_ready)) {
+      // ---- the unit's output: thread i = head_dim row i of O^T
+      const bool out_ready = wait_bounded(o_done, j & 1, p.err, abort_flag);
+      if (!softmax_bar_and(out_ready)) break;
       tc_fence_after();
-      // per-head totals over the 128 token threads: lane h of each warp gets head h
       float tmp[32];
 #pragma unroll
       for (int h = 0; h < 32; ++h) tmp[h] = lp[h];
-      red[warp * 32 + lane] = warp_sum_scatter(tmp, lane);
+      red[warp * 32 + lane] = warp_sum_scatter(tmp, lane);  // per-head sums over the token threads
+      uint32_t o[32];
+      tmem_ld32(tmem_o + lane_off, o);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive1(o_free);  // O^T may be overwritten by the next unit
+      ++j;
       softmax_bar();
       const float lh = red[lane] + red[32 + lane] + red[64 + lane] + red[96 + lane];  // head = lane
       float mrl = 0.f;  // mr[lane]
 #pragma unroll
       for (int h = 0; h < 32; ++h) mrl = h == lane ? mr[h] : mrl;
-      uint32_t o[32];
-      tmem_ld32(tmem_o + lane_off, o);
-      tmem_wait_ld();
-      if (ns == 1) {
+      if (e.ns == 1) {
 #pragma unroll
         for (int h = 0; h < 32; ++h) {
           const float inv = 1.f / __shfl_sync(0xffffffffu, lh, h);
-          if (h < gl) p.out[b * p.o_sb + (int64_t)(h0 + h) * p.o_sh + i] = to_bf16_bits(__uint_as_float(o[h]) * inv);
+          if (h < gl) p.out[e.b * p.o_sb + (int64_t)(h0 + h) * p.o_sh + i] = to_bf16_bits(__uint_as_float(o[h]) * inv);
         }
         if (warp == 0 && lane < gl && p.lse != nullptr)
-          p.lse[b * p.lse_sb + (int64_t)(h0 + lane) * p.lse_sh] = (mrl + log2f(lh)) * kLn2u;
+          p.lse[e.b * p.lse_sb + (int64_t)(h0 + lane) * p.lse_sh] = (mrl + log2f(lh)) * kLn2u;
       } else {
-        const int64_t row0 = ((int64_t)b * p.Hq + h0) * p.S + s;
+        const int64_t row0 = ((int64_t)e.b * p.Hq + h0) * p.S + e.s;
 #pragma unroll
         for (int h = 0; h < 32; ++h) {
           const float inv = 1.f / __shfl_sync(0xffffffffu, lh, h);
@@ -479,22 +609,22 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_kernel(const __grid_cons
         }
         if (warp == 0 && lane < gl) p.lse_part[row0 + (int64_t)lane * p.S] = (mrl + log2f(lh)) * kLn2u;
       }
+      softmax_bar();  // `red` is read by every warp before it is written again
+      if (e.ns > 1 && claim_last_partition(p, e.b, e.kvh, e.ht, e.ns, reinterpret_cast<int *>(words + 1), Warps0to3Sync()))
+        merge_partials<kD, kSoftmaxWarps * 32>(p, e.b, h0, gl, e.ns, reinterpret_cast<float *>(smem + SM::mw),
+                                               Warps0to3Sync());
     }
   }
 
-  // ---------------- all warps: release TMEM, then the split merge ----------------
+  // ---------------- all warps: release TMEM ----------------
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     // every MMA has completed before its accumulators are freed
     wait_bounded(mma_idle, 0, p.err, abort_flag, true);
     tc_fence_after();
-    tmem_dealloc(tmem, 64);
+    tmem_dealloc(tmem, 128);
   }
-  if (*abort_flag) return;
-  if (ns == 1) return;
-  if (claim_last_partition(p, b, kvh, ht, ns, reinterpret_cast<int *>(words + 1)))
-    merge_partials<kD, kUmmaThreads>(p, b, h0, gl, ns, reinterpret_cast<float *>(smem + SM::ring));
 }
 
 int umma_stages() { return kUmmaStages; }

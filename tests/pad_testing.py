@@ -39,9 +39,10 @@ class DeviceWorkload:
         self.lens = torch.from_numpy(w.seq_lens).to(dev)
         self.dev = dev
 
-    def run(self, num_splits=None, lse=True, poison=True):
+    def run(self, num_splits=None, lse=True, poison=True, entry=None):
         import paged_kv_attention_partition_b200 as pad
 
+        entry = pad.pad_decode if entry is None else entry
         w = self.w
         out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=self.dev)
         lse_t = torch.empty((w.B, w.Hq), dtype=torch.float32, device=self.dev) if lse else None
@@ -50,8 +51,7 @@ class DeviceWorkload:
             if lse_t is not None:
                 lse_t.fill_(float("nan"))
         splits = w.num_splits if num_splits is None else num_splits
-        pad.pad_decode(self.q, self.k, self.v, self.tables, self.lens, w.scale, num_splits=splits,
-                       out=out, lse=lse_t)
+        entry(self.q, self.k, self.v, self.tables, self.lens, w.scale, num_splits=splits, out=out, lse=lse_t)
         torch.cuda.synchronize(self.dev)
         return out, lse_t
 

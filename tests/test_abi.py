@@ -89,9 +89,11 @@ def test_heuristic_plans(lib):
         # bytes) at most 1/16 of the K/V bytes it streams (4*D*P)
         if p["num_splits"] > 1:
             assert p["partition_tokens"] >= 64 and g / p["partition_tokens"] <= 1 / 16 + 1e-9
-    # large batches keep 256-token partitions; a small batch is cut finer (down to
-    # 64 tokens) until it fills about two waves of CTAs on 148 SMs
-    assert pad.pad_decode_plan(32, 32, 8, 128, 16, 256, num_splits=0, device=0)["partition_tokens"] == 256
+    # a large batch gets max(512, 64 g) tokens per partition (a power of two); a
+    # small batch is cut finer (down to 64 tokens) until it fills about two
+    # waves of CTAs on 148 SMs
+    assert pad.pad_decode_plan(32, 32, 8, 128, 16, 256, num_splits=0, device=0)["partition_tokens"] == 512
+    assert pad.pad_decode_plan(256, 32, 1, 128, 32, 1024, num_splits=0, device=0)["partition_tokens"] == 2048
     assert pad.pad_decode_plan(1, 32, 8, 128, 16, 256, num_splits=0, device=0)["partition_tokens"] == 64
     assert pad.pad_decode_plan(4, 32, 8, 128, 16, 256, num_splits=0, device=0)["partition_tokens"] == 128
     # group 20: one 32-head tile at D=128, two 16-head tiles at D=256; group 64: two tiles
