@@ -49,10 +49,10 @@ def _load(path: str = _LIB):
         lib = ctypes.CDLL(path)
         p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
         lib.oracle_decode.argtypes = [p, p, p, p, p, p, i64, p, i64, i64, i64, i64, i64,
-                                      ctypes.c_double, p, p, i32]
+                                      ctypes.c_double, i64, p, p, p, i32]
         lib.oracle_decode.restype = ctypes.c_int
         lib.oracle_decode_pairs.argtypes = [p, p, p, p, p, p, i64, p, i64, i64, i64, i64, i64,
-                                            ctypes.c_double, p, i64, p, p, i32]
+                                            ctypes.c_double, i64, p, p, i64, p, p, i32]
         lib.oracle_decode_pairs.restype = ctypes.c_int
         _libs[path] = lib
     return _libs[path]
@@ -74,12 +74,20 @@ def _check(q, k, v, tables, lens):
     assert lens.dtype == np.int32 and lens.ndim == 1 and lens.flags.c_contiguous
 
 
-def decode(q, k_cache, v_cache, block_tables, seq_lens, scale, nthreads=None, lib_path=_LIB):
+def _sinks_arg(sinks, Hq):
+    if sinks is None:
+        return None, None
+    arr = np.ascontiguousarray(np.asarray(sinks, dtype=np.float32).reshape(Hq))
+    return arr, arr.ctypes.data
+
+
+def decode(q, k_cache, v_cache, block_tables, seq_lens, scale, nthreads=None, lib_path=_LIB, window=0, sinks=None):
     """Full oracle: returns (out [B, Hq, D] float64, lse [B, Hq] float64).
 
     q: uint16 bf16 bits [B, Hq, D]; k_cache/v_cache: uint16 [num_blocks, Hkv, bs, D]
     (any strides, e.g. a transposed view of an NHD cache); block_tables int32
-    [B, W]; seq_lens int32 [B]."""
+    [B, W]; seq_lens int32 [B].  window: 0 = every token, W > 0 = each
+    sequence's last W tokens; sinks: None, or fp32 [Hq] sink logits."""
     _check(q, k_cache, v_cache, block_tables, seq_lens)
     B, Hq, D = q.shape
     _, Hkv, bs, Dk = k_cache.shape
@@ -87,16 +95,18 @@ def decode(q, k_cache, v_cache, block_tables, seq_lens, scale, nthreads=None, li
     out = np.zeros((B, Hq, D), dtype=np.float64)
     lse = np.zeros((B, Hq), dtype=np.float64)
     qs, ks = _estrides(q), _estrides(k_cache)
+    keep, sp = _sinks_arg(sinks, Hq)
     rc = _load(lib_path).oracle_decode(
         q.ctypes.data, qs.ctypes.data, k_cache.ctypes.data, v_cache.ctypes.data, ks.ctypes.data,
         block_tables.ctypes.data, block_tables.shape[1], seq_lens.ctypes.data, B, Hq, Hkv, D, bs,
-        float(scale), out.ctypes.data, lse.ctypes.data, nthreads or default_threads())
+        float(scale), int(window), sp, out.ctypes.data, lse.ctypes.data, nthreads or default_threads())
     if rc:
         raise RuntimeError(f"oracle_decode failed ({rc})")
     return out, lse
 
 
-def decode_pairs(q, k_cache, v_cache, block_tables, seq_lens, scale, pairs, nthreads=None, lib_path=_LIB):
+def decode_pairs(q, k_cache, v_cache, block_tables, seq_lens, scale, pairs, nthreads=None, lib_path=_LIB, window=0,
+                 sinks=None):
     """Oracle for selected (b, h) pairs: returns (out [n, D], lse [n])."""
     _check(q, k_cache, v_cache, block_tables, seq_lens)
     B, Hq, D = q.shape
@@ -106,16 +116,18 @@ def decode_pairs(q, k_cache, v_cache, block_tables, seq_lens, scale, pairs, nthr
     out = np.zeros((n, D), dtype=np.float64)
     lse = np.zeros((n,), dtype=np.float64)
     qs, ks = _estrides(q), _estrides(k_cache)
+    keep, sp = _sinks_arg(sinks, Hq)
     rc = _load(lib_path).oracle_decode_pairs(
         q.ctypes.data, qs.ctypes.data, k_cache.ctypes.data, v_cache.ctypes.data, ks.ctypes.data,
         block_tables.ctypes.data, block_tables.shape[1], seq_lens.ctypes.data, B, Hq, Hkv, D, bs,
-        float(scale), pairs.ctypes.data, n, out.ctypes.data, lse.ctypes.data,
+        float(scale), int(window), sp, pairs.ctypes.data, n, out.ctypes.data, lse.ctypes.data,
         nthreads or default_threads())
     if rc:
         raise RuntimeError(f"oracle_decode_pairs failed ({rc})")
     return out, lse
 
 
-def decode_workload(w, nthreads=None):
+def decode_workload(w, nthreads=None, window=0, sinks=None):
     """Oracle over a ``synth.Workload``."""
-    return decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, nthreads)
+    return decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, nthreads, window=window,
+                  sinks=sinks)

@@ -24,6 +24,16 @@
  *     lse   = M + ln Z                    (natural log, includes `scale`)
  *   L_b = 0 gives out = 0 and lse = -inf.
  *
+ * Two options of the decode path that "Attention parity: run every attention
+ * type on the best available path on both targets" (section "Current state")
+ * lists next to dense GQA:
+ *   sliding window W > 0: only tokens t >= L_b - W take part (the last W
+ *     tokens; all of them when W >= L_b);
+ *   attention sinks: a per-head logit sigma_h, in the units of s_t, joins the
+ *     softmax with a zero value row:  M = max(max_t s_t, sigma_h),
+ *     Z = sum_t exp(s_t - M) + exp(sigma_h - M); out and lse as above.  With
+ *     L_b = 0: out = 0, lse = sigma_h.
+ *
  * Exact two-pass softmax: no splits, no online rescaling.  bf16 inputs are
  * widened exactly to double.  Strides are in elements; every dimension may be
  * strided.  Work is spread over (b, kh) pairs with pthreads, which changes no
@@ -52,6 +62,8 @@ typedef struct {
   int64_t q_str[3];   /* b, h, d */
   int64_t kv_str[4];  /* block, kv head, slot, d (same for K and V) */
   double scale;
+  int64_t window;     /* 0: every token; W > 0: the last W tokens */
+  const float *sinks; /* NULL, or sink logit per query head [Hq] */
   double *out;        /* [B, Hq, D] contiguous */
   double *lse;        /* [B, Hq] */
 } problem;
@@ -62,36 +74,43 @@ static void attend_one(const problem *p, int64_t b, int64_t h, double *s, double
   const int64_t kh = h / g;
   const int64_t L = p->lens[b];
   const uint16_t *qrow = p->q + b * p->q_str[0] + h * p->q_str[1];
+  const int has_sink = p->sinks != NULL;
+  const double sink = has_sink ? (double)p->sinks[h] : 0.0;
   for (int64_t d = 0; d < p->D; ++d) o[d] = 0.0;
   if (L <= 0) {
-    *lse = -INFINITY;
+    *lse = has_sink ? sink : -INFINITY;
     return;
   }
-  /* scores */
-  for (int64_t t = 0; t < L; ++t) {
+  /* the tokens that take part: [lo, L) */
+  const int64_t lo = (p->window > 0 && L > p->window) ? L - p->window : 0;
+  /* scores, s[t - lo] for token t */
+  for (int64_t t = lo; t < L; ++t) {
     int64_t phys = p->tables[b * p->table_width + t / p->bs];
     int64_t slot = t % p->bs;
     const uint16_t *krow = p->k + phys * p->kv_str[0] + kh * p->kv_str[1] + slot * p->kv_str[2];
     double acc = 0.0;
     for (int64_t d = 0; d < p->D; ++d)
       acc += bf16_to_double(qrow[d * p->q_str[2]]) * bf16_to_double(krow[d * p->kv_str[3]]);
-    s[t] = p->scale * acc;
+    s[t - lo] = p->scale * acc;
   }
-  /* exact softmax */
+  const int64_t n = L - lo;
+  /* exact softmax (the sink, if any, joins the max and the denominator) */
   double M = s[0];
-  for (int64_t t = 1; t < L; ++t)
+  for (int64_t t = 1; t < n; ++t)
     if (s[t] > M) M = s[t];
+  if (has_sink && sink > M) M = sink;
   double Z = 0.0;
-  for (int64_t t = 0; t < L; ++t) {
+  for (int64_t t = 0; t < n; ++t) {
     s[t] = exp(s[t] - M);
     Z += s[t];
   }
-  /* weighted sum of values */
-  for (int64_t t = 0; t < L; ++t) {
+  if (has_sink) Z += exp(sink - M);
+  /* weighted sum of values (the sink's value row is zero) */
+  for (int64_t t = lo; t < L; ++t) {
     int64_t phys = p->tables[b * p->table_width + t / p->bs];
     int64_t slot = t % p->bs;
     const uint16_t *vrow = p->v + phys * p->kv_str[0] + kh * p->kv_str[1] + slot * p->kv_str[2];
-    double w = s[t] / Z;
+    double w = s[t - lo] / Z;
     for (int64_t d = 0; d < p->D; ++d) o[d] += w * bf16_to_double(vrow[d * p->kv_str[3]]);
   }
   *lse = M + log(Z);
@@ -156,8 +175,11 @@ static int run(const problem *p, const int32_t *pairs, int64_t npairs, int nthre
 static int fill(problem *p, const uint16_t *q, const int64_t *q_str, const uint16_t *k,
                 const uint16_t *v, const int64_t *kv_str, const int32_t *tables,
                 int64_t table_width, const int32_t *lens, int64_t B, int64_t Hq, int64_t Hkv,
-                int64_t D, int64_t bs, double scale, double *out, double *lse) {
-  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || bs <= 0) return 2;
+                int64_t D, int64_t bs, double scale, int64_t window, const float *sinks, double *out,
+                double *lse) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || bs <= 0 || window < 0) return 2;
+  p->window = window;
+  p->sinks = sinks;
   p->q = q;
   p->k = k;
   p->v = v;
@@ -177,14 +199,16 @@ static int fill(problem *p, const uint16_t *q, const int64_t *q_str, const uint1
   return 0;
 }
 
-/* Every (b, h): out [B, Hq, D] and lse [B, Hq], double.  Returns 0 on success. */
+/* Every (b, h): out [B, Hq, D] and lse [B, Hq], double.  `window` 0 = every
+ * token; `sinks` NULL = none.  Returns 0 on success. */
 int oracle_decode(const uint16_t *q, const int64_t *q_str, const uint16_t *k_cache,
                   const uint16_t *v_cache, const int64_t *kv_str, const int32_t *block_tables,
                   int64_t table_width, const int32_t *seq_lens, int64_t B, int64_t Hq, int64_t Hkv,
-                  int64_t D, int64_t bs, double scale, double *out, double *lse, int nthreads) {
+                  int64_t D, int64_t bs, double scale, int64_t window, const float *sinks, double *out,
+                  double *lse, int nthreads) {
   problem p;
   int rc = fill(&p, q, q_str, k_cache, v_cache, kv_str, block_tables, table_width, seq_lens, B,
-                Hq, Hkv, D, bs, scale, out, lse);
+                Hq, Hkv, D, bs, scale, window, sinks, out, lse);
   return rc ? rc : run(&p, NULL, 0, nthreads);
 }
 
@@ -193,11 +217,11 @@ int oracle_decode_pairs(const uint16_t *q, const int64_t *q_str, const uint16_t 
                         const uint16_t *v_cache, const int64_t *kv_str,
                         const int32_t *block_tables, int64_t table_width, const int32_t *seq_lens,
                         int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t bs, double scale,
-                        const int32_t *pairs, int64_t npairs, double *out, double *lse,
-                        int nthreads) {
+                        int64_t window, const float *sinks, const int32_t *pairs, int64_t npairs,
+                        double *out, double *lse, int nthreads) {
   problem p;
   int rc = fill(&p, q, q_str, k_cache, v_cache, kv_str, block_tables, table_width, seq_lens, B,
-                Hq, Hkv, D, bs, scale, out, lse);
+                Hq, Hkv, D, bs, scale, window, sinks, out, lse);
   for (int64_t i = 0; !rc && i < npairs; ++i)
     if (pairs[2 * i] < 0 || pairs[2 * i] >= B || pairs[2 * i + 1] < 0 || pairs[2 * i + 1] >= Hq)
       rc = 2;

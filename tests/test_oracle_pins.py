@@ -16,7 +16,12 @@ section "Summary"):
 * closed forms: q = 0 (uniform weights, lse = ln L, out = mean V), L = 1
   (out = v_0, lse = scale q.k_0), a dominant score (out = v_argmax), L = 0;
 * split combine: attention over disjoint token ranges merged by log-sum-exp
-  equals attention over the union (the identity the split-KV reduce relies on).
+  equals attention over the union (the identity the split-KV reduce relies on);
+* sliding window: equals torch's SDPA over each sequence's last W contiguous
+  tokens; W = 1 gives the last value row exactly;
+* attention sinks: equals scipy's softmax over the scores with the sink logit
+  appended (zero value row); a -inf sink changes nothing; an empty sequence
+  gives out = 0, lse = sink.
 
 ``test_planted_mistakes_are_caught`` compiles copies of the oracle with one
 plausible mistake each and checks that some pin fails for every one.
@@ -244,9 +249,89 @@ def pin_split_combine(lib):
             np.testing.assert_allclose(merged, full_out[b], rtol=0, atol=1e-12)
 
 
+WINDOW_CASES = [
+    # B, Hq, Hkv, D, bs, lens, window
+    (2, 4, 1, 16, 4, [5, 15], 3),
+    (3, 8, 2, 32, 16, [16, 17, 40], 16),
+    (2, 10, 2, 16, 4, [40, 1], 7),
+    (1, 5, 1, 64, 16, [33], 33),
+    (2, 6, 6, 8, 1, [7, 3], 100),
+]
+
+
+def pin_window_bruteforce(lib):
+    # Sliding window ("Attention parity: run every attention type on the best
+    # available path on both targets", section "Current state"): the last W
+    # tokens of each sequence, against SDPA on exactly those contiguous rows.
+    for i, (B, Hq, Hkv, D, bs, lens, W) in enumerate(WINDOW_CASES):
+        lens = np.asarray(lens, dtype=np.int32)
+        q, kc, vc = random_case(300 + i, B, Hq, Hkv, D, bs, lens)
+        kp, vp, tables = scatter_to_pages(kc, vc, lens, bs, extra_blocks=2, seed=400 + i)
+        scale = 1.0 / math.sqrt(D)
+        out, lse = oracle.decode(q, kp, vp, tables, lens, scale, lib_path=lib, window=W)
+        lo = np.maximum(lens - W, 0)
+        wl = (lens - lo).astype(np.int32)
+        kw = np.zeros_like(kc)
+        vw = np.zeros_like(vc)
+        for b in range(B):
+            kw[b, :, : wl[b]] = kc[b, :, lo[b]: lens[b]]
+            vw[b, :, : wl[b]] = vc[b, :, lo[b]: lens[b]]
+        ref_out, ref_lse = library_attention(q, kw, vw, wl, scale)
+        np.testing.assert_allclose(out, ref_out, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-12)
+
+
+def pin_window_one(lib):
+    # W = 1: the weight of the last token is 1: out = v_{L-1}, lse = s_{L-1}
+    lens = np.asarray([9, 1, 30], dtype=np.int32)
+    q, kc, vc = random_case(500, 3, 4, 2, 16, 4, lens)
+    kp, vp, tables = scatter_to_pages(kc, vc, lens, 4, extra_blocks=1, seed=501)
+    out, lse = oracle.decode(q, kp, vp, tables, lens, 0.25, lib_path=lib, window=1)
+    for b in range(3):
+        for h in range(4):
+            kh = h // 2
+            last = int(lens[b]) - 1
+            np.testing.assert_array_equal(out[b, h], _f(vc[b, kh, last]))
+            assert abs(lse[b, h] - 0.25 * float(_f(q[b, h]) @ _f(kc[b, kh, last]))) <= 1e-12
+
+
+def pin_sinks_are_softmax_terms(lib):
+    # Attention sinks (same page, same section): the sink logit joins the
+    # softmax with a zero value row -- scipy's softmax over [scores, sink].
+    lens = np.asarray([5, 15, 1], dtype=np.int32)
+    B, Hq, Hkv, D, bs = 3, 4, 2, 16, 4
+    q, kc, vc = random_case(600, B, Hq, Hkv, D, bs, lens)
+    kp, vp, tables = scatter_to_pages(kc, vc, lens, bs, extra_blocks=1, seed=601)
+    sinks = np.asarray([0.5, -1.0, 3.0, -30.0], dtype=np.float32)
+    scale = 0.25
+    out, lse = oracle.decode(q, kp, vp, tables, lens, scale, lib_path=lib, sinks=sinks)
+    for b in range(B):
+        L = int(lens[b])
+        for h in range(Hq):
+            kh = h // (Hq // Hkv)
+            sc = scale * (_f(kc[b, kh, :L]) @ _f(q[b, h]))
+            logits = np.concatenate([sc, [float(sinks[h])]])
+            w = scipy.special.softmax(logits)
+            np.testing.assert_allclose(out[b, h], w[:L] @ _f(vc[b, kh, :L]), rtol=0, atol=1e-12)
+            assert abs(lse[b, h] - scipy.special.logsumexp(logits)) <= 1e-12
+
+
+def pin_sink_limits(lib):
+    # a -inf sink is no sink; an empty sequence with a sink: out = 0, lse = sink
+    w = synth.make_workload("sinklim", 3, 4, 1, 32, 8, [20, 0, 3], seed=21)
+    plain = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, lib_path=lib)
+    ninf = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, lib_path=lib,
+                         sinks=np.full(4, -np.inf, dtype=np.float32))
+    assert np.array_equal(plain[0], ninf[0]) and np.array_equal(plain[1], ninf[1])
+    sinks = np.asarray([1.0, -2.0, 0.0, 5.0], dtype=np.float32)
+    out, lse = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, lib_path=lib,
+                             sinks=sinks)
+    assert np.all(out[1] == 0.0) and np.array_equal(lse[1], sinks.astype(np.float64))
+
+
 PINS = [pin_bruteforce, pin_weights_are_softmax, pin_permutation_invariance, pin_layout_invariance,
         pin_constant_v, pin_zero_query, pin_single_token, pin_dominant_score, pin_empty_sequence,
-        pin_split_combine]
+        pin_split_combine, pin_window_bruteforce, pin_window_one, pin_sinks_are_softmax_terms, pin_sink_limits]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -275,19 +360,26 @@ def test_thread_count_does_not_change_results():
 # ---------------------------------------------------------------------------
 
 MUTATIONS = {
-    "scale_dropped": ("s[t] = p->scale * acc;", "s[t] = acc;"),
+    "scale_dropped": ("s[t - lo] = p->scale * acc;", "s[t - lo] = acc;"),
     "head_map_modulo": ("const int64_t kh = h / g;", "const int64_t kh = h % p->Hkv;"),
     "slot_from_division": ("int64_t slot = t % p->bs;\n    const uint16_t *krow",
                            "int64_t slot = (t / p->bs) % p->bs;\n    const uint16_t *krow"),
     "first_page_only": ("int64_t phys = p->tables[b * p->table_width + t / p->bs];\n    int64_t slot = t % p->bs;\n    const uint16_t *vrow",
                         "int64_t phys = p->tables[b * p->table_width];\n    int64_t slot = t % p->bs;\n    const uint16_t *vrow"),
-    "unnormalised_weights": ("double w = s[t] / Z;", "double w = s[t];"),
+    "unnormalised_weights": ("double w = s[t - lo] / Z;", "double w = s[t - lo];"),
     "lse_without_max": ("*lse = M + log(Z);", "*lse = log(Z);"),
     "lse_log2": ("*lse = M + log(Z);", "*lse = M + log2(Z);"),
-    "last_token_dropped": ("for (int64_t t = 0; t < L; ++t) {\n    int64_t phys = p->tables[b * p->table_width + t / p->bs];\n    int64_t slot = t % p->bs;\n    const uint16_t *vrow",
-                           "for (int64_t t = 0; t < L - 1; ++t) {\n    int64_t phys = p->tables[b * p->table_width + t / p->bs];\n    int64_t slot = t % p->bs;\n    const uint16_t *vrow"),
-    "max_over_first_half": ("for (int64_t t = 1; t < L; ++t)\n    if (s[t] > M) M = s[t];",
-                            "for (int64_t t = 1; t < L / 2; ++t)\n    if (s[t] > M) M = s[t];"),
+    "last_token_dropped": ("for (int64_t t = lo; t < L; ++t) {\n    int64_t phys = p->tables[b * p->table_width + t / p->bs];\n    int64_t slot = t % p->bs;\n    const uint16_t *vrow",
+                           "for (int64_t t = lo; t < L - 1; ++t) {\n    int64_t phys = p->tables[b * p->table_width + t / p->bs];\n    int64_t slot = t % p->bs;\n    const uint16_t *vrow"),
+    "max_over_first_half": ("for (int64_t t = 1; t < n; ++t)\n    if (s[t] > M) M = s[t];",
+                            "for (int64_t t = 1; t < n / 2; ++t)\n    if (s[t] > M) M = s[t];"),
+    "window_off_by_one": ("L > p->window) ? L - p->window : 0;", "L > p->window) ? L - p->window + 1 : 0;"),
+    "window_ignored": ("const int64_t lo = (p->window > 0 && L > p->window) ? L - p->window : 0;",
+                       "const int64_t lo = 0;"),
+    "sink_ignored": ("if (has_sink) Z += exp(sink - M);", ""),
+    "sink_scaled": ("const double sink = has_sink ? (double)p->sinks[h] : 0.0;",
+                    "const double sink = has_sink ? (double)p->sinks[h] * p->scale : 0.0;"),
+    "empty_sequence_drops_sink": ("*lse = has_sink ? sink : -INFINITY;", "*lse = -INFINITY;"),
     "query_of_kv_head": ("h * p->q_str[1];", "kh * p->q_str[1];"),
     "exp_without_shift": ("s[t] = exp(s[t] - M);", "s[t] = exp(s[t]);"),
 }
