@@ -133,6 +133,36 @@ pad_status pad_decode(const pad_tensor *q, const pad_tensor *k_cache, const pad_
                       int32_t num_splits, pad_tensor *out, pad_tensor *lse, void *stream);
 
 /*
+ * Options of pad_decode_ex: two attention types that "Attention parity: run
+ * every attention type on the best available path on both targets" (section
+ * "Current state") lists next to dense GQA.
+ *   window_left  0: every token; W > 0: each sequence attends to its last W
+ *                tokens only (tokens L_b - W .. L_b - 1; all of them when
+ *                W >= L_b).  Partitions and pages wholly before the window
+ *                are never read.
+ *   sinks        NULL, or a pad_tensor of fp32 [Hq] on the device: the sink
+ *                logit of each query head, in the units of scale * q.k.  It
+ *                joins the softmax with a zero value row:
+ *                  M = max(max_t s_t, sink_h), Z = sum_t exp(s_t - M) +
+ *                  exp(sink_h - M), out = sum_t exp(s_t - M) v_t / Z,
+ *                  lse = M + ln Z;  L_b = 0 gives out = 0, lse = sink_h.
+ */
+typedef struct pad_decode_options {
+  int32_t window_left;
+  const pad_tensor *sinks;
+} pad_decode_options;
+
+/*
+ * pad_decode_ex -- pad_decode with options (NULL options = pad_decode).  Same
+ * arguments, scratch, results and errors; `options->window_left` < 0, or a
+ * sinks tensor that is not fp32 [Hq] device memory, is PAD_ERR_INVALID_ARG.
+ */
+pad_status pad_decode_ex(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
+                         const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
+                         int32_t num_splits, const pad_decode_options *options, pad_tensor *out,
+                         pad_tensor *lse, void *stream);
+
+/*
  * pad_decode_with_workspace -- pad_decode with its scratch supplied by the
  * caller instead of the library ("perf(rocke): prepare saved paged decode
  * bindings once", section "Technical Changes": a binding owns its private

@@ -43,6 +43,11 @@ class PadPlan(ctypes.Structure):
         return {name: getattr(self, name) for name, _ in self._fields_}
 
 
+class PadOptions(ctypes.Structure):
+    """pad_decode_options: sliding window and attention sinks."""
+    _fields_ = [("window_left", ctypes.c_int32), ("sinks", ctypes.POINTER(PadTensor))]
+
+
 class PadError(RuntimeError):
     def __init__(self, status: int, message: str):
         super().__init__(f"{_status_name(status)}: {message}")
@@ -72,6 +77,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pad_decode_static_scratch.restype = ctypes.c_int
     lib.pad_decode_tcgen05.argtypes = lib.pad_decode.argtypes
     lib.pad_decode_tcgen05.restype = ctypes.c_int
+    lib.pad_decode_ex.argtypes = [P, P, P, P, P, ctypes.c_float, ctypes.c_int32, ctypes.POINTER(PadOptions), P, P,
+                                  ctypes.c_void_p]
+    lib.pad_decode_ex.restype = ctypes.c_int
     lib.pad_decode_with_workspace.argtypes = [P, P, P, P, P, ctypes.c_float, ctypes.c_int32, P, P, ctypes.c_void_p,
                                               ctypes.c_size_t, ctypes.c_void_p]
     lib.pad_decode_with_workspace.restype = ctypes.c_int
@@ -134,14 +142,18 @@ def _stream_handle(stream, device) -> int:
 
 def pad_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
                seq_lens: torch.Tensor, scale: float, num_splits: int = 0, out: Optional[torch.Tensor] = None,
-               lse: Union[None, bool, torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """Paged single-token decode attention (see ``pad_decode`` in include/pad.h).
+               lse: Union[None, bool, torch.Tensor] = None, stream=None, window: int = 0,
+               sinks: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Paged single-token decode attention (see ``pad_decode`` / ``pad_decode_ex``
+    in include/pad.h).
 
     q [B, Hq, D] bf16; k_cache/v_cache [num_blocks, Hkv, block_size, D] bf16 (any
     16-byte-multiple strides on dims 0-2, e.g. ``nhd.transpose(1, 2)``);
     block_tables [B, W] int32; seq_lens [B] int32.  ``lse=True`` allocates the
     fp32 [B, Hq] log-sum-exp output, a tensor receives it, None skips it.
-    Returns (out, lse).  Asynchronous on ``stream`` (default: torch's current)."""
+    ``window`` > 0 attends to each sequence's last ``window`` tokens; ``sinks``
+    is an fp32 [Hq] CUDA tensor of per-head sink logits.  Returns (out, lse).
+    Asynchronous on ``stream`` (default: torch's current)."""
     dev = q.device
     if dev.type != "cuda":
         raise ValueError("q must be a CUDA tensor")
@@ -158,13 +170,23 @@ def pad_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, bl
     for name, t in (("out", out), ("lse", lse)):
         if t is not None and t.device != dev:
             raise ValueError(f"{name} is on {t.device}, q on {dev}")
+    if sinks is not None and sinks.device != dev:
+        raise ValueError(f"sinks is on {sinks.device}, q on {dev}")
     lib = load_library()
     dq, dk, dv, dt, dl, do = (describe(t) for t in (q, k_cache, v_cache, block_tables, seq_lens, out))
     dlse = describe(lse) if lse is not None else None
     with torch.cuda.device(dev):
-        st = lib.pad_decode(ctypes.byref(dq), ctypes.byref(dk), ctypes.byref(dv), ctypes.byref(dt),
-                            ctypes.byref(dl), float(scale), int(num_splits), ctypes.byref(do),
-                            ctypes.byref(dlse) if dlse is not None else None, _stream_handle(stream, dev))
+        if window or sinks is not None:
+            dsk = describe(sinks) if sinks is not None else None
+            opts = PadOptions(int(window), ctypes.pointer(dsk) if dsk is not None else None)
+            st = lib.pad_decode_ex(ctypes.byref(dq), ctypes.byref(dk), ctypes.byref(dv), ctypes.byref(dt),
+                                   ctypes.byref(dl), float(scale), int(num_splits), ctypes.byref(opts),
+                                   ctypes.byref(do), ctypes.byref(dlse) if dlse is not None else None,
+                                   _stream_handle(stream, dev))
+        else:
+            st = lib.pad_decode(ctypes.byref(dq), ctypes.byref(dk), ctypes.byref(dv), ctypes.byref(dt),
+                                ctypes.byref(dl), float(scale), int(num_splits), ctypes.byref(do),
+                                ctypes.byref(dlse) if dlse is not None else None, _stream_handle(stream, dev))
     _raise(st)
     return out, lse
 
@@ -269,4 +291,4 @@ def pad_release_workspace(device: int = -1) -> None:
 __all__ = ["pad_decode", "pad_decode_with_workspace", "pad_decode_static_scratch", "pad_decode_tcgen05", "pad_decode_plan",
            "pad_check_device_errors", "pad_release_workspace",
            "pad_status_string", "pad_last_error", "pad_abi_version", "describe", "load_library",
-           "PadError", "PadTensor", "PadPlan"]
+           "PadError", "PadTensor", "PadPlan", "PadOptions"]

@@ -312,7 +312,7 @@ struct Prepared {
 pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
                    const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale, int32_t num_splits,
                    const pad_tensor *out, const pad_tensor *lse, Prepared *pr, bool *empty,
-                   bool tcgen05 = false) {
+                   bool tcgen05 = false, const pad_decode_options *opts = nullptr) {
   pad_status st;
   *empty = false;
   if ((st = check_tensor(q, "q", PAD_BF16, 3)) != PAD_OK) return st;
@@ -416,6 +416,19 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
   p.S = pr->plan.num_splits;
   p.n_units = (uint32_t)units;
   p.scale_log2 = scale * 1.4426950408889634f;
+  if (opts != nullptr) {
+    if (opts->window_left < 0) return fail(PAD_ERR_INVALID_ARG, "window_left must be >= 0 (got %d)", opts->window_left);
+    p.window = opts->window_left;
+    if (opts->sinks != nullptr) {
+      const pad_tensor *sk = opts->sinks;
+      if ((st = check_tensor(sk, "sinks", PAD_F32, 1)) != PAD_OK) return st;
+      if (sk->shape[0] != Hq) return fail(PAD_ERR_INVALID_ARG, "sinks must be fp32 [Hq] = [%lld]", (long long)Hq);
+      if (sk->stride[0] != 1 && Hq > 1) return fail(PAD_ERR_INVALID_ARG, "sinks must be contiguous");
+      if (reinterpret_cast<uintptr_t>(sk->data) % 4) return fail(PAD_ERR_INVALID_ARG, "sinks must be 4-byte aligned");
+      if ((st = check_device_ptr(sk->data, device, "sinks")) != PAD_OK) return st;
+      p.sinks = static_cast<const float *>(sk->data);
+    }
+  }
   p.out = static_cast<uint16_t *>(out->data);
   p.o_sb = out->stride[0];
   p.o_sh = out->stride[1];
@@ -524,6 +537,23 @@ pad_status pad_decode(const pad_tensor *q, const pad_tensor *k_cache, const pad_
   Prepared pr;
   bool empty = false;
   pad_status st = prepare(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, &pr, &empty);
+  if (st != PAD_OK || empty) return st;
+  void *ws = nullptr, *ctl = nullptr;
+  if (pr.ws.total > 0 && (st = get_buffer(g_ws, pr.device, stream, pr.ws.total, &ws)) != PAD_OK) return st;
+  if (pr.cl.total > 0 && (st = get_buffer(g_ctl, pr.device, stream, pr.cl.total, &ctl)) != PAD_OK) return st;
+  bind_buffers(pr, ws, ctl);
+  return run(pr, stream);
+}
+
+pad_status pad_decode_ex(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
+                         const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
+                         int32_t num_splits, const pad_decode_options *options, pad_tensor *out, pad_tensor *lse,
+                         void *stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  Prepared pr;
+  bool empty = false;
+  pad_status st =
+      prepare(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, &pr, &empty, false, options);
   if (st != PAD_OK || empty) return st;
   void *ws = nullptr, *ctl = nullptr;
   if (pr.ws.total > 0 && (st = get_buffer(g_ws, pr.device, stream, pr.ws.total, &ws)) != PAD_OK) return st;

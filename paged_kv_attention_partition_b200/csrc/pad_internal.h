@@ -95,6 +95,8 @@ struct PartitionParams {
   int32_t S;        // partitions per sequence (ceil(capacity / P) <= kMaxSplits)
   uint32_t n_units; // B * Hkv * HT * S, one CTA each
   float scale_log2; // scale * log2(e)
+  int32_t window;     // 0: every token; W > 0: each sequence's last W tokens
+  const float *sinks; // null, or a sink logit per query head [Hq] (natural log, units of scale q.k)
   uint16_t *out;
   int64_t o_sb, o_sh;
   float *lse;  // may be null

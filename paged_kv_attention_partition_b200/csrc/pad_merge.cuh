@@ -5,8 +5,10 @@
 // Every partition of a sequence with ns > 1 non-empty partitions writes its
 // partial output o_s (normalised by its own sum) and lse_s.  The CTA whose
 // count brings the (b, KV head, head tile) counter to ns merges the set:
-//   M = max_s lse_s,  w_s = exp(lse_s - M) / sum_s' exp(lse_s' - M),
-//   out = sum_s w_s o_s,  lse = M + log sum_s exp(lse_s - M).
+//   M = max_s lse_s,  lse = M + log sum_s exp(lse_s - M),
+//   out = sum_s w_s o_s with w_s = exp(lse_s - lse).
+// With attention sinks the head's sink logit joins the denominator:
+//   lse' = logaddexp(lse, sink), w_s = exp(lse_s - lse').
 #pragma once
 
 #include <math.h>
@@ -52,14 +54,15 @@ __device__ __forceinline__ bool claim_last_partition(const PartitionParams &p, i
   return last;
 }
 
-// Merges the ns partials of query heads h0 .. h0+gl-1 of sequence b into bf16
-// out (+ lse).  `wt` is shared memory for gl * ns floats.  The NTHREADS
-// participating threads (threadIdx.x 0 .. NTHREADS-1) call it.
+// Merges partials s_first .. s_first+ns-1 of query heads h0 .. h0+gl-1 of
+// sequence b into bf16 out (+ lse).  `wt` is shared memory for gl * ns floats.
+// The NTHREADS participating threads (threadIdx.x 0 .. NTHREADS-1) call it.
 template <int D, int NTHREADS, class Sync = CtaSync>
-__device__ void merge_partials(const PartitionParams &p, int b, int h0, int gl, int ns, float *wt, Sync sync = Sync()) {
+__device__ void merge_partials(const PartitionParams &p, int b, int h0, int gl, int s_first, int ns, float *wt,
+                               Sync sync = Sync()) {
   constexpr int D4 = D / 4, NW = NTHREADS / 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t row0 = ((int64_t)b * p.Hq + h0) * p.S;
+  const int64_t row0 = ((int64_t)b * p.Hq + h0) * p.S + s_first;
   for (int i = tid; i < gl * ns; i += NTHREADS) {
     const int hl = i / ns, si = i % ns;
     wt[hl * ns + si] = ld_cg_f32(p.lse_part + row0 + (int64_t)hl * p.S + si);
@@ -74,10 +77,14 @@ __device__ void merge_partials(const PartitionParams &p, int b, int h0, int gl, 
     for (int si = lane; si < ns; si += 32) sum += __expf(wt[hl * ns + si] - M);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    const float inv = 1.f / sum;
+    float lse = M + logf(sum);
+    if (p.sinks != nullptr) {
+      const float sg = p.sinks[h0 + hl];
+      lse = fmaxf(lse, sg) + log1pf(__expf(-fabsf(lse - sg)));
+    }
     __syncwarp();
-    for (int si = lane; si < ns; si += 32) wt[hl * ns + si] = __expf(wt[hl * ns + si] - M) * inv;
-    if (lane == 0 && p.lse != nullptr) p.lse[b * p.lse_sb + (int64_t)(h0 + hl) * p.lse_sh] = M + logf(sum);
+    for (int si = lane; si < ns; si += 32) wt[hl * ns + si] = __expf(wt[hl * ns + si] - lse);
+    if (lane == 0 && p.lse != nullptr) p.lse[b * p.lse_sb + (int64_t)(h0 + hl) * p.lse_sh] = lse;
   }
   sync();
   for (int i = tid; i < gl * D4; i += NTHREADS) {

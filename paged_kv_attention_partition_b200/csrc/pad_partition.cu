@@ -120,12 +120,15 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
   const uint32_t box_bytes = (uint32_t)ROWB << bsb_log2;
   const int32_t *trow = p.tables + (int64_t)b * p.table_stride;
 
-  // Warp 0 fetches the block ids of the first NST stages while the length is
-  // still in flight (clamped to the table row; an id is used only for a stage
-  // that holds live tokens): lane j holds box j, j + 32, ... of a stage.
+  // Stages are counted from tu, the first stage holding a token of the unit:
+  // t0 unless a sliding window starts later.  Warp 0 fetches the block ids of
+  // the first NST stages while the length is still in flight (clamped to the
+  // table row; an id is used only for a stage that holds live tokens): lane j
+  // holds box j, j + 32, ... of a stage.
+  int tu = t0;
   int ids[NST][IDW];
   auto load_ids = [&](int (&dst)[IDW], int st) {
-    const int page0 = (t0 + st * ST) >> p.bs_log2;
+    const int page0 = (tu + st * ST) >> p.bs_log2;
 #pragma unroll
     for (int w = 0; w < IDW; ++w) {
       const int j = lane + 32 * w;
@@ -147,33 +150,49 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
     if (tid == 0 && s == 0 && kvh == 0 && ht == 0) atomicOr(p.err, kErrSeqLen);
     L = L < 0 ? 0 : capacity;
   }
+  // tokens that take part: [lo, L) -- the last window tokens under a sliding
+  // window ("Attention parity: run every attention type on the best available
+  // path on both targets", section "Current state": out-of-window block skip);
+  // this unit covers [tlo, t1) of them
+  const int lo = (p.window > 0 && L > p.window) ? L - p.window : 0;
   const int t1 = min(t0 + p.P, L);
-  if (t0 >= t1) {
-    if (L == 0 && s == 0) {  // empty sequence: out = 0, lse = -inf
+  const int tlo = max(t0, lo);
+  if (tlo >= t1) {
+    if (L == 0 && s == 0) {  // empty sequence: out = 0, lse = -inf (or the sink)
       for (int i = tid; i < gl * D; i += kThreads)
         p.out[b * p.o_sb + (int64_t)(h0 + i / D) * p.o_sh + (i % D)] = 0;
-      if (p.lse != nullptr && tid < gl) p.lse[b * p.lse_sb + (int64_t)(h0 + tid) * p.lse_sh] = -INFINITY;
+      if (p.lse != nullptr && tid < gl)
+        p.lse[b * p.lse_sb + (int64_t)(h0 + tid) * p.lse_sh] = p.sinks != nullptr ? p.sinks[h0 + tid] : -INFINITY;
     }
-    return;
+    return;  // pages wholly outside [lo, L) are never read
   }
-  const int ns = (L + p.P - 1) / p.P;  // non-empty partitions of sequence b
-  const int nstages = (t1 - t0 + ST - 1) / ST;
+  const int s_first = lo / p.P;                      // first non-empty partition of sequence b
+  const int ns = (L + p.P - 1) / p.P - s_first;     // non-empty partitions
+  if (tlo >= t0 + ST) {  // stages wholly before the window are skipped
+    tu = t0 + ((tlo - t0) / ST) * ST;
+    if (warp == 0) {
+#pragma unroll
+      for (int k = 0; k < NST; ++k) load_ids(ids[k], k);
+    }
+  }
+  const int nstages = (t1 - tu + ST - 1) / ST;
   __syncthreads();  // the stage barriers are initialised
 
   // Stage st into ring slot st % NST (called by all of warp 0; lane 0 issues).
-  // Only boxes holding live tokens are copied.
+  // Only boxes holding live tokens ([tlo, t1)) are copied.
   auto issue = [&](const int (&sid)[IDW], int st) {
-    const int tb = t0 + st * ST;
+    const int tb = tu + st * ST;
+    const int jb = tb < tlo ? (tlo - tb) >> bsb_log2 : 0;
     const int nb = min(nbox, (t1 - tb + (1 << bsb_log2) - 1) >> bsb_log2);
     uint8_t *sK = smem + (st % NST) * STAGE_BYTES;
     uint8_t *sV = sK + ST * ROWB;
     const uint32_t bar = smem_addr(full + st % NST);
     const int slot0 = tb & ((1 << p.bs_log2) - 1);  // row of the box inside its page
-    if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)nb * box_bytes * 2);
+    if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(nb - jb) * box_bytes * 2);
 #pragma unroll
     for (int w = 0; w < IDW; ++w) {
 #pragma unroll 1
-      for (int jj = 0; jj < 32 && 32 * w + jj < nb; ++jj) {
+      for (int jj = max(0, jb - 32 * w); jj < 32 && 32 * w + jj < nb; ++jj) {
         const int j = 32 * w + jj;
         const int id = __shfl_sync(0xffffffffu, sid[w], jj);
         if (lane == 0) {
@@ -251,14 +270,15 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
 
     uint8_t *sK = smem + (st % NST) * STAGE_BYTES;
     uint8_t *sV = sK + ST * ROWB;
-    const int tb = t0 + st * ST;
-    if (tb + ST > t1) {
-      // the last stage: V rows past t1 (slots past L_b, rows of boxes not
-      // copied) are zeroed so that their zero weights meet finite values
+    const int tb = tu + st * ST;
+    if (tb + ST > t1 || tb < tlo) {
+      // the first and last stages: V rows outside [tlo, t1) (slots past L_b,
+      // tokens before the window, rows of boxes not copied) are zeroed so that
+      // their zero weights meet finite values
 #pragma unroll 1
       for (int e = lane; e < 16 * CH; e += 32) {
         const int r = tg * 16 + e / CH, c = e % CH;
-        if (tb + r >= t1) {
+        if (tb + r >= t1 || tb + r < tlo) {
           uint32_t rb, rk;
           row_base(r, rb, rk);
           *reinterpret_cast<uint4 *>(sV + chunk(rb, rk, c >> 3, c & 7)) = make_uint4(0, 0, 0, 0);
@@ -268,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
       __syncwarp();
     }
     const int tbase = tb + tg * 16;
-    if (tbase < t1) {
+    if (tbase < t1 && tbase + 16 > tlo) {  // the tile holds a live token
       // ---- S^T = K . Q^T over this token group's 16 tokens
       float sc[NT][4], sc2[NT][4];
 #pragma unroll
@@ -289,8 +309,9 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
       }
 
       // ---- online softmax (rows lane/4 and lane/4 + 8; columns 2(lane%4) + {0,1})
-      const bool okA = tbase + (lane >> 2) < t1;
-      const bool okB = tbase + (lane >> 2) + 8 < t1;
+      const int ra = tbase + (lane >> 2), rb8 = ra + 8;
+      const bool okA = ra >= tlo && ra < t1;
+      const bool okB = rb8 >= tlo && rb8 < t1;
       uint32_t pb[NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -311,8 +332,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
         // it by more than kRescaleSlack (log2 units), so weights stay below
         // 2^kRescaleSlack and the O^T rescale is skipped on almost every tile.
         // Any reference point gives the same out and lse as long as l and O^T
-        // share it.  Row 0 of the tile is a live token, so mx0/mx1 are finite
-        // and the first tile always sets the reference.
+        // share it.  The tile holds a live token, so mx0/mx1 are finite and
+        // the first tile always sets the reference.
         if (__any_sync(0xffffffffu, mx0 > m_run[nt][0] + kRescaleSlack || mx1 > m_run[nt][1] + kRescaleSlack)) {
           const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
           const float al0 = fast_exp2(m_run[nt][0] - mn0), al1 = fast_exp2(m_run[nt][1] - mn1);
@@ -421,11 +442,19 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
     const float lse_nat = (m + log2f(l)) * kLn2;
     const int h = h0 + hl;
     if (ns == 1) {
+      float sc = inv, lse_out = lse_nat;
+      if (p.sinks != nullptr) {
+        // the head's sink logit joins the softmax (same page and section:
+        // attention sinks): lse' = logaddexp(lse, sink), out scaled by exp(lse - lse')
+        const float sg = p.sinks[h];
+        lse_out = fmaxf(lse_nat, sg) + log1pf(__expf(-fabsf(lse_nat - sg)));
+        sc *= __expf(lse_nat - lse_out);
+      }
       uint2 packed;
-      packed.x = pack_bf16x2(o.x * inv, o.y * inv);
-      packed.y = pack_bf16x2(o.z * inv, o.w * inv);
+      packed.x = pack_bf16x2(o.x * sc, o.y * sc);
+      packed.y = pack_bf16x2(o.z * sc, o.w * sc);
       *reinterpret_cast<uint2 *>(p.out + b * p.o_sb + (int64_t)h * p.o_sh + d) = packed;
-      if (d == 0 && p.lse != nullptr) p.lse[b * p.lse_sb + (int64_t)h * p.lse_sh] = lse_nat;
+      if (d == 0 && p.lse != nullptr) p.lse[b * p.lse_sb + (int64_t)h * p.lse_sh] = lse_out;
     } else {
       const int64_t row = ((int64_t)b * p.Hq + h) * p.S + s;
       *reinterpret_cast<float4 *>(p.o_part + row * D + d) = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
@@ -434,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
   }
   if (ns == 1) return;
   if (claim_last_partition(p, b, kvh, ht, ns, flag))
-    merge_partials<D, kThreads>(p, b, h0, gl, ns, reinterpret_cast<float *>(smem));  // the ring is free
+    merge_partials<D, kThreads>(p, b, h0, gl, s_first, ns, reinterpret_cast<float *>(smem));  // the ring is free
 }
 
 int partition_stages(int D, int hpt) { return stages_for(D, hpt); }

@@ -611,7 +611,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_kernel(const __grid_cons
       }
       softmax_bar();  // `red` is read by every warp before it is written again
       if (e.ns > 1 && claim_last_partition(p, e.b, e.kvh, e.ht, e.ns, reinterpret_cast<int *>(words + 1), Warps0to3Sync()))
-        merge_partials<kD, kSoftmaxWarps * 32>(p, e.b, h0, gl, e.ns, reinterpret_cast<float *>(smem + SM::mw),
+        merge_partials<kD, kSoftmaxWarps * 32>(p, e.b, h0, gl, 0, e.ns, reinterpret_cast<float *>(smem + SM::mw),
                                                Warps0to3Sync());
     }
   }
