@@ -51,6 +51,10 @@ def parse():
                     help="first B sequences of the workload (reduced profiling cases); default: the full batch")
     ap.add_argument("--compact-pool", action="store_true",
                     help="block pool = exactly the blocks the batch uses, no page shared (llama8b: no-alias variant)")
+    ap.add_argument("--window", type=int, default=0,
+                    help="sliding window: each sequence attends to its last W tokens (pad_decode_ex)")
+    ap.add_argument("--sinks", action="store_true", help="per-head attention sink logits (pad_decode_ex)")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay of the end-to-end step")
     return ap.parse_args()
 
 
@@ -274,15 +278,26 @@ def main():
         flush.fill_(float(i))
         torch.sum(flush_rd, 0, out=flush_acc)
 
+    sinks_dev = (torch.from_numpy(np.random.default_rng(w.seed).standard_normal(w.Hq).astype(np.float32)).to(dev)
+                 if args.sinks else None)
+
+    def call(stream_):
+        # the public one-call API, with the decode options when asked for
+        return pad.pad_decode(q, k, v, tables, lens, w.scale, num_splits=splits, out=out, lse=lse, stream=stream_,
+                              window=args.window, sinks=sinks_dev)
+
     def step():
         # the whole hot path: one launch (partition + fused reduce)
-        pad.pad_decode_with_workspace(q, k, v, tables, lens, w.scale, splits, out, lse, ws, stream)
+        if args.window or args.sinks:
+            call(stream)
+        else:
+            pad.pad_decode_with_workspace(q, k, v, tables, lens, w.scale, splits, out, lse, ws, stream)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             flush_l2(1)
             step()
-            pad.pad_decode(q, k, v, tables, lens, w.scale, num_splits=splits, out=out, lse=lse, stream=stream)
+            call(stream)
     stream.synchronize()
 
     # ---- timed region: exactly K steps, device events around each launch ----
@@ -303,7 +318,8 @@ def main():
         dist.barrier()
     step_ms = [e[0].elapsed_time(e[1]) for e in events]
     part_ms = step_ms  # the step is exactly one launch of the partition kernel
-    total_ms, all_bytes = max_time_sum_bytes(sum(step_ms), w.algorithmic_bytes() * args.steps, dev, world)
+    alg_bytes = w.algorithmic_bytes(window=args.window, sinks=args.sinks)
+    total_ms, all_bytes = max_time_sum_bytes(sum(step_ms), alg_bytes * args.steps, dev, world)
     value = all_bytes / (total_ms / 1e3) / 1e9
 
     # ---- end to end through the public one-call API, host buffers -----------
@@ -327,7 +343,7 @@ def main():
             q.copy_(hq, non_blocking=True)
             tables.copy_(ht, non_blocking=True)
             lens.copy_(hl, non_blocking=True)
-            pad.pad_decode(q, k, v, tables, lens, w.scale, num_splits=splits, out=out, lse=lse, stream=stream)
+            call(stream)
             hout.copy_(out, non_blocking=True)
             if hlse is not None:
                 hlse.copy_(lse, non_blocking=True)
@@ -339,6 +355,37 @@ def main():
     e2e_total = max_over_ranks(e2e_ms / max(e2e_steps, 1) * args.steps if e2e_steps else 0.0, dev, world)
     e2e_value = all_bytes / (e2e_total / 1e3) / 1e9 if e2e_steps else float("nan")
 
+    # ---- the same end-to-end step captured once as a CUDA graph and replayed
+    # (copies in, the call, copies out): what is left of the host's cost.  The
+    # library's scratch for this shape and stream exists already, so capture
+    # allocates nothing.
+    graph_steps = e2e_steps if not args.no_graph else 0
+    graph_ms = 0.0
+    if graph_steps:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            q.copy_(hq, non_blocking=True)
+            tables.copy_(ht, non_blocking=True)
+            lens.copy_(hl, non_blocking=True)
+            call(stream)
+            hout.copy_(out, non_blocking=True)
+            if hlse is not None:
+                hlse.copy_(lse, non_blocking=True)
+        g_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(graph_steps)]
+        with torch.cuda.stream(stream):
+            for i in range(-3, graph_steps):
+                flush_l2(i)
+                if i >= 0:
+                    g_ev[i][0].record(stream)
+                g.replay()
+                if i >= 0:
+                    g_ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        graph_ms = sum(e[0].elapsed_time(e[1]) for e in g_ev)
+        del g
+    graph_total = max_over_ranks(graph_ms / max(graph_steps, 1) * args.steps if graph_steps else 0.0, dev, world)
+    graph_value = all_bytes / (graph_total / 1e3) / 1e9 if graph_steps else float("nan")
+
     errs = pad.pad_check_device_errors(stream)
     if errs:
         raise SystemExit(f"device error word {errs:#x}")
@@ -347,7 +394,7 @@ def main():
         peak, peak_kind = measured_peaks()
         # the only kernel of the step writes out/lse itself: its algorithmic bytes
         # are the whole call's
-        p_bytes = w.algorithmic_bytes()
+        p_bytes = alg_bytes
         p_ms = statistics.mean(part_ms)
         achieved = p_bytes / (p_ms / 1e3) / 1e9
         sha = kernel_source_sha()
@@ -360,7 +407,9 @@ def main():
             "ms_per_step": round(total_ms / args.steps, 5), "us_per_call": round(total_ms / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded counter-based generator; no dataset)",
-            "config": workload_config(w, plan),
+            "config": {**workload_config(w, plan),
+                       **({"window": args.window, "kv_tokens": w.kv_tokens(args.window)} if args.window else {}),
+                       **({"sinks": "one N(0,1) logit per query head"} if args.sinks else {})},
             "hbm_frac_of_peak": round(value / peak, 4),
             "us_per_call_min_max": [round(min(step_ms) * 1e3, 2), round(max(step_ms) * 1e3, 2)],
             "roofline": {"kernel": kname, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
@@ -369,6 +418,9 @@ def main():
             "e2e": None if not e2e_steps else {
                 "value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "us_per_call": round(e2e_total / args.steps * 1e3, 2), "api": "pad_decode"},
+            "e2e_graph": None if not graph_steps else {
+                "value": round(graph_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "us_per_call": round(graph_total / args.steps * 1e3, 2), "api": "pad_decode, replayed as a CUDA graph"},
             "gpu_launches": args.steps,  # one kernel launch per step
             "clocks": clocks.summary(),
         }

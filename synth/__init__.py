@@ -145,18 +145,24 @@ class Workload:
     def max_blocks_per_seq(self) -> int:
         return self.block_tables.shape[1]
 
-    def kv_tokens(self) -> int:
-        return int(self.seq_lens.astype(np.int64).sum())
-
-    def algorithmic_bytes(self) -> int:
-        """Minimum bytes one call must move (K+V pages read once, q read, out
-        written, live table entries, seq_lens, lse when requested)."""
+    def kv_tokens(self, window: int = 0) -> int:
         L = self.seq_lens.astype(np.int64)
-        kv = int((4 * L * self.Hkv * self.D).sum())
+        return int((np.minimum(L, window) if window > 0 else L).sum())
+
+    def algorithmic_bytes(self, window: int = 0, sinks: bool = False) -> int:
+        """Minimum bytes one call must move (K+V pages read once, q read, out
+        written, live table entries, seq_lens, lse when requested).  With a
+        sliding window only the window's tokens and the table entries of the
+        pages they touch count; sinks add one fp32 logit per query head."""
+        L = self.seq_lens.astype(np.int64)
+        lo = np.maximum(L - window, 0) if window > 0 else np.zeros_like(L)
+        kv = int((4 * (L - lo) * self.Hkv * self.D).sum())
         qo = 4 * self.B * self.Hq * self.D
-        table = int(4 * ((L + self.block_size - 1) // self.block_size).sum())
+        bs = self.block_size
+        pages = np.where(L > lo, (L + bs - 1) // bs - lo // bs, 0)
+        table = int(4 * pages.sum())
         lse = 4 * self.B * self.Hq if self.want_lse else 0
-        return kv + qo + table + 4 * self.B + lse
+        return kv + qo + table + 4 * self.B + lse + (4 * self.Hq if sinks else 0)
 
 
 def make_workload(
