@@ -34,6 +34,17 @@
  *     Z = sum_t exp(s_t - M) + exp(sigma_h - M); out and lse as above.  With
  *     L_b = 0: out = 0, lse = sigma_h.
  *
+ * The cache may also hold 8-bit codes: "perf(rocke): prepare saved paged
+ * decode bindings once" (sections "Summary" and the review's item N1) names an
+ * FP8 decode path beside the non-FP8 one but fixes no format or scale.  The
+ * reading taken: OCP FP8 E4M3 codes (OCP 8-bit Floating Point Specification,
+ * E4M3: sign bit 7, exponent bits 6..3 with bias 7, mantissa bits 2..0,
+ * exponent 0 for the subnormals m/8 * 2^-6, S.1111.111 is NaN, no infinities,
+ * largest finite value 448) and one scale per tensor:
+ *     k_t[d] = k_scale * E4M3(K code),  v_t[d] = v_scale * E4M3(V code),
+ * after which everything above applies unchanged.  A bf16 cache is the same
+ * with both scales 1.
+ *
  * Exact two-pass softmax: no splits, no online rescaling.  bf16 inputs are
  * widened exactly to double.  Strides are in elements; every dimension may be
  * strided.  Work is spread over (b, kh) pairs with pthreads, which changes no
@@ -52,10 +63,24 @@ static double bf16_to_double(uint16_t bits) {
   return (double)f;
 }
 
+/* The value of an E4M3 code, from the format's definition (header). */
+static double e4m3_to_double(uint8_t code) {
+  const int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+  double mag;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0)
+    mag = ldexp((double)m / 8.0, -6);
+  else
+    mag = ldexp(1.0 + (double)m / 8.0, e - 7);
+  return sign ? -mag : mag;
+}
+
 typedef struct {
   const uint16_t *q;
-  const uint16_t *k;
-  const uint16_t *v;
+  const void *k;      /* bf16 bits (uint16) or E4M3 codes (uint8) */
+  const void *v;
+  int kv_fp8;         /* 0: bf16 cache; 1: E4M3 cache */
+  double k_scale, v_scale;
   const int32_t *tables;
   const int32_t *lens;
   int64_t B, Hq, Hkv, D, bs, table_width;
@@ -67,6 +92,13 @@ typedef struct {
   double *out;        /* [B, Hq, D] contiguous */
   double *lse;        /* [B, Hq] */
 } problem;
+
+/* Element idx of a K or V cache, widened exactly to double, times the
+ * tensor's scale. */
+static double kv_value(const problem *p, const void *cache, int64_t idx, double tensor_scale) {
+  if (p->kv_fp8) return tensor_scale * e4m3_to_double(((const uint8_t *)cache)[idx]);
+  return tensor_scale * bf16_to_double(((const uint16_t *)cache)[idx]);
+}
 
 /* One query head of one sequence: the definition above, term by term. */
 static void attend_one(const problem *p, int64_t b, int64_t h, double *s, double *o, double *lse) {
@@ -87,10 +119,10 @@ static void attend_one(const problem *p, int64_t b, int64_t h, double *s, double
   for (int64_t t = lo; t < L; ++t) {
     int64_t phys = p->tables[b * p->table_width + t / p->bs];
     int64_t slot = t % p->bs;
-    const uint16_t *krow = p->k + phys * p->kv_str[0] + kh * p->kv_str[1] + slot * p->kv_str[2];
+    const int64_t krow = phys * p->kv_str[0] + kh * p->kv_str[1] + slot * p->kv_str[2];
     double acc = 0.0;
     for (int64_t d = 0; d < p->D; ++d)
-      acc += bf16_to_double(qrow[d * p->q_str[2]]) * bf16_to_double(krow[d * p->kv_str[3]]);
+      acc += bf16_to_double(qrow[d * p->q_str[2]]) * kv_value(p, p->k, krow + d * p->kv_str[3], p->k_scale);
     s[t - lo] = p->scale * acc;
   }
   const int64_t n = L - lo;
@@ -109,9 +141,9 @@ static void attend_one(const problem *p, int64_t b, int64_t h, double *s, double
   for (int64_t t = lo; t < L; ++t) {
     int64_t phys = p->tables[b * p->table_width + t / p->bs];
     int64_t slot = t % p->bs;
-    const uint16_t *vrow = p->v + phys * p->kv_str[0] + kh * p->kv_str[1] + slot * p->kv_str[2];
+    const int64_t vrow = phys * p->kv_str[0] + kh * p->kv_str[1] + slot * p->kv_str[2];
     double w = s[t - lo] / Z;
-    for (int64_t d = 0; d < p->D; ++d) o[d] += w * bf16_to_double(vrow[d * p->kv_str[3]]);
+    for (int64_t d = 0; d < p->D; ++d) o[d] += w * kv_value(p, p->v, vrow + d * p->kv_str[3], p->v_scale);
   }
   *lse = M + log(Z);
 }
@@ -172,12 +204,16 @@ static int run(const problem *p, const int32_t *pairs, int64_t npairs, int nthre
   return rc;
 }
 
-static int fill(problem *p, const uint16_t *q, const int64_t *q_str, const uint16_t *k,
-                const uint16_t *v, const int64_t *kv_str, const int32_t *tables,
+static int fill(problem *p, const uint16_t *q, const int64_t *q_str, const void *k,
+                const void *v, const int64_t *kv_str, const int32_t *tables,
                 int64_t table_width, const int32_t *lens, int64_t B, int64_t Hq, int64_t Hkv,
-                int64_t D, int64_t bs, double scale, int64_t window, const float *sinks, double *out,
-                double *lse) {
+                int64_t D, int64_t bs, double scale, int64_t window, const float *sinks, int64_t kv_fp8,
+                double k_scale, double v_scale, double *out, double *lse) {
   if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || bs <= 0 || window < 0) return 2;
+  if (kv_fp8 != 0 && kv_fp8 != 1) return 2;
+  p->kv_fp8 = (int)kv_fp8;
+  p->k_scale = k_scale;
+  p->v_scale = v_scale;
   p->window = window;
   p->sinks = sinks;
   p->q = q;
@@ -200,28 +236,30 @@ static int fill(problem *p, const uint16_t *q, const int64_t *q_str, const uint1
 }
 
 /* Every (b, h): out [B, Hq, D] and lse [B, Hq], double.  `window` 0 = every
- * token; `sinks` NULL = none.  Returns 0 on success. */
-int oracle_decode(const uint16_t *q, const int64_t *q_str, const uint16_t *k_cache,
-                  const uint16_t *v_cache, const int64_t *kv_str, const int32_t *block_tables,
-                  int64_t table_width, const int32_t *seq_lens, int64_t B, int64_t Hq, int64_t Hkv,
-                  int64_t D, int64_t bs, double scale, int64_t window, const float *sinks, double *out,
-                  double *lse, int nthreads) {
+ * token; `sinks` NULL = none; `kv_fp8` 0: k_cache/v_cache hold bf16 bits
+ * (uint16), 1: E4M3 codes (uint8), dequantised with k_scale / v_scale (pass 1
+ * for a bf16 cache).  Strides are in elements.  Returns 0 on success. */
+int oracle_decode(const uint16_t *q, const int64_t *q_str, const void *k_cache, const void *v_cache,
+                  const int64_t *kv_str, const int32_t *block_tables, int64_t table_width,
+                  const int32_t *seq_lens, int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t bs,
+                  double scale, int64_t window, const float *sinks, int64_t kv_fp8, double k_scale,
+                  double v_scale, double *out, double *lse, int nthreads) {
   problem p;
   int rc = fill(&p, q, q_str, k_cache, v_cache, kv_str, block_tables, table_width, seq_lens, B,
-                Hq, Hkv, D, bs, scale, window, sinks, out, lse);
+                Hq, Hkv, D, bs, scale, window, sinks, kv_fp8, k_scale, v_scale, out, lse);
   return rc ? rc : run(&p, NULL, 0, nthreads);
 }
 
 /* Selected (b, h) pairs only: out [npairs, D], lse [npairs]. */
-int oracle_decode_pairs(const uint16_t *q, const int64_t *q_str, const uint16_t *k_cache,
-                        const uint16_t *v_cache, const int64_t *kv_str,
-                        const int32_t *block_tables, int64_t table_width, const int32_t *seq_lens,
-                        int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t bs, double scale,
-                        int64_t window, const float *sinks, const int32_t *pairs, int64_t npairs,
-                        double *out, double *lse, int nthreads) {
+int oracle_decode_pairs(const uint16_t *q, const int64_t *q_str, const void *k_cache,
+                        const void *v_cache, const int64_t *kv_str, const int32_t *block_tables,
+                        int64_t table_width, const int32_t *seq_lens, int64_t B, int64_t Hq,
+                        int64_t Hkv, int64_t D, int64_t bs, double scale, int64_t window,
+                        const float *sinks, int64_t kv_fp8, double k_scale, double v_scale,
+                        const int32_t *pairs, int64_t npairs, double *out, double *lse, int nthreads) {
   problem p;
   int rc = fill(&p, q, q_str, k_cache, v_cache, kv_str, block_tables, table_width, seq_lens, B,
-                Hq, Hkv, D, bs, scale, window, sinks, out, lse);
+                Hq, Hkv, D, bs, scale, window, sinks, kv_fp8, k_scale, v_scale, out, lse);
   for (int64_t i = 0; !rc && i < npairs; ++i)
     if (pairs[2 * i] < 0 || pairs[2 * i] >= B || pairs[2 * i + 1] < 0 || pairs[2 * i + 1] >= Hq)
       rc = 2;

@@ -15,15 +15,20 @@ prepare saved paged decode bindings once", section "Runnable saved-binding
 HIP-event comparison"). No dataset or checkpoint is involved.
 
 Poisoning: every table entry past ceil(L_b / block_size) points at an extra
-physical block filled with bf16 NaN, and (unless a block is shared by several
-sequences) the cache slots past L_b inside a sequence's last block are NaN too.
-A kernel that reads either place produces NaN and fails parity instead of
-reading out of bounds.
+physical block filled with NaN (bf16 NaN, or the E4M3 NaN code), and (unless a
+block is shared by several sequences) the cache slots past L_b inside a
+sequence's last block are NaN too.  A kernel that reads either place produces
+NaN and fails parity instead of reading out of bounds.
+
+An 8-bit cache (``kv_dtype="e4m3"``) holds OCP FP8 E4M3 codes with one scale per
+tensor: the codes are the seeded samples divided by ``k_scale`` / ``v_scale``
+and rounded onto the E4M3 grid, so ``scale * code`` approximates the sample.
 """
 from __future__ import annotations
 
 import ctypes
 import dataclasses
+import functools
 import math
 import os
 import subprocess
@@ -38,6 +43,10 @@ _LIB = os.path.join(_HERE, "libsynth.so")
 DIST_NORMAL = 0
 DIST_UNIFORM_PM1 = 1
 BF16_NAN = 0x7FC0
+E4M3_NAN = 0x7F
+# default per-tensor scales of an E4M3 cache: not powers of two, exact in fp32
+E4M3_K_SCALE = 3.0 / 64.0
+E4M3_V_SCALE = 5.0 / 256.0
 
 # stream ids: one independent counter space per drawn quantity
 S_Q, S_K, S_V, S_LENS, S_PERM, S_EXTRA = 1, 2, 3, 4, 5, 6
@@ -64,6 +73,8 @@ def _l():
         p = ctypes.c_void_p
         lib.synth_fill_bf16.argtypes = [p, i64, i64, u64, u64, ctypes.c_int, ctypes.c_int]
         lib.synth_fill_blocks_bf16.argtypes = [p, p, i64, i64, u64, u64, ctypes.c_int, ctypes.c_int]
+        lib.synth_fill_blocks_e4m3.argtypes = [p, p, i64, i64, u64, u64, ctypes.c_int, ctypes.c_double,
+                                               ctypes.c_int]
         lib.synth_uniform_f64.argtypes = [p, i64, u64, u64]
         lib.synth_permutation_prefix.argtypes = [p, p, i64, i64, u64, u64]
         lib.synth_uniform_int.argtypes = [p, i64, i32, i32, u64, u64]
@@ -114,7 +125,8 @@ def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
 
 @dataclasses.dataclass
 class Workload:
-    """One decode step's inputs (host arrays, raw bf16 bits as uint16)."""
+    """One decode step's inputs (host arrays: raw bf16 bits as uint16; an E4M3
+    cache as uint8 codes)."""
 
     name: str
     B: int
@@ -123,8 +135,8 @@ class Workload:
     D: int
     block_size: int
     q: np.ndarray             # uint16 [B, Hq, D]
-    k_cache: np.ndarray       # uint16 [num_blocks, Hkv, block_size, D] (logical order)
-    v_cache: np.ndarray       # uint16 same shape
+    k_cache: np.ndarray       # uint16 bf16 / uint8 E4M3 [num_blocks, Hkv, block_size, D] (logical order)
+    v_cache: np.ndarray       # same dtype and shape
     block_tables: np.ndarray  # int32 [B, max_blocks_per_seq]
     seq_lens: np.ndarray      # int32 [B]
     scale: float
@@ -132,6 +144,13 @@ class Workload:
     want_lse: bool
     seed: int
     recipe: str = ""
+    kv_dtype: str = "bf16"    # "bf16" or "e4m3"
+    k_scale: float = 1.0      # dequantisation scales of an E4M3 cache (1 for bf16)
+    v_scale: float = 1.0
+
+    @property
+    def kv_elem_bytes(self) -> int:
+        return 1 if self.kv_dtype == "e4m3" else 2
 
     @property
     def num_blocks(self) -> int:
@@ -156,7 +175,7 @@ class Workload:
         pages they touch count; sinks add one fp32 logit per query head."""
         L = self.seq_lens.astype(np.int64)
         lo = np.maximum(L - window, 0) if window > 0 else np.zeros_like(L)
-        kv = int((4 * (L - lo) * self.Hkv * self.D).sum())
+        kv = int((2 * self.kv_elem_bytes * (L - lo) * self.Hkv * self.D).sum())
         qo = 4 * self.B * self.Hq * self.D
         bs = self.block_size
         pages = np.where(L > lo, (L + bs - 1) // bs - lo // bs, 0)
@@ -185,6 +204,9 @@ def make_workload(
     want_lse: bool = True,
     poison: bool = True,
     recipe: str = "",
+    kv_dtype: str = "bf16",
+    k_scale: Optional[float] = None,
+    v_scale: Optional[float] = None,
 ) -> Workload:
     """Build a workload.
 
@@ -222,33 +244,45 @@ def make_workload(
         tables[b, :n] = ids[off:off + n]
         off += n
 
+    if kv_dtype not in ("bf16", "e4m3"):
+        raise ValueError(kv_dtype)
+    fp8 = kv_dtype == "e4m3"
+    ks = float(np.float32(k_scale if k_scale is not None else (E4M3_K_SCALE if fp8 else 1.0)))
+    vs = float(np.float32(v_scale if v_scale is not None else (E4M3_V_SCALE if fp8 else 1.0)))
     shape = (num_blocks, Hkv, bs, D)
-    k = np.zeros(shape, dtype=np.uint16)
-    v = np.zeros(shape, dtype=np.uint16)
+    k = np.zeros(shape, dtype=np.uint8 if fp8 else np.uint16)
+    v = np.zeros_like(k)
     used = np.unique(ids.astype(np.int64)) if demand else np.zeros(0, np.int64)
     block_elems = Hkv * bs * D
     lib = _l()
     if used.size:
         used = np.ascontiguousarray(used)
-        lib.synth_fill_blocks_bf16(k.ctypes.data, used.ctypes.data, used.size, block_elems, seed, S_K, k_dist, _threads())
-        lib.synth_fill_blocks_bf16(v.ctypes.data, used.ctypes.data, used.size, block_elems, seed, S_V, v_dist, _threads())
+        for arr, stream, dist, sc in ((k, S_K, k_dist, ks), (v, S_V, v_dist, vs)):
+            if fp8:
+                lib.synth_fill_blocks_e4m3(arr.ctypes.data, used.ctypes.data, used.size, block_elems, seed, stream,
+                                           dist, 1.0 / sc, _threads())
+            else:
+                lib.synth_fill_blocks_bf16(arr.ctypes.data, used.ctypes.data, used.size, block_elems, seed, stream,
+                                           dist, _threads())
+    nan = E4M3_NAN if fp8 else BF16_NAN
     if poison:
-        k[poison_block] = BF16_NAN
-        v[poison_block] = BF16_NAN
+        k[poison_block] = nan
+        v[poison_block] = nan
         counts = np.bincount(ids.astype(np.int64), minlength=num_blocks) if demand else None
         for b in range(B):
             L = int(seq_lens[b])
             if L % bs and counts is not None:
                 last = int(tables[b, L // bs])
                 if counts[last] == 1:
-                    k[last, :, L % bs:, :] = BF16_NAN
-                    v[last, :, L % bs:, :] = BF16_NAN
+                    k[last, :, L % bs:, :] = nan
+                    v[last, :, L % bs:, :] = nan
     q = bf16_array((B, Hq, D), seed, S_Q)
     return Workload(
         name=name, B=B, Hq=Hq, Hkv=Hkv, D=D, block_size=bs, q=q, k_cache=k, v_cache=v,
         block_tables=tables, seq_lens=seq_lens,
         scale=float(scale if scale is not None else 1.0 / math.sqrt(D)),
         num_splits=num_splits, want_lse=want_lse, seed=seed, recipe=recipe,
+        kv_dtype=kv_dtype, k_scale=ks, v_scale=vs,
     )
 
 
@@ -260,7 +294,7 @@ CONFIG_NAMES = ("tiny", "llama8b", "qwen14b", "longctx_d256", "ragged_mqa")
 
 
 def config(name: str, seed: Optional[int] = None, batch: Optional[int] = None,
-           compact_pool: bool = False) -> Workload:
+           compact_pool: bool = False, kv_dtype: str = "bf16") -> Workload:
     """The named decode workloads (seeds 0..4 by default).
 
     `batch` keeps every other parameter and takes the first `batch` sequences
@@ -268,7 +302,17 @@ def config(name: str, seed: Optional[int] = None, batch: Optional[int] = None,
     batch's).  `compact_pool` makes the block pool exactly the blocks the batch
     uses, drawn without replacement: no page is shared between sequences and the
     device holds only what is read.  Both serve reduced profiling cases; the
-    llama8b workload with `compact_pool` is also its no-alias variant."""
+    llama8b workload with `compact_pool` is also its no-alias variant.
+    `kv_dtype="e4m3"` stores the same samples as E4M3 codes with the default
+    per-tensor scales (the 8-bit-cache variant of each workload)."""
+    w = _config(name, seed, batch, compact_pool, kv_dtype)
+    if kv_dtype == "e4m3":
+        w.recipe += f"; E4M3 cache, codes = RNE(sample / scale), k_scale {w.k_scale:g}, v_scale {w.v_scale:g}"
+    return w
+
+
+def _config(name, seed, batch, compact_pool, kv_dtype):
+    make_workload = functools.partial(_make_workload, kv_dtype=kv_dtype)
     idx = CONFIG_NAMES.index(name)
     seed = idx if seed is None else seed
 
@@ -312,3 +356,6 @@ def config(name: str, seed: Optional[int] = None, batch: Optional[int] = None,
             num_splits=0,
             recipe="B256 Hq32/Hkv1 D128 bs32, L log-uniform [16,32768], N(0,1), without replacement from a 300000-block pool")
     raise KeyError(name)
+
+
+_make_workload = make_workload

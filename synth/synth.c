@@ -15,6 +15,10 @@
  *   normal:              Box-Muller, sqrt(-2 ln u1) * cos(2 pi u2), with u1,u2
  *                        from the hashes of counters 2i and 2i+1
  *   bf16:                round-to-nearest-even of the fp32 value
+ *   E4M3 codes:          the sample times a gain (1 / the tensor's scale),
+ *                        rounded to nearest even onto the OCP FP8 E4M3 grid
+ *                        (3 mantissa bits, exponent bias 7, subnormals below
+ *                        2^-6), saturated at +-448, never NaN
  */
 #include <math.h>
 #include <pthread.h>
@@ -57,10 +61,30 @@ static inline uint16_t f32_to_bf16_rne(float f) {
   return (uint16_t)(b >> 16);
 }
 
+static inline uint8_t f64_to_e4m3_rne(double x) {
+  const uint8_t sign = signbit(x) ? 0x80 : 0;
+  const double a = fabs(x);
+  if (!(a > 0.0)) return sign;
+  if (a >= 448.0) return sign | 0x7E;
+  int e;
+  frexp(a, &e);
+  int E = e - 1; /* a in [2^E, 2^(E+1)) */
+  if (E < -6) return sign | (uint8_t)nearbyint(a * 512.0); /* quantum 2^-9; 8 is the smallest normal */
+  double m = nearbyint((a / ldexp(1.0, E) - 1.0) * 8.0);
+  if (m == 8.0) {
+    m = 0.0;
+    E += 1;
+  }
+  if (E > 8 || (E == 8 && m > 6.0)) return sign | 0x7E;
+  return sign | (uint8_t)(((E + 7) << 3) | (int)m);
+}
+
 /* ---- threaded driver ---------------------------------------------------- */
 
 typedef struct {
-  uint16_t *dst;
+  void *dst;             /* uint16 bf16 bits, or uint8 E4M3 codes when e4m3 */
+  int e4m3;
+  double gain;           /* E4M3 only: the sample is multiplied by it before rounding */
   const int64_t *blocks; /* NULL: dst is one flat range starting at counter `first` */
   int64_t nunits;        /* number of blocks, or number of elements when blocks==NULL */
   int64_t unit_elems;    /* elements per block (1 when blocks==NULL) */
@@ -70,19 +94,24 @@ typedef struct {
   int nthreads, tid;
 } fill_job;
 
+static inline void put(const fill_job *j, int64_t at, int64_t counter) {
+  const double x = sample(j->key, (uint64_t)counter, j->dist);
+  if (j->e4m3)
+    ((uint8_t *)j->dst)[at] = f64_to_e4m3_rne(x * j->gain);
+  else
+    ((uint16_t *)j->dst)[at] = f32_to_bf16_rne((float)x);
+}
+
 static void *fill_worker(void *arg) {
   fill_job *j = (fill_job *)arg;
   int64_t lo = j->nunits * j->tid / j->nthreads;
   int64_t hi = j->nunits * (j->tid + 1) / j->nthreads;
   for (int64_t u = lo; u < hi; ++u) {
     if (j->blocks) {
-      int64_t blk = j->blocks[u];
-      uint16_t *out = j->dst + blk * j->unit_elems;
-      int64_t base = blk * j->unit_elems;
-      for (int64_t e = 0; e < j->unit_elems; ++e)
-        out[e] = f32_to_bf16_rne((float)sample(j->key, (uint64_t)(base + e), j->dist));
+      int64_t base = j->blocks[u] * j->unit_elems;
+      for (int64_t e = 0; e < j->unit_elems; ++e) put(j, base + e, base + e);
     } else {
-      j->dst[u] = f32_to_bf16_rne((float)sample(j->key, (uint64_t)(j->first + u), j->dist));
+      put(j, u, j->first + u);
     }
   }
   return NULL;
@@ -107,7 +136,7 @@ static void run_fill(fill_job proto, int nthreads) {
 /* Fill dst[0..n) with bf16 samples of counters first..first+n-1. */
 void synth_fill_bf16(uint16_t *dst, int64_t n, int64_t first, uint64_t seed, uint64_t stream,
                      int dist, int nthreads) {
-  fill_job j = {dst, NULL, n, 1, first, stream_key(seed, stream), dist, 1, 0};
+  fill_job j = {dst, 0, 1.0, NULL, n, 1, first, stream_key(seed, stream), dist, 1, 0};
   run_fill(j, nthreads);
 }
 
@@ -116,7 +145,15 @@ void synth_fill_bf16(uint16_t *dst, int64_t n, int64_t first, uint64_t seed, uin
 void synth_fill_blocks_bf16(uint16_t *dst, const int64_t *blocks, int64_t nblocks,
                             int64_t block_elems, uint64_t seed, uint64_t stream, int dist,
                             int nthreads) {
-  fill_job j = {dst, blocks, nblocks, block_elems, 0, stream_key(seed, stream), dist, 1, 0};
+  fill_job j = {dst, 0, 1.0, blocks, nblocks, block_elems, 0, stream_key(seed, stream), dist, 1, 0};
+  run_fill(j, nthreads);
+}
+
+/* As synth_fill_blocks_bf16, with E4M3 codes of gain * sample (uint8). */
+void synth_fill_blocks_e4m3(uint8_t *dst, const int64_t *blocks, int64_t nblocks,
+                            int64_t block_elems, uint64_t seed, uint64_t stream, int dist,
+                            double gain, int nthreads) {
+  fill_job j = {dst, 1, gain, blocks, nblocks, block_elems, 0, stream_key(seed, stream), dist, 1, 0};
   run_fill(j, nthreads);
 }
 

@@ -93,4 +93,5 @@ def sample_pairs(w: synth.Workload, n: int, seed: int):
 
 
 def oracle_pairs(w: synth.Workload, pairs):
-    return oracle.decode_pairs(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, pairs)
+    return oracle.decode_pairs(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale, pairs,
+                               k_scale=w.k_scale, v_scale=w.v_scale)

@@ -22,6 +22,13 @@ section "Summary"):
 * attention sinks: equals scipy's softmax over the scores with the sink logit
   appended (zero value row); a -inf sink changes nothing; an empty sequence
   gives out = 0, lse = sink.
+* E4M3 cache: every one of the 256 codes, read back through one-token
+  sequences, equals torch's float8_e4m3fn widening (and the values the OCP FP8
+  definition fixes: 448, 2^-9, 2^-6, +-1, two NaNs) times the tensor's scale;
+  the paged oracle equals SDPA on the dequantised contiguous K/V; a
+  power-of-two k_scale is the same as scaling the scores, v_scale scales out
+  and leaves lse alone; with both scales 1 it equals the bf16 path on the same
+  values, bitwise.
 
 ``test_planted_mistakes_are_caught`` compiles copies of the oracle with one
 plausible mistake each and checks that some pin fails for every one.
@@ -50,16 +57,18 @@ def _f(bits):
 
 def scatter_to_pages(k_contig, v_contig, lens, bs, extra_blocks, seed):
     """Separate routine (not the oracle's gather): place contiguous per-sequence
-    K/V [B, Hkv, Lmax, D] into a paged cache at randomly chosen physical blocks."""
+    K/V [B, Hkv, Lmax, D] (bf16 bits or E4M3 codes) into a paged cache at
+    randomly chosen physical blocks."""
     B, Hkv, Lmax, D = k_contig.shape
+    nan = synth.E4M3_NAN if k_contig.dtype == np.uint8 else synth.BF16_NAN
     need = [(int(L) + bs - 1) // bs for L in lens]
     nblocks = sum(need) + extra_blocks
     perm = _rng(seed).permutation(nblocks)
     width = max(max(need), 1)
     # entries past the live blocks point at a NaN-filled spare block
     tables = np.full((B, width), int(perm[-1]), dtype=np.int32)
-    kc = np.full((nblocks, Hkv, bs, D), synth.BF16_NAN, dtype=np.uint16)
-    vc = np.full((nblocks, Hkv, bs, D), synth.BF16_NAN, dtype=np.uint16)
+    kc = np.full((nblocks, Hkv, bs, D), nan, dtype=k_contig.dtype)
+    vc = np.full((nblocks, Hkv, bs, D), nan, dtype=k_contig.dtype)
     nxt = 0
     for b in range(B):
         for j in range(need[b]):
@@ -72,9 +81,12 @@ def scatter_to_pages(k_contig, v_contig, lens, bs, extra_blocks, seed):
     return kc, vc, tables
 
 
-def library_attention(q, k_contig, v_contig, lens, scale):
+def library_attention(q, k_contig, v_contig, lens, scale, kf=None, vf=None):
     """torch float64 SDPA (+ torch.logsumexp) on contiguous K/V, per sequence.
-    Query head h reads KV head h // (Hq/Hkv) via repeat_interleave."""
+    Query head h reads KV head h // (Hq/Hkv) via repeat_interleave.  kf / vf
+    widen the stored K / V elements (default: bf16 bits)."""
+    kf = kf or _f
+    vf = vf or _f
     B, Hq, D = q.shape
     Hkv = k_contig.shape[1]
     g = Hq // Hkv
@@ -83,8 +95,8 @@ def library_attention(q, k_contig, v_contig, lens, scale):
     for b in range(B):
         L = int(lens[b])
         qt = torch.from_numpy(_f(q[b]))[:, None, :]                      # [Hq, 1, D]
-        kt = torch.from_numpy(_f(k_contig[b, :, :L])).repeat_interleave(g, 0)  # [Hq, L, D]
-        vt = torch.from_numpy(_f(v_contig[b, :, :L])).repeat_interleave(g, 0)
+        kt = torch.from_numpy(kf(k_contig[b, :, :L])).repeat_interleave(g, 0)  # [Hq, L, D]
+        vt = torch.from_numpy(vf(v_contig[b, :, :L])).repeat_interleave(g, 0)
         o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=scale)
         out[b] = o[:, 0, :].numpy()
         lse[b] = torch.logsumexp(scale * (qt @ kt.transpose(1, 2))[:, 0, :], dim=-1).numpy()
@@ -329,9 +341,102 @@ def pin_sink_limits(lib):
     assert np.all(out[1] == 0.0) and np.array_equal(lse[1], sinks.astype(np.float64))
 
 
+# ---- E4M3 cache ("perf(rocke): prepare saved paged decode bindings once" names
+# an FP8 decode path; format and per-tensor scales are the reading in the
+# oracle's header)
+
+def _e4m3_ref(codes):
+    """torch's widening of E4M3 codes (uint8) to float64."""
+    return torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def _e4m3_codes(x):
+    """torch's round-to-nearest of float values onto E4M3 codes."""
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def pin_e4m3_code_values(lib):
+    codes = np.arange(256, dtype=np.uint8)
+    ref = _e4m3_ref(codes)
+    # the library agrees with values the format's definition fixes
+    for c, val in {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0, 0x40: 2.0,
+                   0x7E: 448.0, 0xB8: -1.0, 0xFE: -448.0}.items():
+        assert ref[c] == val
+    assert np.isnan(ref[0x7F]) and np.isnan(ref[0xFF]) and int(np.isnan(ref).sum()) == 2
+    assert math.copysign(1.0, ref[0x80]) < 0 and ref[0x80] == 0.0
+    # head h reads KV head h; one token; q = e_0 (bf16 1.0 at d = 0)
+    D, H = 8, 256
+    q = np.zeros((1, H, D), np.uint16)
+    q[0, :, 0] = 0x3F80
+    tables, lens = np.asarray([[0]], np.int32), np.asarray([1], np.int32)
+    ks, vs, scale = 0.75, 0.3, 0.5
+    # K codes vary, V zero: lse_h = scale * k_scale * value(code h)
+    k = np.zeros((2, H, 1, D), np.uint8)
+    k[0, :, 0, 0] = codes
+    _, lse = oracle.decode(q, k, np.zeros_like(k), tables, lens, scale, lib_path=lib, k_scale=ks, v_scale=vs)
+    np.testing.assert_array_equal(lse[0], scale * (ks * ref))
+    # K zero, V codes vary: weight 1, out_h[0] = v_scale * value(code h)
+    v = np.zeros((2, H, 1, D), np.uint8)
+    v[0, :, 0, 0] = codes
+    out, lse = oracle.decode(q, np.zeros_like(v), v, tables, lens, scale, lib_path=lib, k_scale=ks, v_scale=vs)
+    np.testing.assert_array_equal(out[0, :, 0], vs * ref)
+    assert np.all(lse == 0.0)
+
+
+E4M3_CASES = [
+    # B, Hq, Hkv, D, bs, lens, k_scale, v_scale
+    (2, 4, 1, 16, 4, [5, 15], 0.046875, 0.01953125),
+    (3, 8, 2, 32, 16, [16, 17, 40], 0.1, 0.02),
+    (2, 6, 6, 8, 1, [7, 3], 1.0, 1.0),
+]
+
+
+def pin_e4m3_bruteforce(lib):
+    for i, (B, Hq, Hkv, D, bs, lens, ks, vs) in enumerate(E4M3_CASES):
+        lens = np.asarray(lens, dtype=np.int32)
+        r = _rng(700 + i)
+        Lmax = int(lens.max())
+        q = _bf16(r.standard_normal((B, Hq, D)))
+        kc = _e4m3_codes(r.standard_normal((B, Hkv, Lmax, D)) / ks)
+        vc = _e4m3_codes(r.standard_normal((B, Hkv, Lmax, D)) / vs)
+        kp, vp, tables = scatter_to_pages(kc, vc, lens, bs, extra_blocks=2, seed=800 + i)
+        scale = 1.0 / math.sqrt(D)
+        out, lse = oracle.decode(q, kp, vp, tables, lens, scale, lib_path=lib, k_scale=ks, v_scale=vs)
+        ref_out, ref_lse = library_attention(q, kc, vc, lens, scale, kf=lambda c: ks * _e4m3_ref(c),
+                                             vf=lambda c: vs * _e4m3_ref(c))
+        np.testing.assert_allclose(out, ref_out, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-12)
+
+
+def pin_e4m3_scales(lib):
+    w = synth.make_workload("e4m3s", 3, 8, 2, 32, 8, [20, 1, 37], seed=22, kv_dtype="e4m3", k_scale=1.0,
+                            v_scale=1.0)
+    base = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, 0.125, lib_path=lib)
+    # k_scale = 2^j is the score scale times 2^j, exactly
+    a = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, 0.125, lib_path=lib, k_scale=0.25)
+    b = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, 0.125 * 0.25, lib_path=lib)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    assert not np.allclose(a[1], base[1])
+    # v_scale multiplies out and leaves lse alone
+    c = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, 0.125, lib_path=lib, v_scale=0.37)
+    np.testing.assert_allclose(c[0], 0.37 * base[0], rtol=0, atol=1e-14)
+    assert np.array_equal(c[1], base[1])
+
+
+def pin_e4m3_equals_bf16_of_same_values(lib):
+    w8 = synth.make_workload("e4m3b", 3, 8, 2, 32, 4, [9, 30, 17], seed=23, kv_dtype="e4m3", k_scale=1.0,
+                             v_scale=1.0, poison=False)
+    kb = _bf16(_e4m3_ref(w8.k_cache))  # E4M3 values are exact in bf16
+    vb = _bf16(_e4m3_ref(w8.v_cache))
+    a = oracle.decode(w8.q, w8.k_cache, w8.v_cache, w8.block_tables, w8.seq_lens, w8.scale, lib_path=lib)
+    b = oracle.decode(w8.q, kb, vb, w8.block_tables, w8.seq_lens, w8.scale, lib_path=lib)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
 PINS = [pin_bruteforce, pin_weights_are_softmax, pin_permutation_invariance, pin_layout_invariance,
         pin_constant_v, pin_zero_query, pin_single_token, pin_dominant_score, pin_empty_sequence,
-        pin_split_combine, pin_window_bruteforce, pin_window_one, pin_sinks_are_softmax_terms, pin_sink_limits]
+        pin_split_combine, pin_window_bruteforce, pin_window_one, pin_sinks_are_softmax_terms, pin_sink_limits,
+        pin_e4m3_code_values, pin_e4m3_bruteforce, pin_e4m3_scales, pin_e4m3_equals_bf16_of_same_values]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -362,15 +467,15 @@ def test_thread_count_does_not_change_results():
 MUTATIONS = {
     "scale_dropped": ("s[t - lo] = p->scale * acc;", "s[t - lo] = acc;"),
     "head_map_modulo": ("const int64_t kh = h / g;", "const int64_t kh = h % p->Hkv;"),
-    "slot_from_division": ("int64_t slot = t % p->bs;\n    const uint16_t *krow",
-                           "int64_t slot = (t / p->bs) % p->bs;\n    const uint16_t *krow"),
-    "first_page_only": ("int64_t phys = p->tables[b * p->table_width + t / p->bs];\n    int64_t slot = t % p->bs;\n    const uint16_t *vrow",
-                        "int64_t phys = p->tables[b * p->table_width];\n    int64_t slot = t % p->bs;\n    const uint16_t *vrow"),
+    "slot_from_division": ("int64_t slot = t % p->bs;\n    const int64_t krow",
+                           "int64_t slot = (t / p->bs) % p->bs;\n    const int64_t krow"),
+    "first_page_only": ("int64_t phys = p->tables[b * p->table_width + t / p->bs];\n    int64_t slot = t % p->bs;\n    const int64_t vrow",
+                        "int64_t phys = p->tables[b * p->table_width];\n    int64_t slot = t % p->bs;\n    const int64_t vrow"),
     "unnormalised_weights": ("double w = s[t - lo] / Z;", "double w = s[t - lo];"),
     "lse_without_max": ("*lse = M + log(Z);", "*lse = log(Z);"),
     "lse_log2": ("*lse = M + log(Z);", "*lse = M + log2(Z);"),
-    "last_token_dropped": ("for (int64_t t = lo; t < L; ++t) {\n    int64_t phys = p->tables[b * p->table_width + t / p->bs];\n    int64_t slot = t % p->bs;\n    const uint16_t *vrow",
-                           "for (int64_t t = lo; t < L - 1; ++t) {\n    int64_t phys = p->tables[b * p->table_width + t / p->bs];\n    int64_t slot = t % p->bs;\n    const uint16_t *vrow"),
+    "last_token_dropped": ("for (int64_t t = lo; t < L; ++t) {\n    int64_t phys = p->tables[b * p->table_width + t / p->bs];\n    int64_t slot = t % p->bs;\n    const int64_t vrow",
+                           "for (int64_t t = lo; t < L - 1; ++t) {\n    int64_t phys = p->tables[b * p->table_width + t / p->bs];\n    int64_t slot = t % p->bs;\n    const int64_t vrow"),
     "max_over_first_half": ("for (int64_t t = 1; t < n; ++t)\n    if (s[t] > M) M = s[t];",
                             "for (int64_t t = 1; t < n / 2; ++t)\n    if (s[t] > M) M = s[t];"),
     "window_off_by_one": ("L > p->window) ? L - p->window : 0;", "L > p->window) ? L - p->window + 1 : 0;"),
@@ -382,6 +487,13 @@ MUTATIONS = {
     "empty_sequence_drops_sink": ("*lse = has_sink ? sink : -INFINITY;", "*lse = -INFINITY;"),
     "query_of_kv_head": ("h * p->q_str[1];", "kh * p->q_str[1];"),
     "exp_without_shift": ("s[t] = exp(s[t] - M);", "s[t] = exp(s[t]);"),
+    "e4m3_subnormal_as_normal": ("mag = ldexp((double)m / 8.0, -6);", "mag = ldexp(1.0 + (double)m / 8.0, -7);"),
+    "e4m3_bias_8": ("mag = ldexp(1.0 + (double)m / 8.0, e - 7);", "mag = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    "e4m3_nan_as_number": ("if (e == 15 && m == 7) return NAN;", ""),
+    "e4m3_sign_dropped": ("return sign ? -mag : mag;", "return mag;"),
+    "k_scale_dropped": ("krow + d * p->kv_str[3], p->k_scale)", "krow + d * p->kv_str[3], 1.0)"),
+    "v_scale_on_keys": ("krow + d * p->kv_str[3], p->k_scale)", "krow + d * p->kv_str[3], p->v_scale)"),
+    "v_scale_dropped": ("vrow + d * p->kv_str[3], p->v_scale)", "vrow + d * p->kv_str[3], 1.0)"),
 }
 
 
