@@ -55,6 +55,8 @@ def parse():
                     help="sliding window: each sequence attends to its last W tokens (pad_decode_ex)")
     ap.add_argument("--sinks", action="store_true", help="per-head attention sink logits (pad_decode_ex)")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay of the end-to-end step")
+    ap.add_argument("--kv-dtype", default="bf16", choices=["bf16", "e4m3"],
+                    help="KV cache element type (e4m3: OCP FP8 E4M3 codes with per-tensor scales)")
     return ap.parse_args()
 
 
@@ -185,7 +187,7 @@ def run_reference(args, rank, world):
     metric = "decode attention µs/call and achieved HBM GB/s vs B200 peak (1 GPU)"
     if rank != 0:
         return
-    w = synth.config(args.workload, batch=args.batch, compact_pool=args.compact_pool)
+    w = synth.config(args.workload, batch=args.batch, compact_pool=args.compact_pool, kv_dtype=args.kv_dtype)
     cb = cpu_baseline(w, args.cpu_seconds)
     us = cb["us_per_call"]
     line = {"impl": "reference", "metric": metric, "value": cb["value"], "unit": "GB/s", "n_gpus": args.gpus,
@@ -251,18 +253,22 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     # weak scaling: every rank decodes its own batch of the same shape
-    base = synth.config(args.workload, batch=args.batch, compact_pool=args.compact_pool)
+    base = synth.config(args.workload, batch=args.batch, compact_pool=args.compact_pool, kv_dtype=args.kv_dtype)
     w = synth.config(args.workload, seed=rank_seed(base.seed, rank), batch=args.batch,
-                     compact_pool=args.compact_pool) if rank else base
+                     compact_pool=args.compact_pool, kv_dtype=args.kv_dtype) if rank else base
     splits = w.num_splits if args.num_splits is None else args.num_splits
     plan = pad.pad_decode_plan(w.B, w.Hq, w.Hkv, w.D, w.block_size, w.max_blocks_per_seq, num_splits=splits,
-                               device=local)
+                               device=local, kv_dtype=args.kv_dtype)
+    fp8 = args.kv_dtype == "e4m3"
     S = plan["num_splits"]
 
     def dev_bf16(a):
         return torch.from_numpy(a).view(torch.bfloat16).to(dev)
 
-    q, k, v = dev_bf16(w.q), dev_bf16(w.k_cache), dev_bf16(w.v_cache)
+    def dev_kv(a):
+        return torch.from_numpy(a).view(torch.float8_e4m3fn if fp8 else torch.bfloat16).to(dev)
+
+    q, k, v = dev_bf16(w.q), dev_kv(w.k_cache), dev_kv(w.v_cache)
     tables = torch.from_numpy(w.block_tables).to(dev)
     lens = torch.from_numpy(w.seq_lens).to(dev)
     out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
@@ -284,11 +290,12 @@ def main():
     def call(stream_):
         # the public one-call API, with the decode options when asked for
         return pad.pad_decode(q, k, v, tables, lens, w.scale, num_splits=splits, out=out, lse=lse, stream=stream_,
-                              window=args.window, sinks=sinks_dev)
+                              window=args.window, sinks=sinks_dev, k_scale=w.k_scale if fp8 else 0.0,
+                              v_scale=w.v_scale if fp8 else 0.0)
 
     def step():
         # the whole hot path: one launch (partition + fused reduce)
-        if args.window or args.sinks:
+        if args.window or args.sinks or fp8:
             call(stream)
         else:
             pad.pad_decode_with_workspace(q, k, v, tables, lens, w.scale, splits, out, lse, ws, stream)
@@ -399,17 +406,19 @@ def main():
         achieved = p_bytes / (p_ms / 1e3) / 1e9
         sha = kernel_source_sha()
         # the recorded ncu traffic is for the named workload at full size
-        traffic = traffic_from_profiles(w.name, sha) if args.batch is None and not args.compact_pool else None
+        traffic = (traffic_from_profiles(w.name + ("_e4m3" if fp8 else ""), sha)
+                   if args.batch is None and not args.compact_pool else None)
         kname = f"partition_kernel<{w.D},{plan['heads_per_tile']}>"
         line = {
             "metric": "decode attention µs/call and achieved HBM GB/s vs B200 peak (1 GPU)",
             "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(total_ms / args.steps, 5), "us_per_call": round(total_ms / args.steps * 1e3, 2),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16",
             "data": "synthetic (seeded counter-based generator; no dataset)",
             "config": {**workload_config(w, plan),
                        **({"window": args.window, "kv_tokens": w.kv_tokens(args.window)} if args.window else {}),
-                       **({"sinks": "one N(0,1) logit per query head"} if args.sinks else {})},
+                       **({"sinks": "one N(0,1) logit per query head"} if args.sinks else {}),
+                       **({"kv_cache": f"e4m3, k_scale {w.k_scale:g}, v_scale {w.v_scale:g}"} if fp8 else {})},
             "hbm_frac_of_peak": round(value / peak, 4),
             "us_per_call_min_max": [round(min(step_ms) * 1e3, 2), round(max(step_ms) * 1e3, 2)],
             "roofline": {"kernel": kname, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,

@@ -65,7 +65,10 @@ typedef enum pad_status {
   PAD_ERR_DEVICE_CHECK = 5  /* a kernel saw an invalid block id or sequence length */
 } pad_status;
 
-typedef enum pad_dtype { PAD_BF16 = 0, PAD_F32 = 1, PAD_I32 = 2 } pad_dtype;
+/* PAD_FP8_E4M3: OCP 8-bit floating point, E4M3 variant (sign, 4 exponent bits
+ * with bias 7, 3 mantissa bits, subnormals, no infinities, S.1111.111 = NaN,
+ * largest finite 448) -- torch.float8_e4m3fn.  Accepted for k_cache/v_cache. */
+typedef enum pad_dtype { PAD_BF16 = 0, PAD_F32 = 1, PAD_I32 = 2, PAD_FP8_E4M3 = 3 } pad_dtype;
 
 /* A strided tensor view.  `stride` is in ELEMENTS.  Unused trailing dims are
  * ignored.  `dtype` holds a pad_dtype value. */
@@ -99,11 +102,14 @@ typedef struct pad_plan {
  * pad_decode -- paged single-token decode attention.
  *
  *  q             bf16 [B, Hq, D], stride[2] == 1, every row 16-byte aligned.
- *  k_cache       bf16 [num_blocks, Hkv, block_size, D], stride[3] == 1; dims 0-2
- *                may have any non-negative strides whose byte size is a multiple
- *                of 16 (so both [blocks, Hkv, bs, D] "HND" and a permuted view of a
- *                [blocks, bs, Hkv, D] "NHD" cache are accepted).  Base 16-byte aligned.
- *  v_cache       bf16, same shape as k_cache, its own strides, same rules.
+ *  k_cache       bf16 or FP8 E4M3 [num_blocks, Hkv, block_size, D], stride[3] ==
+ *                1; dims 0-2 may have any non-negative strides whose byte size
+ *                is a multiple of 16 (so both [blocks, Hkv, bs, D] "HND" and a
+ *                permuted view of a [blocks, bs, Hkv, D] "NHD" cache are
+ *                accepted).  Base 16-byte aligned.  An E4M3 cache holds codes
+ *                dequantised as k_scale * code (pad_decode_options; 1 here).
+ *  v_cache       same dtype and shape as k_cache, its own strides, same rules;
+ *                E4M3 codes are dequantised as v_scale * code.
  *  block_tables  int32 [B, max_blocks_per_seq], stride[1] == 1.  Entries past
  *                ceil(L_b / block_size) may hold anything: their values are never
  *                used (the kernel may read them, within the row, before it knows
@@ -146,16 +152,26 @@ pad_status pad_decode(const pad_tensor *q, const pad_tensor *k_cache, const pad_
  *                  M = max(max_t s_t, sink_h), Z = sum_t exp(s_t - M) +
  *                  exp(sink_h - M), out = sum_t exp(s_t - M) v_t / Z,
  *                  lse = M + ln Z;  L_b = 0 gives out = 0, lse = sink_h.
+ *   k_scale,     dequantisation scales of an E4M3 cache (the FP8 decode path
+ *   v_scale      "perf(rocke): prepare saved paged decode bindings once" names
+ *                beside the non-FP8 one, section "Summary"; one scale per
+ *                tensor is the reading taken): k_t = k_scale * code, v_t =
+ *                v_scale * code.  0 reads as 1; otherwise finite and > 0.  With a
+ *                bf16 cache both must be 0 or 1.
+ * Zero-initialised options are pad_decode exactly.
  */
 typedef struct pad_decode_options {
   int32_t window_left;
   const pad_tensor *sinks;
+  float k_scale;
+  float v_scale;
 } pad_decode_options;
 
 /*
  * pad_decode_ex -- pad_decode with options (NULL options = pad_decode).  Same
- * arguments, scratch, results and errors; `options->window_left` < 0, or a
- * sinks tensor that is not fp32 [Hq] device memory, is PAD_ERR_INVALID_ARG.
+ * arguments, scratch, results and errors; `options->window_left` < 0, a sinks
+ * tensor that is not fp32 [Hq] device memory, or a scale that is negative,
+ * non-finite, or other than 0/1 for a bf16 cache, is PAD_ERR_INVALID_ARG.
  */
 pad_status pad_decode_ex(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
                          const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
@@ -225,8 +241,9 @@ pad_status pad_decode_static_scratch(const pad_tensor *q, const pad_tensor *k_ca
  * tensor memory, K/V/q streamed by TMA in 8-token boxes, the softmax in four warps
  * that own one token (one TMEM lane) each, one persistent CTA per SM walking the
  * (sequence, KV head, partition) units.  Same arguments, results, scratch and
- * errors as pad_decode.  It takes groups of 17..32 query heads per KV head at
- * head_dim 128 with block_size >= 8 and returns PAD_ERR_UNSUPPORTED otherwise.
+ * errors as pad_decode.  It takes a bf16 cache with groups of 17..32 query
+ * heads per KV head at head_dim 128 and block_size >= 8, and returns
+ * PAD_ERR_UNSUPPORTED otherwise.
  * pad_decode does not call it: on the workloads measured on B200 the mma.sync
  * kernel behind pad_decode is faster (its chunk pipeline waits on page-copy
  * latency with two 64 KB chunks in flight).
@@ -246,6 +263,16 @@ pad_status pad_decode_tcgen05(const pad_tensor *q, const pad_tensor *k_cache, co
 pad_status pad_decode_plan(int64_t batch, int64_t num_q_heads, int64_t num_kv_heads,
                            int64_t head_dim, int64_t block_size, int64_t max_blocks_per_seq,
                            int32_t num_splits, int32_t device, pad_plan *plan);
+
+/*
+ * pad_decode_plan_ex -- pad_decode_plan for a cache of dtype `kv_dtype`
+ * (PAD_BF16, as pad_decode_plan, or PAD_FP8_E4M3: the same partitions and
+ * scratch, deeper pipeline stages of half the bytes).  Any other kv_dtype is
+ * PAD_ERR_INVALID_ARG.
+ */
+pad_status pad_decode_plan_ex(int64_t batch, int64_t num_q_heads, int64_t num_kv_heads,
+                              int64_t head_dim, int64_t block_size, int64_t max_blocks_per_seq,
+                              int32_t num_splits, int32_t kv_dtype, int32_t device, pad_plan *plan);
 
 /* Static string for a status code. */
 const char *pad_status_string(pad_status status);

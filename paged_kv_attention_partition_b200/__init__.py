@@ -23,8 +23,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpad.so")
 
 PAD_OK, PAD_ERR_INVALID_ARG, PAD_ERR_UNSUPPORTED, PAD_ERR_WORKSPACE, PAD_ERR_CUDA, PAD_ERR_DEVICE_CHECK = range(6)
-PAD_BF16, PAD_F32, PAD_I32 = 0, 1, 2
-_DTYPES = {torch.bfloat16: PAD_BF16, torch.float32: PAD_F32, torch.int32: PAD_I32}
+PAD_BF16, PAD_F32, PAD_I32, PAD_FP8_E4M3 = 0, 1, 2, 3
+_DTYPES = {torch.bfloat16: PAD_BF16, torch.float32: PAD_F32, torch.int32: PAD_I32,
+           torch.float8_e4m3fn: PAD_FP8_E4M3}
+_KV_DTYPES = {"bf16": PAD_BF16, "e4m3": PAD_FP8_E4M3, torch.bfloat16: PAD_BF16, torch.float8_e4m3fn: PAD_FP8_E4M3}
 
 
 class PadTensor(ctypes.Structure):
@@ -44,8 +46,9 @@ class PadPlan(ctypes.Structure):
 
 
 class PadOptions(ctypes.Structure):
-    """pad_decode_options: sliding window and attention sinks."""
-    _fields_ = [("window_left", ctypes.c_int32), ("sinks", ctypes.POINTER(PadTensor))]
+    """pad_decode_options: sliding window, attention sinks, E4M3 cache scales."""
+    _fields_ = [("window_left", ctypes.c_int32), ("sinks", ctypes.POINTER(PadTensor)),
+                ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float)]
 
 
 class PadError(RuntimeError):
@@ -85,6 +88,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pad_decode_with_workspace.restype = ctypes.c_int
     lib.pad_decode_plan.argtypes = [ctypes.c_int64] * 6 + [ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(PadPlan)]
     lib.pad_decode_plan.restype = ctypes.c_int
+    lib.pad_decode_plan_ex.argtypes = [ctypes.c_int64] * 6 + [ctypes.c_int32] * 3 + [ctypes.POINTER(PadPlan)]
+    lib.pad_decode_plan_ex.restype = ctypes.c_int
     lib.pad_status_string.argtypes = [ctypes.c_int]
     lib.pad_status_string.restype = ctypes.c_char_p
     lib.pad_last_error.argtypes = []
@@ -143,17 +148,19 @@ def _stream_handle(stream, device) -> int:
 def pad_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
                seq_lens: torch.Tensor, scale: float, num_splits: int = 0, out: Optional[torch.Tensor] = None,
                lse: Union[None, bool, torch.Tensor] = None, stream=None, window: int = 0,
-               sinks: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+               sinks: Optional[torch.Tensor] = None, k_scale: float = 0.0,
+               v_scale: float = 0.0) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Paged single-token decode attention (see ``pad_decode`` / ``pad_decode_ex``
     in include/pad.h).
 
-    q [B, Hq, D] bf16; k_cache/v_cache [num_blocks, Hkv, block_size, D] bf16 (any
-    16-byte-multiple strides on dims 0-2, e.g. ``nhd.transpose(1, 2)``);
-    block_tables [B, W] int32; seq_lens [B] int32.  ``lse=True`` allocates the
-    fp32 [B, Hq] log-sum-exp output, a tensor receives it, None skips it.
-    ``window`` > 0 attends to each sequence's last ``window`` tokens; ``sinks``
-    is an fp32 [Hq] CUDA tensor of per-head sink logits.  Returns (out, lse).
-    Asynchronous on ``stream`` (default: torch's current)."""
+    q [B, Hq, D] bf16; k_cache/v_cache [num_blocks, Hkv, block_size, D] bf16 or
+    float8_e4m3fn (any 16-byte-multiple strides on dims 0-2, e.g.
+    ``nhd.transpose(1, 2)``); block_tables [B, W] int32; seq_lens [B] int32.
+    ``lse=True`` allocates the fp32 [B, Hq] log-sum-exp output, a tensor
+    receives it, None skips it.  ``window`` > 0 attends to each sequence's last
+    ``window`` tokens; ``sinks`` is an fp32 [Hq] CUDA tensor of per-head sink
+    logits; ``k_scale`` / ``v_scale`` dequantise an E4M3 cache (0 = 1).
+    Returns (out, lse).  Asynchronous on ``stream`` (default: torch's current)."""
     dev = q.device
     if dev.type != "cuda":
         raise ValueError("q must be a CUDA tensor")
@@ -176,9 +183,10 @@ def pad_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, bl
     dq, dk, dv, dt, dl, do = (describe(t) for t in (q, k_cache, v_cache, block_tables, seq_lens, out))
     dlse = describe(lse) if lse is not None else None
     with torch.cuda.device(dev):
-        if window or sinks is not None:
+        if window or sinks is not None or k_scale or v_scale:
             dsk = describe(sinks) if sinks is not None else None
-            opts = PadOptions(int(window), ctypes.pointer(dsk) if dsk is not None else None)
+            opts = PadOptions(int(window), ctypes.pointer(dsk) if dsk is not None else None, float(k_scale),
+                              float(v_scale))
             st = lib.pad_decode_ex(ctypes.byref(dq), ctypes.byref(dk), ctypes.byref(dv), ctypes.byref(dt),
                                    ctypes.byref(dl), float(scale), int(num_splits), ctypes.byref(opts),
                                    ctypes.byref(do), ctypes.byref(dlse) if dlse is not None else None,
@@ -261,11 +269,17 @@ def pad_decode_with_workspace(q, k_cache, v_cache, block_tables, seq_lens, scale
 
 
 def pad_decode_plan(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, block_size: int,
-                    max_blocks_per_seq: int, num_splits: int = 0, device: int = -1) -> dict:
-    """Launch geometry pad_decode would use for this shape (no launch)."""
+                    max_blocks_per_seq: int, num_splits: int = 0, device: int = -1, kv_dtype="bf16") -> dict:
+    """Launch geometry pad_decode would use for this shape (no launch);
+    ``kv_dtype`` "bf16" or "e4m3" (or the torch dtype) names the cache."""
     plan = PadPlan()
-    st = load_library().pad_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, block_size,
-                                        max_blocks_per_seq, num_splits, device, ctypes.byref(plan))
+    lib = load_library()
+    if kv_dtype in ("bf16", torch.bfloat16):
+        st = lib.pad_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                                 num_splits, device, ctypes.byref(plan))
+    else:
+        st = lib.pad_decode_plan_ex(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                                    num_splits, _KV_DTYPES.get(kv_dtype, -1), device, ctypes.byref(plan))
     _raise(st)
     return plan.as_dict()
 

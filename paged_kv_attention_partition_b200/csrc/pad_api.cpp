@@ -48,6 +48,7 @@ int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
 struct Shape {
   int64_t B, Hq, Hkv, D, bs, W, g;
+  bool fp8;  // E4M3 cache
 };
 
 pad_status check_shape(const Shape &s, int32_t num_splits) {
@@ -123,10 +124,10 @@ void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan, b
   plan->partition_tokens = (int32_t)P;
   plan->heads_per_tile = hpt;
   plan->head_tiles = (int32_t)HT;
-  const bool umma = tcgen05 && pad::umma_eligible((int)s.D, hpt, (int)s.bs);
+  const bool umma = tcgen05 && !s.fp8 && pad::umma_eligible((int)s.D, hpt, (int)s.bs);
   plan->warps_per_cta = umma ? pad::kUmmaWarps : pad::kWarps;
-  plan->stage_tokens = umma ? pad::kUmmaStageTokens : pad::stage_tokens_for((int)s.D, hpt);
-  plan->stages = umma ? pad::umma_stages() : pad::partition_stages((int)s.D, hpt);
+  plan->stage_tokens = umma ? pad::kUmmaStageTokens : pad::stage_tokens_for((int)s.D, hpt, s.fp8);
+  plan->stages = umma ? pad::umma_stages() : pad::partition_stages((int)s.D, hpt, s.fp8);
   // one CTA per unit; the tcgen05 kernel is persistent: one CTA per SM walks the units
   const int64_t sms = sm_count(device < 0 ? 0 : device);
   plan->ctas = (int32_t)(umma ? (units < sms ? units : sms) : (units > 0x7fffffffll ? 0x7fffffffll : units));
@@ -166,17 +167,22 @@ pad_status encode_cache_map(CUtensorMap *map, const pad_tensor *t, int box_rows_
   EncodeTiledFn enc = tensor_map_encoder();
   if (enc == nullptr) return fail(PAD_ERR_CUDA, "the CUDA driver does not provide cuTensorMapEncodeTiled");
   const int64_t NB = t->shape[0], Hkv = t->shape[1], bs = t->shape[2], D = t->shape[3];
+  const bool fp8 = t->dtype == PAD_FP8_E4M3;
+  const int64_t eb = fp8 ? 1 : 2;                 // bytes per element
+  const int64_t rowb = D * eb, rw = rowb < 128 ? rowb : 128;  // row bytes; bytes per column block
   auto stride_bytes = [&](int i, int64_t natural) -> cuuint64_t {
-    return (cuuint64_t)(t->shape[i] > 1 ? t->stride[i] * 2 : natural);
+    return (cuuint64_t)(t->shape[i] > 1 ? t->stride[i] * eb : natural);
   };
-  const cuuint64_t dims[5] = {64, (cuuint64_t)bs, (cuuint64_t)(D / 64), (cuuint64_t)Hkv, (cuuint64_t)NB};
-  const cuuint64_t strides[4] = {stride_bytes(2, D * 2), 128, stride_bytes(1, bs * D * 2),
-                                 stride_bytes(0, Hkv * bs * D * 2)};
-  const cuuint32_t box[5] = {64, (cuuint32_t)box_rows_, (cuuint32_t)(D / 64), 1, 1};
+  const cuuint64_t dims[5] = {(cuuint64_t)(rw / eb), (cuuint64_t)bs, (cuuint64_t)(rowb / rw), (cuuint64_t)Hkv,
+                              (cuuint64_t)NB};
+  const cuuint64_t strides[4] = {stride_bytes(2, rowb), (cuuint64_t)rw, stride_bytes(1, bs * rowb),
+                                 stride_bytes(0, Hkv * bs * rowb)};
+  const cuuint32_t box[5] = {(cuuint32_t)(rw / eb), (cuuint32_t)box_rows_, (cuuint32_t)(rowb / rw), 1, 1};
   const cuuint32_t elem[5] = {1, 1, 1, 1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, t->data, dims, strides, box, elem,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r = enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, t->data,
+                         dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         rw == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(PAD_ERR_INVALID_ARG, "%s: strides/shape not expressible as a TMA tensor (cuTensorMapEncodeTiled %d)",
                 name, (int)r);
@@ -215,14 +221,14 @@ pad_status check_tensor(const pad_tensor *t, const char *name, pad_dtype dt, int
   return PAD_OK;
 }
 
-// rows of 16-bit elements along the last dim must be contiguous and 16-byte aligned
-pad_status check_rows16(const pad_tensor *t, const char *name) {
+// rows of `elem_bytes`-byte elements along the last dim must be contiguous and 16-byte aligned
+pad_status check_rows16(const pad_tensor *t, const char *name, int64_t elem_bytes = 2) {
   const int last = t->ndim - 1;
   if (t->stride[last] != 1) return fail(PAD_ERR_INVALID_ARG, "%s: last dim must be contiguous", name);
   if (reinterpret_cast<uintptr_t>(t->data) % 16 != 0)
     return fail(PAD_ERR_INVALID_ARG, "%s: data must be 16-byte aligned", name);
   for (int i = 0; i < last; ++i)
-    if ((t->stride[i] * 2) % 16 != 0 && t->shape[i] > 1)
+    if ((t->stride[i] * elem_bytes) % 16 != 0 && t->shape[i] > 1)
       return fail(PAD_ERR_INVALID_ARG, "%s: stride[%d]=%lld is not a multiple of 16 bytes", name, i,
                   (long long)t->stride[i]);
   return PAD_OK;
@@ -307,6 +313,7 @@ struct Prepared {
   pad::ControlLayout cl;
   int D;
   int device;
+  bool kv_fp8;
 };
 
 pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
@@ -316,8 +323,11 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
   pad_status st;
   *empty = false;
   if ((st = check_tensor(q, "q", PAD_BF16, 3)) != PAD_OK) return st;
-  if ((st = check_tensor(k_cache, "k_cache", PAD_BF16, 4)) != PAD_OK) return st;
-  if ((st = check_tensor(v_cache, "v_cache", PAD_BF16, 4)) != PAD_OK) return st;
+  // the cache is bf16 or E4M3, K and V alike
+  const bool fp8 = k_cache != nullptr && k_cache->dtype == PAD_FP8_E4M3;
+  const pad_dtype kv_dt = fp8 ? PAD_FP8_E4M3 : PAD_BF16;
+  if ((st = check_tensor(k_cache, "k_cache", kv_dt, 4)) != PAD_OK) return st;
+  if ((st = check_tensor(v_cache, "v_cache", kv_dt, 4)) != PAD_OK) return st;
   if ((st = check_tensor(block_tables, "block_tables", PAD_I32, 2)) != PAD_OK) return st;
   if ((st = check_tensor(seq_lens, "seq_lens", PAD_I32, 1)) != PAD_OK) return st;
   if ((st = check_tensor(out, "out", PAD_BF16, 3)) != PAD_OK) return st;
@@ -344,15 +354,26 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
   if (!isfinite(scale)) return fail(PAD_ERR_INVALID_ARG, "scale must be finite");
   if (NB <= 0 || NB > 0x7fffffffll) return fail(PAD_ERR_INVALID_ARG, "num_blocks %lld out of range", (long long)NB);
   if ((st = check_rows16(q, "q")) != PAD_OK) return st;
-  if ((st = check_rows16(k_cache, "k_cache")) != PAD_OK) return st;
-  if ((st = check_rows16(v_cache, "v_cache")) != PAD_OK) return st;
+  if ((st = check_rows16(k_cache, "k_cache", fp8 ? 1 : 2)) != PAD_OK) return st;
+  if ((st = check_rows16(v_cache, "v_cache", fp8 ? 1 : 2)) != PAD_OK) return st;
   if ((st = check_rows16(out, "out")) != PAD_OK) return st;
   if (reinterpret_cast<uintptr_t>(block_tables->data) % 4 || reinterpret_cast<uintptr_t>(seq_lens->data) % 4 ||
       (lse != nullptr && reinterpret_cast<uintptr_t>(lse->data) % 4))
     return fail(PAD_ERR_INVALID_ARG, "int32/fp32 tensors must be 4-byte aligned");
 
-  Shape s{B, Hq, Hkv, D, bs, block_tables->shape[1], Hkv > 0 ? Hq / Hkv : 0};
+  Shape s{B, Hq, Hkv, D, bs, block_tables->shape[1], Hkv > 0 ? Hq / Hkv : 0, fp8};
   if ((st = check_shape(s, num_splits)) != PAD_OK) return st;
+  // dequantisation scales: 0 reads as 1; an E4M3 cache takes any finite
+  // positive value, a bf16 cache only 1
+  float k_scale = 1.f, v_scale = 1.f;
+  if (opts != nullptr) {
+    k_scale = opts->k_scale == 0.f ? 1.f : opts->k_scale;
+    v_scale = opts->v_scale == 0.f ? 1.f : opts->v_scale;
+    if (!(isfinite(k_scale) && k_scale > 0.f) || !(isfinite(v_scale) && v_scale > 0.f))
+      return fail(PAD_ERR_INVALID_ARG, "k_scale and v_scale must be finite and positive (or 0 for 1)");
+    if (!fp8 && (k_scale != 1.f || v_scale != 1.f))
+      return fail(PAD_ERR_INVALID_ARG, "k_scale / v_scale apply to an E4M3 cache only (bf16 cache: 0 or 1)");
+  }
   if (B == 0) {
     *empty = true;
     return PAD_OK;
@@ -369,11 +390,11 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
   if ((st = check_device_ptr(out->data, device, "out")) != PAD_OK) return st;
   if (lse != nullptr && (st = check_device_ptr(lse->data, device, "lse")) != PAD_OK) return st;
 
-  if (tcgen05 && !pad::umma_eligible((int)D, s.g <= 8 ? 8 : (s.g <= 16 ? 16 : 32), (int)bs))
+  if (tcgen05 && (fp8 || !pad::umma_eligible((int)D, s.g <= 8 ? 8 : (s.g <= 16 ? 16 : 32), (int)bs)))
     return fail(PAD_ERR_UNSUPPORTED,
-                "the tcgen05 kernel takes groups of 17..32 query heads per KV head at head_dim 128 with a block "
-                "size of at least 8 (got group %lld, head_dim %lld, block size %lld)",
-                (long long)s.g, (long long)D, (long long)bs);
+                "the tcgen05 kernel takes a bf16 cache with groups of 17..32 query heads per KV head at head_dim "
+                "128 and a block size of at least 8 (got %s, group %lld, head_dim %lld, block size %lld)",
+                fp8 ? "E4M3" : "bf16", (long long)s.g, (long long)D, (long long)bs);
   make_plan(s, num_splits, device, &pr->plan, tcgen05);
   const int64_t units = B * Hkv * pr->plan.head_tiles * (int64_t)pr->plan.num_splits;
   if (units > 0x7fffffffll) return fail(PAD_ERR_UNSUPPORTED, "too many work units (%lld) for one launch", (long long)units);
@@ -386,7 +407,7 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
   pad::PartitionParams &p = pr->p;
   p = pad::PartitionParams{};
   pr->umma = tcgen05;
-  const int rows = pr->umma ? 8 : pad::box_rows((int)bs, (int)D, pr->plan.heads_per_tile);
+  const int rows = pr->umma ? 8 : pad::box_rows((int)bs, (int)D, pr->plan.heads_per_tile, fp8);
   if ((st = encode_cache_map(&p.tmk, k_cache, rows, "k_cache")) != PAD_OK) return st;
   if ((st = encode_cache_map(&p.tmv, v_cache, rows, "v_cache")) != PAD_OK) return st;
   if (pr->umma && (st = encode_q_map(&p.tmq, q, pr->plan.heads_per_tile)) != PAD_OK) return st;
@@ -415,7 +436,8 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
   p.P = pr->plan.partition_tokens;
   p.S = pr->plan.num_splits;
   p.n_units = (uint32_t)units;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale_log2 = (float)((double)scale * (double)k_scale * 1.4426950408889634);
+  p.v_scale = v_scale;
   if (opts != nullptr) {
     if (opts->window_left < 0) return fail(PAD_ERR_INVALID_ARG, "window_left must be >= 0 (got %d)", opts->window_left);
     p.window = opts->window_left;
@@ -438,6 +460,7 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
   p.err = err;
   pr->D = (int)D;
   pr->device = device;
+  pr->kv_fp8 = fp8;
   return PAD_OK;
 }
 
@@ -459,7 +482,8 @@ pad_status check_caller_buffer(const Prepared &pr, void *buf, size_t bytes, size
 
 pad_status run(const Prepared &pr, cudaStream_t stream) {
   cudaError_t e = pr.umma ? pad::launch_umma(pr.p, pr.plan.ctas, stream)
-                          : pad::launch_partition(pr.p, pr.D, pr.plan.heads_per_tile, pr.plan.ctas, stream);
+                          : pad::launch_partition(pr.p, pr.D, pr.plan.heads_per_tile, pr.kv_fp8, pr.plan.ctas,
+                                                  stream);
   return e == cudaSuccess ? PAD_OK : cuda_fail(e, "partition kernel launch");
 }
 
@@ -511,9 +535,18 @@ const char *pad_last_error(void) { return g_last_error.c_str(); }
 pad_status pad_decode_plan(int64_t batch, int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
                            int64_t block_size, int64_t max_blocks_per_seq, int32_t num_splits, int32_t device,
                            pad_plan *plan) {
+  return pad_decode_plan_ex(batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_splits,
+                            PAD_BF16, device, plan);
+}
+
+pad_status pad_decode_plan_ex(int64_t batch, int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
+                              int64_t block_size, int64_t max_blocks_per_seq, int32_t num_splits, int32_t kv_dtype,
+                              int32_t device, pad_plan *plan) {
   if (plan == nullptr) return fail(PAD_ERR_INVALID_ARG, "plan is NULL");
+  if (kv_dtype != PAD_BF16 && kv_dtype != PAD_FP8_E4M3)
+    return fail(PAD_ERR_INVALID_ARG, "kv_dtype must be PAD_BF16 or PAD_FP8_E4M3 (got %d)", kv_dtype);
   Shape s{batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
-          num_kv_heads > 0 ? num_q_heads / num_kv_heads : 0};
+          num_kv_heads > 0 ? num_q_heads / num_kv_heads : 0, kv_dtype == PAD_FP8_E4M3};
   pad_status st = check_shape(s, num_splits);
   if (st != PAD_OK) return st;
   if (device < 0) {

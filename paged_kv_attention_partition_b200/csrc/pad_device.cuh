@@ -1,9 +1,10 @@
 // Small device helpers: TMA tensor copies and mbarriers, ldmatrix/movmatrix,
-// bf16 tensor-core MMA, L2-coherent loads.
+// bf16 and f16 tensor-core MMA, E4M3 widening, L2-coherent loads.
 #pragma once
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace pad {
@@ -92,6 +93,38 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4],
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D(16x8, f32) += A(16x16, f16, row) * B(16x8, f16, col)
+__device__ __forceinline__ void mma_16816_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two E4M3 codes (low byte -> low half) widened to f16x2.  Exact: every E4M3
+// value, subnormals and NaN included, is an f16 value.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  uint32_t h;
+  const uint16_t x = (uint16_t)two_codes;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;\n" : "=r"(h) : "h"(x));
+  return h;
+}
+
+// Two E4M3 codes widened to bf16x2, through f16 and f32.  Exact: an E4M3 value
+// has at most 4 significant bits and its exponent range lies inside bf16's.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two_codes) {
+  const uint32_t f = e4m3x2_to_f16x2(two_codes);
+  const float lo = __half2float(__ushort_as_half((unsigned short)(f & 0xffffu)));
+  const float hi = __half2float(__ushort_as_half((unsigned short)(f >> 16)));
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Bytes of x selected by `sel` (4 nibbles, byte indices 0-3 of x).
+__device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t sel) { return __byte_perm(x, 0, sel); }
+
 // 2^x on the special-function unit (ex2.approx: about 2 ulp, 2^-inf = +0).
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -101,6 +134,11 @@ __device__ __forceinline__ float fast_exp2(float x) {
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);
 }
 

@@ -31,14 +31,37 @@ constexpr int kMaxSplits = 256;      // partitions per sequence (bounds the merg
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 __host__ __device__ constexpr int dsplit_for(int D, int hpt) { return D == 256 ? 2 : 1; }
-__host__ __device__ constexpr int stage_tokens_for(int D, int hpt) { return 16 * kWarps / dsplit_for(D, hpt); }
+// 16-token tiles a token group computes per stage.  An E4M3 stage carries the
+// same bytes as a bf16 one with twice the tokens: with 8- or 16-head tiles at
+// D >= 128 each group takes two tiles per stage (two independent QK chains,
+// one max exchange and one rescale check for both), which the math needs to
+// keep up with the halved bytes per token.
+__host__ __device__ constexpr int tiles_per_group(int D, int hpt, bool f8 = false) {
+  return f8 && D >= 128 && hpt <= 16 ? 2 : 1;
+}
+__host__ __device__ constexpr int stage_tokens_for(int D, int hpt, bool f8 = false) {
+  return 16 * kWarps / dsplit_for(D, hpt) * tiles_per_group(D, hpt, f8);
+}
 
-// Pipeline depth and resident CTAs per SM of one (head_dim, heads-per-tile)
-// instantiation.  The ring is kept small so that several CTAs share each SM:
-// their loads, math and start/finish latencies overlap one another.
-__host__ __device__ constexpr int stages_for(int D, int hpt) { return D == 64 || (D == 128 && hpt == 32) ? 3 : 2; }
-__host__ __device__ constexpr int ctas_per_sm_for(int D, int hpt) {
+// Pipeline depth and resident CTAs per SM of one (head_dim, heads-per-tile,
+// cache type) instantiation.  The ring is kept small so that several CTAs
+// share each SM: their loads, math and start/finish latencies overlap one
+// another.  An E4M3 stage of one tile per group holds the same tokens in half
+// the bytes, so it runs twice the stages (the same bytes in flight); at D = 64
+// its 64-byte rows sit in boxes of at least 128 bytes, which caps it at three.
+// With two tiles per group an E4M3 stage is as large as a bf16 one.
+__host__ __device__ constexpr int stages_for(int D, int hpt, bool f8 = false) {
+  return f8 ? (tiles_per_group(D, hpt, f8) == 2 ? 2 : D == 64 ? 3 : 6)
+            : (D == 64 || (D == 128 && hpt == 32) ? 3 : 2);
+}
+__host__ __device__ constexpr int ctas_per_sm_for(int D, int hpt, bool f8 = false) {
   return D == 64 ? (hpt == 32 ? 3 : 4) : D == 128 ? (hpt == 32 ? 2 : 3) : (hpt == 16 ? 2 : 3);
+}
+// Bytes of one K (or V) half-stage: bf16 rows of 2D bytes; E4M3 rows of D
+// bytes, in boxes padded to at least 128 bytes (only D = 64 with one-row boxes
+// needs it).
+__host__ __device__ constexpr int half_stage_bytes(int D, int hpt, bool f8) {
+  return stage_tokens_for(D, hpt, f8) * (f8 ? (D < 128 ? 128 : D) : 2 * D);
 }
 
 // Shared memory of one CTA (from a 1024-byte aligned base): the K/V ring,
@@ -50,11 +73,11 @@ struct SmemPlan {
   size_t stage_bytes, ring_bytes, warp_merge_bytes, split_merge_bytes, region_bytes, total;
 };
 
-__host__ __device__ constexpr SmemPlan smem_plan_for(int D, int hpt) {
+__host__ __device__ constexpr SmemPlan smem_plan_for(int D, int hpt, bool f8 = false) {
   SmemPlan s{};
-  s.stages = stages_for(D, hpt);
-  s.stage_tokens = stage_tokens_for(D, hpt);
-  s.stage_bytes = (size_t)s.stage_tokens * D * 2 * 2;  // K and V rows of one stage
+  s.stages = stages_for(D, hpt, f8);
+  s.stage_tokens = stage_tokens_for(D, hpt, f8);
+  s.stage_bytes = (size_t)half_stage_bytes(D, hpt, f8) * 2;  // K and V rows of one stage
   s.ring_bytes = (size_t)s.stages * s.stage_bytes;
   s.warp_merge_bytes = (size_t)(kWarps / dsplit_for(D, hpt)) * hpt * (D + 4 + 2) * 4;  // padded rows, m, l
   s.split_merge_bytes = (size_t)hpt * (kMaxSplits + 1) * 4;
@@ -70,9 +93,11 @@ __host__ __device__ constexpr SmemPlan smem_plan_for(int D, int hpt) {
 inline int max_heads_per_tile(int D) { return D <= 128 ? 32 : 16; }
 
 struct PartitionParams {
-  // K and V caches as 5-D tiled tensors (64 head_dim elements, slot, head_dim
-  // / 64, kv head, block), one box = one page (or a stage's worth of a larger
-  // page; 8 rows for the tcgen05 kernel) with the 128-byte swizzle.
+  // K and V caches as 5-D tiled tensors (128 bytes of head_dim, slot, the
+  // rest of head_dim in 128-byte blocks, kv head, block), one box = one page
+  // (or a stage's worth of a larger page; 8 rows for the tcgen05 kernel) with
+  // the 128-byte swizzle.  An E4M3 cache at D = 64 has one 64-byte block and
+  // the 64-byte swizzle.
   CUtensorMap tmk, tmv;
   // q as a 4-D tiled tensor (64 head_dim elements, head, head_dim / 64, b), one
   // box = a 32-head tile (tcgen05 kernel only).
@@ -94,7 +119,8 @@ struct PartitionParams {
   int32_t P;        // tokens per partition (multiple of the block size)
   int32_t S;        // partitions per sequence (ceil(capacity / P) <= kMaxSplits)
   uint32_t n_units; // B * Hkv * HT * S, one CTA each
-  float scale_log2; // scale * log2(e)
+  float scale_log2; // scale * k_scale * log2(e)
+  float v_scale;    // E4M3 V dequantisation scale (1 for bf16)
   int32_t window;     // 0: every token; W > 0: each sequence's last W tokens
   const float *sinks; // null, or a sink logit per query head [Hq] (natural log, units of scale q.k)
   uint16_t *out;
@@ -136,7 +162,8 @@ inline ControlLayout control_layout(int64_t B, int64_t Hkv, int64_t HT, int64_t 
   return c;
 }
 
-cudaError_t launch_partition(const PartitionParams &p, int D, int heads_per_tile, int grid, cudaStream_t s);
+cudaError_t launch_partition(const PartitionParams &p, int D, int heads_per_tile, bool kv_fp8, int grid,
+                             cudaStream_t s);
 // The tcgen05 kernel (pad_umma.cu) takes 32-head tiles at head_dim 128 with
 // pages of at least 8 tokens (its K/V boxes are 8 rows of one page).
 inline bool umma_eligible(int D, int hpt, int block_size) { return D == 128 && hpt == 32 && block_size >= 8; }
@@ -146,11 +173,11 @@ constexpr int kUmmaStageTokens = 128;
 constexpr int kUmmaWarps = 6;
 
 // Rows of one TMA box: a page, or a stage's worth of rows of a larger page.
-inline int box_rows(int block_size, int D, int hpt) {
-  const int st = stage_tokens_for(D, hpt);
+inline int box_rows(int block_size, int D, int hpt, bool f8) {
+  const int st = stage_tokens_for(D, hpt, f8);
   return block_size < st ? block_size : st;
 }
-int partition_stages(int D, int heads_per_tile);
+int partition_stages(int D, int heads_per_tile, bool kv_fp8);
 cudaError_t device_error_word(int device, uint32_t **ptr);
 void set_last_error(const char *msg);
 

@@ -31,6 +31,18 @@
 //   P^T = exp2(S^T * scale*log2e - m)
 //   O^T += V^T . P^T              (P^T moved into the B-operand layout by movmatrix)
 //
+// An E4M3 cache ("perf(rocke): prepare saved paged decode bindings once",
+// section "Summary": the FP8 decode path beside the non-FP8 one) streams 8-bit
+// codes, half the bytes, through the same stages.  K operands are loaded four
+// codes per register and widened exactly to bf16 (E4M3 -> f16 -> f32 -> bf16),
+// so the QK product stays exact against bf16 q; the head_dim order inside each
+// 16-wide k-step is permuted (codes 4c..4c+3 of a row go to k = 2c, 2c+1,
+// 2c+8, 2c+9), and the q fragments take the same permutation, which a dot
+// product allows.  V operands come from a transposed ldmatrix of the codes and
+// a byte permute, widened to f16 (exact) for an f16 PV product with f16
+// weights; the m-tile rows are head_dim 2i and 2i+1 instead of i and i+8.
+// k_scale is folded into the score scale, v_scale into the final 1/l.
+//
 // A sequence with one non-empty partition writes bf16 out (+ lse) directly.
 // Otherwise each partition writes its fp32 output (normalised by its own sum)
 // and its lse, and the CTA that finishes the last partition of the (b, KV head,
@@ -74,25 +86,29 @@ __device__ bool wait_stage(uint32_t bar, uint32_t parity, uint32_t *err) {
 }
 }  // namespace
 
-template <int D, int HPT>
-__global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
+template <int D, int HPT, bool F8>
+__global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
     partition_kernel(const __grid_constant__ PartitionParams p) {
-  constexpr SmemPlan SP = smem_plan_for(D, HPT);
+  constexpr SmemPlan SP = smem_plan_for(D, HPT, F8);
   constexpr int NST = SP.stages;
   constexpr uint32_t STAGE_BYTES = (uint32_t)SP.stage_bytes;
   constexpr int ST = SP.stage_tokens;      // tokens per stage
-  constexpr int ST_LOG2 = ST == 64 ? 6 : 5;
+  constexpr int ST_LOG2 = ST == 128 ? 7 : ST == 64 ? 6 : 5;
   constexpr int DS = dsplit_for(D, HPT);   // warps sharing a token group (head_dim split)
   constexpr int TG = kWarps / DS;          // token groups
+  constexpr int TPW = tiles_per_group(D, HPT, F8);  // 16-token tiles per token group per stage
   constexpr int NT = HPT / 8;              // 8-head n-tiles
   constexpr int KT = D / 16;               // QK k-steps
   constexpr int MT = KT / DS;              // PV m-tiles (16 head_dim rows each) per warp
-  constexpr int CH = D / 8;                // 16-byte chunks per K/V row
-  constexpr int NH = D / 64;               // 128-byte column blocks per row
-  constexpr int ROWB = D * 2;
+  constexpr int ROWB = F8 ? D : D * 2;     // bytes per K/V row
+  constexpr int RW = ROWB < 128 ? ROWB : 128;  // bytes of a row in one column block
+  constexpr int CH = ROWB / 16;            // 16-byte chunks per K/V row
+  constexpr int CPB = RW / 16;             // 16-byte chunks per column block
+  constexpr int HALF = half_stage_bytes(D, HPT, F8);  // K (or V) rows of one stage
   constexpr int IDW = (ST + 31) / 32;      // block ids per lane of warp 0 for one stage
   constexpr bool SPLIT_QK = NT <= 2;       // two QK accumulation chains when registers allow
-  static_assert(ST == 16 * TG && (1 << ST_LOG2) == ST, "stage shape");
+  static_assert(ST == 16 * TG * TPW && (1 << ST_LOG2) == ST, "stage shape");
+  static_assert(!F8 || (KT % 2 == 0 && MT % 2 == 0), "E4M3 operands are loaded two k-steps / m-tiles at a time");
   static_assert(NST >= 2 && NST <= 8, "at least one stage in flight during the math; barrier area");
   static_assert(SP.total <= (size_t)kSmemBudget, "shared-memory plan over budget");
   extern __shared__ uint8_t smem_raw[];
@@ -115,9 +131,12 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
   const int t0 = s * p.P;
 
   // A box holds bsb rows: a whole page, or a stage's worth of a larger page.
+  // Boxes sit box_pitch bytes apart: their size, but at least 128 bytes (a
+  // one-row E4M3 box at D = 64 is 64 bytes), so every copy lands 128-byte aligned.
   const int bsb_log2 = min(p.bs_log2, ST_LOG2);
   const int nbox = ST >> bsb_log2;  // boxes per stage
   const uint32_t box_bytes = (uint32_t)ROWB << bsb_log2;
+  const uint32_t box_pitch = box_bytes < 128u ? 128u : box_bytes;
   const int32_t *trow = p.tables + (int64_t)b * p.table_stride;
 
   // Stages are counted from tu, the first stage holding a token of the unit:
@@ -185,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
     const int jb = tb < tlo ? (tlo - tb) >> bsb_log2 : 0;
     const int nb = min(nbox, (t1 - tb + (1 << bsb_log2) - 1) >> bsb_log2);
     uint8_t *sK = smem + (st % NST) * STAGE_BYTES;
-    uint8_t *sV = sK + ST * ROWB;
+    uint8_t *sV = sK + HALF;
     const uint32_t bar = smem_addr(full + st % NST);
     const int slot0 = tb & ((1 << p.bs_log2) - 1);  // row of the box inside its page
     if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(nb - jb) * box_bytes * 2);
@@ -197,8 +216,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
         const int id = __shfl_sync(0xffffffffu, sid[w], jj);
         if (lane == 0) {
           if ((unsigned)id >= (unsigned)p.num_blocks) atomicOr(p.err, kErrBlockId);  // the box reads as zeros
-          tma_load_5d(smem_addr(sK + j * box_bytes), &p.tmk, 0, slot0, 0, kvh, id, bar);
-          tma_load_5d(smem_addr(sV + j * box_bytes), &p.tmv, 0, slot0, 0, kvh, id, bar);
+          tma_load_5d(smem_addr(sK + j * box_pitch), &p.tmk, 0, slot0, 0, kvh, id, bar);
+          tma_load_5d(smem_addr(sV + j * box_pitch), &p.tmv, 0, slot0, 0, kvh, id, bar);
         }
       }
     }
@@ -210,36 +229,86 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
   }
   int (&idn)[IDW] = ids[NST - 1];  // block ids of the next stage to issue
 
-  // Address of 16-byte chunk (column block h, chunk c7 of it) of row r in a K
+  // Address of 16-byte chunk (column block h, chunk c of it) of row r in a K
   // or V half-stage: rows grouped in boxes of 2^bsb_log2 rows, each box laid out
-  // [D/64][rows][128 B], and the TMA's 128-byte swizzle XORs the chunk index
-  // with bits 7-9 of the address.  rbase/rkey depend on the row only.
+  // [column blocks][rows][RW bytes].  The TMA's 128-byte swizzle XORs the chunk
+  // index with address bits 7-9; the 64-byte swizzle (E4M3 rows at D = 64, one
+  // column block) XORs chunk bits 4-5 with address bits 7-8.  rbase/rkey depend
+  // on the row only.
   auto row_base = [&](int r, uint32_t &rbase, uint32_t &rkey) {
     const int slot = r & ((1 << bsb_log2) - 1);
-    rbase = (uint32_t)((r - slot) * ROWB + slot * 128);
-    rkey = (uint32_t)((r - slot) * NH + slot);
+    rbase = (uint32_t)(r >> bsb_log2) * box_pitch + (uint32_t)(slot * RW);
+    rkey = rbase >> 7;
   };
-  auto chunk = [&](uint32_t rbase, uint32_t rkey, int h, int c7) -> uint32_t {
-    return rbase + ((uint32_t)h << (bsb_log2 + 7)) + ((((uint32_t)c7) ^ ((rkey + ((uint32_t)h << bsb_log2)) & 7u)) << 4);
+  auto chunk = [&](uint32_t rbase, uint32_t rkey, int h, int c) -> uint32_t {
+    if constexpr (RW == 128)
+      return rbase + ((uint32_t)h << (bsb_log2 + 7)) + ((((uint32_t)c) ^ ((rkey + ((uint32_t)h << bsb_log2)) & 7u)) << 4);
+    else
+      return rbase + ((((uint32_t)c) ^ (rkey & 3u)) << 4);
   };
-  // QK operand rows (ldmatrix of K) and PV operand rows (transposed ldmatrix of V)
-  uint32_t kb, kk_key, vb, vkey;
-  row_base(tg * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, kb, kk_key);
-  row_base(tg * 16 + (lane & 7) + ((lane >> 4) & 1) * 8, vb, vkey);
+  // QK operand rows (ldmatrix of K) and PV operand rows (transposed ldmatrix
+  // of V) of this warp's tiles: tile i of token group tg is stage rows
+  // 16 (i TG + tg) .. +15.  (E4M3: both operands' matrices 0/1 are tokens
+  // 0-7/8-15 of the first 16 bytes, matrices 2/3 the same tokens of the next 16.)
+  uint32_t kb[TPW], kk_key[TPW], vb[TPW], vkey[TPW];
+#pragma unroll
+  for (int i = 0; i < TPW; ++i) {
+    const int r0 = 16 * (i * TG + tg) + (lane & 7);
+    row_base(r0 + ((lane >> 3) & 1) * 8, kb[i], kk_key[i]);
+    row_base(r0 + ((F8 ? (lane >> 3) : (lane >> 4)) & 1) * 8, vb[i], vkey[i]);
+  }
 
   // Q^T fragments (B operand of S^T = K.Q^T): lane holds head nt*8 + lane/4,
-  // dims 16kk + 2(lane%4) + {0,1} and + {8,9}.  Padded heads are zero.
+  // dims 16kk + 2(lane%4) + {0,1} and + {8,9} -- with an E4M3 cache, in the
+  // permuted order of its K operands, 16kk + 4(lane%4) + {0,1} and + {2,3}.
+  // Padded heads are zero.  With an E4M3 cache the fragments are f16: q times
+  // 2^qe, qe chosen so that the tile's largest |q| lies in [2^14, 2^15), which
+  // keeps every bf16 value exact (down to 2^-28 of that largest, where f16 turns
+  // subnormal), and 2^-qe joins the score scale.
   uint32_t qf[KT][NT][2];
+  float sl2 = p.scale_log2;
+  auto q_row = [&](int nt, bool &ok) -> const uint16_t * {
+    const int hl = nt * 8 + (lane >> 2);
+    ok = hl < gl;
+    return p.q + b * p.q_sb + (int64_t)(h0 + (ok ? hl : 0)) * p.q_sh + (lane & 3) * (F8 ? 4 : 2);
+  };
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const int hl = nt * 8 + (lane >> 2);
-    const bool ok = hl < gl;
-    const uint16_t *qr = p.q + b * p.q_sb + (int64_t)(h0 + (ok ? hl : 0)) * p.q_sh + (lane & 3) * 2;
+    bool ok;
+    const uint16_t *qr = q_row(nt, ok);
 #pragma unroll
     for (int kk = 0; kk < KT; ++kk) {
       qf[kk][nt][0] = ok ? __ldg(reinterpret_cast<const uint32_t *>(qr + kk * 16)) : 0u;
-      qf[kk][nt][1] = ok ? __ldg(reinterpret_cast<const uint32_t *>(qr + kk * 16 + 8)) : 0u;
+      qf[kk][nt][1] = ok ? __ldg(reinterpret_cast<const uint32_t *>(qr + kk * 16 + (F8 ? 2 : 8))) : 0u;
     }
+  }
+  if constexpr (F8) {
+    float amax = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int kk = 0; kk < KT; ++kk)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const uint32_t w = qf[kk][nt][j];
+          amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w << 16)), fabsf(__uint_as_float(w & 0xffff0000u))));
+        }
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    int e2 = 0;
+    if (amax > 0.f && amax <= 3.0e38f) frexpf(amax, &e2);  // amax = f 2^e2, f in [0.5, 1)
+    const int qe = amax > 0.f && amax <= 3.0e38f ? min(100, max(-100, 15 - e2)) : 0;
+    const float qs = __int_as_float((127 + qe) << 23);
+    sl2 = p.scale_log2 * __int_as_float((127 - qe) << 23);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int kk = 0; kk < KT; ++kk)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const uint32_t w = qf[kk][nt][j];
+          qf[kk][nt][j] = pack_f16x2(__uint_as_float(w << 16) * qs, __uint_as_float(w & 0xffff0000u) * qs);
+        }
   }
 
   float oacc[MT][NT][4];
@@ -269,60 +338,106 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
     const bool landed = wait_stage(smem_addr(full + st % NST), (st / NST) & 1, p.err);
 
     uint8_t *sK = smem + (st % NST) * STAGE_BYTES;
-    uint8_t *sV = sK + ST * ROWB;
+    uint8_t *sV = sK + HALF;
     const int tb = tu + st * ST;
     if (tb + ST > t1 || tb < tlo) {
       // the first and last stages: V rows outside [tlo, t1) (slots past L_b,
       // tokens before the window, rows of boxes not copied) are zeroed so that
       // their zero weights meet finite values
 #pragma unroll 1
-      for (int e = lane; e < 16 * CH; e += 32) {
-        const int r = tg * 16 + e / CH, c = e % CH;
+      for (int e = lane; e < TPW * 16 * CH; e += 32) {
+        const int r = 16 * ((e / (16 * CH)) * TG + tg) + (e / CH) % 16, c = e % CH;
         if (tb + r >= t1 || tb + r < tlo) {
           uint32_t rb, rk;
           row_base(r, rb, rk);
-          *reinterpret_cast<uint4 *>(sV + chunk(rb, rk, c >> 3, c & 7)) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4 *>(sV + chunk(rb, rk, c / CPB, c % CPB)) = make_uint4(0, 0, 0, 0);
         }
       }
       fence_proxy_async_smem();  // before the slot's next TMA write
       __syncwarp();
     }
-    const int tbase = tb + tg * 16;
-    if (tbase < t1 && tbase + 16 > tlo) {  // the tile holds a live token
-      // ---- S^T = K . Q^T over this token group's 16 tokens
-      float sc[NT][4], sc2[NT][4];
+    int tbase[TPW];
+    bool live = false;
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+    for (int i = 0; i < TPW; ++i) {
+      tbase[i] = tb + 16 * (i * TG + tg);
+      live = live || (tbase[i] < t1 && tbase[i] + 16 > tlo);
+    }
+    if (live) {  // one of the warp's tiles holds a live token
+      // ---- S^T = K . Q^T over each tile's 16 tokens
+      float sc[TPW][NT][4], sc2[TPW][NT][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) sc[nt][i] = sc2[nt][i] = 0.f;
+      for (int i = 0; i < TPW; ++i)
 #pragma unroll
-      for (int kk = 0; kk < KT; ++kk) {
-        uint32_t a[4];
-        ldsm_x4(a, smem_addr(sK + chunk(kb, kk_key, kk >> 2, ((kk * 2) & 7) + (lane >> 4))));
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          if (SPLIT_QK && (kk & 1))
-            mma_16816(sc2[nt], a, qf[kk][nt][0], qf[kk][nt][1]);
-          else
-            mma_16816(sc[nt], a, qf[kk][nt][0], qf[kk][nt][1]);
+          for (int j = 0; j < 4; ++j) sc[i][nt][j] = sc2[i][nt][j] = 0.f;
+#pragma unroll
+      for (int i = 0; i < TPW; ++i) {
+        if constexpr (F8) {
+          // one ldmatrix.x4 per two k-steps: r[0]/r[1] hold codes 32kp +
+          // 4(lane%4) .. +3 of tokens lane/4 and lane/4 + 8, r[2]/r[3] the next
+          // 16 bytes; each pair of codes widens to f16x2 exactly
+#pragma unroll
+          for (int kp = 0; kp < KT / 2; ++kp) {
+            uint32_t r[4];
+            const int cb = kp * 32 + (lane >> 4) * 16;
+            ldsm_x4(r, smem_addr(sK + chunk(kb[i], kk_key[i], cb / RW, (cb % RW) >> 4)));
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              const int kk = 2 * kp + hf;
+              uint32_t a[4];
+              a[0] = e4m3x2_to_f16x2(r[2 * hf]);
+              a[1] = e4m3x2_to_f16x2(r[2 * hf + 1]);
+              a[2] = e4m3x2_to_f16x2(r[2 * hf] >> 16);
+              a[3] = e4m3x2_to_f16x2(r[2 * hf + 1] >> 16);
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                if (SPLIT_QK && (kk & 1))
+                  mma_16816_f16(sc2[i][nt], a, qf[kk][nt][0], qf[kk][nt][1]);
+                else
+                  mma_16816_f16(sc[i][nt], a, qf[kk][nt][0], qf[kk][nt][1]);
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < KT; ++kk) {
+            uint32_t a[4];
+            ldsm_x4(a, smem_addr(sK + chunk(kb[i], kk_key[i], kk >> 2, ((kk * 2) & 7) + (lane >> 4))));
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              if (SPLIT_QK && (kk & 1))
+                mma_16816(sc2[i][nt], a, qf[kk][nt][0], qf[kk][nt][1]);
+              else
+                mma_16816(sc[i][nt], a, qf[kk][nt][0], qf[kk][nt][1]);
+            }
+          }
         }
       }
 
-      // ---- online softmax (rows lane/4 and lane/4 + 8; columns 2(lane%4) + {0,1})
-      const int ra = tbase + (lane >> 2), rb8 = ra + 8;
-      const bool okA = ra >= tlo && ra < t1;
-      const bool okB = rb8 >= tlo && rb8 < t1;
-      uint32_t pb[NT][2];
+      // ---- online softmax over the warp's tiles (rows lane/4 and lane/4 + 8 of
+      // each; columns 2(lane%4) + {0,1})
+      uint32_t pb[TPW][NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        if (SPLIT_QK)
+        float sv[TPW][4];
+        float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) sc[nt][i] += sc2[nt][i];
-        const float s0 = okA ? sc[nt][0] * p.scale_log2 : -INFINITY;
-        const float s1 = okA ? sc[nt][1] * p.scale_log2 : -INFINITY;
-        const float s2 = okB ? sc[nt][2] * p.scale_log2 : -INFINITY;
-        const float s3 = okB ? sc[nt][3] * p.scale_log2 : -INFINITY;
-        float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+        for (int i = 0; i < TPW; ++i) {
+          const int ra = tbase[i] + (lane >> 2), rb8 = ra + 8;
+          const bool okA = ra >= tlo && ra < t1;
+          const bool okB = rb8 >= tlo && rb8 < t1;
+          if (SPLIT_QK)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) sc[i][nt][j] += sc2[i][nt][j];
+          sv[i][0] = okA ? sc[i][nt][0] * sl2 : -INFINITY;
+          sv[i][1] = okA ? sc[i][nt][1] * sl2 : -INFINITY;
+          sv[i][2] = okB ? sc[i][nt][2] * sl2 : -INFINITY;
+          sv[i][3] = okB ? sc[i][nt][3] * sl2 : -INFINITY;
+          mx0 = fmaxf(mx0, fmaxf(sv[i][0], sv[i][2]));
+          mx1 = fmaxf(mx1, fmaxf(sv[i][1], sv[i][3]));
+        }
 #pragma unroll
         for (int off = 4; off < 32; off <<= 1) {
           mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
@@ -332,8 +447,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
         // it by more than kRescaleSlack (log2 units), so weights stay below
         // 2^kRescaleSlack and the O^T rescale is skipped on almost every tile.
         // Any reference point gives the same out and lse as long as l and O^T
-        // share it.  The tile holds a live token, so mx0/mx1 are finite and
-        // the first tile always sets the reference.
+        // share it.  A tile holds a live token, so mx0/mx1 are finite and the
+        // first step always sets the reference.
         if (__any_sync(0xffffffffu, mx0 > m_run[nt][0] + kRescaleSlack || mx1 > m_run[nt][1] + kRescaleSlack)) {
           const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
           const float al0 = fast_exp2(m_run[nt][0] - mn0), al1 = fast_exp2(m_run[nt][1] - mn1);
@@ -349,27 +464,61 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
             oacc[mt][nt][3] *= al1;
           }
         }
-        const float e0 = fast_exp2(s0 - m_run[nt][0]), e1 = fast_exp2(s1 - m_run[nt][1]);
-        const float e2 = fast_exp2(s2 - m_run[nt][0]), e3 = fast_exp2(s3 - m_run[nt][1]);
-        const uint32_t pA = pack_bf16x2(e0, e1);
-        const uint32_t pB = pack_bf16x2(e2, e3);
-        // The running sum takes the fp32 weights: summing the bf16-rounded ones
-        // moves the LSE of a short sequence by up to 2^-9 (one weight's rounding).
-        l_run[nt][0] += e0 + e2;
-        l_run[nt][1] += e1 + e3;
-        pb[nt][0] = movmatrix_t(pA);
-        pb[nt][1] = movmatrix_t(pB);
+#pragma unroll
+        for (int i = 0; i < TPW; ++i) {
+          const float e0 = fast_exp2(sv[i][0] - m_run[nt][0]), e1 = fast_exp2(sv[i][1] - m_run[nt][1]);
+          const float e2 = fast_exp2(sv[i][2] - m_run[nt][0]), e3 = fast_exp2(sv[i][3] - m_run[nt][1]);
+          const uint32_t pA = F8 ? pack_f16x2(e0, e1) : pack_bf16x2(e0, e1);
+          const uint32_t pB = F8 ? pack_f16x2(e2, e3) : pack_bf16x2(e2, e3);
+          // The running sum takes the fp32 weights: summing the rounded ones
+          // moves the LSE of a short sequence by up to 2^-9 (one weight's rounding).
+          l_run[nt][0] += e0 + e2;
+          l_run[nt][1] += e1 + e3;
+          pb[i][nt][0] = movmatrix_t(pA);
+          pb[i][nt][1] = movmatrix_t(pB);
+        }
       }
 
-      // ---- O^T += V^T . P^T over this warp's head_dim rows (rows past t1 were
-      // zero-filled, their weights are 0)
+      // ---- O^T += V^T . P^T over this warp's head_dim rows (rows outside
+      // [tlo, t1) were zero-filled, their weights are 0)
+      if constexpr (F8) {
+        // one transposed ldmatrix.x4 per two m-tiles: r[0]/r[1] hold, for
+        // tokens 2(lane%4) and +1 (of 0-7 / 8-15), the codes of head_dim
+        // 16gm + 2(lane/4) and +1; r[2]/r[3] the same of m-tile gm + 1.  A
+        // byte permute pairs the two tokens of each head_dim row.
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        const int gm = dh * MT + mt;  // m-tile of head_dim rows
-        uint32_t a[4];
-        ldsm_x4_t(a, smem_addr(sV + chunk(vb, vkey, gm >> 2, ((gm * 2) & 7) + ((lane >> 3) & 1))));
+        for (int mp = 0; mp < MT / 2; ++mp) {
+          const int gm = dh * MT + 2 * mp;
+          const int cb = (gm + (lane >> 4)) * 16;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_16816(oacc[mt][nt], a, pb[nt][0], pb[nt][1]);
+          for (int i = 0; i < TPW; ++i) {
+            uint32_t r[4];
+            ldsm_x4_t(r, smem_addr(sV + chunk(vb[i], vkey[i], cb / RW, (cb % RW) >> 4)));
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              const uint32_t x0 = byte_perm(r[2 * hf], 0x3120), x1 = byte_perm(r[2 * hf + 1], 0x3120);
+              uint32_t a[4];
+              a[0] = e4m3x2_to_f16x2(x0);
+              a[1] = e4m3x2_to_f16x2(x0 >> 16);
+              a[2] = e4m3x2_to_f16x2(x1);
+              a[3] = e4m3x2_to_f16x2(x1 >> 16);
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) mma_16816_f16(oacc[2 * mp + hf][nt], a, pb[i][nt][0], pb[i][nt][1]);
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const int gm = dh * MT + mt;  // m-tile of head_dim rows
+#pragma unroll
+          for (int i = 0; i < TPW; ++i) {
+            uint32_t a[4];
+            ldsm_x4_t(a, smem_addr(sV + chunk(vb[i], vkey[i], gm >> 2, ((gm * 2) & 7) + ((lane >> 3) & 1))));
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_16816(oacc[mt][nt], a, pb[i][nt][0], pb[i][nt][1]);
+          }
+        }
       }
     }
     // every warp is done with slot st % NST before it is refilled; a stage
@@ -408,12 +557,14 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
     }
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
-      const int d = (dh * MT + mt) * 16 + (lane >> 2);
+      // accumulator rows lane/4 and lane/4 + 8 are head_dim rows d and d2
+      const int d = (dh * MT + mt) * 16 + (F8 ? 2 : 1) * (lane >> 2);
+      const int d2 = d + (F8 ? 1 : 8);
       float *o0 = sm_o + (tg * HPT + nt * 8 + (lane & 3) * 2) * MROW;
       o0[d] = oacc[mt][nt][0];
       o0[MROW + d] = oacc[mt][nt][1];
-      o0[d + 8] = oacc[mt][nt][2];
-      o0[MROW + d + 8] = oacc[mt][nt][3];
+      o0[d2] = oacc[mt][nt][2];
+      o0[MROW + d2] = oacc[mt][nt][3];
     }
   }
   __syncthreads();
@@ -438,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
       o.z += f * ow.z;
       o.w += f * ow.w;
     }
-    const float inv = 1.f / l;
+    const float inv = (F8 ? p.v_scale : 1.f) / l;  // out carries v_scale, lse does not
     const float lse_nat = (m + log2f(l)) * kLn2;
     const int h = h0 + hl;
     if (ns == 1) {
@@ -466,38 +617,44 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT))
     merge_partials<D, kThreads>(p, b, h0, gl, s_first, ns, reinterpret_cast<float *>(smem));  // the ring is free
 }
 
-int partition_stages(int D, int hpt) { return stages_for(D, hpt); }
+int partition_stages(int D, int hpt, bool kv_fp8) { return stages_for(D, hpt, kv_fp8); }
 
-template <int D, int HPT>
+template <int D, int HPT, bool F8>
 static cudaError_t launch_t(const PartitionParams &p, int grid, cudaStream_t stream) {
   static std::atomic<uint64_t> attr_done{0};
-  constexpr SmemPlan SP = smem_plan_for(D, HPT);
+  constexpr SmemPlan SP = smem_plan_for(D, HPT, F8);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_done.load(std::memory_order_acquire) & bit)) {
-    e = cudaFuncSetAttribute(partition_kernel<D, HPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SP.total);
+    e = cudaFuncSetAttribute(partition_kernel<D, HPT, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SP.total);
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(bit, std::memory_order_acq_rel);
   }
-  partition_kernel<D, HPT><<<grid, kThreads, SP.total, stream>>>(p);
+  partition_kernel<D, HPT, F8><<<grid, kThreads, SP.total, stream>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_partition(const PartitionParams &p, int D, int heads_per_tile, int grid, cudaStream_t s) {
-  if (heads_per_tile > max_heads_per_tile(D)) return cudaErrorInvalidValue;
+template <bool F8>
+static cudaError_t launch_f(const PartitionParams &p, int D, int heads_per_tile, int grid, cudaStream_t s) {
   switch (D * 64 + heads_per_tile) {
-    case 64 * 64 + 8: return launch_t<64, 8>(p, grid, s);
-    case 64 * 64 + 16: return launch_t<64, 16>(p, grid, s);
-    case 64 * 64 + 32: return launch_t<64, 32>(p, grid, s);
-    case 128 * 64 + 8: return launch_t<128, 8>(p, grid, s);
-    case 128 * 64 + 16: return launch_t<128, 16>(p, grid, s);
-    case 128 * 64 + 32: return launch_t<128, 32>(p, grid, s);
-    case 256 * 64 + 8: return launch_t<256, 8>(p, grid, s);
-    case 256 * 64 + 16: return launch_t<256, 16>(p, grid, s);
+    case 64 * 64 + 8: return launch_t<64, 8, F8>(p, grid, s);
+    case 64 * 64 + 16: return launch_t<64, 16, F8>(p, grid, s);
+    case 64 * 64 + 32: return launch_t<64, 32, F8>(p, grid, s);
+    case 128 * 64 + 8: return launch_t<128, 8, F8>(p, grid, s);
+    case 128 * 64 + 16: return launch_t<128, 16, F8>(p, grid, s);
+    case 128 * 64 + 32: return launch_t<128, 32, F8>(p, grid, s);
+    case 256 * 64 + 8: return launch_t<256, 8, F8>(p, grid, s);
+    case 256 * 64 + 16: return launch_t<256, 16, F8>(p, grid, s);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_partition(const PartitionParams &p, int D, int heads_per_tile, bool kv_fp8, int grid,
+                             cudaStream_t s) {
+  if (heads_per_tile > max_heads_per_tile(D)) return cudaErrorInvalidValue;
+  return kv_fp8 ? launch_f<true>(p, D, heads_per_tile, grid, s) : launch_f<false>(p, D, heads_per_tile, grid, s);
 }
 
 cudaError_t device_error_word(int device, uint32_t **ptr) {

@@ -19,6 +19,12 @@ def bf16_dev(a: np.ndarray, dev) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).to(dev)
 
 
+def kv_dev(a: np.ndarray, dev) -> torch.Tensor:
+    """A cache array on the device: uint16 bf16 bits, or uint8 E4M3 codes."""
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    return t.view(torch.float8_e4m3fn if a.dtype == np.uint8 else torch.bfloat16).to(dev)
+
+
 class DeviceWorkload:
     """A workload's tensors on the device.  layout "hnd" keeps the cache as
     [blocks, Hkv, bs, D]; "nhd" stores it [blocks, bs, Hkv, D] and passes the
@@ -28,11 +34,11 @@ class DeviceWorkload:
         self.w = w
         self.q = bf16_dev(w.q, dev)
         if layout == "hnd":
-            self.k = bf16_dev(w.k_cache, dev)
-            self.v = bf16_dev(w.v_cache, dev)
+            self.k = kv_dev(w.k_cache, dev)
+            self.v = kv_dev(w.v_cache, dev)
         elif layout == "nhd":
-            self.k = bf16_dev(w.k_cache.transpose(0, 2, 1, 3), dev).transpose(1, 2)
-            self.v = bf16_dev(w.v_cache.transpose(0, 2, 1, 3), dev).transpose(1, 2)
+            self.k = kv_dev(w.k_cache.transpose(0, 2, 1, 3), dev).transpose(1, 2)
+            self.v = kv_dev(w.v_cache.transpose(0, 2, 1, 3), dev).transpose(1, 2)
         else:
             raise ValueError(layout)
         self.tables = torch.from_numpy(w.block_tables).to(dev)
@@ -51,7 +57,9 @@ class DeviceWorkload:
             if lse_t is not None:
                 lse_t.fill_(float("nan"))
         splits = w.num_splits if num_splits is None else num_splits
-        entry(self.q, self.k, self.v, self.tables, self.lens, w.scale, num_splits=splits, out=out, lse=lse_t)
+        scales = dict(k_scale=w.k_scale, v_scale=w.v_scale) if w.kv_dtype == "e4m3" else {}
+        entry(self.q, self.k, self.v, self.tables, self.lens, w.scale, num_splits=splits, out=out, lse=lse_t,
+              **scales)
         torch.cuda.synchronize(self.dev)
         return out, lse_t
 
