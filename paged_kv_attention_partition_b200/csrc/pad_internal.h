@@ -31,13 +31,11 @@ constexpr int kMaxSplits = 256;      // partitions per sequence (bounds the merg
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 __host__ __device__ constexpr int dsplit_for(int D, int hpt) { return D == 256 ? 2 : 1; }
-// 16-token tiles a token group computes per stage.  An E4M3 stage carries the
-// same bytes as a bf16 one with twice the tokens: with 8- or 16-head tiles at
-// D >= 128 each group takes two tiles per stage (two independent QK chains,
-// one max exchange and one rescale check for both), which the math needs to
-// keep up with the halved bytes per token.
+// 16-token tiles a token group computes per stage: two for an E4M3 cache at
+// D = 256 (8- or 16-head tiles), whose stage then carries as many bytes as a
+// bf16 one with twice the tokens; one elsewhere.
 __host__ __device__ constexpr int tiles_per_group(int D, int hpt, bool f8 = false) {
-  return f8 && D >= 128 && hpt <= 16 ? 2 : 1;
+  return f8 && D == 256 && hpt <= 16 ? 2 : 1;
 }
 __host__ __device__ constexpr int stage_tokens_for(int D, int hpt, bool f8 = false) {
   return 16 * kWarps / dsplit_for(D, hpt) * tiles_per_group(D, hpt, f8);
@@ -46,16 +44,20 @@ __host__ __device__ constexpr int stage_tokens_for(int D, int hpt, bool f8 = fal
 // Pipeline depth and resident CTAs per SM of one (head_dim, heads-per-tile,
 // cache type) instantiation.  The ring is kept small so that several CTAs
 // share each SM: their loads, math and start/finish latencies overlap one
-// another.  An E4M3 stage of one tile per group holds the same tokens in half
-// the bytes, so it runs twice the stages (the same bytes in flight); at D = 64
-// its 64-byte rows sit in boxes of at least 128 bytes, which caps it at three.
-// With two tiles per group an E4M3 stage is as large as a bf16 one.
+// another.  The math is latency bound, so resident warps decide the speed:
+// an E4M3 cache at D = 128 with 8 or 16 heads per tile keeps two 16 KB stages
+// and runs five (8 heads) or four (16 heads, whose accumulators would spill at
+// five) CTAs per SM, registers capped to fit -- measured against deeper rings
+// and two-tile stages at 2-4 CTAs per SM, which were slower.
+// At D = 64 its 64-byte rows sit in boxes of at least 128 bytes, which caps
+// it at three stages; 32-head tiles keep six stages of half the bf16 bytes.
 __host__ __device__ constexpr int stages_for(int D, int hpt, bool f8 = false) {
-  return f8 ? (tiles_per_group(D, hpt, f8) == 2 ? 2 : D == 64 ? 3 : 6)
+  return f8 ? (tiles_per_group(D, hpt, f8) == 2 || (D == 128 && hpt <= 16) ? 2 : D == 64 ? 3 : 6)
             : (D == 64 || (D == 128 && hpt == 32) ? 3 : 2);
 }
 __host__ __device__ constexpr int ctas_per_sm_for(int D, int hpt, bool f8 = false) {
-  return D == 64 ? (hpt == 32 ? 3 : 4) : D == 128 ? (hpt == 32 ? 2 : 3) : (hpt == 16 ? 2 : 3);
+  return f8 && D == 128 && hpt <= 16 ? (hpt == 8 ? 5 : 4)
+                                     : D == 64 ? (hpt == 32 ? 3 : 4) : D == 128 ? (hpt == 32 ? 2 : 3) : (hpt == 16 ? 2 : 3);
 }
 // Bytes of one K (or V) half-stage: bf16 rows of 2D bytes; E4M3 rows of D
 // bytes, in boxes padded to at least 128 bytes (only D = 64 with one-row boxes

@@ -106,7 +106,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
   constexpr int CPB = RW / 16;             // 16-byte chunks per column block
   constexpr int HALF = half_stage_bytes(D, HPT, F8);  // K (or V) rows of one stage
   constexpr int IDW = (ST + 31) / 32;      // block ids per lane of warp 0 for one stage
-  constexpr bool SPLIT_QK = NT <= 2;       // two QK accumulation chains when registers allow
+  constexpr int NCH = NT == 1 ? 4 : NT == 2 ? 2 : 1;  // independent QK accumulation chains (registers allow)
+  static_assert(KT % NCH == 0, "k-steps split evenly over the chains");
   static_assert(ST == 16 * TG * TPW && (1 << ST_LOG2) == ST, "stage shape");
   static_assert(!F8 || (KT % 2 == 0 && MT % 2 == 0), "E4M3 operands are loaded two k-steps / m-tiles at a time");
   static_assert(NST >= 2 && NST <= 8, "at least one stage in flight during the math; barrier area");
@@ -364,14 +365,17 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
       live = live || (tbase[i] < t1 && tbase[i] + 16 > tlo);
     }
     if (live) {  // one of the warp's tiles holds a live token
-      // ---- S^T = K . Q^T over each tile's 16 tokens
-      float sc[TPW][NT][4], sc2[TPW][NT][4];
+      // ---- S^T = K . Q^T over each tile's 16 tokens; k-step kk accumulates
+      // into chain kk % NCH, so NCH MMA chains run side by side
+      float sc[NCH][TPW][NT][4];
 #pragma unroll
-      for (int i = 0; i < TPW; ++i)
+      for (int c = 0; c < NCH; ++c)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int i = 0; i < TPW; ++i)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) sc[i][nt][j] = sc2[i][nt][j] = 0.f;
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) sc[c][i][nt][j] = 0.f;
 #pragma unroll
       for (int i = 0; i < TPW; ++i) {
         if constexpr (F8) {
@@ -392,12 +396,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
               a[2] = e4m3x2_to_f16x2(r[2 * hf] >> 16);
               a[3] = e4m3x2_to_f16x2(r[2 * hf + 1] >> 16);
 #pragma unroll
-              for (int nt = 0; nt < NT; ++nt) {
-                if (SPLIT_QK && (kk & 1))
-                  mma_16816_f16(sc2[i][nt], a, qf[kk][nt][0], qf[kk][nt][1]);
-                else
-                  mma_16816_f16(sc[i][nt], a, qf[kk][nt][0], qf[kk][nt][1]);
-              }
+              for (int nt = 0; nt < NT; ++nt) mma_16816_f16(sc[kk % NCH][i][nt], a, qf[kk][nt][0], qf[kk][nt][1]);
             }
           }
         } else {
@@ -406,12 +405,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
             uint32_t a[4];
             ldsm_x4(a, smem_addr(sK + chunk(kb[i], kk_key[i], kk >> 2, ((kk * 2) & 7) + (lane >> 4))));
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              if (SPLIT_QK && (kk & 1))
-                mma_16816(sc2[i][nt], a, qf[kk][nt][0], qf[kk][nt][1]);
-              else
-                mma_16816(sc[i][nt], a, qf[kk][nt][0], qf[kk][nt][1]);
-            }
+            for (int nt = 0; nt < NT; ++nt) mma_16816(sc[kk % NCH][i][nt], a, qf[kk][nt][0], qf[kk][nt][1]);
           }
         }
       }
@@ -422,34 +416,47 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         float sv[TPW][4];
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+        bool over = false;  // a score of this lane passes its head's reference by more than the slack
 #pragma unroll
         for (int i = 0; i < TPW; ++i) {
           const int ra = tbase[i] + (lane >> 2), rb8 = ra + 8;
           const bool okA = ra >= tlo && ra < t1;
           const bool okB = rb8 >= tlo && rb8 < t1;
-          if (SPLIT_QK)
+          float acc[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) sc[i][nt][j] += sc2[i][nt][j];
-          sv[i][0] = okA ? sc[i][nt][0] * sl2 : -INFINITY;
-          sv[i][1] = okA ? sc[i][nt][1] * sl2 : -INFINITY;
-          sv[i][2] = okB ? sc[i][nt][2] * sl2 : -INFINITY;
-          sv[i][3] = okB ? sc[i][nt][3] * sl2 : -INFINITY;
-          mx0 = fmaxf(mx0, fmaxf(sv[i][0], sv[i][2]));
-          mx1 = fmaxf(mx1, fmaxf(sv[i][1], sv[i][3]));
-        }
+          for (int j = 0; j < 4; ++j) {
+            acc[j] = sc[0][i][nt][j];
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+            for (int c = 1; c < NCH; ++c) acc[j] += sc[c][i][nt][j];
+          }
+          sv[i][0] = okA ? acc[0] * sl2 : -INFINITY;
+          sv[i][1] = okA ? acc[1] * sl2 : -INFINITY;
+          sv[i][2] = okB ? acc[2] * sl2 : -INFINITY;
+          sv[i][3] = okB ? acc[3] * sl2 : -INFINITY;
+          over = over || fmaxf(sv[i][0], sv[i][2]) > m_run[nt][0] + kRescaleSlack ||
+                 fmaxf(sv[i][1], sv[i][3]) > m_run[nt][1] + kRescaleSlack;
         }
         // Lazy rescale: a head's reference max moves only when a score passes
         // it by more than kRescaleSlack (log2 units), so weights stay below
         // 2^kRescaleSlack and the O^T rescale is skipped on almost every tile.
         // Any reference point gives the same out and lse as long as l and O^T
-        // share it.  A tile holds a live token, so mx0/mx1 are finite and the
-        // first step always sets the reference.
-        if (__any_sync(0xffffffffu, mx0 > m_run[nt][0] + kRescaleSlack || mx1 > m_run[nt][1] + kRescaleSlack)) {
+        // share it.  The reference is uniform over the eight lanes that hold a
+        // head, so each lane tests its own scores and one vote decides; the
+        // tile's maximum (three shuffle rounds) is taken only when the
+        // reference moves.  A tile holds a live token and the first reference is
+        // -inf, so the first step always sets it.
+        if (__any_sync(0xffffffffu, over)) {
+          float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < TPW; ++i) {
+            mx0 = fmaxf(mx0, fmaxf(sv[i][0], sv[i][2]));
+            mx1 = fmaxf(mx1, fmaxf(sv[i][1], sv[i][3]));
+          }
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+          }
           const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
           const float al0 = fast_exp2(m_run[nt][0] - mn0), al1 = fast_exp2(m_run[nt][1] - mn1);
           m_run[nt][0] = mn0;

@@ -187,12 +187,12 @@ def test_binding_has_no_cpu_path():
 
 def test_e4m3_plan_keeps_partitions_and_scratch(lib):
     # an E4M3 cache streams the same tokens in half the bytes: the same
-    # partitions and scratch; stages of twice the tokens (two 16-token tiles per
-    # token group) where the group fits 8 or 16 heads at D >= 128, else twice
-    # the stages (three at D = 64)
-    for shape, stage_tokens, stages in (((32, 32, 8, 128, 16, 256), 128, 2), ((256, 32, 1, 128, 32, 1024), 64, 6),
+    # partitions and scratch; at D = 128 (8/16-head tiles) two 64-token stages
+    # of half the bytes, at D = 256 two stages of twice the tokens, at D = 64
+    # three stages, for 32-head tiles six
+    for shape, stage_tokens, stages in (((32, 32, 8, 128, 16, 256), 64, 2), ((256, 32, 1, 128, 32, 1024), 64, 6),
                                         ((16, 16, 4, 256, 16, 2048), 64, 2), ((4, 16, 2, 64, 4, 100), 64, 3),
-                                        ((2, 32, 2, 128, 16, 64), 128, 2)):
+                                        ((2, 32, 2, 128, 16, 64), 64, 2)):
         b = pad.pad_decode_plan(*shape, num_splits=0, device=0)
         f = pad.pad_decode_plan(*shape, num_splits=0, device=0, kv_dtype="e4m3")
         for k in ("num_splits", "partition_tokens", "heads_per_tile", "head_tiles", "ctas", "workspace_bytes",
