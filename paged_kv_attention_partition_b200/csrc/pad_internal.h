@@ -17,12 +17,17 @@ enum : uint32_t {
 };
 
 // Kernel geometry: one CTA of 4 warps per work unit; one thread issues the
-// stage copies (TMA), all four warps compute.  The warps form kWarps / dsplit token groups of dsplit warps each: token group
-// tg computes tokens 16 tg .. 16 tg + 15 of every shared-memory stage (so a
-// stage holds 16 kWarps / dsplit tokens), and warp dh of the group keeps the
-// dh-th 1/dsplit of the head_dim rows of O^T (both warps of a group compute
-// the same scores).  Splitting head_dim halves the stage and the accumulator
-// where they would otherwise limit residency: at D = 256 (64 KB stages).
+// stage copies (TMA), all four warps compute.  A warp is (token group tg, head
+// group hg, head_dim part dh):
+//   - head groups split a head tile's 8-head n-tiles between warps: with 16 or
+//     32 heads per tile each warp owns one n-tile and computes every token of the
+//     stage for it (a quarter or half of the accumulator a warp holding the whole
+//     tile would need, and each head's softmax stays inside one warp);
+//   - head_dim parts split O^T's rows between the two warps of a pair that
+//     compute the same scores (D = 256, where a stage and the accumulator would
+//     otherwise limit residency);
+//   - the remaining warps form token groups: group tg computes 16-token tiles
+//     tg, tg + TG, ... of every stage, and the groups merge at the end.
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kSmemBudget = 232448;  // 227 KiB per CTA
@@ -31,14 +36,22 @@ constexpr int kMaxSplits = 256;      // partitions per sequence (bounds the merg
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 __host__ __device__ constexpr int dsplit_for(int D, int hpt) { return D == 256 ? 2 : 1; }
-// 16-token tiles a token group computes per stage: two for an E4M3 cache at
-// D = 256 (8- or 16-head tiles), whose stage then carries as many bytes as a
-// bf16 one with twice the tokens; one elsewhere.
-__host__ __device__ constexpr int tiles_per_group(int D, int hpt, bool f8 = false) {
-  return f8 && D == 256 && hpt <= 16 ? 2 : 1;
+__host__ __device__ constexpr int head_groups_for(int D, int hpt) {
+  return (hpt / 8) * dsplit_for(D, hpt) <= kWarps ? hpt / 8 : kWarps / dsplit_for(D, hpt);
 }
+__host__ __device__ constexpr int token_groups_for(int D, int hpt) {
+  return kWarps / (dsplit_for(D, hpt) * head_groups_for(D, hpt));
+}
+// Tokens of one pipeline stage: 64; 32 at D = 256, whose rows are twice as
+// long, and for bf16 32-head tiles at D = 128, whose 16 KB stages let four CTAs
+// share an SM; an E4M3 cache at D = 256 with 8 or 16 heads per tile doubles
+// them, so its stage carries as many bytes as a bf16 one.
 __host__ __device__ constexpr int stage_tokens_for(int D, int hpt, bool f8 = false) {
-  return 16 * kWarps / dsplit_for(D, hpt) * tiles_per_group(D, hpt, f8);
+  return (D == 256 || (D == 128 && hpt == 32 && !f8) ? 32 : 64) * (f8 && D == 256 && hpt <= 16 ? 2 : 1);
+}
+// 16-token tiles a warp computes per stage.
+__host__ __device__ constexpr int tiles_per_group(int D, int hpt, bool f8 = false) {
+  return stage_tokens_for(D, hpt, f8) / (16 * token_groups_for(D, hpt));
 }
 
 // Pipeline depth and resident CTAs per SM of one (head_dim, heads-per-tile,
@@ -50,14 +63,16 @@ __host__ __device__ constexpr int stage_tokens_for(int D, int hpt, bool f8 = fal
 // five) CTAs per SM, registers capped to fit -- measured against deeper rings
 // and two-tile stages at 2-4 CTAs per SM, which were slower.
 // At D = 64 its 64-byte rows sit in boxes of at least 128 bytes, which caps
-// it at three stages; 32-head tiles keep six stages of half the bf16 bytes.
+// it at three stages.  32-head tiles at D = 128 (one n-tile per warp, 128
+// registers) run three 16 KB stages and four CTAs per SM for either cache
+// type, measured against two 32 KB stages at three CTAs (ragged MQA batch:
+// 177 -> 157 us bf16, 165 -> 159 us E4M3).
 __host__ __device__ constexpr int stages_for(int D, int hpt, bool f8 = false) {
-  return f8 ? (tiles_per_group(D, hpt, f8) == 2 || (D == 128 && hpt <= 16) ? 2 : D == 64 ? 3 : 6)
-            : (D == 64 || (D == 128 && hpt == 32) ? 3 : 2);
+  return f8 ? (D == 256 || (D == 128 && hpt <= 16) ? 2 : 3) : (D == 64 || (D == 128 && hpt == 32) ? 3 : 2);
 }
 __host__ __device__ constexpr int ctas_per_sm_for(int D, int hpt, bool f8 = false) {
-  return f8 && D == 128 && hpt <= 16 ? (hpt == 8 ? 5 : 4)
-                                     : D == 64 ? (hpt == 32 ? 3 : 4) : D == 128 ? (hpt == 32 ? 2 : 3) : (hpt == 16 ? 2 : 3);
+  return f8 && D == 128 ? (hpt == 8 ? 5 : 4)
+                        : D == 64 ? (hpt == 32 ? 3 : 4) : D == 128 ? (hpt == 32 ? 4 : 3) : (hpt == 16 ? 2 : 3);
 }
 // Bytes of one K (or V) half-stage: bf16 rows of 2D bytes; E4M3 rows of D
 // bytes, in boxes padded to at least 128 bytes (only D = 64 with one-row boxes
@@ -81,7 +96,7 @@ __host__ __device__ constexpr SmemPlan smem_plan_for(int D, int hpt, bool f8 = f
   s.stage_tokens = stage_tokens_for(D, hpt, f8);
   s.stage_bytes = (size_t)half_stage_bytes(D, hpt, f8) * 2;  // K and V rows of one stage
   s.ring_bytes = (size_t)s.stages * s.stage_bytes;
-  s.warp_merge_bytes = (size_t)(kWarps / dsplit_for(D, hpt)) * hpt * (D + 4 + 2) * 4;  // padded rows, m, l
+  s.warp_merge_bytes = (size_t)token_groups_for(D, hpt) * hpt * (D + 4 + 2) * 4;  // padded rows, m, l
   s.split_merge_bytes = (size_t)hpt * (kMaxSplits + 1) * 4;
   size_t m = s.ring_bytes;
   if (s.warp_merge_bytes > m) m = s.warp_merge_bytes;

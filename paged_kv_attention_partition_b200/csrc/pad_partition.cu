@@ -94,10 +94,12 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
   constexpr uint32_t STAGE_BYTES = (uint32_t)SP.stage_bytes;
   constexpr int ST = SP.stage_tokens;      // tokens per stage
   constexpr int ST_LOG2 = ST == 128 ? 7 : ST == 64 ? 6 : 5;
-  constexpr int DS = dsplit_for(D, HPT);   // warps sharing a token group (head_dim split)
-  constexpr int TG = kWarps / DS;          // token groups
-  constexpr int TPW = tiles_per_group(D, HPT, F8);  // 16-token tiles per token group per stage
-  constexpr int NT = HPT / 8;              // 8-head n-tiles
+  constexpr int DS = dsplit_for(D, HPT);   // warps sharing a token group's scores (head_dim split)
+  constexpr int HG = head_groups_for(D, HPT);  // warps splitting the tile's n-tiles
+  constexpr int TG = token_groups_for(D, HPT);  // token groups
+  constexpr int TPW = tiles_per_group(D, HPT, F8);  // 16-token tiles per warp per stage
+  constexpr int NT = HPT / 8;              // 8-head n-tiles of the head tile
+  constexpr int NTW = NT / HG;             // n-tiles of one warp
   constexpr int KT = D / 16;               // QK k-steps
   constexpr int MT = KT / DS;              // PV m-tiles (16 head_dim rows each) per warp
   constexpr int ROWB = F8 ? D : D * 2;     // bytes per K/V row
@@ -106,9 +108,11 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
   constexpr int CPB = RW / 16;             // 16-byte chunks per column block
   constexpr int HALF = half_stage_bytes(D, HPT, F8);  // K (or V) rows of one stage
   constexpr int IDW = (ST + 31) / 32;      // block ids per lane of warp 0 for one stage
-  constexpr int NCH = NT == 1 ? 4 : NT == 2 ? 2 : 1;  // independent QK accumulation chains (registers allow)
+  // independent QK accumulation chains per tile (four in all where registers allow)
+  constexpr int NCH = NTW == 1 ? (TPW >= 4 ? 1 : 4 / TPW) : NTW == 2 && TPW == 1 ? 2 : 1;
   static_assert(KT % NCH == 0, "k-steps split evenly over the chains");
   static_assert(ST == 16 * TG * TPW && (1 << ST_LOG2) == ST, "stage shape");
+  static_assert(DS * HG * TG == kWarps && NTW * HG == NT, "warp roles");
   static_assert(!F8 || (KT % 2 == 0 && MT % 2 == 0), "E4M3 operands are loaded two k-steps / m-tiles at a time");
   static_assert(NST >= 2 && NST <= 8, "at least one stage in flight during the math; barrier area");
   static_assert(SP.total <= (size_t)kSmemBudget, "shared-memory plan over budget");
@@ -118,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
   int *flag = reinterpret_cast<int *>(smem + SP.region_bytes + 64);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tg = warp / DS, dh = warp % DS;  // token group, head_dim part
+  const int dh = warp % DS, hg = (warp / DS) % HG, tg = warp / (DS * HG);  // head_dim part, head group, token group
   uint32_t u = blockIdx.x;
   const int s = (int)(u % (uint32_t)p.S);
   u /= (uint32_t)p.S;
@@ -266,15 +270,15 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
   // 2^qe, qe chosen so that the tile's largest |q| lies in [2^14, 2^15), which
   // keeps every bf16 value exact (down to 2^-28 of that largest, where f16 turns
   // subnormal), and 2^-qe joins the score scale.
-  uint32_t qf[KT][NT][2];
+  uint32_t qf[KT][NTW][2];
   float sl2 = p.scale_log2;
   auto q_row = [&](int nt, bool &ok) -> const uint16_t * {
-    const int hl = nt * 8 + (lane >> 2);
+    const int hl = (hg * NTW + nt) * 8 + (lane >> 2);
     ok = hl < gl;
     return p.q + b * p.q_sb + (int64_t)(h0 + (ok ? hl : 0)) * p.q_sh + (lane & 3) * (F8 ? 4 : 2);
   };
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
+  for (int nt = 0; nt < NTW; ++nt) {
     bool ok;
     const uint16_t *qr = q_row(nt, ok);
 #pragma unroll
@@ -286,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
   if constexpr (F8) {
     float amax = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int nt = 0; nt < NTW; ++nt)
 #pragma unroll
       for (int kk = 0; kk < KT; ++kk)
 #pragma unroll
@@ -302,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
     const float qs = __int_as_float((127 + qe) << 23);
     sl2 = p.scale_log2 * __int_as_float((127 - qe) << 23);
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int nt = 0; nt < NTW; ++nt)
 #pragma unroll
       for (int kk = 0; kk < KT; ++kk)
 #pragma unroll
@@ -312,10 +316,10 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
         }
   }
 
-  float oacc[MT][NT][4];
-  float m_run[NT][2], l_run[NT][2];
+  float oacc[MT][NTW][4];
+  float m_run[NTW][2], l_run[NTW][2];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
+  for (int nt = 0; nt < NTW; ++nt) {
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       m_run[nt][j] = -INFINITY;
@@ -367,13 +371,13 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
     if (live) {  // one of the warp's tiles holds a live token
       // ---- S^T = K . Q^T over each tile's 16 tokens; k-step kk accumulates
       // into chain kk % NCH, so NCH MMA chains run side by side
-      float sc[NCH][TPW][NT][4];
+      float sc[NCH][TPW][NTW][4];
 #pragma unroll
       for (int c = 0; c < NCH; ++c)
 #pragma unroll
         for (int i = 0; i < TPW; ++i)
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
+          for (int nt = 0; nt < NTW; ++nt)
 #pragma unroll
             for (int j = 0; j < 4; ++j) sc[c][i][nt][j] = 0.f;
 #pragma unroll
@@ -396,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
               a[2] = e4m3x2_to_f16x2(r[2 * hf] >> 16);
               a[3] = e4m3x2_to_f16x2(r[2 * hf + 1] >> 16);
 #pragma unroll
-              for (int nt = 0; nt < NT; ++nt) mma_16816_f16(sc[kk % NCH][i][nt], a, qf[kk][nt][0], qf[kk][nt][1]);
+              for (int nt = 0; nt < NTW; ++nt) mma_16816_f16(sc[kk % NCH][i][nt], a, qf[kk][nt][0], qf[kk][nt][1]);
             }
           }
         } else {
@@ -405,16 +409,16 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
             uint32_t a[4];
             ldsm_x4(a, smem_addr(sK + chunk(kb[i], kk_key[i], kk >> 2, ((kk * 2) & 7) + (lane >> 4))));
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_16816(sc[kk % NCH][i][nt], a, qf[kk][nt][0], qf[kk][nt][1]);
+            for (int nt = 0; nt < NTW; ++nt) mma_16816(sc[kk % NCH][i][nt], a, qf[kk][nt][0], qf[kk][nt][1]);
           }
         }
       }
 
       // ---- online softmax over the warp's tiles (rows lane/4 and lane/4 + 8 of
       // each; columns 2(lane%4) + {0,1})
-      uint32_t pb[TPW][NT][2];
+      uint32_t pb[TPW][NTW][2];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
+      for (int nt = 0; nt < NTW; ++nt) {
         float sv[TPW][4];
         bool over = false;  // a score of this lane passes its head's reference by more than the slack
 #pragma unroll
@@ -510,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
               a[2] = e4m3x2_to_f16x2(x1);
               a[3] = e4m3x2_to_f16x2(x1 >> 16);
 #pragma unroll
-              for (int nt = 0; nt < NT; ++nt) mma_16816_f16(oacc[2 * mp + hf][nt], a, pb[i][nt][0], pb[i][nt][1]);
+              for (int nt = 0; nt < NTW; ++nt) mma_16816_f16(oacc[2 * mp + hf][nt], a, pb[i][nt][0], pb[i][nt][1]);
             }
           }
         }
@@ -523,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
             uint32_t a[4];
             ldsm_x4_t(a, smem_addr(sV + chunk(vb[i], vkey[i], gm >> 2, ((gm * 2) & 7) + ((lane >> 3) & 1))));
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_16816(oacc[mt][nt], a, pb[i][nt][0], pb[i][nt][1]);
+            for (int nt = 0; nt < NTW; ++nt) mma_16816(oacc[mt][nt], a, pb[i][nt][0], pb[i][nt][1]);
           }
         }
       }
@@ -545,21 +549,22 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
 
   // ---- merge the token groups' states through shared memory (the ring is
   // free); rows padded to D+4 floats so the fragment stores are conflict free.
-  // The warps of a group hold identical (m, l); the first one stores them.
+  // The warps of a head_dim pair hold identical (m, l); the first one stores them.
   constexpr int MROW = D + 4;
   float *sm_o = reinterpret_cast<float *>(smem);  // [TG][HPT][MROW]
   float *sm_m = sm_o + TG * HPT * MROW;            // [TG][HPT]
   float *sm_l = sm_m + TG * HPT;                   // [TG][HPT]
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
+  for (int nt = 0; nt < NTW; ++nt) {
+    const int hn = (hg * NTW + nt) * 8;  // first head of this n-tile in the head tile
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       float l = l_run[nt][j];
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
       if (dh == 0 && lane < 4) {
-        sm_m[tg * HPT + nt * 8 + 2 * lane + j] = m_run[nt][j];
-        sm_l[tg * HPT + nt * 8 + 2 * lane + j] = l;
+        sm_m[tg * HPT + hn + 2 * lane + j] = m_run[nt][j];
+        sm_l[tg * HPT + hn + 2 * lane + j] = l;
       }
     }
 #pragma unroll
@@ -567,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
       // accumulator rows lane/4 and lane/4 + 8 are head_dim rows d and d2
       const int d = (dh * MT + mt) * 16 + (F8 ? 2 : 1) * (lane >> 2);
       const int d2 = d + (F8 ? 1 : 8);
-      float *o0 = sm_o + (tg * HPT + nt * 8 + (lane & 3) * 2) * MROW;
+      float *o0 = sm_o + (tg * HPT + hn + (lane & 3) * 2) * MROW;
       o0[d] = oacc[mt][nt][0];
       o0[MROW + d] = oacc[mt][nt][1];
       o0[d2] = oacc[mt][nt][2];
