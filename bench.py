@@ -176,7 +176,7 @@ def traffic_from_profiles(workload, kernel_sha):
 
 def kernel_source_sha():
     h = hashlib.sha256()
-    for f in ("pad_partition.cu", "pad_device.cuh", "pad_internal.h"):
+    for f in ("pad_partition.cu", "pad_merge.cuh", "pad_device.cuh", "pad_internal.h"):
         with open(os.path.join(ROOT, "paged_kv_attention_partition_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
