@@ -332,14 +332,41 @@ def main():
     # ---- end to end through the public one-call API, host buffers -----------
     # Per step: pinned host -> device copy of the step's inputs (q, block table,
     # seq_lens; the KV cache stays resident in HBM as in a decode loop), the call,
-    # device -> host copy of out and lse.
-    hq = torch.from_numpy(w.q).view(torch.bfloat16).pin_memory()
-    ht = torch.from_numpy(w.block_tables).pin_memory()
-    hl = torch.from_numpy(w.seq_lens).pin_memory()
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory() if lse is not None else None
-    h2d = hq.numel() * 2 + ht.numel() * 4 + hl.numel() * 4
-    d2h = hout.numel() * 2 + (hlse.numel() * 4 if hlse is not None else 0)
+    # device -> host copy of out and lse.  The inputs share one pinned staging
+    # buffer and one device buffer (each tensor at a 256-byte aligned offset), and
+    # out and lse share one device buffer, so a step makes one copy each way.
+    def pack(parts):
+        offs, total = [], 0
+        for t in parts:
+            offs.append(total)
+            total += (t.numel() * t.element_size() + 255) // 256 * 256
+        return offs, total
+
+    def view(buf, off, like):
+        return buf[off:off + like.numel() * like.element_size()].view(like.dtype).view(like.shape)
+
+    in_parts = [q, tables, lens]
+    in_offs, in_total = pack(in_parts)
+    din = torch.empty(in_total, dtype=torch.uint8, device=dev)
+    hin = torch.zeros(in_total, dtype=torch.uint8).pin_memory()
+    for off, t, a in zip(in_offs, in_parts, (w.q, w.block_tables, w.seq_lens)):
+        view(hin, off, t).copy_(torch.from_numpy(a).view(t.dtype))
+    qe, te, le = (view(din, off, t) for off, t in zip(in_offs, in_parts))
+    out_parts = [out] + ([lse] if lse is not None else [])
+    out_offs, out_total = pack(out_parts)
+    dout = torch.empty(out_total, dtype=torch.uint8, device=dev)
+    hout = torch.empty(out_total, dtype=torch.uint8).pin_memory()
+    oute = view(dout, out_offs[0], out)
+    lsee = view(dout, out_offs[1], lse) if lse is not None else None
+    h2d, d2h = in_total, out_total
+
+    def e2e_step(stream_):
+        din.copy_(hin, non_blocking=True)
+        pad.pad_decode(qe, k, v, te, le, w.scale, num_splits=splits, out=oute, lse=lsee, stream=stream_,
+                       window=args.window, sinks=sinks_dev, k_scale=w.k_scale if fp8 else 0.0,
+                       v_scale=w.v_scale if fp8 else 0.0)
+        hout.copy_(dout, non_blocking=True)
+
     e2e_steps = 0 if args.no_e2e else max(10, args.steps // 2)
     e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(e2e_steps)]
     with torch.cuda.stream(stream):
@@ -347,16 +374,12 @@ def main():
             flush_l2(i)
             if i >= 0:
                 e2e_ev[i][0].record(stream)
-            q.copy_(hq, non_blocking=True)
-            tables.copy_(ht, non_blocking=True)
-            lens.copy_(hl, non_blocking=True)
-            call(stream)
-            hout.copy_(out, non_blocking=True)
-            if hlse is not None:
-                hlse.copy_(lse, non_blocking=True)
+            e2e_step(stream)
             if i >= 0:
                 e2e_ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
+    if e2e_steps and not torch.equal(view(hout, out_offs[0], out), out.cpu()):
+        raise SystemExit("the end-to-end step's output differs from the kernel leg's")
     e2e_ms = sum(e[0].elapsed_time(e[1]) for e in e2e_ev) if e2e_steps else float("nan")
     # every rank takes the same collective steps, e2e leg or not
     e2e_total = max_over_ranks(e2e_ms / max(e2e_steps, 1) * args.steps if e2e_steps else 0.0, dev, world)
@@ -371,13 +394,7 @@ def main():
     if graph_steps:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            q.copy_(hq, non_blocking=True)
-            tables.copy_(ht, non_blocking=True)
-            lens.copy_(hl, non_blocking=True)
-            call(stream)
-            hout.copy_(out, non_blocking=True)
-            if hlse is not None:
-                hlse.copy_(lse, non_blocking=True)
+            e2e_step(stream)
         g_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(graph_steps)]
         with torch.cuda.stream(stream):
             for i in range(-3, graph_steps):
