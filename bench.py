@@ -294,11 +294,11 @@ def main():
                               v_scale=w.v_scale if fp8 else 0.0)
 
     def step():
-        # the whole hot path: one launch (partition + fused reduce)
-        if args.window or args.sinks or fp8:
-            call(stream)
-        else:
-            pad.pad_decode_with_workspace(q, k, v, tables, lens, w.scale, splits, out, lse, ws, stream)
+        # the whole hot path: one launch (partition + fused reduce), partials in
+        # the caller-owned workspace
+        pad.pad_decode_with_workspace(q, k, v, tables, lens, w.scale, splits, out, lse, ws, stream,
+                                      window=args.window, sinks=sinks_dev, k_scale=w.k_scale if fp8 else 0.0,
+                                      v_scale=w.v_scale if fp8 else 0.0)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):

@@ -203,6 +203,18 @@ pad_status pad_decode_with_workspace(const pad_tensor *q, const pad_tensor *k_ca
                                      size_t workspace_bytes, void *stream);
 
 /*
+ * pad_decode_with_workspace_ex -- pad_decode_with_workspace with the options of
+ * pad_decode_ex (window, sinks, E4M3 scales; NULL = none).  Same arguments,
+ * scratch rules, results and errors as those two.
+ */
+pad_status pad_decode_with_workspace_ex(const pad_tensor *q, const pad_tensor *k_cache,
+                                        const pad_tensor *v_cache, const pad_tensor *block_tables,
+                                        const pad_tensor *seq_lens, float scale, int32_t num_splits,
+                                        const pad_decode_options *options, pad_tensor *out,
+                                        pad_tensor *lse, void *workspace, size_t workspace_bytes,
+                                        void *stream);
+
+/*
  * pad_decode_static_scratch -- pad_decode for callers that cannot allocate device
  * memory.  The source pages have no counterpart of this entry point.
  *

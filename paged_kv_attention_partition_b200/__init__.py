@@ -86,6 +86,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pad_decode_with_workspace.argtypes = [P, P, P, P, P, ctypes.c_float, ctypes.c_int32, P, P, ctypes.c_void_p,
                                               ctypes.c_size_t, ctypes.c_void_p]
     lib.pad_decode_with_workspace.restype = ctypes.c_int
+    lib.pad_decode_with_workspace_ex.argtypes = [P, P, P, P, P, ctypes.c_float, ctypes.c_int32,
+                                                 ctypes.POINTER(PadOptions), P, P, ctypes.c_void_p, ctypes.c_size_t,
+                                                 ctypes.c_void_p]
+    lib.pad_decode_with_workspace_ex.restype = ctypes.c_int
     lib.pad_decode_plan.argtypes = [ctypes.c_int64] * 6 + [ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(PadPlan)]
     lib.pad_decode_plan.restype = ctypes.c_int
     lib.pad_decode_plan_ex.argtypes = [ctypes.c_int64] * 6 + [ctypes.c_int32] * 3 + [ctypes.POINTER(PadPlan)]
@@ -248,23 +252,36 @@ def pad_decode_tcgen05(q, k_cache, v_cache, block_tables, seq_lens, scale, num_s
 
 
 def pad_decode_with_workspace(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, workspace,
-                              stream=None) -> None:
+                              stream=None, window: int = 0, sinks: Optional[torch.Tensor] = None,
+                              k_scale: float = 0.0, v_scale: float = 0.0) -> None:
     """pad_decode with caller-owned partials scratch (see include/pad.h):
     ``workspace`` is a contiguous device tensor of at least
     ``pad_decode_plan(...)["workspace_bytes"]`` bytes (any contents), or None
-    when that is 0."""
+    when that is 0.  The options are those of ``pad_decode``
+    (``pad_decode_with_workspace_ex`` when any is set)."""
     dev = q.device
     if workspace is not None and (workspace.device != dev or not workspace.is_contiguous()):
         raise ValueError("workspace must be a contiguous tensor on q's device")
+    if sinks is not None and sinks.device != dev:
+        raise ValueError(f"sinks is on {sinks.device}, q on {dev}")
     descs = [describe(t) for t in (q, k_cache, v_cache, block_tables, seq_lens, out)]
     dlse = describe(lse) if lse is not None else None
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    lib = load_library()
     with torch.cuda.device(dev):
-        st = load_library().pad_decode_with_workspace(
-            *(ctypes.byref(d) for d in descs[:5]), float(scale), int(num_splits), ctypes.byref(descs[5]),
-            ctypes.byref(dlse) if dlse is not None else None,
-            workspace.data_ptr() if workspace is not None else None,
-            workspace.numel() * workspace.element_size() if workspace is not None else 0,
-            _stream_handle(stream, dev))
+        if window or sinks is not None or k_scale or v_scale:
+            dsk = describe(sinks) if sinks is not None else None
+            opts = PadOptions(int(window), ctypes.pointer(dsk) if dsk is not None else None, float(k_scale),
+                              float(v_scale))
+            st = lib.pad_decode_with_workspace_ex(
+                *(ctypes.byref(d) for d in descs[:5]), float(scale), int(num_splits), ctypes.byref(opts),
+                ctypes.byref(descs[5]), ctypes.byref(dlse) if dlse is not None else None, ws_ptr, ws_bytes,
+                _stream_handle(stream, dev))
+        else:
+            st = lib.pad_decode_with_workspace(
+                *(ctypes.byref(d) for d in descs[:5]), float(scale), int(num_splits), ctypes.byref(descs[5]),
+                ctypes.byref(dlse) if dlse is not None else None, ws_ptr, ws_bytes, _stream_handle(stream, dev))
     _raise(st)
 
 

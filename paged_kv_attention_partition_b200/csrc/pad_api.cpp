@@ -614,10 +614,19 @@ pad_status pad_decode_with_workspace(const pad_tensor *q, const pad_tensor *k_ca
                                      const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
                                      int32_t num_splits, pad_tensor *out, pad_tensor *lse, void *workspace,
                                      size_t workspace_bytes, void *stream_) {
+  return pad_decode_with_workspace_ex(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, nullptr, out,
+                                      lse, workspace, workspace_bytes, stream_);
+}
+
+pad_status pad_decode_with_workspace_ex(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
+                                        const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
+                                        int32_t num_splits, const pad_decode_options *options, pad_tensor *out,
+                                        pad_tensor *lse, void *workspace, size_t workspace_bytes, void *stream_) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   Prepared pr;
   bool empty = false;
-  pad_status st = prepare(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, &pr, &empty);
+  pad_status st =
+      prepare(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, &pr, &empty, false, options);
   if (st != PAD_OK || empty) return st;
   if ((st = check_caller_buffer(pr, workspace, workspace_bytes, pr.ws.total, "workspace")) != PAD_OK) return st;
   void *ctl = nullptr;

@@ -118,3 +118,25 @@ def test_e4m3_invalid_arguments(cuda_device):
         DeviceWorkload(w32, cuda_device).run(
             entry=lambda *a, k_scale=None, v_scale=None, **kw: pad.pad_decode_tcgen05(*a, **kw))
     assert e.value.status == pad.PAD_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("splits", [1, 5, 0])
+def test_caller_workspace_with_options(cuda_device, splits):
+    # pad_decode_with_workspace_ex: caller-owned partials with E4M3 scales, a
+    # window and sinks together
+    w = _case("e4m3_ws_ex", 3, 16, 2, 128, 16, [700, 90, 1200])
+    sinks = np.linspace(-2.0, 3.0, w.Hq).astype(np.float32)
+    W = 333
+    ref_out, ref_lse = oracle.decode_workload(w, window=W, sinks=sinks)
+    plan = pad.pad_decode_plan(w.B, w.Hq, w.Hkv, w.D, w.block_size, w.max_blocks_per_seq, num_splits=splits,
+                               kv_dtype="e4m3")
+    ws = torch.full((plan["workspace_bytes"] // 4 + 64,), float("nan"), dtype=torch.float32, device=cuda_device)
+    dev_sinks = torch.from_numpy(sinks).to(cuda_device)
+
+    def entry(q, k, v, t, l, scale, num_splits, out, lse, **kw):
+        pad.pad_decode_with_workspace(q, k, v, t, l, scale, num_splits, out, lse, ws if plan["workspace_bytes"] else None,
+                                      window=W, sinks=dev_sinks, **kw)
+
+    out, lse = DeviceWorkload(w, cuda_device).run(num_splits=splits, entry=entry)
+    check_parity(to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, f"workspace_ex/S={splits}")
+    assert pad.pad_check_device_errors() == 0
