@@ -112,16 +112,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
   return h;
 }
 
-// Two E4M3 codes widened to bf16x2, through f16 and f32.  Exact: an E4M3 value
-// has at most 4 significant bits and its exponent range lies inside bf16's.
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two_codes) {
-  const uint32_t f = e4m3x2_to_f16x2(two_codes);
-  const float lo = __half2float(__ushort_as_half((unsigned short)(f & 0xffffu)));
-  const float hi = __half2float(__ushort_as_half((unsigned short)(f >> 16)));
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t *>(&v);
-}
-
 // Bytes of x selected by `sel` (4 nibbles, byte indices 0-3 of x).
 __device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t sel) { return __byte_perm(x, 0, sel); }
 

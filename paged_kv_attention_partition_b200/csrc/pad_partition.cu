@@ -20,12 +20,15 @@
 // are whole, so the last page's slots past L_b arrive too: their scores are
 // masked and their V rows zeroed before use.
 //
-// The warps form token groups: group tg computes tokens 16tg .. 16tg+15 of every
-// stage and keeps its own running max and sum per head (the warp-strided online
-// softmax of the same section; the groups are merged at the end, so the sum is
-// taken in another order than a sequential kernel's).  At head_dim 256 a group
-// is two warps that compute the same scores and each keep half of the head_dim
-// rows of O^T, which halves the stage and the accumulator.
+// With 8 heads per tile the warps form token groups: group tg computes 16-token
+// tiles tg, tg + 4, ... of every stage and keeps its own running max and sum
+// per head (the warp-strided online softmax of the same section; the groups
+// are merged at the end, so the sum is taken in another order than a
+// sequential kernel's).  With 16 or 32 heads per tile the warps are head
+// groups instead: each owns one 8-head n-tile and computes every token of the
+// stage for it.  At head_dim 256 two warps compute the same scores and each
+// keep half of the head_dim rows of O^T, which halves the stage and the
+// accumulator.
 // Per 16-token tile and 8-head n-tile:
 //   S^T = K . Q^T                 (mma.m16n8k16 bf16, fp32 accumulate)
 //   P^T = exp2(S^T * scale*log2e - m)
@@ -34,9 +37,10 @@
 // An E4M3 cache ("perf(rocke): prepare saved paged decode bindings once",
 // section "Summary": the FP8 decode path beside the non-FP8 one) streams 8-bit
 // codes, half the bytes, through the same stages.  K operands are loaded four
-// codes per register and widened exactly to bf16 (E4M3 -> f16 -> f32 -> bf16),
-// so the QK product stays exact against bf16 q; the head_dim order inside each
-// 16-wide k-step is permuted (codes 4c..4c+3 of a row go to k = 2c, 2c+1,
+// codes per register and widened exactly to f16 (one cvt per pair: every E4M3
+// value is an f16 value); q enters the f16 QK product scaled by a power of two
+// per head tile so that its bf16 values stay exact.  The head_dim order inside
+// each 16-wide k-step is permuted (codes 4c..4c+3 of a row go to k = 2c, 2c+1,
 // 2c+8, 2c+9), and the q fragments take the same permutation, which a dot
 // product allows.  V operands come from a transposed ldmatrix of the codes and
 // a byte permute, widened to f16 (exact) for an f16 PV product with f16
