@@ -19,9 +19,11 @@
 //   MMA thread:     S^T[128 tok x 32 heads] = K . Q^T        (tcgen05.mma, TMEM)
 //                   O^T[128 d x 32 heads]  += V^T . P^T      (tcgen05.mma, TMEM)
 //   softmax warps:  thread i owns token i (TMEM lane i): reads its 32 scores,
-//                   per-head max over the chunk (shuffle transpose-reduce and a
-//                   4-warp combine), lazy running max (moves only when a score
-//                   passes it by more than 2^8), weights in fp32 summed per
+//                   lazy running max per head (moves only when a score passes
+//                   it by more than 2^8: each thread tests its token and one
+//                   barrier-reduce decides; only then the chunk's per-head
+//                   maximum, a shuffle transpose-reduce and a 4-warp combine),
+//                   weights in fp32 summed per
 //                   thread, P^T row written to shared memory (MN-major, 128-byte
 //                   swizzle) as the B operand of the PV product.  At the end
 //                   thread i owns head_dim row i of O^T.
@@ -498,27 +500,32 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_kernel(const __grid_cons
         }
         const int tb = e.t0 + c * kChunk;
         const bool live = landed && tb + i < e.t1;
-        float sc[32], cm[32];
+        float sc[32];
+        bool over = false;  // a score of this token passes its head's reference by more than the slack
 #pragma unroll
         for (int h = 0; h < 32; ++h) {
           sc[h] = live ? __uint_as_float(raw[h]) * p.scale_log2 : -INFINITY;
-          cm[h] = sc[h];
+          over |= sc[h] > mr[h] + kSlack;
         }
-        // per-head maximum over the chunk's 128 tokens (token 0 of the chunk is live)
-        red[warp * 32 + lane] = warp_max_scatter(cm, lane);
         if (!softmax_bar_and(landed)) {  // one decision for all 128 threads
           ok = false;
           break;
         }
-        const float mh = fmaxf(fmaxf(red[lane], red[32 + lane]), fmaxf(red[64 + lane], red[96 + lane]));  // head = lane
-        bool grow = false;
+        // The reference maxima are the same in every thread, so each thread
+        // tests its own token and one barrier-reduce decides; the chunk's
+        // per-head maximum (a transpose-reduce and a 4-warp combine) is taken
+        // only when a reference moves.  Token 0 of a chunk is live and the first
+        // reference is -inf, so a unit's first chunk always sets it.
+        if (!softmax_bar_and(!over)) {  // the same decision in every thread
+          float cm[32];
 #pragma unroll
-        for (int h = 0; h < 32; ++h) {
-          cm[h] = __shfl_sync(0xffffffffu, mh, h);
-          grow |= cm[h] > mr[h] + kSlack;
-        }
-        softmax_bar();  // every warp has read `red` before its next use
-        if (grow) {  // the same decision in every thread: the values are identical
+          for (int h = 0; h < 32; ++h) cm[h] = sc[h];
+          red[warp * 32 + lane] = warp_max_scatter(cm, lane);
+          softmax_bar();
+          const float mh = fmaxf(fmaxf(red[lane], red[32 + lane]), fmaxf(red[64 + lane], red[96 + lane]));  // head = lane
+#pragma unroll
+          for (int h = 0; h < 32; ++h) cm[h] = __shfl_sync(0xffffffffu, mh, h);
+          softmax_bar();  // every warp has read `red` before its next use
           float al[32];
 #pragma unroll
           for (int h = 0; h < 32; ++h) {
