@@ -84,8 +84,24 @@ def workload_config(w, plan):
     return cfg
 
 
-def cpu_baseline(w, budget_s, runs_max=50):
-    """Time the oracle as it stands on this host's cores on a bounded sample."""
+def split_scratch_bytes(w, plan, window=0):
+    """Bytes of split partials one launch writes and the merge reads back (fp32
+    o_s and lse_s of every partition of every sequence with more than one
+    non-empty partition): reported beside the algorithmic bytes, not credited."""
+    P = plan["partition_tokens"]
+    total = 0
+    for L in w.seq_lens.tolist():
+        lo = max(0, L - window) if window else 0
+        ns = (-(-L // P) - lo // P) if L > lo else 0
+        if ns > 1:
+            total += 2 * ns * w.Hq * (w.D + 1) * 4
+    return total
+
+
+def cpu_baseline(w, budget_s, runs_max=50, prefix=None):
+    """Time the oracle as it stands on this host's cores on a bounded sample,
+    plus a one-thread figure (on the whole batch, or on its first sequences
+    when that would take more than a few seconds; `prefix(k)` builds that batch)."""
     import oracle
     threads = oracle.default_threads()
     bytes_per = w.algorithmic_bytes()
@@ -98,10 +114,19 @@ def cpu_baseline(w, budget_s, runs_max=50):
         if time.perf_counter() - t_all > budget_s or len(times) >= runs_max:
             break
     med = statistics.median(times)
+    one = None
+    est1 = med * threads  # rough one-thread time of the whole batch
+    w1 = w if est1 <= 4.0 or prefix is None else prefix(max(1, int(w.B * 4.0 / est1)))
+    t0 = time.perf_counter()
+    oracle.decode_workload(w1, nthreads=1)
+    t1 = time.perf_counter() - t0
+    one = {"value": round(w1.algorithmic_bytes() / t1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+           "sample": (f"whole {w.name} batch" if w1 is w else f"first {w1.B} of {w.B} {w.name} sequences")
+                     + f", one run, {t1 * 1e6:.0f} us"}
     return {"value": round(bytes_per / med / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": f"whole {w.name} batch, {len(times)} run(s), median {med * 1e6:.0f} us/call "
                       f"(double precision, {threads} threads)",
-            "us_per_call": round(med * 1e6, 1)}
+            "us_per_call": round(med * 1e6, 1), "one_thread": one}
 
 
 class ClockSampler:
@@ -188,13 +213,14 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     w = synth.config(args.workload, batch=args.batch, compact_pool=args.compact_pool, kv_dtype=args.kv_dtype)
-    cb = cpu_baseline(w, args.cpu_seconds)
+    cb = cpu_baseline(w, args.cpu_seconds, prefix=lambda k: synth.config(
+        args.workload, batch=k, compact_pool=args.compact_pool, kv_dtype=args.kv_dtype))
     us = cb["us_per_call"]
     line = {"impl": "reference", "metric": metric, "value": cb["value"], "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1e3, 4), "us_per_call": us,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded generator, no dataset)", "config": workload_config(w, None),
-            "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+            "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample", "one_thread")},
             "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line), flush=True)
@@ -440,7 +466,8 @@ def main():
             "us_per_call_min_max": [round(min(step_ms) * 1e3, 2), round(max(step_ms) * 1e3, 2)],
             "roofline": {"kernel": kname, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "peak_kind": f"{peak_kind} copy bandwidth", "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "algorithmic_bytes_per_launch": p_bytes, "traffic": traffic, "source_sha": sha},
+                         "algorithmic_bytes_per_launch": p_bytes, "traffic": traffic, "source_sha": sha,
+                         "split_scratch_bytes_per_launch": split_scratch_bytes(w, plan, args.window)},
             "e2e": None if not e2e_steps else {
                 "value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "us_per_call": round(e2e_total / args.steps * 1e3, 2), "api": "pad_decode"},
@@ -451,8 +478,9 @@ def main():
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
-            cb = cpu_baseline(w, args.cpu_seconds)
-            line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+            cb = cpu_baseline(w, args.cpu_seconds, prefix=lambda k: synth.config(
+                args.workload, batch=k, compact_pool=args.compact_pool, kv_dtype=args.kv_dtype))
+            line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample", "one_thread")}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
