@@ -90,8 +90,7 @@ typedef struct pad_plan {
                                 producer, MMA) */
   int32_t stage_tokens;      /* tokens per shared-memory pipeline stage */
   int32_t stages;            /* pipeline depth */
-  int32_t ctas;              /* CTAs launched: one per unit (B * Hkv * head_tiles * num_splits), or
-                                for the persistent tcgen05 kernel min(units, SM count) */
+  int32_t ctas;              /* CTAs launched: one per unit (B * Hkv * head_tiles * num_splits) */
   int32_t reduce;            /* 1 when partitions may need merging (S > 1) */
   int64_t workspace_bytes;   /* partial-output scratch (0 when S == 1) */
   int64_t control_bytes;     /* merge counters, 0 when S == 1 (library-owned except
@@ -251,8 +250,8 @@ pad_status pad_decode_static_scratch(const pad_tensor *q, const pad_tensor *k_ca
  * pad_decode_tcgen05 -- pad_decode computed by the 5th-generation tensor-core
  * kernel: S^T = K.Q^T and O^T += V^T.P^T as tcgen05.mma with the accumulators in
  * tensor memory, K/V/q streamed by TMA in 8-token boxes, the softmax in four warps
- * that own one token (one TMEM lane) each, one persistent CTA per SM walking the
- * (sequence, KV head, partition) units.  Same arguments, results, scratch and
+ * that own one token (one TMEM lane) each, one CTA per (sequence, KV head,
+ * partition) unit, two per SM.  Same arguments, results, scratch and
  * errors as pad_decode.  It takes a bf16 cache with groups of 17..32 query
  * heads per KV head at head_dim 128 and block_size >= 8, and returns
  * PAD_ERR_UNSUPPORTED otherwise.

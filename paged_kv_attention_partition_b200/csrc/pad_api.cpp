@@ -128,9 +128,8 @@ void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan, b
   plan->warps_per_cta = umma ? pad::kUmmaWarps : pad::kWarps;
   plan->stage_tokens = umma ? pad::kUmmaStageTokens : pad::stage_tokens_for((int)s.D, hpt, s.fp8);
   plan->stages = umma ? pad::umma_stages() : pad::partition_stages((int)s.D, hpt, s.fp8);
-  // one CTA per unit; the tcgen05 kernel is persistent: one CTA per SM walks the units
-  const int64_t sms = sm_count(device < 0 ? 0 : device);
-  plan->ctas = (int32_t)(umma ? (units < sms ? units : sms) : (units > 0x7fffffffll ? 0x7fffffffll : units));
+  // one CTA per unit (both kernels)
+  plan->ctas = (int32_t)(units > 0x7fffffffll ? 0x7fffffffll : units);
   plan->reduce = S > 1 ? 1 : 0;
   plan->workspace_bytes = (int64_t)pad::workspace_layout(s.B, s.Hq, S, s.D).total;
   plan->control_bytes = (int64_t)pad::control_layout(s.B, s.Hkv, HT, S).total;

@@ -1,21 +1,23 @@
 // Partition kernel on the 5th-generation tensor cores, for 32-head tiles at
 // head_dim 128 (large GQA groups and MQA, where the group's QK and PV are dense
-// enough -- 32 flop per K/V byte -- for the mma.sync path to run out of
-// registers and issue slots).
+// enough -- 32 flop per K/V byte -- to be a real contraction).
 //
 // Same work unit and result as partition_kernel (pad_partition.cu): one CTA per
 // (sequence b, KV head, head tile, partition s), the query heads of the tile
 // against tokens [s*P, min((s+1)*P, L_b)) ("perf(rocke): prepare saved paged
 // decode bindings once", section "Summary"), every head served from one K/V read
 // ("spec(BACKEND-ROCM): the ROCm head_dim=128 decode arm", section "It is a
-// mirror of merged work, not new design").  The partition is processed in
-// chunks of 128 tokens:
+// mirror of merged work, not new design").  Two CTAs share an SM, so one's
+// start, epilogue and split merge overlap the other's streaming.  The
+// partition is processed in chunks of 128 tokens:
 //
 //   producer warp:  TMA of the chunk's K and V, boxes of 8 tokens x 128 head_dim
 //                   (two 64-element column blocks, 128-byte swizzle), so that
 //                   8-token groups sit 2 KB apart: the canonical tcgen05
 //                   operand layout for K (K-major) and for V (MN-major).  The
-//                   q rows of the tile arrive the same way.
+//                   q rows of the tile arrive the same way.  One K and one V
+//                   chunk buffer: K(c+1) streams once S(c) has read K(c), V(c+1)
+//                   once PV(c) has read V(c).
 //   MMA thread:     S^T[128 tok x 32 heads] = K . Q^T        (tcgen05.mma, TMEM)
 //                   O^T[128 d x 32 heads]  += V^T . P^T      (tcgen05.mma, TMEM)
 //   softmax warps:  thread i owns token i (TMEM lane i): reads its 32 scores,
@@ -23,15 +25,12 @@
 //                   it by more than 2^8: each thread tests its token and one
 //                   barrier-reduce decides; only then the chunk's per-head
 //                   maximum, a shuffle transpose-reduce and a 4-warp combine),
-//                   weights in fp32 summed per
-//                   thread, P^T row written to shared memory (MN-major, 128-byte
-//                   swizzle) as the B operand of the PV product.  At the end
-//                   thread i owns head_dim row i of O^T.
+//                   weights in fp32 summed per thread, P^T row written to shared
+//                   memory (MN-major, 128-byte swizzle) as the B operand of the
+//                   PV product.  At the end thread i owns head_dim row i of O^T.
 //
-// S^T and P^T are double buffered: the MMA thread issues QK(c+1) as soon as
-// chunk c+1 has landed, so the softmax warps find the next scores ready, and
-// PV(c) runs while the softmax works on chunk c+1.  A rescale of O^T waits for
-// PV(c-1); a P^T buffer is rewritten once PV(c-2) has read it.
+// S^T and P^T are double buffered.  A rescale of O^T waits for PV(c-1); a P^T
+// buffer is rewritten once PV(c-2) has read it.
 //
 // Output and split handling are those of partition_kernel: one non-empty
 // partition writes bf16 out (+ lse), otherwise fp32 partials and the last CTA of
@@ -63,7 +62,6 @@ constexpr uint32_t kPBytes = kChunk * 128;                 // one P^T buffer: 12
 constexpr int kSoftmaxWarps = 4;
 constexpr int kProducerWarp = 4, kMmaWarp = 5;
 constexpr int kUmmaThreads = 6 * 32;
-constexpr int kUmmaStages = 2;  // K/V chunks in flight
 
 // ---- tcgen05 wrappers (sm_100a) ----------------------------------------------
 
@@ -196,78 +194,89 @@ __device__ __forceinline__ float warp_sum_scatter(float (&v)[32], int lane) {
 
 }  // namespace
 
-// One queued work unit.  nch > 0: chunks to stream; 0: an empty sequence (the
-// unit writes out = 0, lse = -inf); -1: no more units.
-struct UnitDesc {
-  int32_t b, kvh, ht, s, t0, t1, ns, nch;
-};
-constexpr int kQueue = 4;
-
-// Shared memory (1024-byte aligned base): q 2 x 8 KB | K/V ring NST x (K 32 KB,
-// V 32 KB) | P^T 2 x 16 KB | merge weights 32 KB | reductions 1 KB | queue,
-// barriers and words.  TMEM: S^T in two 32-column buffers, O^T after them.
-template <int NST>
+// Shared memory (1024-byte aligned base): q 8 KB | K chunk 32 KB | V chunk
+// 32 KB | P^T 2 x 16 KB | reductions 1 KB | barriers and words.  The K and V
+// chunk buffers are reused for the split merge's weights after the last chunk.
+// TMEM: S^T in two 32-column buffers, O^T after them (128 columns; two CTAs per
+// SM take 256 of the 512).
 struct UmmaSmem {
   static constexpr uint32_t q = 0;
-  static constexpr uint32_t ring = 2 * kQBytes;
-  static constexpr uint32_t pt = ring + NST * 2 * kHalfBytes;
-  static constexpr uint32_t mw = pt + 2 * kPBytes;
-  static constexpr uint32_t red = mw + kHeads * kMaxSplits * 4;
-  static constexpr uint32_t queue = red + 1024;
-  static constexpr uint32_t bars = queue + kQueue * sizeof(UnitDesc);
-  static constexpr uint32_t total = bars + 512 + 1024 /* alignment slack */;
+  static constexpr uint32_t k = kQBytes;
+  static constexpr uint32_t v = k + kHalfBytes;
+  static constexpr uint32_t pt = v + kHalfBytes;
+  static constexpr uint32_t red = pt + 2 * kPBytes;
+  static constexpr uint32_t bars = red + 1024;
+  static constexpr uint32_t total = bars + 256 + 1024 /* alignment slack */;
 };
+static_assert(2 * kHalfBytes >= kHeads * kMaxSplits * 4, "merge weights fit the K and V buffers");
 
-// Persistent: one CTA per SM walks the units blockIdx.x, blockIdx.x + G, ...
-// The producer warp finds the non-empty ones 32 at a time and queues them; the
-// MMA thread and the softmax warps consume the queue.  Chunk buffers, q
-// buffers, TMEM and barrier phases carry over from unit to unit, so the next
-// unit's copies stream while the current one finishes.
-template <int NST>
-__global__ void __launch_bounds__(kUmmaThreads, 1) umma_kernel(const __grid_constant__ PartitionParams p) {
-  using SM = UmmaSmem<NST>;
+// One CTA per work unit (sequence b, KV head, head tile, partition s), two
+// CTAs per SM: while one streams, the other's start, epilogue and split merge
+// proceed.  Roles: warps 0-3 softmax and epilogue (thread i = token i of a
+// chunk, then head_dim row i of O^T), warp 4 copies (TMA), warp 5 issues the
+// MMAs (one thread).  Per chunk c of 128 tokens:
+//   K(c) lands -> S(c) = K(c).Q^T into S buffer c%2 -> K buffer refilled with K(c+1)
+//   softmax(c) reads S(c), writes P^T(c) -> PV(c): O^T += V(c)^T.P^T(c)
+//   -> V buffer refilled with V(c+1)
+// The MMA thread issues S(0), then PV(c), S(c+1) for each c, so K(c+1) and
+// V(c+1) stream while the softmax works on chunk c.
+__global__ void __launch_bounds__(kUmmaThreads, 2) umma_kernel(const __grid_constant__ PartitionParams p) {
+  using SM = UmmaSmem;
   static_assert(SM::total <= (uint32_t)kSmemBudget, "shared-memory plan over budget");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::bars);
-  UnitDesc *queue = reinterpret_cast<UnitDesc *>(smem + SM::queue);
-  // barriers: chunk ring, q buffers, S^T and P^T buffers (x2), O^T, unit queue
-  const uint32_t kv_full0 = smem_addr(bars), kv_empty0 = smem_addr(bars + NST);
-  const uint32_t q_full0 = smem_addr(bars + 2 * NST), q_empty0 = smem_addr(bars + 2 * NST + 2);
-  const uint32_t s_full0 = smem_addr(bars + 2 * NST + 4), s_free0 = smem_addr(bars + 2 * NST + 6);
-  const uint32_t p_full0 = smem_addr(bars + 2 * NST + 8), p_free0 = smem_addr(bars + 2 * NST + 10);
-  const uint32_t o_done = smem_addr(bars + 2 * NST + 12), o_free = smem_addr(bars + 2 * NST + 13);
-  const uint32_t uq_full0 = smem_addr(bars + 2 * NST + 14), uq_empty0 = smem_addr(bars + 2 * NST + 14 + kQueue);
-  const uint32_t mma_idle = smem_addr(bars + 2 * NST + 14 + 2 * kQueue);
-  uint32_t *words = reinterpret_cast<uint32_t *>(bars + 2 * NST + 15 + 2 * kQueue);  // [0] tmem, [1] flag
+  const uint32_t q_full = smem_addr(bars + 0);
+  const uint32_t k_full = smem_addr(bars + 1), k_free = smem_addr(bars + 2);
+  const uint32_t v_full = smem_addr(bars + 3), v_free = smem_addr(bars + 4);
+  const uint32_t s_full0 = smem_addr(bars + 5), s_free0 = smem_addr(bars + 7);
+  const uint32_t p_full0 = smem_addr(bars + 9), p_free0 = smem_addr(bars + 11);
+  const uint32_t o_done = smem_addr(bars + 13), mma_idle = smem_addr(bars + 14);
+  uint32_t *words = reinterpret_cast<uint32_t *>(bars + 16);  // [0] tmem, [1] flag, [2] abort
   volatile int *abort_flag = reinterpret_cast<volatile int *>(words + 2);
   float *red = reinterpret_cast<float *>(smem + SM::red);  // [4][32]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint32_t u = blockIdx.x;
+  const int s = (int)(u % (uint32_t)p.S);
+  u /= (uint32_t)p.S;
+  const int ht = (int)(u % (uint32_t)p.HT);
+  u /= (uint32_t)p.HT;
+  const int kvh = (int)(u % (uint32_t)p.Hkv);
+  const int b = (int)(u / (uint32_t)p.Hkv);
+  const int h0 = kvh * p.g + ht * kHeads;
+  const int gl = min(kHeads, p.g - ht * kHeads);
   const int capacity = p.max_blocks << p.bs_log2;
+  int L = __ldg(p.seq_lens + b);
+  if (L < 0 || L > capacity) {
+    if (tid == 0 && s == 0 && kvh == 0 && ht == 0) atomicOr(p.err, kErrSeqLen);
+    L = L < 0 ? 0 : capacity;
+  }
+  const int t0 = s * p.P, t1 = min(t0 + p.P, L);
+  if (t0 >= t1) {
+    if (L == 0 && s == 0) {  // empty sequence: out = 0, lse = -inf
+      for (int x = tid; x < gl * kD; x += kUmmaThreads)
+        p.out[b * p.o_sb + (int64_t)(h0 + x / kD) * p.o_sh + (x % kD)] = 0;
+      if (p.lse != nullptr && tid < gl) p.lse[b * p.lse_sb + (int64_t)(h0 + tid) * p.lse_sh] = -INFINITY;
+    }
+    return;  // nothing issued, nothing allocated
+  }
+  const int ns = (L + p.P - 1) / p.P;
+  const int nch = (t1 - t0 + kChunk - 1) / kChunk;
 
   if (tid == 0) {
-#pragma unroll
-    for (int i = 0; i < NST; ++i) {
-      mbar_init(kv_full0 + 8 * i, 1);
-      mbar_init(kv_empty0 + 8 * i, 1);
-    }
+    mbar_init(q_full, 1);
+    mbar_init(k_full, 1);
+    mbar_init(k_free, 1);
+    mbar_init(v_full, 1);
+    mbar_init(v_free, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(q_full0 + 8 * i, 1);
-      mbar_init(q_empty0 + 8 * i, 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(s_full0 + 8 * i, 1);                     // QK commit
-      mbar_init(s_free0 + 8 * i, kSoftmaxWarps * 32);    // every softmax thread has read S^T
-      mbar_init(p_full0 + 8 * i, kSoftmaxWarps * 32);    // every softmax thread has written its P^T row
-      mbar_init(p_free0 + 8 * i, 1);                     // PV commit
+      mbar_init(s_full0 + 8 * i, 1);                   // QK commit
+      mbar_init(s_free0 + 8 * i, kSoftmaxWarps * 32);  // every softmax thread has read S^T
+      mbar_init(p_full0 + 8 * i, kSoftmaxWarps * 32);  // every softmax thread has written its P^T row
+      mbar_init(p_free0 + 8 * i, 1);                   // PV commit
     }
     mbar_init(o_done, 1);
-    mbar_init(o_free, kSoftmaxWarps * 32);
-    for (int i = 0; i < kQueue; ++i) {
-      mbar_init(uq_full0 + 8 * i, 1);
-      mbar_init(uq_empty0 + 8 * i, 1 + kSoftmaxWarps * 32);  // the MMA thread and every softmax thread
-    }
     mbar_init(mma_idle, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -283,128 +292,58 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_kernel(const __grid_cons
   const uint32_t tmem_o = tmem + 64;
 
   if (warp == kProducerWarp) {
-    // ---------------- scheduler + TMA producer ----------------
-    const uint32_t G = gridDim.x;
-    int k = 0;      // units queued
-    int j = 0;      // units with chunks (q buffer use)
-    int g = 0;      // chunks issued
+    // ---------------- TMA: q, then each chunk's K and V (lane l copies box l) ----------------
+    const int32_t *trow = p.tables + (int64_t)b * p.table_stride;
+    int kq = 0, vq = 0;  // K and V chunks issued
     bool ok = true;
-    auto push = [&](const UnitDesc &d) -> bool {
-      const int qs = k % kQueue;
-      if (k >= kQueue && !wait_bounded(uq_empty0 + 8 * qs, ((k / kQueue) - 1) & 1, p.err, abort_flag)) return false;
-      if (lane == 0) {
-        queue[qs] = d;
-        mbar_arrive1(uq_full0 + 8 * qs);  // releases the entry
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, kQBytes);
+      tma_load_4d(smem_addr(smem + SM::q), &p.tmq, 0, h0, 0, b, q_full);
+    }
+    for (int c = 0; ok && c < nch; ++c) {
+      const int tb = t0 + c * kChunk;
+      const int nbox = min(kChunk / kBoxRows, (t1 - tb + kBoxRows - 1) / kBoxRows);
+      const int tok = tb + kBoxRows * lane;
+      const int id = lane < nbox ? __ldg(trow + (tok >> p.bs_log2)) : 0;
+      const int slot0 = tok & ((1 << p.bs_log2) - 1);
+      if (lane < nbox && (unsigned)id >= (unsigned)p.num_blocks) atomicOr(p.err, kErrBlockId);  // reads as zeros
+      // K(c) once S(c-1) has read the K buffer
+      if (c > 0 && !wait_bounded(k_free, (c - 1) & 1, p.err, abort_flag)) {
+        ok = false;
+        break;
       }
+      if (lane == 0) mbar_arrive_expect_tx(k_full, (uint32_t)nbox * kBoxBytes);
       __syncwarp();
-      ++k;
-      return true;
-    };
-    for (uint32_t base = blockIdx.x; ok && base < p.n_units; base += 32 * G) {
-      // lane l looks at unit base + l G
-      const uint32_t uu = base + (uint32_t)lane * G;
-      UnitDesc d{};
-      bool live = false;
-      if (uu < p.n_units) {
-        uint32_t u = uu;
-        d.s = (int)(u % (uint32_t)p.S);
-        u /= (uint32_t)p.S;
-        d.ht = (int)(u % (uint32_t)p.HT);
-        u /= (uint32_t)p.HT;
-        d.kvh = (int)(u % (uint32_t)p.Hkv);
-        d.b = (int)(u / (uint32_t)p.Hkv);
-        int L = __ldg(p.seq_lens + d.b);
-        if (L < 0 || L > capacity) {
-          if (d.s == 0 && d.kvh == 0 && d.ht == 0) atomicOr(p.err, kErrSeqLen);
-          L = L < 0 ? 0 : capacity;
-        }
-        d.t0 = d.s * p.P;
-        d.t1 = min(d.t0 + p.P, L);
-        d.ns = (L + p.P - 1) / p.P;
-        d.nch = d.t0 < d.t1 ? (d.t1 - d.t0 + kChunk - 1) / kChunk : 0;
-        live = d.t0 < d.t1 || (L == 0 && d.s == 0);
+      if (lane < nbox) tma_load_5d(smem_addr(smem + SM::k + lane * kBoxBytes), &p.tmk, 0, slot0, 0, kvh, id, k_full);
+      ++kq;
+      // V(c) once PV(c-1) has read the V buffer
+      if (c > 0 && !wait_bounded(v_free, (c - 1) & 1, p.err, abort_flag)) {
+        ok = false;
+        break;
       }
-      uint32_t mask = __ballot_sync(0xffffffffu, live);
-      while (ok && mask) {
-        const int src = __ffs(mask) - 1;
-        mask &= mask - 1;
-        UnitDesc e;
-        e.b = __shfl_sync(0xffffffffu, d.b, src);
-        e.kvh = __shfl_sync(0xffffffffu, d.kvh, src);
-        e.ht = __shfl_sync(0xffffffffu, d.ht, src);
-        e.s = __shfl_sync(0xffffffffu, d.s, src);
-        e.t0 = __shfl_sync(0xffffffffu, d.t0, src);
-        e.t1 = __shfl_sync(0xffffffffu, d.t1, src);
-        e.ns = __shfl_sync(0xffffffffu, d.ns, src);
-        e.nch = __shfl_sync(0xffffffffu, d.nch, src);
-        if (!push(e)) {
-          ok = false;
-          break;
-        }
-        if (e.nch == 0) continue;
-        // q rows of the tile -> q buffer j % 2
-        const int h0 = e.kvh * p.g + e.ht * kHeads;
-        const int qs = j % 2;
-        if (j >= 2 && !wait_bounded(q_empty0 + 8 * qs, ((j / 2) - 1) & 1, p.err, abort_flag)) {
-          ok = false;
-          break;
-        }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(q_full0 + 8 * qs, kQBytes);
-          tma_load_4d(smem_addr(smem + SM::q + qs * kQBytes), &p.tmq, 0, h0, 0, e.b, q_full0 + 8 * qs);
-        }
-        ++j;
-        // the unit's chunks: lane l < 16 copies box l (tokens tb + 8l .. +7) of K and of V
-        const int32_t *trow = p.tables + (int64_t)e.b * p.table_stride;
-        for (int c = 0; c < e.nch; ++c, ++g) {
-          const int slot = g % NST;
-          const int tb = e.t0 + c * kChunk;
-          const int nbox = min(kChunk / kBoxRows, (e.t1 - tb + kBoxRows - 1) / kBoxRows);
-          const int tok = tb + kBoxRows * lane;
-          const int id = lane < nbox ? __ldg(trow + (tok >> p.bs_log2)) : 0;
-          if (g >= NST && !wait_bounded(kv_empty0 + 8 * slot, ((g / NST) - 1) & 1, p.err, abort_flag)) {
-            ok = false;
-            break;
-          }
-          if (lane == 0) mbar_arrive_expect_tx(kv_full0 + 8 * slot, (uint32_t)nbox * kBoxBytes * 2);
-          __syncwarp();
-          if (lane < nbox) {
-            if ((unsigned)id >= (unsigned)p.num_blocks) atomicOr(p.err, kErrBlockId);  // reads as zeros
-            const int slot0 = tok & ((1 << p.bs_log2) - 1);
-            uint8_t *kdst = smem + SM::ring + slot * 2 * kHalfBytes + lane * kBoxBytes;
-            tma_load_5d(smem_addr(kdst), &p.tmk, 0, slot0, 0, e.kvh, id, kv_full0 + 8 * slot);
-            tma_load_5d(smem_addr(kdst + kHalfBytes), &p.tmv, 0, slot0, 0, e.kvh, id, kv_full0 + 8 * slot);
-          }
-        }
-      }
+      if (lane == 0) mbar_arrive_expect_tx(v_full, (uint32_t)nbox * kBoxBytes);
+      __syncwarp();
+      if (lane < nbox) tma_load_5d(smem_addr(smem + SM::v + lane * kBoxBytes), &p.tmv, 0, slot0, 0, kvh, id, v_full);
+      ++vq;
     }
-    if (ok) {
-      UnitDesc t{};
-      t.nch = -1;
-      push(t);
-    }
-    if (*abort_flag && lane == 0) {
-      // leave no copy in flight: the last NST chunks and the last two q tiles
-      for (int c = max(0, g - NST); c < g; ++c)
-        wait_bounded(kv_full0 + 8 * (c % NST), (c / NST) & 1, p.err, abort_flag, true);
-      for (int x = max(0, j - 2); x < j; ++x) wait_bounded(q_full0 + 8 * (x % 2), (x / 2) & 1, p.err, abort_flag, true);
+    if (!ok && lane == 0) {
+      // leave no copy in flight: the last K and V chunks and q
+      if (kq > 0) wait_bounded(k_full, (kq - 1) & 1, p.err, abort_flag, true);
+      if (vq > 0) wait_bounded(v_full, (vq - 1) & 1, p.err, abort_flag, true);
+      wait_bounded(q_full, 0, p.err, abort_flag, true);
     }
   } else if (warp == kMmaWarp) {
-    // ---------------- MMA issue (one thread) ----------------
-    // Per unit: QK of the first chunk, then for every chunk c: QK(c+1) into the
-    // other S^T buffer as soon as its copies landed, and PV(c) once the softmax
-    // has written P^T(c).  g counts chunks over all units (buffer = g % 2).
+    // ---------------- MMA issue (one thread): S(0), then PV(c), S(c+1) ----------------
     if (lane == 0) {
       constexpr uint32_t IQK = umma_idesc(false, false), IPV = umma_idesc(true, true);
-      int k = 0, j = 0, g = 0;
-      bool ok = true;
-      auto qk = [&](int gc, int qs) -> bool {
-        if (!wait_bounded(kv_full0 + 8 * (gc % NST), (gc / NST) & 1, p.err, abort_flag)) return false;
-        if (gc >= 2 && !wait_bounded(s_free0 + 8 * (gc & 1), ((gc >> 1) - 1) & 1, p.err, abort_flag)) return false;
+      bool ok = wait_bounded(q_full, 0, p.err, abort_flag);
+      auto qk = [&](int c) -> bool {
+        if (!wait_bounded(k_full, c & 1, p.err, abort_flag)) return false;
+        if (c >= 2 && !wait_bounded(s_free0 + 8 * (c & 1), ((c >> 1) - 1) & 1, p.err, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t kb = smem_addr(smem + SM::ring + (gc % NST) * 2 * kHalfBytes);
-        const uint32_t qb = smem_addr(smem + SM::q + qs * kQBytes);
-        const uint32_t sd = tmem + (uint32_t)(gc & 1) * 32;
+        const uint32_t kb = smem_addr(smem + SM::k);
+        const uint32_t qb = smem_addr(smem + SM::q);
+        const uint32_t sd = tmem + (uint32_t)(c & 1) * 32;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           // K: rows of 128 B in 8-row groups 2 KB apart, column block kk/4 at +1 KB
@@ -413,176 +352,142 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_kernel(const __grid_cons
           const uint64_t bq = smem_desc(qb + (kk >> 2) * 4096 + (kk & 3) * 32, 16, 1024);
           umma_bf16(sd, a, bq, IQK, kk > 0);
         }
-        umma_commit(s_full0 + 8 * (gc & 1));
+        umma_commit(s_full0 + 8 * (c & 1));
+        umma_commit(k_free);  // the K buffer may take the next chunk
         return true;
       };
-      auto pv = [&](int gc, bool first) -> bool {
-        if (!wait_bounded(p_full0 + 8 * (gc & 1), (gc >> 1) & 1, p.err, abort_flag)) return false;
-        // before a unit's first PV product overwrites O^T, the previous unit's
-        // epilogue has read it
-        if (first && j > 0 && !wait_bounded(o_free, (j - 1) & 1, p.err, abort_flag)) return false;
+      auto pv = [&](int c) -> bool {
+        if (!wait_bounded(p_full0 + 8 * (c & 1), (c >> 1) & 1, p.err, abort_flag)) return false;
+        if (!wait_bounded(v_full, c & 1, p.err, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t vb = smem_addr(smem + SM::ring + (gc % NST) * 2 * kHalfBytes + kHalfBytes);
-        const uint32_t pb = smem_addr(smem + SM::pt + (gc & 1) * kPBytes);
+        const uint32_t vb = smem_addr(smem + SM::v);
+        const uint32_t pb = smem_addr(smem + SM::pt + (c & 1) * kPBytes);
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk) {
           // V^T (MN-major): 64-d column blocks 1 KB apart, 8-token groups 2 KB apart
           const uint64_t a = smem_desc(vb + kk * 2 * kBoxBytes, 1024, 2 * 1024);
           // P^T (MN-major): token rows of 128 B, 8-token groups 1 KB apart
           const uint64_t bp = smem_desc(pb + kk * 2 * 1024, 1024, 1024);
-          umma_bf16(tmem_o, a, bp, IPV, !first || kk > 0);
+          umma_bf16(tmem_o, a, bp, IPV, c > 0 || kk > 0);
         }
-        umma_commit(kv_empty0 + 8 * (gc % NST));  // the chunk's K and V are consumed
-        umma_commit(p_free0 + 8 * (gc & 1));       // P^T buffer free; O^T holds chunks ..gc
+        umma_commit(p_free0 + 8 * (c & 1));  // P^T buffer free; O^T holds chunks ..c
+        umma_commit(v_free);                 // the V buffer may take the next chunk
         return true;
       };
-      while (ok) {
-        const int qe = k % kQueue;
-        if (!wait_bounded(uq_full0 + 8 * qe, (k / kQueue) & 1, p.err, abort_flag)) break;
-        const int nch = queue[qe].nch;
-        mbar_arrive1(uq_empty0 + 8 * qe);
-        ++k;
-        if (nch < 0) break;
-        if (nch == 0) continue;
-        const int qs = j % 2;
-        if (!wait_bounded(q_full0 + 8 * qs, (j / 2) & 1, p.err, abort_flag) || !qk(g, qs)) break;
-        for (int c = 0; ok && c < nch; ++c) {
-          const int gc = g + c;
-          if (c + 1 < nch) ok = qk(gc + 1, qs);
-          if (ok && c + 1 == nch) umma_commit(q_empty0 + 8 * qs);  // the tile's last QK read of q
-          if (ok) ok = pv(gc, c == 0);
-        }
-        if (!ok) break;
-        umma_commit(o_done);
-        g += nch;
-        ++j;
+      ok = ok && qk(0);
+      for (int c = 0; ok && c < nch; ++c) {
+        ok = pv(c);
+        if (ok && c + 1 < nch) ok = qk(c + 1);
       }
+      if (ok) umma_commit(o_done);
       umma_commit(mma_idle);  // every MMA issued above has completed when this arrives
     }
   } else {
     // ---------------- softmax warps: thread i = token i of a chunk, then head_dim row i ----------------
     const int i = tid;  // 0..127 == TMEM lane
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    int k = 0, j = 0, g = 0;
-    while (true) {
-      const int qe = k % kQueue;
-      const bool got = wait_bounded(uq_full0 + 8 * qe, (k / kQueue) & 1, p.err, abort_flag);
-      if (!softmax_bar_and(got)) break;
-      const UnitDesc e = queue[qe];
-      mbar_arrive1(uq_empty0 + 8 * qe);
-      ++k;
-      if (e.nch < 0) break;
-      const int h0 = e.kvh * p.g + e.ht * kHeads;
-      const int gl = min(kHeads, p.g - e.ht * kHeads);
-      if (e.nch == 0) {  // empty sequence: out = 0, lse = -inf
-        for (int x = i; x < gl * kD; x += kSoftmaxWarps * 32)
-          p.out[e.b * p.o_sb + (int64_t)(h0 + x / kD) * p.o_sh + (x % kD)] = 0;
-        if (p.lse != nullptr && i < gl) p.lse[e.b * p.lse_sb + (int64_t)(h0 + i) * p.lse_sh] = -INFINITY;
-        continue;
+    float mr[32], lp[32];
+#pragma unroll
+    for (int h = 0; h < 32; ++h) {
+      mr[h] = -INFINITY;
+      lp[h] = 0.f;
+    }
+    bool ok = true;
+    for (int c = 0; c < nch; ++c) {
+      // warp-uniform: tcgen05.ld is a warp-collective instruction
+      const bool landed = __all_sync(0xffffffffu, wait_bounded(s_full0 + 8 * (c & 1), (c >> 1) & 1, p.err, abort_flag));
+      uint32_t raw[32];
+      if (landed) {
+        tc_fence_after();
+        tmem_ld32(tmem + (uint32_t)(c & 1) * 32 + lane_off, raw);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive1(s_free0 + 8 * (c & 1));  // the next-but-one QK may overwrite this buffer
       }
-      float mr[32], lp[32];
+      const int tb = t0 + c * kChunk;
+      const bool live = landed && tb + i < t1;
+      float sc[32];
+      bool over = false;  // a score of this token passes its head's reference by more than the slack
 #pragma unroll
       for (int h = 0; h < 32; ++h) {
-        mr[h] = -INFINITY;
-        lp[h] = 0.f;
+        sc[h] = live ? __uint_as_float(raw[h]) * p.scale_log2 : -INFINITY;
+        over |= sc[h] > mr[h] + kSlack;
       }
-      bool ok = true;
-      for (int c = 0; c < e.nch; ++c, ++g) {
-        // warp-uniform: tcgen05.ld is a warp-collective instruction
-        const bool landed = __all_sync(0xffffffffu, wait_bounded(s_full0 + 8 * (g & 1), (g >> 1) & 1, p.err, abort_flag));
-        uint32_t raw[32];
-        if (landed) {
-          tc_fence_after();
-          tmem_ld32(tmem + (uint32_t)(g & 1) * 32 + lane_off, raw);
-          tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive1(s_free0 + 8 * (g & 1));  // the next-but-one QK may overwrite this buffer
-        }
-        const int tb = e.t0 + c * kChunk;
-        const bool live = landed && tb + i < e.t1;
-        float sc[32];
-        bool over = false;  // a score of this token passes its head's reference by more than the slack
+      if (!softmax_bar_and(landed)) {  // one decision for all 128 threads
+        ok = false;
+        break;
+      }
+      // The reference maxima are the same in every thread, so each thread
+      // tests its own token and one barrier-reduce decides; the chunk's
+      // per-head maximum (a transpose-reduce and a 4-warp combine) is taken
+      // only when a reference moves.  Token 0 of a chunk is live and the first
+      // reference is -inf, so the first chunk always sets it.
+      if (!softmax_bar_and(!over)) {  // the same decision in every thread
+        float cm[32];
+#pragma unroll
+        for (int h = 0; h < 32; ++h) cm[h] = sc[h];
+        red[warp * 32 + lane] = warp_max_scatter(cm, lane);
+        softmax_bar();
+        const float mh = fmaxf(fmaxf(red[lane], red[32 + lane]), fmaxf(red[64 + lane], red[96 + lane]));  // head = lane
+#pragma unroll
+        for (int h = 0; h < 32; ++h) cm[h] = __shfl_sync(0xffffffffu, mh, h);
+        softmax_bar();  // every warp has read `red` before its next use
+        float al[32];
 #pragma unroll
         for (int h = 0; h < 32; ++h) {
-          sc[h] = live ? __uint_as_float(raw[h]) * p.scale_log2 : -INFINITY;
-          over |= sc[h] > mr[h] + kSlack;
+          const float mn = fmaxf(mr[h], cm[h]);
+          al[h] = fast_exp2(mr[h] - mn);
+          mr[h] = mn;
+          lp[h] *= al[h];
         }
-        if (!softmax_bar_and(landed)) {  // one decision for all 128 threads
-          ok = false;
-          break;
+        // row i of O^T holds chunks 0..c-1 once PV(c-1) has completed
+        if (c > 0 &&
+            __all_sync(0xffffffffu, wait_bounded(p_free0 + 8 * ((c - 1) & 1), ((c - 1) >> 1) & 1, p.err, abort_flag))) {
+          tc_fence_after();
+          uint32_t o[32];
+          tmem_ld32(tmem_o + lane_off, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < 32; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * al[h]);
+          tmem_st32(tmem_o + lane_off, o);
+          tmem_wait_st();
         }
-        // The reference maxima are the same in every thread, so each thread
-        // tests its own token and one barrier-reduce decides; the chunk's
-        // per-head maximum (a transpose-reduce and a 4-warp combine) is taken
-        // only when a reference moves.  Token 0 of a chunk is live and the first
-        // reference is -inf, so a unit's first chunk always sets it.
-        if (!softmax_bar_and(!over)) {  // the same decision in every thread
-          float cm[32];
-#pragma unroll
-          for (int h = 0; h < 32; ++h) cm[h] = sc[h];
-          red[warp * 32 + lane] = warp_max_scatter(cm, lane);
-          softmax_bar();
-          const float mh = fmaxf(fmaxf(red[lane], red[32 + lane]), fmaxf(red[64 + lane], red[96 + lane]));  // head = lane
-#pragma unroll
-          for (int h = 0; h < 32; ++h) cm[h] = __shfl_sync(0xffffffffu, mh, h);
-          softmax_bar();  // every warp has read `red` before its next use
-          float al[32];
-#pragma unroll
-          for (int h = 0; h < 32; ++h) {
-            const float mn = fmaxf(mr[h], cm[h]);
-            al[h] = fast_exp2(mr[h] - mn);
-            mr[h] = mn;
-            lp[h] *= al[h];
-          }
-          // row i of O^T holds chunks 0..c-1 once PV(c-1) has completed
-          if (c > 0 &&
-              __all_sync(0xffffffffu, wait_bounded(p_free0 + 8 * ((g - 1) & 1), ((g - 1) >> 1) & 1, p.err, abort_flag))) {
-            tc_fence_after();
-            uint32_t o[32];
-            tmem_ld32(tmem_o + lane_off, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int h = 0; h < 32; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * al[h]);
-            tmem_st32(tmem_o + lane_off, o);
-            tmem_wait_st();
-          }
-        }
-        // weights, the fp32 running sums, and the P^T row of token i (into the
-        // buffer PV(g-2) has finished reading)
-        if (g >= 2) wait_bounded(p_free0 + 8 * (g & 1), ((g >> 1) - 1) & 1, p.err, abort_flag);
-        uint8_t *pt = smem + SM::pt + (g & 1) * kPBytes;
-        uint32_t pk[16];
-#pragma unroll
-        for (int h = 0; h < 32; h += 2) {
-          const float e0 = fast_exp2(sc[h] - mr[h]), e1 = fast_exp2(sc[h + 1] - mr[h + 1]);
-          lp[h] += e0;
-          lp[h + 1] += e1;
-          pk[h / 2] = pack_bf16x2(e0, e1);
-        }
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          *reinterpret_cast<uint4 *>(pt + i * 128 + ((q4 ^ (i & 7)) << 4)) =
-              make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-        if (!live) {
-          // V row of a token past t1 (a slot past L_b or a box not copied):
-          // zeros, after the chunk's copies have landed
-          wait_bounded(kv_full0 + 8 * (g % NST), (g / NST) & 1, p.err, abort_flag);
-          uint8_t *vrow = smem + SM::ring + (g % NST) * 2 * kHalfBytes + kHalfBytes + (i >> 3) * kBoxBytes + (i & 7) * 128;
-#pragma unroll
-          for (int q8 = 0; q8 < 8; ++q8) {
-            *reinterpret_cast<uint4 *>(vrow + q8 * 16) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4 *>(vrow + 1024 + q8 * 16) = make_uint4(0, 0, 0, 0);
-          }
-        }
-        fence_proxy_async_smem();  // P^T and zeroed rows, before the tensor core reads them
-        tc_fence_before();
-        mbar_arrive1(p_full0 + 8 * (g & 1));
       }
-      if (!ok) break;
+      // weights, the fp32 running sums, and the P^T row of token i (into the
+      // buffer PV(c-2) has finished reading)
+      if (c >= 2) wait_bounded(p_free0 + 8 * (c & 1), ((c >> 1) - 1) & 1, p.err, abort_flag);
+      uint8_t *pt = smem + SM::pt + (c & 1) * kPBytes;
+      uint32_t pk[16];
+#pragma unroll
+      for (int h = 0; h < 32; h += 2) {
+        const float e0 = fast_exp2(sc[h] - mr[h]), e1 = fast_exp2(sc[h + 1] - mr[h + 1]);
+        lp[h] += e0;
+        lp[h + 1] += e1;
+        pk[h / 2] = pack_bf16x2(e0, e1);
+      }
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4)
+        *reinterpret_cast<uint4 *>(pt + i * 128 + ((q4 ^ (i & 7)) << 4)) =
+            make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+      if (!live) {
+        // V row of a token past t1 (a slot past L_b or a box not copied):
+        // zeros, after the chunk's copies have landed
+        wait_bounded(v_full, c & 1, p.err, abort_flag);
+        uint8_t *vrow = smem + SM::v + (i >> 3) * kBoxBytes + (i & 7) * 128;
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) {
+          *reinterpret_cast<uint4 *>(vrow + q8 * 16) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4 *>(vrow + 1024 + q8 * 16) = make_uint4(0, 0, 0, 0);
+        }
+      }
+      fence_proxy_async_smem();  // P^T and zeroed rows, before the tensor core reads them
+      tc_fence_before();
+      mbar_arrive1(p_full0 + 8 * (c & 1));
+    }
 
-      // ---- the unit's output: thread i = head_dim row i of O^T
-      const bool out_ready = wait_bounded(o_done, j & 1, p.err, abort_flag);
-      if (!softmax_bar_and(out_ready)) break;
+    // ---- the unit's output: thread i = head_dim row i of O^T
+    if (ok) ok = softmax_bar_and(wait_bounded(o_done, 0, p.err, abort_flag));
+    if (ok) {
       tc_fence_after();
       float tmp[32];
 #pragma unroll
@@ -592,23 +497,21 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_kernel(const __grid_cons
       tmem_ld32(tmem_o + lane_off, o);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive1(o_free);  // O^T may be overwritten by the next unit
-      ++j;
       softmax_bar();
       const float lh = red[lane] + red[32 + lane] + red[64 + lane] + red[96 + lane];  // head = lane
       float mrl = 0.f;  // mr[lane]
 #pragma unroll
       for (int h = 0; h < 32; ++h) mrl = h == lane ? mr[h] : mrl;
-      if (e.ns == 1) {
+      if (ns == 1) {
 #pragma unroll
         for (int h = 0; h < 32; ++h) {
           const float inv = 1.f / __shfl_sync(0xffffffffu, lh, h);
-          if (h < gl) p.out[e.b * p.o_sb + (int64_t)(h0 + h) * p.o_sh + i] = to_bf16_bits(__uint_as_float(o[h]) * inv);
+          if (h < gl) p.out[b * p.o_sb + (int64_t)(h0 + h) * p.o_sh + i] = to_bf16_bits(__uint_as_float(o[h]) * inv);
         }
         if (warp == 0 && lane < gl && p.lse != nullptr)
-          p.lse[e.b * p.lse_sb + (int64_t)(h0 + lane) * p.lse_sh] = (mrl + log2f(lh)) * kLn2u;
+          p.lse[b * p.lse_sb + (int64_t)(h0 + lane) * p.lse_sh] = (mrl + log2f(lh)) * kLn2u;
       } else {
-        const int64_t row0 = ((int64_t)e.b * p.Hq + h0) * p.S + e.s;
+        const int64_t row0 = ((int64_t)b * p.Hq + h0) * p.S + s;
 #pragma unroll
         for (int h = 0; h < 32; ++h) {
           const float inv = 1.f / __shfl_sync(0xffffffffu, lh, h);
@@ -616,9 +519,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_kernel(const __grid_cons
         }
         if (warp == 0 && lane < gl) p.lse_part[row0 + (int64_t)lane * p.S] = (mrl + log2f(lh)) * kLn2u;
       }
-      softmax_bar();  // `red` is read by every warp before it is written again
-      if (e.ns > 1 && claim_last_partition(p, e.b, e.kvh, e.ht, e.ns, reinterpret_cast<int *>(words + 1), Warps0to3Sync()))
-        merge_partials<kD, kSoftmaxWarps * 32>(p, e.b, h0, gl, 0, e.ns, reinterpret_cast<float *>(smem + SM::mw),
+      softmax_bar();  // `red` is read by every warp before the merge reuses shared memory
+      // every chunk has been consumed: the K and V buffers hold the merge's weights
+      if (ns > 1 && claim_last_partition(p, b, kvh, ht, ns, reinterpret_cast<int *>(words + 1), Warps0to3Sync()))
+        merge_partials<kD, kSoftmaxWarps * 32>(p, b, h0, gl, 0, ns, reinterpret_cast<float *>(smem + SM::k),
                                                Warps0to3Sync());
     }
   }
@@ -634,21 +538,20 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_kernel(const __grid_cons
   }
 }
 
-int umma_stages() { return kUmmaStages; }
+int umma_stages() { return 1; }
 
 cudaError_t launch_umma(const PartitionParams &p, int grid, cudaStream_t stream) {
   static std::atomic<uint64_t> attr_done{0};
-  using SM = UmmaSmem<kUmmaStages>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_done.load(std::memory_order_acquire) & bit)) {
-    e = cudaFuncSetAttribute(umma_kernel<kUmmaStages>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::total);
+    e = cudaFuncSetAttribute(umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)UmmaSmem::total);
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(bit, std::memory_order_acq_rel);
   }
-  umma_kernel<kUmmaStages><<<grid, kUmmaThreads, SM::total, stream>>>(p);
+  umma_kernel<<<grid, kUmmaThreads, UmmaSmem::total, stream>>>(p);
   return cudaGetLastError();
 }
 
