@@ -30,22 +30,23 @@ struct Warps0to3Sync {
 
 // Counts this partition; true (in every participating thread) for the CTA that
 // completes the set, which also resets the counter for the next launch.  The
-// barrier orders every participant's partial stores before thread 0's fence,
-// which publishes them (cumulatively) before the count.  Every participating
-// thread calls it; thread 0 must be one of them.
+// barrier orders every participant's partial stores before thread 0's count, a
+// release-acquire atomic at GPU scope: its release publishes them
+// (cumulatively), and in the CTA that completes the set its acquire orders the
+// other partitions' stores, published by their releases to the same counter,
+// before the merge's loads (which the next barrier passes on to every
+// participant).  Every participating thread calls it; thread 0 must be one of
+// them.
 template <class Sync = CtaSync>
 __device__ __forceinline__ bool claim_last_partition(const PartitionParams &p, int b, int kvh, int ht, int ns,
                                                      int *flag, Sync sync = Sync()) {
   sync();
   if (threadIdx.x == 0) {
     const uint32_t pair = ((uint32_t)b * p.Hkv + kvh) * p.HT + ht;
-    __threadfence();
-    const uint32_t done = atomicAdd(p.counters + pair, 1u);
+    uint32_t done;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;\n" : "=r"(done) : "l"(p.counters + pair) : "memory");
     const int last = done + 1 == (uint32_t)ns;
-    if (last) {
-      atomicExch(p.counters + pair, 0u);  // ready for the next launch
-      __threadfence();                    // the other partials' stores, before the loads below
-    }
+    if (last) atomicExch(p.counters + pair, 0u);  // ready for the next launch
     *flag = last;
   }
   sync();
