@@ -140,3 +140,36 @@ def test_caller_workspace_with_options(cuda_device, splits):
     out, lse = DeviceWorkload(w, cuda_device).run(num_splits=splits, entry=entry)
     check_parity(to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, f"workspace_ex/S={splits}")
     assert pad.pad_check_device_errors() == 0
+
+
+def test_e4m3_graph_replay_reads_live_inputs(cuda_device):
+    # a captured E4M3 decode (scales, window, sinks) replayed after q changed in
+    # place: the graph reads the tensors' current contents
+    w = _case("e4m3_graph", 3, 8, 2, 128, 16, [300, 45, 700])
+    sinks = np.asarray([0.5, -1.0, 2.0, 0.0, -3.0, 1.0, 0.25, -0.5], dtype=np.float32)
+    dev_sinks = torch.from_numpy(sinks).to(cuda_device)
+    W = 200
+    dw = DeviceWorkload(w, cuda_device)
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=cuda_device)
+    lse = torch.empty((w.B, w.Hq), device=cuda_device)
+    s = torch.cuda.Stream()
+
+    def call():
+        pad.pad_decode(dw.q, dw.k, dw.v, dw.tables, dw.lens, w.scale, num_splits=3, out=out, lse=lse, window=W,
+                       sinks=dev_sinks, k_scale=w.k_scale, v_scale=w.v_scale)
+
+    with torch.cuda.stream(s):
+        call()  # the library's scratch for this shape exists before capture
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        call()
+    q2 = synth.bf16_array(w.q.shape, 999, 1)
+    dw.q.copy_(torch.from_numpy(q2).view(torch.bfloat16).to(cuda_device))
+    out.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    w2 = synth.Workload(**{**w.__dict__, "q": q2})
+    ref_out, ref_lse = oracle.decode_workload(w2, window=W, sinks=sinks)
+    check_parity(to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, "e4m3 graph replay")
+    assert pad.pad_check_device_errors() == 0

@@ -48,6 +48,20 @@ def test_static_scratch_matches_pad_decode_twice(cuda_device):
         _compare(out, lse, ref_out, ref_lse)
 
 
+def test_static_scratch_e4m3_cache(cuda_device):
+    # an E4M3 cache of unit scales (the entry takes no options) through the
+    # static array, against pad_decode on the same inputs
+    w = synth.make_workload("na_e4m3", 6, 16, 4, 128, 16, [900, 40, 1024, 0, 333, 129], seed=64,
+                            max_blocks_per_seq=64, kv_dtype="e4m3", k_scale=1.0, v_scale=1.0)
+    dw = DeviceWorkload(w, cuda_device)
+    ref_out, ref_lse = pad.pad_decode(dw.q, dw.k, dw.v, dw.tables, dw.lens, w.scale, num_splits=8, lse=True)
+    out = torch.full((w.B, w.Hq, w.D), float("nan"), dtype=torch.bfloat16, device=cuda_device)
+    lse = torch.full((w.B, w.Hq), float("nan"), device=cuda_device)
+    pad.pad_decode_static_scratch(dw.q, dw.k, dw.v, dw.tables, dw.lens, w.scale, num_splits=8, out=out, lse=lse)
+    torch.cuda.synchronize()
+    _compare(out, lse, ref_out, ref_lse)
+
+
 def test_static_scratch_rejects_shapes_beyond_its_size(cuda_device):
     w = synth.make_workload("na_big", 2, 64, 1, 256, 16, [40, 40], seed=63, max_blocks_per_seq=4096)
     dw = DeviceWorkload(w, cuda_device)
