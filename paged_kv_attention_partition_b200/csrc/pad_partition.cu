@@ -127,9 +127,17 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int dh = warp % DS, hg = (warp / DS) % HG, tg = warp / (DS * HG);  // head_dim part, head group, token group
+  // Grid order: partition index descending, outermost.  The highest partitions
+  // exist only for the longest sequences, so their work starts first and the
+  // empty ones (short sequences) exit early; the last waves are every
+  // sequence's first partition, full for every sequence that reaches P tokens.
+  // Measured on B200: llama8b (lengths 512..4096) 59.4 -> 56.1 us against
+  // partition-innermost order; batches of uniform full lengths lose ~3% (every
+  // merge then falls in the last wave).
   uint32_t u = blockIdx.x;
-  const int s = (int)(u % (uint32_t)p.S);
-  u /= (uint32_t)p.S;
+  const uint32_t pairs = (uint32_t)p.B * p.Hkv * p.HT;
+  const int s = p.S - 1 - (int)(u / pairs);
+  u %= pairs;
   const int ht = (int)(u % (uint32_t)p.HT);
   u /= (uint32_t)p.HT;
   const int kvh = (int)(u % (uint32_t)p.Hkv);
