@@ -1,0 +1,78 @@
+"""Host-side helpers of bench.py, on CPU: the split-scratch byte count, the
+recorded-traffic lookup (and its source-hash check), and the CPU baseline's
+bounded samples."""
+import importlib.util
+import os
+
+import numpy as np
+
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_split_scratch_bytes_counts_multi_partition_sequences():
+    bench = _bench()
+    w = synth.make_workload("sc", 4, 8, 2, 64, 16, [0, 100, 512, 1000], seed=3, max_blocks_per_seq=64)
+    P = 256
+    # brute force: per sequence, the partitions that hold a token
+    expect = 0
+    for L in w.seq_lens.tolist():
+        ns = len({t // P for t in range(L)})
+        if ns > 1:
+            expect += 2 * ns * w.Hq * (w.D + 1) * 4
+    assert bench.split_scratch_bytes(w, {"partition_tokens": P}) == expect
+    # a window keeps only the partitions that hold its tokens
+    W = 300
+    expect_w = 0
+    for L in w.seq_lens.tolist():
+        ns = len({t // P for t in range(max(0, L - W), L)})
+        if ns > 1:
+            expect_w += 2 * ns * w.Hq * (w.D + 1) * 4
+    assert bench.split_scratch_bytes(w, {"partition_tokens": P}, window=W) == expect_w
+
+
+def test_traffic_is_read_only_for_the_recorded_source(tmp_path, monkeypatch):
+    bench = _bench()
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "partition_kernel_demo.md").write_text("# demo\n\nsource_sha256: abc123\ndram_bytes_per_launch: 4242\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_from_profiles("demo", "abc123") == 4242
+    assert bench.traffic_from_profiles("demo", "other") is None  # the kernel changed since the capture
+    assert bench.traffic_from_profiles("missing", "abc123") is None
+
+
+def test_kernel_source_hash_covers_the_kernel_headers():
+    bench = _bench()
+    sha = bench.kernel_source_sha()
+    assert len(sha) == 16 and sha == bench.kernel_source_sha()
+
+
+def test_cpu_baseline_samples_are_bounded_and_described(monkeypatch):
+    bench = _bench()
+    w = synth.config("tiny")
+    cb = bench.cpu_baseline(w, budget_s=0.2, runs_max=3)
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] > 0
+    one = cb["one_thread"]
+    assert one["cores"] == 1 and one["value"] > 0 and "whole tiny batch" in one["sample"]
+    # a batch too slow for one thread is sampled through its first sequences
+    big = synth.make_workload("big", 3, 8, 2, 128, 16, [4096] * 3, seed=4, max_blocks_per_seq=256)
+    calls = []
+
+    def prefix(k):
+        calls.append(k)
+        return synth.make_workload("big", k, 8, 2, 128, 16, [4096] * k, seed=4, max_blocks_per_seq=256)
+
+    clock = iter(np.arange(0, 1e6, 50.0))  # every timed oracle call "takes" 50 s
+    monkeypatch.setattr(bench.time, "perf_counter", lambda: float(next(clock)))
+    cb2 = bench.cpu_baseline(big, budget_s=1.0, runs_max=1, prefix=prefix)
+    assert calls and calls[0] < big.B
+    assert cb2["one_thread"]["sample"].startswith(f"first {calls[0]} of {big.B}")
