@@ -286,6 +286,30 @@ pad_status pad_decode_plan_ex(int64_t batch, int64_t num_q_heads, int64_t num_kv
                               int64_t head_dim, int64_t block_size, int64_t max_blocks_per_seq,
                               int32_t num_splits, int32_t kv_dtype, int32_t device, pad_plan *plan);
 
+/*
+ * pad_launch_witness / pad_last_launch -- what the most recent decode launch
+ * on the current device recorded from inside the kernel (block 0, before
+ * anything else): which kernel ran and the plan it was compiled and launched
+ * with.  A test compares it with pad_decode_plan[_ex] to show that the planned
+ * kernel is the one that executed ("Attention parity: run every attention type
+ * on the best available path on both targets": a silent fallback counts as a
+ * failure).  pad_last_launch synchronises the device; concurrent launches on
+ * several streams leave the record of whichever wrote last.
+ */
+typedef struct pad_launch_witness {
+  int32_t kernel;            /* 1: partition kernel (mma.sync), 2: tcgen05 kernel; 0: none yet */
+  int32_t head_dim;          /* D the kernel was compiled for */
+  int32_t heads_per_tile;    /* query heads per unit it was compiled for */
+  int32_t kv_dtype;          /* pad_dtype of the cache it was compiled for */
+  int32_t stages;            /* pipeline stages it was compiled with */
+  int32_t stage_tokens;      /* tokens per stage (chunk) */
+  int32_t num_splits;        /* S it was launched with */
+  int32_t partition_tokens;  /* P it was launched with */
+  int32_t ctas;              /* grid size */
+} pad_launch_witness;
+
+pad_status pad_last_launch(pad_launch_witness *witness);
+
 /* Static string for a status code. */
 const char *pad_status_string(pad_status status);
 

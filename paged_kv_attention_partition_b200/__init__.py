@@ -51,6 +51,12 @@ class PadOptions(ctypes.Structure):
                 ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float)]
 
 
+class PadLaunchWitness(ctypes.Structure):
+    """pad_launch_witness: what the most recent launch recorded from inside the kernel."""
+    _fields_ = [(n, ctypes.c_int32) for n in ("kernel", "head_dim", "heads_per_tile", "kv_dtype", "stages",
+                                                  "stage_tokens", "num_splits", "partition_tokens", "ctas")]
+
+
 class PadError(RuntimeError):
     def __init__(self, status: int, message: str):
         super().__init__(f"{_status_name(status)}: {message}")
@@ -94,6 +100,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pad_decode_plan.restype = ctypes.c_int
     lib.pad_decode_plan_ex.argtypes = [ctypes.c_int64] * 6 + [ctypes.c_int32] * 3 + [ctypes.POINTER(PadPlan)]
     lib.pad_decode_plan_ex.restype = ctypes.c_int
+    lib.pad_last_launch.argtypes = [ctypes.POINTER(PadLaunchWitness)]
+    lib.pad_last_launch.restype = ctypes.c_int
     lib.pad_status_string.argtypes = [ctypes.c_int]
     lib.pad_status_string.restype = ctypes.c_char_p
     lib.pad_last_error.argtypes = []
@@ -314,6 +322,17 @@ def pad_check_device_errors(stream=None, device=None) -> int:
     return bits.value
 
 
+def pad_last_launch(device=None) -> dict:
+    """What the most recent decode launch on the device recorded from inside the
+    kernel: ``kernel`` (1 partition kernel, 2 tcgen05 kernel) and the plan it ran
+    with.  Synchronises the device."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    w = PadLaunchWitness()
+    with torch.cuda.device(dev):
+        _raise(load_library().pad_last_launch(ctypes.byref(w)))
+    return {name: getattr(w, name) for name, _ in w._fields_}
+
+
 def pad_release_workspace(device: int = -1) -> None:
     """Free the library's split scratch for one device (all when < 0)."""
     _raise(load_library().pad_release_workspace(device))
@@ -322,4 +341,4 @@ def pad_release_workspace(device: int = -1) -> None:
 __all__ = ["pad_decode", "pad_decode_with_workspace", "pad_decode_static_scratch", "pad_decode_tcgen05", "pad_decode_plan",
            "pad_check_device_errors", "pad_release_workspace",
            "pad_status_string", "pad_last_error", "pad_abi_version", "describe", "load_library",
-           "PadError", "PadTensor", "PadPlan", "PadOptions"]
+           "PadError", "PadTensor", "PadPlan", "PadOptions", "PadLaunchWitness", "pad_last_launch"]

@@ -457,6 +457,7 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
   p.lse_sb = lse != nullptr ? lse->stride[0] : 0;
   p.lse_sh = lse != nullptr ? lse->stride[1] : 0;
   p.err = err;
+  if ((e = pad::device_witness(device, &p.witness)) != cudaSuccess) return cuda_fail(e, "launch witness");
   pr->D = (int)D;
   pr->device = device;
   pr->kv_fp8 = fp8;
@@ -632,6 +633,28 @@ pad_status pad_decode_with_workspace_ex(const pad_tensor *q, const pad_tensor *k
   if (pr.cl.total > 0 && (st = get_buffer(g_ctl, pr.device, stream, pr.cl.total, &ctl)) != PAD_OK) return st;
   bind_buffers(pr, workspace, ctl);
   return run(pr, stream);
+}
+
+pad_status pad_last_launch(pad_launch_witness *w) {
+  if (w == nullptr) return fail(PAD_ERR_INVALID_ARG, "witness is NULL");
+  int device = 0;
+  cudaError_t e = cudaGetDevice(&device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  pad::LaunchWitness *dw = nullptr;
+  if ((e = pad::device_witness(device, &dw)) != cudaSuccess) return cuda_fail(e, "launch witness");
+  if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  pad::LaunchWitness h{};
+  if ((e = cudaMemcpy(&h, dw, sizeof(h), cudaMemcpyDeviceToHost)) != cudaSuccess) return cuda_fail(e, "read witness");
+  w->kernel = h.kernel;
+  w->head_dim = h.head_dim;
+  w->heads_per_tile = h.heads_per_tile;
+  w->kv_dtype = h.kv_dtype;
+  w->stages = h.stages;
+  w->stage_tokens = h.stage_tokens;
+  w->num_splits = h.num_splits;
+  w->partition_tokens = h.partition_tokens;
+  w->ctas = h.ctas;
+  return PAD_OK;
 }
 
 pad_status pad_check_device_errors(void *stream_, uint32_t *bits) {

@@ -109,6 +109,11 @@ __host__ __device__ constexpr SmemPlan smem_plan_for(int D, int hpt, bool f8 = f
 // Largest query-head tile whose fp32 O^T accumulator (D x heads) fits one warp's registers.
 inline int max_heads_per_tile(int D) { return D <= 128 ? 32 : 16; }
 
+// What a launch records from inside the kernel (pad_last_launch).
+struct LaunchWitness {
+  int32_t kernel, head_dim, heads_per_tile, kv_dtype, stages, stage_tokens, num_splits, partition_tokens, ctas;
+};
+
 struct PartitionParams {
   // K and V caches as 5-D tiled tensors (128 bytes of head_dim, slot, the
   // rest of head_dim in 128-byte blocks, kv head, block), one box = one page
@@ -148,6 +153,7 @@ struct PartitionParams {
   float *lse_part;     // [B, Hq, S] fp32 (natural log)
   uint32_t *counters;  // [B * Hkv * HT] partitions finished per (b, kv head, head tile)
   uint32_t *err;
+  LaunchWitness *witness;  // written by block 0 of every launch
 };
 
 // Partials layout inside a workspace buffer (offsets 256-byte aligned); empty
@@ -196,6 +202,7 @@ inline int box_rows(int block_size, int D, int hpt, bool f8) {
 }
 int partition_stages(int D, int heads_per_tile, bool kv_fp8);
 cudaError_t device_error_word(int device, uint32_t **ptr);
+cudaError_t device_witness(int device, LaunchWitness **ptr);
 void set_last_error(const char *msg);
 
 // pad_decode with explicit buffers: `partials` (>= the plan's workspace_bytes,

@@ -69,6 +69,7 @@
 namespace pad {
 
 __device__ uint32_t g_err_word;
+__device__ LaunchWitness g_witness;
 
 namespace {
 constexpr float kLn2 = 0.69314718055994530942f;
@@ -127,6 +128,9 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int dh = warp % DS, hg = (warp / DS) % HG, tg = warp / (DS * HG);  // head_dim part, head group, token group
+  if (blockIdx.x == 0 && tid == 0)  // which kernel ran, and with what plan
+    *p.witness = LaunchWitness{1, D, HPT, F8 ? (int32_t)PAD_FP8_E4M3 : (int32_t)PAD_BF16, NST, ST, p.S, p.P,
+                               (int32_t)gridDim.x};
   // Grid order: partition index descending, outermost.  The highest partitions
   // exist only for the longest sequences, so their work starts first and the
   // empty ones (short sequences) exit early; the last waves are every
@@ -679,6 +683,21 @@ cudaError_t launch_partition(const PartitionParams &p, int D, int heads_per_tile
                              cudaStream_t s) {
   if (heads_per_tile > max_heads_per_tile(D)) return cudaErrorInvalidValue;
   return kv_fp8 ? launch_f<true>(p, D, heads_per_tile, grid, s) : launch_f<false>(p, D, heads_per_tile, grid, s);
+}
+
+cudaError_t device_witness(int device, LaunchWitness **ptr) {
+  static std::atomic<LaunchWitness *> cache[64];
+  if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
+  LaunchWitness *v = cache[device].load(std::memory_order_acquire);
+  if (v == nullptr) {
+    void *addr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&addr, g_witness);
+    if (e != cudaSuccess) return e;
+    v = static_cast<LaunchWitness *>(addr);
+    cache[device].store(v, std::memory_order_release);
+  }
+  *ptr = v;
+  return cudaSuccess;
 }
 
 cudaError_t device_error_word(int device, uint32_t **ptr) {
