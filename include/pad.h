@@ -291,10 +291,13 @@ pad_status pad_decode_plan_ex(int64_t batch, int64_t num_q_heads, int64_t num_kv
  * on the current device recorded from inside the kernel (block 0, before
  * anything else): which kernel ran and the plan it was compiled and launched
  * with.  A test compares it with pad_decode_plan[_ex] to show that the planned
- * kernel is the one that executed ("Attention parity: run every attention type
- * on the best available path on both targets": a silent fallback counts as a
- * failure).  pad_last_launch synchronises the device; concurrent launches on
- * several streams leave the record of whichever wrote last.
+ * kernel is the one that executed: kernel-resident witnesses of which arm ran
+ * ("perf(BACKEND-ROCM): cooperate across Q8_K activation blocks", section
+ * "What changed"), because selection can land silently on another path
+ * ("Attention parity: run every attention type on the best available path on
+ * both targets", opening summary).  pad_last_launch synchronises the device;
+ * concurrent launches on several streams leave the record of whichever wrote
+ * last.
  */
 typedef struct pad_launch_witness {
   int32_t kernel;            /* 1: partition kernel (mma.sync), 2: tcgen05 kernel; 0: none yet */

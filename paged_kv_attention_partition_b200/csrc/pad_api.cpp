@@ -7,9 +7,11 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <map>
+#include <set>
 #include <mutex>
 #include <string>
 #include <utility>
@@ -97,6 +99,39 @@ int sm_count(int device) {
 // partitions for the llama8b (512) and ragged_mqa (2048) batches.  At most
 // kMaxSplits partitions per sequence.  One CTA per unit; units past a
 // sequence's length exit at once.
+// PAD_LOG=1: one line on stderr for each distinct (shape, request, device,
+// kernel) the library plans, the first time it plans it -- the launch geometry
+// the decode entry points and pad_decode_plan choose.  Unset, empty or "0":
+// silent.
+// Any other value: one warning, then silent (a logging switch never fails a call).
+bool plan_log_enabled() {
+  static const bool on = [] {
+    const char *v = getenv("PAD_LOG");
+    if (v == nullptr || v[0] == '\0' || strcmp(v, "0") == 0) return false;
+    if (strcmp(v, "1") == 0) return true;
+    fprintf(stderr, "pad: PAD_LOG=%s ignored (0 or 1)\n", v);
+    return false;
+  }();
+  return on;
+}
+
+void log_plan(const Shape &s, int32_t requested, int device, const pad_plan &p, bool umma) {
+  if (!plan_log_enabled()) return;
+  char line[512];
+  snprintf(line, sizeof line,
+           "pad: plan B=%lld Hq=%lld Hkv=%lld D=%lld bs=%lld capacity=%lld kv=%s num_splits=%d device=%d -> "
+           "kernel=%s S=%d P=%d heads_per_tile=%d head_tiles=%d stages=%dx%d warps=%d ctas=%d "
+           "workspace_bytes=%lld control_bytes=%lld\n",
+           (long long)s.B, (long long)s.Hq, (long long)s.Hkv, (long long)s.D, (long long)s.bs,
+           (long long)(s.W * s.bs), s.fp8 ? "e4m3" : "bf16", requested, device, umma ? "tcgen05" : "partition",
+           p.num_splits, p.partition_tokens, p.heads_per_tile, p.head_tiles, p.stages, p.stage_tokens,
+           p.warps_per_cta, p.ctas, (long long)p.workspace_bytes, (long long)p.control_bytes);
+  static std::mutex mu;
+  static std::set<std::string> seen;
+  std::lock_guard<std::mutex> lock(mu);
+  if (seen.insert(line).second) fputs(line, stderr);
+}
+
 void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan, bool tcgen05 = false) {
   const int64_t C = s.W * s.bs;
   int hpt = s.g <= 8 ? 8 : (s.g <= 16 ? 16 : 32);
@@ -133,6 +168,7 @@ void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan, b
   plan->reduce = S > 1 ? 1 : 0;
   plan->workspace_bytes = (int64_t)pad::workspace_layout(s.B, s.Hq, S, s.D).total;
   plan->control_bytes = (int64_t)pad::control_layout(s.B, s.Hkv, HT, S).total;
+  log_plan(s, num_splits, device, *plan, umma);
 }
 
 // ---- TMA tensor maps of the K/V caches --------------------------------------
@@ -465,9 +501,11 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
 }
 
 void bind_buffers(Prepared &pr, void *partials, void *control) {
+  // No partials buffer (one partition per sequence, nothing to merge): the
+  // kernel never reads these, and no offset is applied to a null pointer.
   char *base = static_cast<char *>(partials);
-  pr.p.o_part = reinterpret_cast<float *>(base + pr.ws.o_part);
-  pr.p.lse_part = reinterpret_cast<float *>(base + pr.ws.lse_part);
+  pr.p.o_part = base != nullptr ? reinterpret_cast<float *>(base + pr.ws.o_part) : nullptr;
+  pr.p.lse_part = base != nullptr ? reinterpret_cast<float *>(base + pr.ws.lse_part) : nullptr;
   pr.p.counters = pr.cl.total > 0 ? reinterpret_cast<uint32_t *>(static_cast<char *>(control) + pr.cl.counters)
                                   : nullptr;
 }

@@ -189,5 +189,6 @@ void synth_uniform_int(int32_t *dst, int64_t n, int32_t lo, int32_t hi, uint64_t
                        uint64_t stream) {
   uint64_t key = stream_key(seed, stream);
   uint64_t span = (uint64_t)((int64_t)hi - (int64_t)lo + 1);
-  for (int64_t i = 0; i < n; ++i) dst[i] = lo + (int32_t)below(draw(key, (uint64_t)i), span);
+  /* the offset is below 2^32; the sum, in [lo, hi], is formed in 64 bits */
+  for (int64_t i = 0; i < n; ++i) dst[i] = (int32_t)((int64_t)lo + (int64_t)below(draw(key, (uint64_t)i), span));
 }

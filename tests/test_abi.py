@@ -202,3 +202,25 @@ def test_e4m3_plan_keeps_partitions_and_scratch(lib):
     with pytest.raises(pad.PadError) as e:
         pad.pad_decode_plan(4, 16, 2, 128, 16, 100, kv_dtype="fp4")
     assert e.value.status == pad.PAD_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("value, lines, warned", [("1", 2, False), (None, 0, False), ("", 0, False), ("0", 0, False),
+                                                  ("yes", 0, True)])
+def test_pad_log_prints_each_plan_once(value, lines, warned):
+    # PAD_LOG=1: the plan chosen for each distinct shape, once; other values
+    # warn once and stay silent; unset, empty or 0 print nothing
+    import sys
+    env = {k: v for k, v in os.environ.items() if k != "PAD_LOG"}
+    if value is not None:
+        env["PAD_LOG"] = value
+    code = ("import paged_kv_attention_partition_b200 as pad\n"
+            "for _ in range(3): pad.pad_decode_plan(32, 32, 8, 128, 16, 256)\n"
+            "pad.pad_decode_plan(64, 40, 8, 128, 16, 512, num_splits=16, kv_dtype='e4m3')\n")
+    res = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env, cwd=ROOT, timeout=120)
+    assert res.returncode == 0, res.stderr
+    plans = [l for l in res.stderr.splitlines() if l.startswith("pad: plan ")]
+    assert len(plans) == lines, res.stderr
+    if lines:
+        assert "B=32 Hq=32 Hkv=8 D=128 bs=16 capacity=4096 kv=bf16 num_splits=0" in plans[0]
+        assert "kv=e4m3 num_splits=16" in plans[1] and " S=16 P=512 " in plans[1]
+    assert ("ignored" in res.stderr) == warned

@@ -1,0 +1,112 @@
+"""Address and undefined-behaviour sanitizer lane for the host code (CPU only).
+
+Two executables, built here with -fsanitize=address,undefined and run without a
+GPU (the CPU lane of "perf(BACKEND-ROCM): cooperate across Q8_K activation
+blocks", vllm.cpp PR #2472, CI classification comment):
+
+* host_lane_oracle.c + oracle/oracle.c + synth/synth.c: the checker and the
+  input generator on small paged problems in every mode;
+* host_lane_abi.c + the library's own sources (pad_api.cpp by g++, the .cu files
+  by nvcc with the same sm_100a flags as the product build, host side
+  instrumented): plans over a grid of shapes, every decode entry point with one
+  argument broken at a time, an empty batch.
+
+The two never share a binary: the checker and the library stay apart.  The GPU
+side has no sanitizer here; its bounds are covered by the kernels' own checks
+(error word) and the parity tests.
+"""
+import os
+import subprocess
+from concurrent.futures import ThreadPoolExecutor
+
+import pytest
+
+from paged_kv_attention_partition_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SAN = ["-fsanitize=address", "-fsanitize=undefined", "-fno-sanitize-recover=all", "-fno-omit-frame-pointer"]
+ENV = dict(os.environ,
+           ASAN_OPTIONS="detect_leaks=1:halt_on_error=1:abort_on_error=0",
+           UBSAN_OPTIONS="print_stacktrace=1:halt_on_error=1")
+
+
+def _cuda_home() -> str:
+    return os.path.dirname(os.path.dirname(os.path.realpath(_build.nvcc())))
+
+
+def _run(cmd, **kw):
+    res = subprocess.run(cmd, capture_output=True, text=True, **kw)
+    assert res.returncode == 0, " ".join(cmd) + "\n" + res.stdout + res.stderr
+    return res
+
+
+def _assert_clean(res):
+    out = res.stdout + res.stderr
+    assert res.returncode == 0, out
+    for marker in ("runtime error", "AddressSanitizer", "LeakSanitizer", "FAIL "):
+        assert marker not in out, out
+    assert "clean" in res.stdout
+
+
+def test_oracle_and_generator_under_sanitizers(tmp_path):
+    exe = tmp_path / "lane_oracle"
+    _run(["gcc", "-std=c11", "-O1", "-g", *SAN, "-Wall", "-Wextra", "-Werror",
+          os.path.join(ROOT, "tests", "host_lane_oracle.c"), os.path.join(ROOT, "oracle", "oracle.c"),
+          os.path.join(ROOT, "synth", "synth.c"), "-lm", "-lpthread", "-o", str(exe)])
+    _assert_clean(subprocess.run([str(exe)], capture_output=True, text=True, env=ENV, timeout=300))
+
+
+def test_c_abi_host_code_under_sanitizers(tmp_path):
+    cuda = _cuda_home()
+    inc = ["-I", _build.INCLUDE, "-I", _build.CSRC]
+    jobs = []
+    objs = []
+    for src in _build.SOURCES:
+        obj = str(tmp_path / (os.path.splitext(src)[0] + ".o"))
+        objs.append(obj)
+        path = os.path.join(_build.CSRC, src)
+        if src.endswith(".cpp"):
+            jobs.append(["g++", "-std=c++17", "-O1", "-g", *SAN, *inc, "-I", os.path.join(cuda, "include"),
+                         "-c", path, "-o", obj])
+        else:
+            xc = [a for flag in SAN for a in ("-Xcompiler", flag)]
+            jobs.append([_build.nvcc(), "-std=c++17", "-O1", "-g", *_build.ARCH_FLAGS, *xc, *inc, "-c", path,
+                         "-o", obj])
+    lane_obj = str(tmp_path / "lane_abi.o")
+    objs.append(lane_obj)
+    jobs.append(["gcc", "-std=c11", "-O1", "-g", *SAN, "-Wall", "-Wextra", "-Werror", "-I", _build.INCLUDE,
+                 "-c", os.path.join(ROOT, "tests", "host_lane_abi.c"), "-o", lane_obj])
+    with ThreadPoolExecutor(max_workers=len(jobs)) as ex:
+        for f in [ex.submit(_run, j) for j in jobs]:
+            f.result()
+    exe = str(tmp_path / "lane_abi")
+    _run(["g++", *SAN, *objs, "-L", os.path.join(cuda, "lib64"), "-lcudart_static", "-ldl", "-lrt", "-lpthread",
+          "-o", exe])
+    res = subprocess.run([exe], capture_output=True, text=True, env=ENV, timeout=300)
+    _assert_clean(res)
+
+
+def test_lane_catches_a_planted_overrun(tmp_path):
+    """Negative control: the same lane on a copy of the checker whose score loop
+    runs one token past the sequence (a plausible off-by-one) must fail -- the
+    last sequence fills its table row, so the extra token reads past the table."""
+    src = open(os.path.join(ROOT, "oracle", "oracle.c")).read()
+    loop = "for (int64_t t = lo; t < L; ++t) {"
+    i = src.index(loop)  # the first token loop: the scores
+    assert src.index("s[t - lo] = p->scale * acc;", i) < src.index(loop, i + 1)
+    bad = tmp_path / "oracle_overrun.c"
+    bad.write_text(src[:i] + loop.replace("t < L", "t <= L") + src[i + len(loop):])
+    exe = tmp_path / "lane_bad"
+    _run(["gcc", "-std=c11", "-O1", "-g", *SAN, os.path.join(ROOT, "tests", "host_lane_oracle.c"), str(bad),
+          os.path.join(ROOT, "synth", "synth.c"), "-lm", "-lpthread", "-o", str(exe)])
+    res = subprocess.run([str(exe)], capture_output=True, text=True, env=ENV, timeout=300)
+    assert res.returncode != 0 and "AddressSanitizer" in res.stderr, res.stdout + res.stderr[-2000:]
+
+
+@pytest.mark.parametrize("lane", ["host_lane_oracle.c", "host_lane_abi.c"])
+def test_lane_sources_do_not_mix_the_checker_and_the_library(lane):
+    text = open(os.path.join(ROOT, "tests", lane)).read()
+    if lane == "host_lane_abi.c":
+        assert "oracle_" not in text and "synth_" not in text
+    else:
+        assert "pad.h" not in text and "pad_decode" not in text

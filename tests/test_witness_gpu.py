@@ -1,9 +1,11 @@
 """The kernel that ran is the kernel that was planned.
 
 Every decode launch records, from inside the kernel (block 0), which kernel ran
-and the plan it was compiled and launched with (pad_last_launch).  A silent
-fallback to another path would show here ("Attention parity: run every attention
-type on the best available path on both targets", section "Current state").
+and the plan it was compiled and launched with (pad_last_launch): a
+kernel-resident witness of the arm that executed ("perf(BACKEND-ROCM): cooperate
+across Q8_K activation blocks", section "What changed").  A silent landing on
+another path ("Attention parity: run every attention type on the best available
+path on both targets", opening summary) would show here.
 """
 import pytest
 import torch
