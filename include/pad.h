@@ -288,9 +288,11 @@ pad_status pad_decode_plan_ex(int64_t batch, int64_t num_q_heads, int64_t num_kv
 
 /*
  * pad_launch_witness / pad_last_launch -- what the most recent decode launch
- * on the current device recorded from inside the kernel (block 0, before
- * anything else): which kernel ran and the plan it was compiled and launched
- * with.  A test compares it with pad_decode_plan[_ex] to show that the planned
+ * on the current device recorded from inside the kernel (thread 0 of block 0:
+ * the partition kernel when its unit is done, the tcgen05 kernel at its
+ * start): which kernel ran and the plan it was compiled and launched with.  A
+ * launch whose block 0 gave up on an internal error (pad_check_device_errors
+ * reports it) leaves the previous record.  A test compares it with pad_decode_plan[_ex] to show that the planned
  * kernel is the one that executed: kernel-resident witnesses of which arm ran
  * ("perf(BACKEND-ROCM): cooperate across Q8_K activation blocks", section
  * "What changed"), because selection can land silently on another path

@@ -91,6 +91,20 @@ __device__ bool wait_stage(uint32_t bar, uint32_t parity, uint32_t *err) {
 }
 }  // namespace
 
+// Which kernel ran, and with what plan: thread 0 of block 0 writes the record
+// when its unit is done (empty, or through the epilogue); a unit that gives up
+// on an internal error records nothing -- the error word reports that case.
+// Out of line and at the exits, the store leaves the main loop's code as it is:
+// inlined (at the start or at the exits) it changed the 32-head bf16
+// instance's schedule at its 128-register cap and cost ragged_mqa 6% on B200;
+// as a call it is within 1% of no record at all.
+template <int D, int HPT, bool F8, int NST, int ST>
+__device__ __noinline__ void record_launch(const PartitionParams &p) {
+  if (blockIdx.x == 0 && threadIdx.x == 0)
+    *p.witness = LaunchWitness{1, D, HPT, F8 ? (int32_t)PAD_FP8_E4M3 : (int32_t)PAD_BF16, NST, ST, p.S, p.P,
+                               (int32_t)gridDim.x};
+}
+
 template <int D, int HPT, bool F8>
 __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
     partition_kernel(const __grid_constant__ PartitionParams p) {
@@ -128,9 +142,6 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int dh = warp % DS, hg = (warp / DS) % HG, tg = warp / (DS * HG);  // head_dim part, head group, token group
-  if (blockIdx.x == 0 && tid == 0)  // which kernel ran, and with what plan
-    *p.witness = LaunchWitness{1, D, HPT, F8 ? (int32_t)PAD_FP8_E4M3 : (int32_t)PAD_BF16, NST, ST, p.S, p.P,
-                               (int32_t)gridDim.x};
   // Grid order: partition index descending, outermost.  The highest partitions
   // exist only for the longest sequences, so their work starts first and the
   // empty ones (short sequences) exit early; the last waves are every
@@ -204,6 +215,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
       if (p.lse != nullptr && tid < gl)
         p.lse[b * p.lse_sb + (int64_t)(h0 + tid) * p.lse_sh] = p.sinks != nullptr ? p.sinks[h0 + tid] : -INFINITY;
     }
+    record_launch<D, HPT, F8, NST, ST>(p);
     return;  // pages wholly outside [lo, L) are never read
   }
   const int s_first = lo / p.P;                      // first non-empty partition of sequence b
@@ -640,6 +652,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
       if (d == 0) p.lse_part[row] = lse_nat;
     }
   }
+  record_launch<D, HPT, F8, NST, ST>(p);
   if (ns == 1) return;
   if (claim_last_partition(p, b, kvh, ht, ns, flag))
     merge_partials<D, kThreads>(p, b, h0, gl, s_first, ns, reinterpret_cast<float *>(smem));  // the ring is free
