@@ -57,7 +57,13 @@ def parse():
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay of the end-to-end step")
     ap.add_argument("--kv-dtype", default="bf16", choices=["bf16", "e4m3"],
                     help="KV cache element type (e4m3: OCP FP8 E4M3 codes with per-tensor scales)")
-    return ap.parse_args()
+    ap.add_argument("--entry", default="default", choices=["default", "tcgen05"],
+                    help="tcgen05: every leg calls pad_decode_tcgen05, the tensor-memory kernel (bf16 cache, "
+                         "head_dim 128, 17-32 query heads per KV head; no window, sinks or E4M3)")
+    args = ap.parse_args()
+    if args.entry == "tcgen05" and (args.kv_dtype != "bf16" or args.window or args.sinks):
+        ap.error("--entry tcgen05 takes a bf16 cache without --window or --sinks")
+    return args
 
 
 def measured_peaks():
@@ -183,9 +189,9 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-def traffic_from_profiles(workload, kernel_sha):
+def traffic_from_profiles(workload, kernel_sha, kernel="partition_kernel"):
     """ncu dram bytes per launch recorded under profiles/, if taken on this kernel source."""
-    path = os.path.join(ROOT, "profiles", f"partition_kernel_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     try:
         txt = open(path).read()
     except OSError:
@@ -199,9 +205,15 @@ def traffic_from_profiles(workload, kernel_sha):
         return None
 
 
-def kernel_source_sha():
+KERNEL_SOURCES = {
+    "partition_kernel": ("pad_partition.cu", "pad_merge.cuh", "pad_device.cuh", "pad_internal.h"),
+    "umma_kernel": ("pad_umma.cu", "pad_merge.cuh", "pad_device.cuh", "pad_internal.h"),
+}
+
+
+def kernel_source_sha(kernel="partition_kernel"):
     h = hashlib.sha256()
-    for f in ("pad_partition.cu", "pad_merge.cuh", "pad_device.cuh", "pad_internal.h"):
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "paged_kv_attention_partition_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -287,6 +299,8 @@ def main():
                                device=local, kv_dtype=args.kv_dtype)
     fp8 = args.kv_dtype == "e4m3"
     S = plan["num_splits"]
+    tc = args.entry == "tcgen05"
+    kernel = "umma_kernel" if tc else "partition_kernel"
 
     def dev_bf16(a):
         return torch.from_numpy(a).view(torch.bfloat16).to(dev)
@@ -313,15 +327,24 @@ def main():
     sinks_dev = (torch.from_numpy(np.random.default_rng(w.seed).standard_normal(w.Hq).astype(np.float32)).to(dev)
                  if args.sinks else None)
 
-    def call(stream_):
+    def decode(q_, tables_, lens_, out_, lse_, stream_):
         # the public one-call API, with the decode options when asked for
-        return pad.pad_decode(q, k, v, tables, lens, w.scale, num_splits=splits, out=out, lse=lse, stream=stream_,
-                              window=args.window, sinks=sinks_dev, k_scale=w.k_scale if fp8 else 0.0,
-                              v_scale=w.v_scale if fp8 else 0.0)
+        if tc:
+            return pad.pad_decode_tcgen05(q_, k, v, tables_, lens_, w.scale, num_splits=splits, out=out_, lse=lse_,
+                                          stream=stream_)
+        return pad.pad_decode(q_, k, v, tables_, lens_, w.scale, num_splits=splits, out=out_, lse=lse_,
+                              stream=stream_, window=args.window, sinks=sinks_dev,
+                              k_scale=w.k_scale if fp8 else 0.0, v_scale=w.v_scale if fp8 else 0.0)
+
+    def call(stream_):
+        return decode(q, tables, lens, out, lse, stream_)
 
     def step():
         # the whole hot path: one launch (partition + fused reduce), partials in
-        # the caller-owned workspace
+        # the caller-owned workspace (the tcgen05 entry: library-owned scratch)
+        if tc:
+            call(stream)
+            return
         pad.pad_decode_with_workspace(q, k, v, tables, lens, w.scale, splits, out, lse, ws, stream,
                                       window=args.window, sinks=sinks_dev, k_scale=w.k_scale if fp8 else 0.0,
                                       v_scale=w.v_scale if fp8 else 0.0)
@@ -388,9 +411,7 @@ def main():
 
     def e2e_step(stream_):
         din.copy_(hin, non_blocking=True)
-        pad.pad_decode(qe, k, v, te, le, w.scale, num_splits=splits, out=oute, lse=lsee, stream=stream_,
-                       window=args.window, sinks=sinks_dev, k_scale=w.k_scale if fp8 else 0.0,
-                       v_scale=w.v_scale if fp8 else 0.0)
+        decode(qe, te, le, oute, lsee, stream_)
         hout.copy_(dout, non_blocking=True)
 
     e2e_steps = 0 if args.no_e2e else max(10, args.steps // 2)
@@ -447,11 +468,12 @@ def main():
         p_bytes = alg_bytes
         p_ms = statistics.mean(part_ms)
         achieved = p_bytes / (p_ms / 1e3) / 1e9
-        sha = kernel_source_sha()
+        sha = kernel_source_sha(kernel)
         # the recorded ncu traffic is for the named workload at full size
-        traffic = (traffic_from_profiles(w.name + ("_e4m3" if fp8 else ""), sha)
+        traffic = (traffic_from_profiles(w.name + ("_e4m3" if fp8 else ""), sha, kernel)
                    if args.batch is None and not args.compact_pool else None)
-        kname = f"partition_kernel<{w.D},{plan['heads_per_tile']}>"
+        kname = f"{kernel}<{w.D},{plan['heads_per_tile']}>"
+        api = "pad_decode_tcgen05" if tc else "pad_decode"
         line = {
             "metric": "decode attention µs/call and achieved HBM GB/s vs B200 peak (1 GPU)",
             "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -459,6 +481,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16",
             "data": "synthetic (seeded counter-based generator; no dataset)",
             "config": {**workload_config(w, plan),
+                       **({"entry": "pad_decode_tcgen05"} if tc else {}),
                        **({"window": args.window, "kv_tokens": w.kv_tokens(args.window)} if args.window else {}),
                        **({"sinks": "one N(0,1) logit per query head"} if args.sinks else {}),
                        **({"kv_cache": f"e4m3, k_scale {w.k_scale:g}, v_scale {w.v_scale:g}"} if fp8 else {})},
@@ -470,10 +493,10 @@ def main():
                          "split_scratch_bytes_per_launch": split_scratch_bytes(w, plan, args.window)},
             "e2e": None if not e2e_steps else {
                 "value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "us_per_call": round(e2e_total / args.steps * 1e3, 2), "api": "pad_decode"},
+                "us_per_call": round(e2e_total / args.steps * 1e3, 2), "api": api},
             "e2e_graph": None if not graph_steps else {
                 "value": round(graph_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "us_per_call": round(graph_total / args.steps * 1e3, 2), "api": "pad_decode, replayed as a CUDA graph"},
+                "us_per_call": round(graph_total / args.steps * 1e3, 2), "api": api + ", replayed as a CUDA graph"},
             "gpu_launches": args.steps,  # one kernel launch per step
             "clocks": clocks.summary(),
         }

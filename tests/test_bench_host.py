@@ -76,3 +76,16 @@ def test_cpu_baseline_samples_are_bounded_and_described(monkeypatch):
     cb2 = bench.cpu_baseline(big, budget_s=1.0, runs_max=1, prefix=prefix)
     assert calls and calls[0] < big.B
     assert cb2["one_thread"]["sample"].startswith(f"first {calls[0]} of {big.B}")
+
+
+def test_each_kernel_has_its_own_source_hash_and_profile(tmp_path, monkeypatch):
+    bench = _bench()
+    assert bench.kernel_source_sha("umma_kernel") != bench.kernel_source_sha("partition_kernel")
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "umma_kernel_demo.md").write_text("source_sha256: u1\ndram_bytes_per_launch: 77\n")
+    (prof / "partition_kernel_demo.md").write_text("source_sha256: p1\ndram_bytes_per_launch: 55\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_from_profiles("demo", "u1", "umma_kernel") == 77
+    assert bench.traffic_from_profiles("demo", "p1") == 55
+    assert bench.traffic_from_profiles("demo", "p1", "umma_kernel") is None
