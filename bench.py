@@ -469,9 +469,11 @@ def main():
         p_ms = statistics.mean(part_ms)
         achieved = p_bytes / (p_ms / 1e3) / 1e9
         sha = kernel_source_sha(kernel)
-        # the recorded ncu traffic is for the named workload at full size
+        # the recorded ncu traffic is for the named workload at full size, as
+        # captured: no window, no sinks
         traffic = (traffic_from_profiles(w.name + ("_e4m3" if fp8 else ""), sha, kernel)
-                   if args.batch is None and not args.compact_pool else None)
+                   if args.batch is None and not args.compact_pool and not args.window and not args.sinks
+                   else None)
         kname = f"{kernel}<{w.D},{plan['heads_per_tile']}>"
         api = "pad_decode_tcgen05" if tc else "pad_decode"
         line = {
