@@ -68,8 +68,15 @@ pad_status check_shape(const Shape &s, int32_t num_splits) {
     return fail(PAD_ERR_UNSUPPORTED, "block_size %lld must be a power of two in [1, 256]", (long long)s.bs);
   if (s.g > 256)
     return fail(PAD_ERR_UNSUPPORTED, "GQA group %lld exceeds 256 query heads per KV head", (long long)s.g);
-  if (s.W * s.bs > (int64_t)1 << 30)
-    return fail(PAD_ERR_UNSUPPORTED, "table capacity %lld tokens too large", (long long)(s.W * s.bs));
+  // Bounds that keep every product below (units, scratch bytes, row indices) in
+  // range: sequences are indexed with 32-bit ints in the kernels, and (b, head)
+  // rows of the split scratch number at most 2^31.
+  if (s.B > 0x7fffffffll || s.Hq > 65536 || s.B * s.Hq > ((int64_t)1 << 31))
+    return fail(PAD_ERR_UNSUPPORTED, "batch %lld x query heads %lld too large (at most 2^31 rows, 65536 heads)",
+                (long long)s.B, (long long)s.Hq);
+  if (s.W > ((int64_t)1 << 30) || s.W * s.bs > ((int64_t)1 << 30))
+    return fail(PAD_ERR_UNSUPPORTED, "table capacity %lld blocks x %lld tokens too large (at most 2^30 tokens)",
+                (long long)s.W, (long long)s.bs);
   return PAD_OK;
 }
 

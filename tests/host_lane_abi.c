@@ -105,6 +105,19 @@ static void check_plans(void) {
   CHECK(pad_decode_plan(-1, 32, 8, 128, 16, 256, 0, 0, &a) != PAD_OK, "negative batch accepted");
   CHECK(pad_decode_plan(32, 32, 8, 128, -16, 256, 0, 0, &a) != PAD_OK, "negative block size accepted");
   CHECK(pad_decode_plan(32, 32, 8, 128, 16, -1, 0, 0, &a) != PAD_OK, "negative table width accepted");
+  /* sizes whose products would overflow 64 bits: rejected, not wrapped */
+  const int64_t huge[][6] = {{(int64_t)1 << 62, 8, 8, 128, 16, 4},   {3, (int64_t)1 << 40, 1 << 20, 128, 16, 4},
+                             {3, 32, 8, 128, 256, (int64_t)1 << 62}, {(int64_t)1 << 31, 2, 1, 64, 16, 4},
+                             {1 << 20, 4096, 16, 128, 16, 4},         {3, 65537 * 2, 2, 128, 16, 4}};
+  for (size_t i = 0; i < sizeof(huge) / sizeof(huge[0]); ++i) {
+    pad_plan p;
+    const int64_t *h = huge[i];
+    CHECK(pad_decode_plan(h[0], h[1], h[2], h[3], h[4], h[5], 0, 0, &p) == PAD_ERR_UNSUPPORTED && has_message(),
+          "oversized shape %zu not rejected", i);
+  }
+  /* the largest accepted sizes plan without overflow */
+  CHECK(pad_decode_plan(1 << 20, 64, 1, 256, 256, 4096, 0, 0, &a) == PAD_OK && a.ctas > 0 && a.workspace_bytes > 0,
+        "largest accepted shape did not plan");
 }
 
 static void *plan_thread(void *arg) {
