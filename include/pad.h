@@ -128,7 +128,9 @@ typedef struct pad_plan {
  *  stream        cudaStream_t.
  *
  * Supported envelope: D in {64, 128, 256}; Hq / Hkv <= 256; block_size a power of
- * two in [1, 256].  Scratch (partials, and a control block of merge counters
+ * two in [1, 256]; B < 2^31, Hq <= 65536 and B * Hq <= 2^31; a table capacity C of
+ * at most 2^30 tokens; at most 2^31 - 1 work units (B * Hkv * head tiles * S) per
+ * launch.  Outside it: PAD_ERR_UNSUPPORTED, nothing launched.  Scratch (partials, and a control block of merge counters
  * that every launch leaves zero) is owned by the library, kept per (device,
  * stream) and grown on demand; growing it while `stream` is being captured into
  * a CUDA graph returns PAD_ERR_WORKSPACE (call once outside capture first).
