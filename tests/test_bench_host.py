@@ -89,3 +89,18 @@ def test_each_kernel_has_its_own_source_hash_and_profile(tmp_path, monkeypatch):
     assert bench.traffic_from_profiles("demo", "u1", "umma_kernel") == 77
     assert bench.traffic_from_profiles("demo", "p1") == 55
     assert bench.traffic_from_profiles("demo", "p1", "umma_kernel") is None
+
+
+def test_tcgen05_entry_rejects_what_that_kernel_does_not_take(monkeypatch):
+    bench = _bench()
+    for extra in (["--kv-dtype", "e4m3"], ["--window", "100"], ["--sinks"]):
+        monkeypatch.setattr("sys.argv", ["bench.py", "--entry", "tcgen05", *extra])
+        try:
+            bench.parse()
+        except SystemExit as e:
+            assert e.code == 2
+        else:
+            raise AssertionError(f"--entry tcgen05 {extra} accepted")
+    monkeypatch.setattr("sys.argv", ["bench.py", "--entry", "tcgen05", "--workload", "ragged_mqa"])
+    args = bench.parse()
+    assert args.entry == "tcgen05" and args.kv_dtype == "bf16"
