@@ -104,3 +104,24 @@ def test_tcgen05_entry_rejects_what_that_kernel_does_not_take(monkeypatch):
     monkeypatch.setattr("sys.argv", ["bench.py", "--entry", "tcgen05", "--workload", "ragged_mqa"])
     args = bench.parse()
     assert args.entry == "tcgen05" and args.kv_dtype == "bf16"
+
+
+def test_reference_arm_prints_one_contract_line():
+    # the oracle arm runs on the host cores, so it is checked here end to end
+    import json
+    import subprocess
+    import sys
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "1", "--cpu-seconds", "1"], capture_output=True, text=True, cwd=ROOT,
+                         timeout=600)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1, res.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"].startswith("decode attention")
+    assert d["unit"] == "GB/s" and d["higher_is_better"] is True and d["value"] > 0
+    assert (d["steps"], d["warmup"], d["n_gpus"]) == (1, 1, 1)
+    assert d["config"]["workload"] == "llama8b"
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
