@@ -134,6 +134,10 @@ typedef struct pad_plan {
  * that every launch leaves zero) is owned by the library, kept per (device,
  * stream) and grown on demand; growing it while `stream` is being captured into
  * a CUDA graph returns PAD_ERR_WORKSPACE (call once outside capture first).
+ * Threads: any number of host threads may call at once on different streams
+ * (each (device, stream) has its own scratch); calls on the same stream must be
+ * serialised by the caller, as their launches would be unordered anyway (a call
+ * may regrow that stream's scratch).
  */
 pad_status pad_decode(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
                       const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,

@@ -10,6 +10,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <map>
 #include <set>
 #include <mutex>
@@ -81,17 +82,19 @@ pad_status check_shape(const Shape &s, int32_t num_splits) {
 }
 
 int sm_count(int device) {
-  static int cache[64] = {0};
+  // per-device cache; threads that plan at once may both query and store the
+  // same value, so the slots are atomic
+  static std::atomic<int> cache[64];
   if (device < 0 || device >= 64) return 148;
-  if (cache[device] == 0) {
-    int n = 0;
+  int n = cache[device].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n <= 0) {
       cudaGetLastError();
       n = 148;
     }
-    cache[device] = n;
+    cache[device].store(n, std::memory_order_relaxed);
   }
-  return cache[device];
+  return n;
 }
 
 // Per-shape launch plan.  The lengths live on the device, so the plan sees only
