@@ -98,6 +98,8 @@ static void check_plans(void) {
   CHECK(ok > 100 && rejected > 100, "plan grid: %ld accepted, %ld rejected", ok, rejected);
   /* the bf16 entry equals the _ex entry with a bf16 cache */
   pad_plan a, b;
+  memset(&a, 0, sizeof(a)); /* the struct has padding: compare what the calls write */
+  memset(&b, 0, sizeof(b));
   CHECK(pad_decode_plan(32, 32, 8, 128, 16, 256, 0, 0, &a) == PAD_OK, "llama8b-shaped plan rejected");
   CHECK(pad_decode_plan_ex(32, 32, 8, 128, 16, 256, 0, PAD_BF16, 0, &b) == PAD_OK, "llama8b-shaped plan_ex rejected");
   CHECK(memcmp(&a, &b, sizeof(a)) == 0, "pad_decode_plan differs from pad_decode_plan_ex(bf16)");
@@ -125,8 +127,10 @@ static void *plan_thread(void *arg) {
   for (int i = 0; i < 2000; ++i) {
     pad_plan p;
     const int64_t mbps = 1 + ((i * 37 + t * 11) % 3000);
+    /* devices 1..8: the threads are the first to fill those slots of the
+       library's per-device caches, at the same time */
     pad_status st = pad_decode_plan_ex(1 + (i % 64), 32, 1 + (i % 4 == 0 ? 0 : 7), 128, 16, mbps, i % 5,
-                                       (i & 1) ? PAD_FP8_E4M3 : PAD_BF16, 0, &p);
+                                       (i & 1) ? PAD_FP8_E4M3 : PAD_BF16, 1 + (i % 8), &p);
     if (st != PAD_OK && !has_message()) return (void *)1;
     if (i % 97 == 0) (void)pad_status_string(st);
   }

@@ -11,7 +11,9 @@ blocks", vllm.cpp PR #2472, CI classification comment):
   instrumented): plans over a grid of shapes, every decode entry point with one
   argument broken at a time, an empty batch.
 
-The two never share a binary: the checker and the library stay apart.  The GPU
+A third build of the library lane under -fsanitize=thread checks the host code
+for data races while several threads plan at once (with a planted race as its
+control).  The two never share a binary: the checker and the library stay apart.  The GPU
 side has no sanitizer here; its bounds are covered by the kernels' own checks
 (error word) and the parity tests.
 """
@@ -57,33 +59,76 @@ def test_oracle_and_generator_under_sanitizers(tmp_path):
 
 
 def test_c_abi_host_code_under_sanitizers(tmp_path):
+    objs = _abi_objects(tmp_path, SAN)
+    res = subprocess.run([_link(objs, SAN, str(tmp_path / "lane_abi"))], capture_output=True, text=True, env=ENV,
+                         timeout=300)
+    _assert_clean(res)
+
+
+def _abi_objects(tmp_path, san, api_src=None):
+    """Object files of the library (host side instrumented with `san`) and the
+    ABI lane, compiled in parallel; `api_src` replaces pad_api.cpp."""
     cuda = _cuda_home()
     inc = ["-I", _build.INCLUDE, "-I", _build.CSRC]
-    jobs = []
-    objs = []
+    jobs, objs = [], []
     for src in _build.SOURCES:
         obj = str(tmp_path / (os.path.splitext(src)[0] + ".o"))
         objs.append(obj)
         path = os.path.join(_build.CSRC, src)
         if src.endswith(".cpp"):
-            jobs.append(["g++", "-std=c++17", "-O1", "-g", *SAN, *inc, "-I", os.path.join(cuda, "include"),
-                         "-c", path, "-o", obj])
+            jobs.append(["g++", "-std=c++17", "-O1", "-g", *san, *inc, "-I", os.path.join(cuda, "include"),
+                         "-c", api_src or path, "-o", obj])
         else:
-            xc = [a for flag in SAN for a in ("-Xcompiler", flag)]
+            xc = [a for flag in san for a in ("-Xcompiler", flag)]
             jobs.append([_build.nvcc(), "-std=c++17", "-O1", "-g", *_build.ARCH_FLAGS, *xc, *inc, "-c", path,
                          "-o", obj])
     lane_obj = str(tmp_path / "lane_abi.o")
     objs.append(lane_obj)
-    jobs.append(["gcc", "-std=c11", "-O1", "-g", *SAN, "-Wall", "-Wextra", "-Werror", "-I", _build.INCLUDE,
+    jobs.append(["gcc", "-std=c11", "-O1", "-g", *san, "-Wall", "-Wextra", "-Werror", "-I", _build.INCLUDE,
                  "-c", os.path.join(ROOT, "tests", "host_lane_abi.c"), "-o", lane_obj])
     with ThreadPoolExecutor(max_workers=len(jobs)) as ex:
         for f in [ex.submit(_run, j) for j in jobs]:
             f.result()
-    exe = str(tmp_path / "lane_abi")
-    _run(["g++", *SAN, *objs, "-L", os.path.join(cuda, "lib64"), "-lcudart_static", "-ldl", "-lrt", "-lpthread",
+    return objs
+
+
+def _link(objs, san, exe):
+    cuda = _cuda_home()
+    _run(["g++", *san, *objs, "-L", os.path.join(cuda, "lib64"), "-lcudart_static", "-ldl", "-lrt", "-lpthread",
           "-o", exe])
-    res = subprocess.run([exe], capture_output=True, text=True, env=ENV, timeout=300)
-    _assert_clean(res)
+    return exe
+
+
+TSAN = ["-fsanitize=thread", "-fno-omit-frame-pointer"]
+TSAN_ENV = dict(os.environ, TSAN_OPTIONS="halt_on_error=1")
+
+
+def test_c_abi_host_code_under_thread_sanitizer(tmp_path):
+    """The ABI lane's four threads plan at once, each the first to fill some
+    slots of the library's per-device caches: no data race may be reported.
+    Negative control: the same lane over a copy of pad_api.cpp whose SM-count
+    cache is a plain int array must be reported."""
+    objs = _abi_objects(tmp_path, TSAN)
+    res = subprocess.run([_link(objs, TSAN, str(tmp_path / "lane_tsan"))], capture_output=True, text=True,
+                         env=TSAN_ENV, timeout=300)
+    out = res.stdout + res.stderr
+    assert res.returncode == 0 and "ThreadSanitizer" not in out and "clean" in res.stdout, out[-3000:]
+
+    src = open(os.path.join(_build.CSRC, "pad_api.cpp")).read()
+    for a, b in (("static std::atomic<int> cache[64];", "static int cache[64];"),
+                 ("cache[device].load(std::memory_order_relaxed)", "cache[device]"),
+                 ("cache[device].store(n, std::memory_order_relaxed);", "cache[device] = n;")):
+        assert src.count(a) == 1, a
+        src = src.replace(a, b)
+    racy = tmp_path / "racy" / "pad_api.cpp"
+    racy.parent.mkdir()
+    racy.write_text(src)
+    obj = str(tmp_path / "pad_api.o")
+    _run(["g++", "-std=c++17", "-O1", "-g", *TSAN, "-I", _build.INCLUDE, "-I", _build.CSRC, "-I",
+          os.path.join(_cuda_home(), "include"), "-c", str(racy), "-o", obj])
+    res = subprocess.run([_link(objs, TSAN, str(tmp_path / "lane_tsan_racy"))], capture_output=True, text=True,
+                         env=TSAN_ENV, timeout=300)
+    assert res.returncode != 0 and "data race" in res.stderr and "sm_count" in res.stderr, res.stderr[-3000:]
 
 
 def test_lane_catches_a_planted_overrun(tmp_path):
