@@ -11,6 +11,9 @@ blocks", vllm.cpp PR #2472, CI classification comment):
   instrumented): plans over a grid of shapes, every decode entry point with one
   argument broken at a time, an empty batch.
 
+A fourth executable links the library's host file with a fake of every CUDA
+call it makes (host_lane_fake_cuda.cpp): what it hands the kernels and how
+injected failures come back, with planted mistakes as its controls.
 A third build of the library lane under -fsanitize=thread checks the host code
 for data races while several threads plan at once (with a planted race as its
 control).  The two never share a binary: the checker and the library stay apart.  The GPU
@@ -129,6 +132,57 @@ def test_c_abi_host_code_under_thread_sanitizer(tmp_path):
     res = subprocess.run([_link(objs, TSAN, str(tmp_path / "lane_tsan_racy"))], capture_output=True, text=True,
                          env=TSAN_ENV, timeout=300)
     assert res.returncode != 0 and "data race" in res.stderr and "sm_count" in res.stderr, res.stderr[-3000:]
+
+
+def _fake_lane(tmp_path, api_src, name):
+    """The library's host file (or a copy of it) over the fake CUDA runtime of
+    host_lane_fake_cuda.cpp, under ASan/UBSan; no CUDA library is linked."""
+    exe = str(tmp_path / name)
+    _run(["g++", "-std=c++17", "-O1", "-g", *SAN, "-I", _build.INCLUDE, "-I", _build.CSRC, "-I",
+          os.path.join(_cuda_home(), "include"), os.path.join(ROOT, "tests", "host_lane_fake_cuda.cpp"), api_src,
+          "-lpthread", "-o", exe])
+    return exe
+
+
+def test_c_abi_over_a_fake_runtime(tmp_path):
+    """What pad_api.cpp hands the kernels (pointers, strides, plan, scratch, TMA
+    maps) and how injected failures come back, with fakes of every CUDA call it
+    makes; the missing-encoder case runs in a process of its own."""
+    exe = _fake_lane(tmp_path, os.path.join(_build.CSRC, "pad_api.cpp"), "lane_fake")
+    for args in ([], ["no-encoder"]):
+        _assert_clean(subprocess.run([exe, *args], capture_output=True, text=True, env=ENV, timeout=300))
+
+
+# Plausible mistakes in the host file, each of which the fake-runtime lane must catch.
+PLANTED = {
+    "partials swapped": ("pr.p.o_part = base != nullptr ? reinterpret_cast<float *>(base + pr.ws.o_part)",
+                         "pr.p.o_part = base != nullptr ? reinterpret_cast<float *>(base + pr.ws.lse_part)"),
+    "freed before the stream drained": ("    e = cudaStreamSynchronize(stream);\n"
+                                        "    if (e != cudaSuccess) return cuda_fail(e, \"cudaStreamSynchronize\");\n"
+                                        "    cudaFree(w.ptr);", "    cudaFree(w.ptr);"),
+    "map strides swapped": ("{stride_bytes(2, rowb), (cuuint64_t)rw, stride_bytes(1, bs * rowb),",
+                            "{stride_bytes(1, bs * rowb), (cuuint64_t)rw, stride_bytes(2, rowb),"),
+    "scratch not cleared": ("  e = cudaMemsetAsync(w.ptr, 0, want, stream);\n"
+                            "  if (e != cudaSuccess) return cuda_fail(e, \"cudaMemsetAsync(library scratch)\");\n",
+                            ""),
+}
+
+
+def test_fake_runtime_lane_catches_planted_mistakes(tmp_path):
+    src = open(os.path.join(_build.CSRC, "pad_api.cpp")).read()
+    exes = {}
+    for i, (name, (a, b)) in enumerate(PLANTED.items()):
+        assert src.count(a) == 1, name
+        d = tmp_path / f"m{i}"
+        d.mkdir()
+        (d / "pad_api.cpp").write_text(src.replace(a, b))
+        exes[name] = str(d / "pad_api.cpp")
+    with ThreadPoolExecutor(max_workers=len(exes)) as ex:
+        built = {n: ex.submit(_fake_lane, tmp_path, p, f"lane_{i}") for i, (n, p) in enumerate(exes.items())}
+        built = {n: f.result() for n, f in built.items()}
+    for name, exe in built.items():
+        res = subprocess.run([exe], capture_output=True, text=True, env=ENV, timeout=300)
+        assert res.returncode != 0 and "FAIL" in res.stderr, f"{name}: not caught\n{res.stdout}{res.stderr[-1500:]}"
 
 
 def test_lane_catches_a_planted_overrun(tmp_path):
