@@ -62,7 +62,8 @@ typedef enum pad_status {
   PAD_ERR_UNSUPPORTED = 2,  /* valid problem outside the compiled envelope */
   PAD_ERR_WORKSPACE = 3,    /* split scratch could not be obtained (e.g. growth under capture) */
   PAD_ERR_CUDA = 4,         /* a CUDA runtime call failed; see pad_last_error() */
-  PAD_ERR_DEVICE_CHECK = 5  /* a kernel saw an invalid block id or sequence length */
+  PAD_ERR_DEVICE_CHECK = 5  /* a kernel saw an invalid block id or sequence length, or a
+                               bounded wait gave up (pad_check_device_errors) */
 } pad_status;
 
 /* PAD_FP8_E4M3: OCP 8-bit floating point, E4M3 variant (sign, 4 exponent bits
@@ -98,7 +99,11 @@ typedef struct pad_plan {
 } pad_plan;
 
 /*
- * pad_decode -- paged single-token decode attention.
+ * pad_decode -- paged single-token decode attention: the operation of
+ * "spec(BACKEND-ROCM): the ROCm head_dim=128 decode arm, the ROCm half of #382"
+ * (section "The gap it specs") computed as the one-token split-KV attention of
+ * "perf(rocke): prepare saved paged decode bindings once" (section "Summary"),
+ * with the optional log-sum-exp output.
  *
  *  q             bf16 [B, Hq, D], stride[2] == 1, every row 16-byte aligned.
  *  k_cache       bf16 or FP8 E4M3 [num_blocks, Hkv, block_size, D], stride[3] ==
@@ -173,7 +178,11 @@ typedef struct pad_decode_options {
 } pad_decode_options;
 
 /*
- * pad_decode_ex -- pad_decode with options (NULL options = pad_decode).  Same
+ * pad_decode_ex -- pad_decode with options (NULL options = pad_decode): the
+ * attention types "Attention parity: run every attention type on the best
+ * available path on both targets" (section "Current state") lists next to
+ * dense GQA, and the FP8 cache of "perf(rocke): prepare saved paged decode
+ * bindings once" (section "Summary").  Same
  * arguments, scratch, results and errors; `options->window_left` < 0, a sinks
  * tensor that is not fp32 [Hq] device memory, or a scale that is negative,
  * non-finite, or other than 0/1 for a bf16 cache, is PAD_ERR_INVALID_ARG.
@@ -209,7 +218,9 @@ pad_status pad_decode_with_workspace(const pad_tensor *q, const pad_tensor *k_ca
 
 /*
  * pad_decode_with_workspace_ex -- pad_decode_with_workspace with the options of
- * pad_decode_ex (window, sinks, E4M3 scales; NULL = none).  Same arguments,
+ * pad_decode_ex (window, sinks, E4M3 scales; NULL = none): caller-owned scratch
+ * ("perf(rocke): prepare saved paged decode bindings once", section "Technical
+ * Changes") for every attention type of pad_decode_ex.  Same arguments,
  * scratch rules, results and errors as those two.
  */
 pad_status pad_decode_with_workspace_ex(const pad_tensor *q, const pad_tensor *k_cache,
@@ -232,15 +243,20 @@ pad_status pad_decode_with_workspace_ex(const pad_tensor *q, const pad_tensor *k
  * compiled into the library, which every GPU that loads the library holds until
  * the process exits.
  *
- * Arguments, results and validation are those of pad_decode.  It calls no
- * allocating routine.  Shapes whose split scratch (pad_decode_plan(...)
- * .workspace_bytes) exceeds 32 MiB are rejected with PAD_ERR_WORKSPACE before
- * anything is launched.
+ * Arguments, results and validation are those of pad_decode, checked in the
+ * same order with the same statuses.  It calls no allocating routine.  A valid
+ * shape whose split scratch (pad_decode_plan(...).control_bytes +
+ * .workspace_bytes) exceeds 32 MiB is then rejected with PAD_ERR_WORKSPACE
+ * before anything is launched.
  *
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call before
- * any stream capture.  All calls on a device share the one array and it keeps
- * the last call's contents; each call clears, on `stream` after validating its
+ * Every call with a non-empty batch that passes validation looks up the
+ * array's device address (cudaGetSymbolAddress, with the call's device current;
+ * kept per device after the first), whether or not that call splits.  Under
+ * CUDA's lazy module loading (the default since CUDA 12.2) that first lookup
+ * loads the library module holding the array, which is when the 32 MiB are
+ * reserved on the device: make the first call on each device before any stream
+ * capture.  All calls on a device share the one array and it keeps the last
+ * call's contents; each call clears, on `stream` after validating its
  * arguments and before its launch (cudaMemsetAsync, which allocates nothing),
  * the counter words that must start at zero.  Calls that may
  * overlap on the GPU -- on different streams without ordering between them, or
@@ -257,8 +273,10 @@ pad_status pad_decode_static_scratch(const pad_tensor *q, const pad_tensor *k_ca
  * kernel: S^T = K.Q^T and O^T += V^T.P^T as tcgen05.mma with the accumulators in
  * tensor memory, K/V/q streamed by TMA in 8-token boxes, the softmax in four warps
  * that own one token (one TMEM lane) each, one CTA per (sequence, KV head,
- * partition) unit, two per SM.  Same arguments, results, scratch and
- * errors as pad_decode.  It takes a bf16 cache with groups of 17..32 query
+ * partition) unit, two per SM -- the GQA-group fusion over one K/V read of
+ * "spec(BACKEND-ROCM): the ROCm head_dim=128 decode arm, the ROCm half of #382"
+ * (section "The gap it specs") on tensor memory.  Same arguments, results,
+ * scratch and errors as pad_decode.  It takes a bf16 cache with groups of 17..32 query
  * heads per KV head at head_dim 128 and block_size >= 8, and returns
  * PAD_ERR_UNSUPPORTED otherwise.
  * pad_decode does not call it: on the workloads measured on B200 the mma.sync
@@ -272,7 +290,9 @@ pad_status pad_decode_tcgen05(const pad_tensor *q, const pad_tensor *k_cache, co
 
 /*
  * pad_decode_plan -- the launch geometry pad_decode would use for this shape
- * (the per-shape heuristic when num_splits == 0).  Pure host computation; no
+ * (the per-shape heuristic when num_splits == 0): the geometry a saved binding
+ * of "perf(rocke): prepare saved paged decode bindings once" prepares once and
+ * reuses for compatible calls (section "Summary").  Pure host computation; no
  * launch.  `device` < 0 means the current device (its SM count feeds the
  * heuristic: a small batch gets shorter partitions, down to 64 tokens, so that
  * it still fills the GPU).  Returns PAD_ERR_INVALID_ARG / PAD_ERR_UNSUPPORTED exactly when
@@ -285,7 +305,9 @@ pad_status pad_decode_plan(int64_t batch, int64_t num_q_heads, int64_t num_kv_he
 /*
  * pad_decode_plan_ex -- pad_decode_plan for a cache of dtype `kv_dtype`
  * (PAD_BF16, as pad_decode_plan, or PAD_FP8_E4M3: the same partitions and
- * scratch, deeper pipeline stages of half the bytes).  Any other kv_dtype is
+ * scratch, deeper pipeline stages of half the bytes) -- the non-FP8 and FP8
+ * decode paths of "perf(rocke): prepare saved paged decode bindings once"
+ * (section "Summary").  Any other kv_dtype is
  * PAD_ERR_INVALID_ARG.
  */
 pad_status pad_decode_plan_ex(int64_t batch, int64_t num_q_heads, int64_t num_kv_heads,
@@ -321,28 +343,67 @@ typedef struct pad_launch_witness {
 
 pad_status pad_last_launch(pad_launch_witness *witness);
 
-/* Static string for a status code. */
+/*
+ * pad_status_string -- static name of a status code.  Every failure is reported
+ * as a status with a message, never dropped: "perf(rocke): prepare saved paged
+ * decode bindings once", review item N1 (an argument the call cannot honour
+ * raises instead of being silently ignored).
+ */
 const char *pad_status_string(pad_status status);
 
-/* Message for the last failure on the calling thread ("" if none). */
+/*
+ * pad_last_error -- message for the last failure on the calling thread ("" if
+ * none); the message half of the same rule ("perf(rocke): prepare saved paged
+ * decode bindings once", review item N1).
+ */
 const char *pad_last_error(void);
 
 /*
  * pad_check_device_errors -- synchronises `stream`, then reads and clears the
- * current device's sticky error word.  Returns PAD_ERR_DEVICE_CHECK if any kernel
- * since the last check saw an invalid block id (bit 0x1) or sequence length
- * (bit 0x2); the bits are stored in *bits when bits != NULL.
+ * current device's sticky error word: the guards that "feat(rocm): wvSplitK
+ * skinny GEMM for decode M<=4" (opening review, findings 1 and 3) asks of
+ * every device access, reported instead of silently producing wrong numbers.
+ * Returns PAD_ERR_DEVICE_CHECK if any kernel since the last check set a bit;
+ * the bits are stored in *bits when bits != NULL:
+ *   0x1  a live table entry outside [0, num_blocks) (the page read as zeros),
+ *   0x2  a sequence length < 0 or > the table capacity (clamped),
+ *   0x4  a bounded wait gave up: a stage's copies did not land within its
+ *        limit (1 s; internal error) or pad_inject_stage_timeout stalled the
+ *        launch.  The CTA that gave up waited (bounded) for its own copies and
+ *        returned without writing its outputs; the merge counters it left set
+ *        in the library-owned control blocks of this device are re-zeroed by
+ *        this call, so the next call is correct.  That launch's out and lse
+ *        are not valid.
  */
 pad_status pad_check_device_errors(void *stream, uint32_t *bits);
 
 /*
+ * pad_inject_stage_timeout -- failure-path test hook ("perf(rocke): prepare
+ * saved paged decode bindings once", section "Risk Assessment": focused tests
+ * of failure recovery).  The next launch of the partition kernel made from the
+ * calling thread (pad_decode, pad_decode_ex, the workspace and static-scratch
+ * entry points; not pad_decode_tcgen05) runs with the CTAs of partition
+ * `partition` waiting, after they issue their first copies, on a barrier that
+ * nothing arrives on.  The wait gives up after a short limit (about 20 us),
+ * sets bit 0x4 of the device error word, drains the CTA's own copies (bounded)
+ * and returns, exactly as on a stage that never lands; the other partitions
+ * count themselves and leave their merge counters set.  No GPU fault, trap or
+ * hang is involved.  One-shot: the launch consumes it.  -1 disarms it; other
+ * values outside [0, 256) are PAD_ERR_INVALID_ARG.
+ */
+pad_status pad_inject_stage_timeout(int32_t partition);
+
+/*
  * pad_release_workspace -- frees the split scratch held for `device` (< 0: all
- * devices) after synchronising that device.  Safe to call at any time outside
- * stream capture; later calls re-grow scratch on demand.
+ * devices) after synchronising that device: the scratch a binding owns and
+ * keeps until its queued work completes ("perf(rocke): prepare saved paged
+ * decode bindings once", section "Technical Changes").  Safe to call at any
+ * time outside stream capture; later calls re-grow scratch on demand.
  */
 pad_status pad_release_workspace(int32_t device);
 
-/* PAD_ABI_VERSION of the loaded library. */
+/* pad_abi_version -- PAD_ABI_VERSION of the loaded library.  The source pages
+ * have no counterpart. */
 int32_t pad_abi_version(void);
 
 #ifdef __cplusplus

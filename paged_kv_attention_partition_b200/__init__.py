@@ -7,7 +7,8 @@ fallback, and the import fails loudly if ``libpad.so`` has not been built
 (``python -m paged_kv_attention_partition_b200._build``).
 
 Functions carry the C names: ``pad_decode``, ``pad_decode_with_workspace``,
-``pad_decode_static_scratch``, ``pad_decode_plan``, ``pad_check_device_errors``,
+``pad_decode_static_scratch``, ``pad_decode_tcgen05``, ``pad_decode_plan``,
+``pad_check_device_errors``, ``pad_inject_stage_timeout``, ``pad_last_launch``,
 ``pad_release_workspace``, ``pad_status_string``, ``pad_last_error``,
 ``pad_abi_version``.
 """
@@ -108,6 +109,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pad_last_error.restype = ctypes.c_char_p
     lib.pad_check_device_errors.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]
     lib.pad_check_device_errors.restype = ctypes.c_int
+    lib.pad_inject_stage_timeout.argtypes = [ctypes.c_int32]
+    lib.pad_inject_stage_timeout.restype = ctypes.c_int
     lib.pad_release_workspace.argtypes = [ctypes.c_int32]
     lib.pad_release_workspace.restype = ctypes.c_int
     lib.pad_abi_version.argtypes = []
@@ -312,7 +315,10 @@ def pad_decode_plan(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: i
 def pad_check_device_errors(stream=None, device=None) -> int:
     """Synchronise, then read and clear the device's sticky error word.  Returns
     the bits: 0 = clean, 0x1 = an out-of-range block id, 0x2 = an out-of-range
-    sequence length.  Raises PadError only when the check itself fails."""
+    sequence length, 0x4 = a bounded wait gave up (a stage's copies did not land
+    in time, or ``pad_inject_stage_timeout`` stalled the launch; that launch's
+    outputs are not valid, and the library's merge counters on the device are
+    re-zeroed by this call).  Raises PadError only when the check itself fails."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     bits = ctypes.c_uint32(0)
     with torch.cuda.device(dev):
@@ -320,6 +326,13 @@ def pad_check_device_errors(stream=None, device=None) -> int:
     if st not in (PAD_OK, PAD_ERR_DEVICE_CHECK):
         _raise(st)
     return bits.value
+
+
+def pad_inject_stage_timeout(partition: int) -> None:
+    """Failure-path test hook (see include/pad.h): the next partition-kernel
+    launch from this thread makes the CTAs of ``partition`` give up on a bounded
+    wait, as on a stage that never lands (error bit 0x4).  -1 disarms it."""
+    _raise(load_library().pad_inject_stage_timeout(int(partition)))
 
 
 def pad_last_launch(device=None) -> dict:
@@ -341,4 +354,5 @@ def pad_release_workspace(device: int = -1) -> None:
 __all__ = ["pad_decode", "pad_decode_with_workspace", "pad_decode_static_scratch", "pad_decode_tcgen05", "pad_decode_plan",
            "pad_check_device_errors", "pad_release_workspace",
            "pad_status_string", "pad_last_error", "pad_abi_version", "describe", "load_library",
-           "PadError", "PadTensor", "PadPlan", "PadOptions", "PadLaunchWitness", "pad_last_launch"]
+           "PadError", "PadTensor", "PadPlan", "PadOptions", "PadLaunchWitness", "pad_last_launch",
+           "pad_inject_stage_timeout"]

@@ -22,6 +22,9 @@
 namespace {
 
 thread_local std::string g_last_error;
+// pad_inject_stage_timeout: partition whose CTAs the next partition-kernel
+// launch from this thread stalls (-1: none)
+thread_local int32_t g_stall_partition = -1;
 
 pad_status fail(pad_status st, const char *fmt, ...) {
   char buf[512];
@@ -503,6 +506,7 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
   p.lse_sb = lse != nullptr ? lse->stride[0] : 0;
   p.lse_sh = lse != nullptr ? lse->stride[1] : 0;
   p.err = err;
+  p.stall_partition = tcgen05 ? -1 : g_stall_partition;
   if ((e = pad::device_witness(device, &p.witness)) != cudaSuccess) return cuda_fail(e, "launch witness");
   pr->D = (int)D;
   pr->device = device;
@@ -532,6 +536,7 @@ pad_status run(const Prepared &pr, cudaStream_t stream) {
   cudaError_t e = pr.umma ? pad::launch_umma(pr.p, pr.plan.ctas, stream)
                           : pad::launch_partition(pr.p, pr.D, pr.plan.heads_per_tile, pr.kv_fp8, pr.plan.ctas,
                                                   stream);
+  if (!pr.umma) g_stall_partition = -1;  // the test hook is one-shot
   return e == cudaSuccess ? PAD_OK : cuda_fail(e, "partition kernel launch");
 }
 
@@ -542,22 +547,31 @@ namespace pad {
 // pad_last_error().
 void set_last_error(const char *msg) { g_last_error = msg; }
 
-pad_status decode_with_buffers(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
-                               const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
-                               int32_t num_splits, pad_tensor *out, pad_tensor *lse, void *partials,
-                               size_t partials_bytes, void *control, size_t control_bytes, bool clear_control,
-                               cudaStream_t stream) {
+pad_status decode_with_scratch_array(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
+                                     const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
+                                     int32_t num_splits, pad_tensor *out, pad_tensor *lse,
+                                     pad_status (*scratch_address)(void **), size_t scratch_bytes,
+                                     cudaStream_t stream) {
   Prepared pr;
   bool empty = false;
   pad_status st = prepare(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse, &pr, &empty);
   if (st != PAD_OK || empty) return st;
-  if ((st = check_caller_buffer(pr, partials, partials_bytes, pr.ws.total, "partials buffer")) != PAD_OK) return st;
-  if ((st = check_caller_buffer(pr, control, control_bytes, pr.cl.total, "control buffer")) != PAD_OK) return st;
-  if (clear_control && pr.cl.total > 0) {
-    cudaError_t e = cudaMemsetAsync(control, 0, pr.cl.total, stream);
+  // the control block sits at the array's start, the partials after it (the
+  // control block's size is a multiple of 256 bytes, so they stay aligned)
+  const size_t need = pr.cl.total + pr.ws.total;
+  if (need > scratch_bytes)
+    return fail(PAD_ERR_WORKSPACE,
+                "this shape needs %zu bytes of split scratch; the static array holds %zu (use fewer splits or "
+                "pad_decode)",
+                need, scratch_bytes);
+  void *base = nullptr;
+  if ((st = scratch_address(&base)) != PAD_OK) return st;
+  if (pr.cl.total > 0) {
+    // the array outlives every call and keeps whatever the last one left
+    cudaError_t e = cudaMemsetAsync(base, 0, pr.cl.total, stream);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(control block)");
   }
-  bind_buffers(pr, partials, control);
+  bind_buffers(pr, pr.ws.total > 0 ? static_cast<char *>(base) + pr.cl.total : nullptr, base);
   return run(pr, stream);
 }
 }  // namespace pad
@@ -730,6 +744,13 @@ pad_status pad_check_device_errors(void *stream_, uint32_t *bits) {
     return fail(PAD_ERR_DEVICE_CHECK, "kernel saw %s%s%s", (v & pad::kErrBlockId) ? "an out-of-range block id; " : "",
                 (v & pad::kErrSeqLen) ? "an out-of-range sequence length; " : "",
                 (v & pad::kErrTimeout) ? "a stage whose copies never completed (internal error)" : "");
+  return PAD_OK;
+}
+
+pad_status pad_inject_stage_timeout(int32_t partition) {
+  if (partition < -1 || partition >= pad::kMaxSplits)
+    return fail(PAD_ERR_INVALID_ARG, "partition must be -1 (none) or in [0, %d) (got %d)", pad::kMaxSplits, partition);
+  g_stall_partition = partition;
   return PAD_OK;
 }
 

@@ -154,6 +154,11 @@ struct PartitionParams {
   uint32_t *counters;  // [B * Hkv * HT] partitions finished per (b, kv head, head tile)
   uint32_t *err;
   LaunchWitness *witness;  // written by block 0 of every launch
+  // Failure-path test hook (pad_inject_stage_timeout): -1 normally; otherwise
+  // the partition kernel's CTAs of partition `stall_partition` wait, after
+  // issuing their first copies, on a barrier nothing arrives on, give up after
+  // a short bounded wait and take the timeout exit.
+  int32_t stall_partition;
 };
 
 // Partials layout inside a workspace buffer (offsets 256-byte aligned); empty
@@ -205,14 +210,17 @@ cudaError_t device_error_word(int device, uint32_t **ptr);
 cudaError_t device_witness(int device, LaunchWitness **ptr);
 void set_last_error(const char *msg);
 
-// pad_decode with explicit buffers: `partials` (>= the plan's workspace_bytes,
-// 256-byte aligned) and `control` (>= the plan's control_bytes; zero at launch,
-// or cleared on `stream` after validation when `clear_control`).  Used by the
-// allocation-free entry point; allocates nothing itself.
-pad_status decode_with_buffers(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
-                               const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
-                               int32_t num_splits, pad_tensor *out, pad_tensor *lse, void *partials,
-                               size_t partials_bytes, void *control, size_t control_bytes, bool clear_control,
-                               cudaStream_t stream);
+// pad_decode with its scratch in a fixed array of `scratch_bytes` bytes:
+// validates and plans exactly as pad_decode, then rejects a shape whose control
+// block and partials exceed the array (PAD_ERR_WORKSPACE), asks
+// `scratch_address` for the array's device address (on every call that gets
+// this far, so the first one does any set-up), clears the control block on
+// `stream` and launches.  Used by the allocation-free entry point; allocates
+// nothing itself.
+pad_status decode_with_scratch_array(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
+                                     const pad_tensor *block_tables, const pad_tensor *seq_lens, float scale,
+                                     int32_t num_splits, pad_tensor *out, pad_tensor *lse,
+                                     pad_status (*scratch_address)(void **), size_t scratch_bytes,
+                                     cudaStream_t stream);
 
 }  // namespace pad

@@ -38,7 +38,11 @@ constexpr size_t kStaticScratchBytes = PAD_STATIC_SCRATCH_BYTES;
 
 std::atomic<void *> g_scratch_addr[64];
 
-// Device address of the array on the current device (set-up on first use).
+// Device address of the array on the current device, looked up on the first
+// call on each device with that device current.  Without -rdc the array lives
+// in a module of its own; under CUDA's lazy module loading (the default since
+// CUDA 12.2) this lookup is what loads that module and reserves the 32 MiB on
+// the device, so it belongs in the first call, made before any stream capture.
 pad_status static_scratch_address(void **out) {
   int device = 0;
   cudaError_t e = cudaGetDevice(&device);
@@ -74,44 +78,14 @@ extern "C" pad_status pad_decode_static_scratch(const pad_tensor *q, const pad_t
                                                 const pad_tensor *v_cache, const pad_tensor *block_tables,
                                                 const pad_tensor *seq_lens, float scale, int32_t num_splits,
                                                 pad_tensor *out, pad_tensor *lse, void *stream) {
-  // The array holds the control block (merge counters) first and the split
-  // partials after it.  Reject shapes that do not fit before launching.
-  size_t control = 0, need = 0;
-  bool empty_batch = false;
-  if (q != nullptr && k_cache != nullptr && block_tables != nullptr && q->ndim == 3 && k_cache->ndim == 4 &&
-      block_tables->ndim == 2) {
-    empty_batch = q->shape[0] == 0;
-    const int32_t kv_dtype = k_cache->dtype == PAD_FP8_E4M3 ? PAD_FP8_E4M3 : PAD_BF16;
-    pad_plan plan;
-    if (pad_decode_plan_ex(q->shape[0], q->shape[1], k_cache->shape[1], q->shape[2], k_cache->shape[2],
-                           block_tables->shape[1], num_splits, kv_dtype, -1, &plan) == PAD_OK) {
-      control = (size_t)plan.control_bytes;
-      need = control + (size_t)plan.workspace_bytes;
-      if (need > pad::kStaticScratchBytes) {
-        char msg[256];
-        snprintf(msg, sizeof msg,
-                 "this shape needs %zu bytes of split scratch; the static array holds %zu "
-                 "(use fewer splits or pad_decode)",
-                 need, pad::kStaticScratchBytes);
-        pad::set_last_error(msg);
-        return PAD_ERR_WORKSPACE;
-      }
-    }
-  }
-  // Only a launch that merges partitions touches the array: an empty batch or
-  // one partition per sequence needs no address, and a malformed call is
-  // rejected by the validation below before any buffer is looked at.
-  void *scratch = nullptr;
-  if (need > 0 && !empty_batch) {
-    pad_status st = pad::static_scratch_address(&scratch);
-    if (st != PAD_OK) return st;
-  }
-  char *partials = scratch != nullptr ? static_cast<char *>(scratch) + control : nullptr;
-  const size_t partials_bytes = scratch != nullptr ? pad::kStaticScratchBytes - control : 0;
-  // The control block must start at zero.  A completed call leaves it zero, but
-  // the array outlives every call, so it is cleared on the stream after the
-  // arguments are validated and before the launch.
-  return pad::decode_with_buffers(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse,
-                                  partials, partials_bytes, scratch, scratch != nullptr ? control : 0,
-                                  /*clear_control=*/true, static_cast<cudaStream_t>(stream));
+  // Arguments are validated and the plan made exactly as for pad_decode (same
+  // statuses, same order); then a shape whose control block and partials do
+  // not fit the array is rejected, and every call that gets that far -- one
+  // partition per sequence included -- looks up the array's address, so the
+  // first such call on a device does the set-up.  The control block (merge
+  // counters) sits at the array's start and is cleared on the stream before
+  // the launch; the partials follow it.
+  return pad::decode_with_scratch_array(q, k_cache, v_cache, block_tables, seq_lens, scale, num_splits, out, lse,
+                                        pad::static_scratch_address, pad::kStaticScratchBytes,
+                                        static_cast<cudaStream_t>(stream));
 }

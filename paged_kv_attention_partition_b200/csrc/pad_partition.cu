@@ -75,19 +75,27 @@ namespace {
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kRescaleSlack = 8.f;                  // log2 units: weights stay below 256
 constexpr uint64_t kWaitLimitNs = 1000000000ull;      // no stage can legitimately take 1 s
+constexpr uint64_t kStallLimitNs = 20000ull;          // the test hook's wait on a barrier nothing arrives on
 
 // Waits for the phase of `bar` with this parity; false (and the timeout bit)
-// after kWaitLimitNs.
-__device__ bool wait_stage(uint32_t bar, uint32_t parity, uint32_t *err) {
+// after `limit_ns`.
+__device__ bool wait_stage(uint32_t bar, uint32_t parity, uint32_t *err, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t start = global_timer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - start > kWaitLimitNs) {
+    if (global_timer_ns() - start > limit_ns) {
       atomicOr(err, kErrTimeout);
       return false;
     }
   }
   return true;
+}
+
+// Failure-path test hook: thread 0 of a CTA of the chosen partition waits on
+// `never` (initialised, never arrived on) until the short limit runs out, as a
+// stage whose copies never land would; true when it gave up.
+__device__ __noinline__ bool stall_for_test(uint32_t never, uint32_t *err) {
+  return !wait_stage(never, 0, err, kStallLimitNs);
 }
 }  // namespace
 
@@ -139,6 +147,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + SP.region_bytes);  // one per stage slot
   int *flag = reinterpret_cast<int *>(smem + SP.region_bytes + 64);
+  uint64_t *never = reinterpret_cast<uint64_t *>(smem + SP.region_bytes + 96);  // test hook only
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int dh = warp % DS, hg = (warp / DS) % HG, tg = warp / (DS * HG);  // head_dim part, head group, token group
@@ -193,6 +202,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
   if (tid == 0) {
 #pragma unroll
     for (int i = 0; i < NST; ++i) mbar_init(smem_addr(full + i), 1);
+    if (p.stall_partition >= 0) mbar_init(smem_addr(never), 1);
     fence_mbar_init();
   }
 
@@ -261,6 +271,18 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
       if (k < nstages) issue(ids[k], k);
   }
   int (&idn)[IDW] = ids[NST - 1];  // block ids of the next stage to issue
+  if (p.stall_partition >= 0) {
+    // failure-path test hook (uniform over the launch): the chosen partition's
+    // CTAs give up as on a stage that never lands, with the first stages'
+    // copies in flight, and drain them (bounded) before returning
+    const bool gave_up = tid == 0 && s == p.stall_partition && stall_for_test(smem_addr(never), p.err);
+    if (__syncthreads_or(gave_up)) {
+      if (tid == 0)
+        for (int j = 0; j < nstages && j < NST - 1; ++j) wait_stage(smem_addr(full + j), 0, p.err);
+      __syncthreads();
+      return;
+    }
+  }
 
   // Address of 16-byte chunk (column block h, chunk c of it) of row r in a K
   // or V half-stage: rows grouped in boxes of 2^bsb_log2 rows, each box laid out

@@ -42,6 +42,37 @@ def test_every_declared_symbol_is_exported(lib):
         getattr(lib, n)
 
 
+# The source pages, by title; a declaration's comment names one of them with a
+# section (or a review finding), or says the pages have no counterpart.
+PAGE_TITLES = (
+    "spec(BACKEND-ROCM): the ROCm head_dim=128 decode arm",
+    "feat(rocm): wvSplitK skinny GEMM for decode M<=4",
+    "perf(BACKEND-ROCM): cooperate across Q8_K activation blocks",
+    "Attention parity: run every attention type on the best available path on both targets",
+    "perf(rocke): prepare saved paged decode bindings once",
+)
+
+
+def test_every_declaration_cites_a_passage_or_says_it_has_none():
+    src = open(os.path.join(ROOT, "include", "pad.h")).read()
+    for name in declared_functions():
+        decl = re.search(r"^[A-Za-z_][\w \*]*?\b" + name + r"\s*\(", src, flags=re.M)
+        assert decl, name
+        # the last block comment starting in column 0 before the declaration
+        blocks = [m for m in re.finditer(r"^/\*.*?\*/", src[:decl.start()], flags=re.M | re.S)]
+        assert blocks, f"{name}: no comment"
+        text = " ".join(re.sub(r"\n\s*\*(?!/)", " ", blocks[-1].group(0)).split())
+        cites = any(t in text for t in PAGE_TITLES) and ("section" in text or "review" in text)
+        assert cites or "no counterpart" in text, f"{name}: its comment names no page section: {text[:120]}"
+
+
+def test_stage_timeout_hook_checks_its_argument(lib):
+    assert lib.pad_inject_stage_timeout(-2) == pad.PAD_ERR_INVALID_ARG
+    assert lib.pad_inject_stage_timeout(256) == pad.PAD_ERR_INVALID_ARG
+    assert lib.pad_inject_stage_timeout(3) == pad.PAD_OK
+    assert lib.pad_inject_stage_timeout(-1) == pad.PAD_OK  # disarmed
+
+
 def test_library_is_built_for_sm100a():
     cmd = _build.compile_command("x.so")
     assert "arch=compute_100a,code=sm_100a" in " ".join(cmd)
