@@ -71,22 +71,22 @@ def test_e4m3_window_and_sinks(cuda_device, D, bs):
     assert pad.pad_check_device_errors() == 0
 
 
-@pytest.mark.parametrize("name", ["llama8b", "qwen14b", "longctx_d256", "ragged_mqa"])
+@pytest.mark.parametrize("name", synth.CONFIG_NAMES)
 def test_e4m3_named_workload_full_size(cuda_device, name):
+    """Each named workload on its E4M3 cache, as benchmarked with --kv-dtype
+    e4m3: every (b, head) row against the oracle over the whole batch, after a
+    sampled quick check."""
     w = synth.config(name, kv_dtype="e4m3")
     dw = DeviceWorkload(w, cuda_device)
     out, lse = dw.run()
-    pairs = sample_pairs(w, 48, seed=11)
-    ref_out, ref_lse = oracle_pairs(w, pairs)
-    idx_b = [b for b, _ in pairs]
-    idx_h = [h for _, h in pairs]
-    check_parity(to_f64(out[idx_b, idx_h]), lse[idx_b, idx_h].cpu().numpy(), ref_out, ref_lse, "e4m3 " + name)
-    # every output is a convex combination of dequantised value rows
-    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
-    live = np.unique(w.block_tables[w.block_tables < w.num_blocks - 1])
-    vals = torch.from_numpy(w.v_cache[live]).view(torch.float8_e4m3fn).float().abs()
-    vmax = w.v_scale * float(vals[~torch.isnan(vals)].max())  # slots past L_b hold the NaN code
-    assert float(out.float().abs().max()) <= vmax * (1 + 2 ** -7)
+    got_out, got_lse = to_f64(out), lse.cpu().numpy()
+    if name != "tiny":
+        pairs = sample_pairs(w, 48, seed=11)
+        ref_o, ref_l = oracle_pairs(w, pairs)
+        idx_b, idx_h = [b for b, _ in pairs], [h for _, h in pairs]
+        check_parity(got_out[idx_b, idx_h], got_lse[idx_b, idx_h], ref_o, ref_l, "e4m3 " + name + " (sampled)")
+    ref_out, ref_lse = oracle.decode_workload(w)
+    check_parity(got_out, got_lse, ref_out, ref_lse, "e4m3 " + name)
     assert pad.pad_check_device_errors() == 0
     del dw
     torch.cuda.empty_cache()

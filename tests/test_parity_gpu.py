@@ -215,29 +215,25 @@ def test_graph_capture_replays(cuda_device):
     assert e.value.status == pad.PAD_ERR_WORKSPACE
 
 
-# ---- the five named workloads at full size (sampled outputs) ----------------
+# ---- the five named workloads at full size, every output -------------------
 
 @pytest.mark.parametrize("name", synth.CONFIG_NAMES)
 def test_named_workload_full_size(cuda_device, name):
+    """The workload exactly as benchmarked (its own partition count, 0 =
+    heuristic), every (b, head) row of out and lse against the oracle over the
+    whole batch; sampled pairs (longest and shortest sequences, first and last
+    heads) run first as a quick check that fails with a small report."""
     w = synth.config(name)
     dw = DeviceWorkload(w, cuda_device)
-    out, lse = dw.run()  # the workload's own partition count (0 = heuristic), as benchmarked
-    if name == "tiny":
-        ref_out, ref_lse = oracle.decode_workload(w)
-        check_parity(to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, name)
-        return
-    pairs = sample_pairs(w, 48, seed=7)
-    ref_out, ref_lse = oracle_pairs(w, pairs)
-    idx_b = [b for b, _ in pairs]
-    idx_h = [h for _, h in pairs]
-    got_out = to_f64(out[idx_b, idx_h])
-    got_lse = lse[idx_b, idx_h].cpu().numpy()
+    out, lse = dw.run()
+    got_out, got_lse = to_f64(out), lse.cpu().numpy()
+    if name != "tiny":
+        pairs = sample_pairs(w, 48, seed=7)
+        ref_o, ref_l = oracle_pairs(w, pairs)
+        idx_b, idx_h = [b for b, _ in pairs], [h for _, h in pairs]
+        check_parity(got_out[idx_b, idx_h], got_lse[idx_b, idx_h], ref_o, ref_l, name + " (sampled)")
+    ref_out, ref_lse = oracle.decode_workload(w)
     check_parity(got_out, got_lse, ref_out, ref_lse, name)
-    # properties that hold at any size, over every output: finite, and each
-    # output is a convex combination of value rows, so bounded by max |V|
-    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
-    vmax = float(np.nanmax(np.abs(synth.bf16_to_f64(w.v_cache[np.unique(w.block_tables[w.block_tables < w.num_blocks - 1])]))))
-    assert float(out.float().abs().max()) <= vmax * (1 + 2 ** -7)
     assert pad.pad_check_device_errors() == 0
     del dw
     torch.cuda.empty_cache()
