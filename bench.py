@@ -2,17 +2,21 @@
 """Benchmark: paged single-token decode attention on B200.
 
 One step = one full pass of the hot path (one launch: partition kernel with the
-split reduce folded in) over one decode batch.  Default workload: the Llama-8B-shaped decode batch
-(B=32, Hq/Hkv=32/8, D=128, block_size 16, seq_lens ~ U{512..4096}, synthetic bf16
-~N(0,1), tables over a 4096-block pool).  --workload picks another named one.
+split reduce folded in) over one decode batch.  Default workload: the
+Qwen3-14B-shaped decode batch (B=64, Hq/Hkv=40/8, D=128, block_size 16, every
+seq_len 8192, synthetic bf16 ~N(0,1), tables over a 32768-block pool, 16 splits of
+512 tokens, LSE on).  --workload picks another named one.
 
 Prints one JSON line (rank 0).  `value` is achieved algorithmic HBM GB/s of the
-whole step (all ranks' bytes / max-over-ranks device time); `us_per_call` is the
-mean device time per step.  Timing: W warm-up steps, then K timed steps, each
-bracketed by CUDA events on the launching stream, with an L2 flush between steps
-outside the events (a 256 MiB write, then a 256 MiB read so that the written
-lines are evicted too: every timed launch starts from a cold L2 holding no dirty
-data); barrier + synchronize around the timed region.
+whole step: all ranks' bytes per step / the max over ranks of the MEDIAN device
+time of a step (seven-sample upper-middle statistics in the pages' CLI; the
+median here); the mean, min and max ride beside it.  Timing: W warm-up steps,
+then K timed steps, each bracketed by CUDA events on the launching stream, with
+an L2 flush between steps outside the events (a 256 MiB write, then a 256 MiB
+read so that the written lines are evicted too: every timed launch starts from a
+cold L2 holding no dirty data); barrier + synchronize around the timed region.
+At N=1 the other named workloads (and every workload on its E4M3 cache) are
+then timed the same way, each with its own events, into `workloads`.
 
 --impl reference times the CPU oracle (the reference arm of this path) on the
 host cores instead; it never touches the GPU.
@@ -42,7 +46,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    ap.add_argument("--workload", default="llama8b")
+    ap.add_argument("--workload", default="qwen14b")
     ap.add_argument("--num-splits", type=int, default=None, help="override the workload's partition count")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline time budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -55,6 +59,9 @@ def parse():
                     help="sliding window: each sequence attends to its last W tokens (pad_decode_ex)")
     ap.add_argument("--sinks", action="store_true", help="per-head attention sink logits (pad_decode_ex)")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay of the end-to-end step")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip timing the other named workloads (the `workloads` table)")
+    ap.add_argument("--side-steps", type=int, default=60, help="timed steps per workload of the `workloads` table")
     ap.add_argument("--kv-dtype", default="bf16", choices=["bf16", "e4m3"],
                     help="KV cache element type (e4m3: OCP FP8 E4M3 codes with per-tensor scales)")
     ap.add_argument("--entry", default="default", choices=["default", "tcgen05"],
@@ -63,7 +70,19 @@ def parse():
     args = ap.parse_args()
     if args.entry == "tcgen05" and (args.kv_dtype != "bf16" or args.window or args.sinks):
         ap.error("--entry tcgen05 takes a bf16 cache without --window or --sinks")
+    check_gpus(args.gpus, int(os.environ.get("WORLD_SIZE", "1")), ap.error)
     return args
+
+
+def check_gpus(n, world, error):
+    """--gpus N is one rank per GPU: N > 1 needs the N ranks a launcher
+    (torch.distributed.run) starts, so a single process never reports n_gpus 1
+    for a request of N."""
+    if n < 1:
+        error(f"--gpus must be >= 1 (got {n})")
+    if n != world:
+        error(f"--gpus {n} but WORLD_SIZE is {world}: launch one rank per GPU, e.g. "
+              f"python -m torch.distributed.run --nproc-per-node {n} bench.py --gpus {n}")
 
 
 def measured_peaks():
@@ -268,6 +287,52 @@ def max_time_sum_bytes(total_ms, my_bytes, device, world):
     return t_max, float(bt.item())
 
 
+# The `workloads` table: every named workload on both caches, and llama8b's
+# no-alias variant (its 4096-block pool is smaller than the pages it needs, so
+# some pages are shared; the compact pool gives every page one reader).
+SIDE_WORKLOADS = [("tiny", "bf16", False), ("llama8b", "bf16", False), ("llama8b", "bf16", True),
+                  ("qwen14b", "bf16", False), ("longctx_d256", "bf16", False), ("ragged_mqa", "bf16", False),
+                  ("llama8b", "e4m3", False), ("qwen14b", "e4m3", False), ("longctx_d256", "e4m3", False),
+                  ("ragged_mqa", "e4m3", False)]
+
+
+def time_workload(pad, torch, w, dev, stream, flush_l2, steps, warmup, kv_dtype):
+    """Device time of K launches of one workload as the main leg times it (caller
+    workspace, L2 flushed between steps outside the events): a dict of the
+    median / mean / min / max us per call and the median's GB/s."""
+    fp8 = kv_dtype == "e4m3"
+    kvt = torch.float8_e4m3fn if fp8 else torch.bfloat16
+    q = torch.from_numpy(w.q).view(torch.bfloat16).to(dev)
+    k = torch.from_numpy(w.k_cache).view(kvt).to(dev)
+    v = torch.from_numpy(w.v_cache).view(kvt).to(dev)
+    tables, lens = torch.from_numpy(w.block_tables).to(dev), torch.from_numpy(w.seq_lens).to(dev)
+    plan = pad.pad_decode_plan(w.B, w.Hq, w.Hkv, w.D, w.block_size, w.max_blocks_per_seq,
+                               num_splits=w.num_splits, device=dev.index, kv_dtype=kv_dtype)
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev) if w.want_lse else None
+    ws = torch.empty(plan["workspace_bytes"] // 4 + 64, dtype=torch.float32, device=dev)
+    sc = dict(k_scale=w.k_scale, v_scale=w.v_scale) if fp8 else {}
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for i in range(-warmup, steps):
+            flush_l2(i)
+            if i >= 0:
+                ev[i][0].record(stream)
+            pad.pad_decode_with_workspace(q, k, v, tables, lens, w.scale, w.num_splits, out, lse, ws, stream, **sc)
+            if i >= 0:
+                ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    if pad.pad_check_device_errors(stream):
+        raise SystemExit(f"device error word set on {w.name} ({kv_dtype})")
+    ms = [a.elapsed_time(b) for a, b in ev]
+    med = statistics.median(ms)
+    gbs = w.algorithmic_bytes() / (med / 1e3) / 1e9
+    return {"us_per_call": round(med * 1e3, 2), "us_mean": round(statistics.mean(ms) * 1e3, 2),
+            "us_min_max": [round(min(ms) * 1e3, 2), round(max(ms) * 1e3, 2)], "GB_s": round(gbs, 1),
+            "algorithmic_bytes": w.algorithmic_bytes(), "num_splits": plan["num_splits"],
+            "partition_tokens": plan["partition_tokens"], "ctas": plan["ctas"], "steps": steps}
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -375,8 +440,11 @@ def main():
     step_ms = [e[0].elapsed_time(e[1]) for e in events]
     part_ms = step_ms  # the step is exactly one launch of the partition kernel
     alg_bytes = w.algorithmic_bytes(window=args.window, sinks=args.sinks)
-    total_ms, all_bytes = max_time_sum_bytes(sum(step_ms), alg_bytes * args.steps, dev, world)
-    value = all_bytes / (total_ms / 1e3) / 1e9
+    # the median step (max over ranks) sets `value`; the mean is reported beside it
+    med_ms, all_bytes = max_time_sum_bytes(statistics.median(step_ms), alg_bytes, dev, world)
+    total_ms = max_over_ranks(sum(step_ms), dev, world)
+    value = all_bytes / (med_ms / 1e3) / 1e9
+    value_mean = all_bytes * args.steps / (total_ms / 1e3) / 1e9
 
     # ---- end to end through the public one-call API, host buffers -----------
     # Per step: pinned host -> device copy of the step's inputs (q, block table,
@@ -427,10 +495,10 @@ def main():
     torch.cuda.synchronize(dev)
     if e2e_steps and not torch.equal(view(hout, out_offs[0], out), out.cpu()):
         raise SystemExit("the end-to-end step's output differs from the kernel leg's")
-    e2e_ms = sum(e[0].elapsed_time(e[1]) for e in e2e_ev) if e2e_steps else float("nan")
+    e2e_ms = statistics.median([e[0].elapsed_time(e[1]) for e in e2e_ev]) if e2e_steps else float("nan")
     # every rank takes the same collective steps, e2e leg or not
-    e2e_total = max_over_ranks(e2e_ms / max(e2e_steps, 1) * args.steps if e2e_steps else 0.0, dev, world)
-    e2e_value = all_bytes / (e2e_total / 1e3) / 1e9 if e2e_steps else float("nan")
+    e2e_med = max_over_ranks(e2e_ms if e2e_steps else 0.0, dev, world)
+    e2e_value = all_bytes / (e2e_med / 1e3) / 1e9 if e2e_steps else float("nan")
 
     # ---- the same end-to-end step captured once as a CUDA graph and replayed
     # (copies in, the call, copies out): what is left of the host's cost.  The
@@ -452,10 +520,10 @@ def main():
                 if i >= 0:
                     g_ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
-        graph_ms = sum(e[0].elapsed_time(e[1]) for e in g_ev)
+        graph_ms = statistics.median([e[0].elapsed_time(e[1]) for e in g_ev])
         del g
-    graph_total = max_over_ranks(graph_ms / max(graph_steps, 1) * args.steps if graph_steps else 0.0, dev, world)
-    graph_value = all_bytes / (graph_total / 1e3) / 1e9 if graph_steps else float("nan")
+    graph_med = max_over_ranks(graph_ms if graph_steps else 0.0, dev, world)
+    graph_value = all_bytes / (graph_med / 1e3) / 1e9 if graph_steps else float("nan")
 
     errs = pad.pad_check_device_errors(stream)
     if errs:
@@ -466,7 +534,7 @@ def main():
         # the only kernel of the step writes out/lse itself: its algorithmic bytes
         # are the whole call's
         p_bytes = alg_bytes
-        p_ms = statistics.mean(part_ms)
+        p_ms = statistics.median(part_ms)
         achieved = p_bytes / (p_ms / 1e3) / 1e9
         sha = kernel_source_sha(kernel)
         # the recorded ncu traffic is for the named workload at full size, as
@@ -479,7 +547,9 @@ def main():
         line = {
             "metric": "decode attention µs/call and achieved HBM GB/s vs B200 peak (1 GPU)",
             "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(total_ms / args.steps, 5), "us_per_call": round(total_ms / args.steps * 1e3, 2),
+            "ms_per_step": round(med_ms, 5), "us_per_call": round(med_ms * 1e3, 2),
+            "timing": "value and us_per_call: median step (max over ranks); mean beside it",
+            "value_mean": round(value_mean, 2), "us_per_call_mean": round(total_ms / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16",
             "data": "synthetic (seeded counter-based generator; no dataset)",
             "config": {**workload_config(w, plan),
@@ -495,13 +565,27 @@ def main():
                          "split_scratch_bytes_per_launch": split_scratch_bytes(w, plan, args.window)},
             "e2e": None if not e2e_steps else {
                 "value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "us_per_call": round(e2e_total / args.steps * 1e3, 2), "api": api},
+                "us_per_call": round(e2e_med * 1e3, 2), "api": api},
             "e2e_graph": None if not graph_steps else {
                 "value": round(graph_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "us_per_call": round(graph_total / args.steps * 1e3, 2), "api": api + ", replayed as a CUDA graph"},
+                "us_per_call": round(graph_med * 1e3, 2), "api": api + ", replayed as a CUDA graph"},
             "gpu_launches": args.steps,  # one kernel launch per step
             "clocks": clocks.summary(),
         }
+        if world == 1 and not args.no_workloads:
+            # every named workload (both caches) as a parity-test case would
+            # run it, timed in this process after the main leg
+            table = {}
+            for name, kvd, compact in SIDE_WORKLOADS:
+                sw = synth.config(name, compact_pool=compact, kv_dtype=kvd)
+                r = time_workload(pad, torch, sw, dev, stream, flush_l2, args.side_steps, 5, kvd)
+                r["frac_of_peak"] = round(r["GB_s"] / peak, 4) if name != "tiny" else None
+                table[name + ("_compact" if compact else "") + ("_e4m3" if kvd == "e4m3" else "")] = r
+                del sw
+                torch.cuda.empty_cache()
+            line["workloads"] = {"note": f"median of {args.side_steps} launches each (5 warm-up), L2 flushed "
+                                         "between launches, caller workspace; frac_of_peak against the same peak "
+                                         "(tiny: launch latency only)", **table}
         if world == 1 and not args.no_cpu_baseline:
             cb = cpu_baseline(w, args.cpu_seconds, prefix=lambda k: synth.config(
                 args.workload, batch=k, compact_pool=args.compact_pool, kv_dtype=args.kv_dtype))

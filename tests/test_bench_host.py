@@ -106,6 +106,34 @@ def test_tcgen05_entry_rejects_what_that_kernel_does_not_take(monkeypatch):
     assert args.entry == "tcgen05" and args.kv_dtype == "bf16"
 
 
+def test_gpus_flag_needs_one_rank_per_gpu(monkeypatch):
+    # a single process asked for N > 1 GPUs refuses instead of reporting n_gpus 1
+    bench = _bench()
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    for argv in (["--gpus", "8"], ["--gpus", "2", "--impl", "reference"], ["--gpus", "0"]):
+        monkeypatch.setattr("sys.argv", ["bench.py", *argv])
+        try:
+            bench.parse()
+        except SystemExit as e:
+            assert e.code == 2
+        else:
+            raise AssertionError(f"{argv} accepted without its ranks")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setattr("sys.argv", ["bench.py", "--gpus", "2"])
+    assert bench.parse().gpus == 2
+    monkeypatch.setattr("sys.argv", ["bench.py", "--gpus", "4"])  # ranks and request disagree
+    try:
+        bench.parse()
+    except SystemExit as e:
+        assert e.code == 2
+    else:
+        raise AssertionError("--gpus 4 accepted with WORLD_SIZE 2")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setattr("sys.argv", ["bench.py"])
+    args = bench.parse()
+    assert args.gpus == 1 and args.workload == "qwen14b"
+
+
 def test_reference_arm_prints_one_contract_line():
     # the oracle arm runs on the host cores, so it is checked here end to end
     import json
@@ -121,7 +149,7 @@ def test_reference_arm_prints_one_contract_line():
     assert d["impl"] == "reference" and d["metric"].startswith("decode attention")
     assert d["unit"] == "GB/s" and d["higher_is_better"] is True and d["value"] > 0
     assert (d["steps"], d["warmup"], d["n_gpus"]) == (1, 1, 1)
-    assert d["config"]["workload"] == "llama8b"
+    assert d["config"]["workload"] == "qwen14b"
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
