@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define PAD_ABI_VERSION 1
+#define PAD_ABI_VERSION 2
 
 typedef enum pad_status {
   PAD_OK = 0,
@@ -87,7 +87,8 @@ typedef struct pad_plan {
   int32_t partition_tokens;  /* P, tokens per partition, a multiple of block_size */
   int32_t heads_per_tile;    /* query heads per work unit, padded (8, 16 or 32) */
   int32_t head_tiles;        /* work units per (sequence, KV head, partition): ceil(group / heads_per_tile) */
-  int32_t warps_per_cta;     /* warps per CTA: 4 (mma.sync kernel), 6 (tcgen05 kernel: 4 softmax,
+  int32_t warps_per_cta;     /* warps per CTA: 4 or 8 (mma.sync kernel, chosen per head_dim, heads
+                                per tile and cache type), 6 (tcgen05 kernel: 4 softmax,
                                 producer, MMA) */
   int32_t stage_tokens;      /* tokens per shared-memory pipeline stage */
   int32_t stages;            /* pipeline depth */
@@ -339,6 +340,7 @@ typedef struct pad_launch_witness {
   int32_t num_splits;        /* S it was launched with */
   int32_t partition_tokens;  /* P it was launched with */
   int32_t ctas;              /* grid size */
+  int32_t warps;             /* warps per CTA it was compiled for */
 } pad_launch_witness;
 
 pad_status pad_last_launch(pad_launch_witness *witness);

@@ -55,7 +55,8 @@ class PadOptions(ctypes.Structure):
 class PadLaunchWitness(ctypes.Structure):
     """pad_launch_witness: what the most recent launch recorded from inside the kernel."""
     _fields_ = [(n, ctypes.c_int32) for n in ("kernel", "head_dim", "heads_per_tile", "kv_dtype", "stages",
-                                                  "stage_tokens", "num_splits", "partition_tokens", "ctas")]
+                                                  "stage_tokens", "num_splits", "partition_tokens", "ctas",
+                                                  "warps")]
 
 
 class PadError(RuntimeError):

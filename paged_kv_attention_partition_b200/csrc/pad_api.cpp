@@ -158,7 +158,7 @@ void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan, b
     P = 512;
     while (P < 64 * s.g) P *= 2;
     const int64_t slots = (int64_t)sm_count(device < 0 ? 0 : device) *
-                          pad::ctas_per_sm_for((int)s.D, hpt);
+                          pad::ctas_per_sm_for((int)s.D, hpt, false);
     const int64_t pairs = s.B * s.Hkv * HT;
     while (P / 2 >= p_floor && P / 2 >= s.bs && pairs * ((C + P - 1) / P) < 2 * slots) P /= 2;
     P = round_up(P, s.bs);
@@ -173,7 +173,7 @@ void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan, b
   plan->heads_per_tile = hpt;
   plan->head_tiles = (int32_t)HT;
   const bool umma = tcgen05 && !s.fp8 && pad::umma_eligible((int)s.D, hpt, (int)s.bs);
-  plan->warps_per_cta = umma ? pad::kUmmaWarps : pad::kWarps;
+  plan->warps_per_cta = umma ? pad::kUmmaWarps : pad::warps_for((int)s.D, hpt, s.fp8);
   plan->stage_tokens = umma ? pad::kUmmaStageTokens : pad::stage_tokens_for((int)s.D, hpt, s.fp8);
   plan->stages = umma ? pad::umma_stages() : pad::partition_stages((int)s.D, hpt, s.fp8);
   // one CTA per unit (both kernels)
@@ -716,6 +716,7 @@ pad_status pad_last_launch(pad_launch_witness *w) {
   w->num_splits = h.num_splits;
   w->partition_tokens = h.partition_tokens;
   w->ctas = h.ctas;
+  w->warps = h.warps;
   return PAD_OK;
 }
 

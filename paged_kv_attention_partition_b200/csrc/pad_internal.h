@@ -16,69 +16,93 @@ enum : uint32_t {
   kErrTimeout = 0x4u,  // a bounded wait for a stage's copies gave up (internal error)
 };
 
-// Kernel geometry: one CTA of 4 warps per work unit; one thread issues the
-// stage copies (TMA), all four warps compute.  A warp is (token group tg, head
-// group hg, head_dim part dh):
+// Kernel geometry: one CTA of NW warps (4 or 8) per work unit; one thread
+// issues the stage copies (TMA), all warps compute.  A warp is (token group tg,
+// head group hg, head_dim part dh):
 //   - head groups split a head tile's 8-head n-tiles between warps: with 16 or
 //     32 heads per tile each warp owns one n-tile and computes every token of the
 //     stage for it (a quarter or half of the accumulator a warp holding the whole
 //     tile would need, and each head's softmax stays inside one warp);
 //   - head_dim parts split O^T's rows between the two warps of a pair that
-//     compute the same scores (D = 256, where a stage and the accumulator would
-//     otherwise limit residency);
+//     compute the same scores (D = 256, and 8-head tiles at D = 128 with 8
+//     warps: where a stage and the accumulator would otherwise limit residency);
 //   - the remaining warps form token groups: group tg computes 16-token tiles
 //     tg, tg + TG, ... of every stage, and the groups merge at the end.
-constexpr int kWarps = 4;
-constexpr int kThreads = kWarps * 32;
 constexpr int kSmemBudget = 232448;  // 227 KiB per CTA
 constexpr int kMaxSplits = 256;      // partitions per sequence (bounds the merge's weight table)
 
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ constexpr int dsplit_for(int D, int hpt) { return D == 256 ? 2 : 1; }
-__host__ __device__ constexpr int head_groups_for(int D, int hpt) {
-  return (hpt / 8) * dsplit_for(D, hpt) <= kWarps ? hpt / 8 : kWarps / dsplit_for(D, hpt);
+// Warps per CTA of each (head_dim, heads-per-tile, cache type) instantiation,
+// the measured choice (4 and 8 were timed on every named workload on B200).
+__host__ __device__ constexpr int warps_for(int D, int hpt, bool f8) { return 4; }
+
+__host__ __device__ constexpr int dsplit_for(int D, int hpt, int nw) {
+  return D == 256 ? 2 : (nw == 8 && D == 128 && hpt == 8 ? 2 : 1);
 }
-__host__ __device__ constexpr int token_groups_for(int D, int hpt) {
-  return kWarps / (dsplit_for(D, hpt) * head_groups_for(D, hpt));
+__host__ __device__ constexpr int head_groups_for(int D, int hpt, int nw) {
+  return (hpt / 8) * dsplit_for(D, hpt, nw) <= nw ? hpt / 8 : nw / dsplit_for(D, hpt, nw);
+}
+__host__ __device__ constexpr int token_groups_for(int D, int hpt, int nw) {
+  return nw / (dsplit_for(D, hpt, nw) * head_groups_for(D, hpt, nw));
 }
 // Tokens of one pipeline stage: 64; 32 at D = 256, whose rows are twice as
 // long, and for bf16 32-head tiles at D = 128, whose 16 KB stages let four CTAs
 // share an SM; an E4M3 cache at D = 256 with 8 or 16 heads per tile doubles
-// them, so its stage carries as many bytes as a bf16 one.
-__host__ __device__ constexpr int stage_tokens_for(int D, int hpt, bool f8 = false) {
-  return (D == 256 || (D == 128 && hpt == 32 && !f8) ? 32 : 64) * (f8 && D == 256 && hpt <= 16 ? 2 : 1);
+// them, so its stage carries as many bytes as a bf16 one.  At least one
+// 16-token tile per token group.
+__host__ __device__ constexpr int stage_tokens_for(int D, int hpt, bool f8, int nw) {
+  int st = (D == 256 || (D == 128 && hpt == 32 && !f8) ? 32 : 64) * (f8 && D == 256 && hpt <= 16 ? 2 : 1);
+  while (st < 16 * token_groups_for(D, hpt, nw)) st *= 2;
+  return st;
 }
 // 16-token tiles a warp computes per stage.
-__host__ __device__ constexpr int tiles_per_group(int D, int hpt, bool f8 = false) {
-  return stage_tokens_for(D, hpt, f8) / (16 * token_groups_for(D, hpt));
+__host__ __device__ constexpr int tiles_per_group(int D, int hpt, bool f8, int nw) {
+  return stage_tokens_for(D, hpt, f8, nw) / (16 * token_groups_for(D, hpt, nw));
 }
 
 // Pipeline depth and resident CTAs per SM of one (head_dim, heads-per-tile,
-// cache type) instantiation.  The ring is kept small so that several CTAs
-// share each SM: their loads, math and start/finish latencies overlap one
-// another.  The math is latency bound, so resident warps decide the speed:
-// an E4M3 cache at D = 128 with 8 or 16 heads per tile keeps two 16 KB stages
-// and runs five (8 heads) or four (16 heads, whose accumulators would spill at
-// five) CTAs per SM, registers capped to fit -- measured against deeper rings
-// and two-tile stages at 2-4 CTAs per SM, which were slower.
+// cache type, warps) instantiation.  The ring is kept small so that several
+// CTAs share each SM: their loads, math and start/finish latencies overlap one
+// another.  The math is latency bound, so resident warps decide the speed.
+// With 4 warps: an E4M3 cache at D = 128 with 8 or 16 heads per tile keeps two
+// 16 KB stages and runs five (8 heads) or four (16 heads, whose accumulators
+// would spill at five) CTAs per SM, registers capped to fit -- measured against
+// deeper rings and two-tile stages at 2-4 CTAs per SM, which were slower.
 // At D = 64 its 64-byte rows sit in boxes of at least 128 bytes, which caps
 // it at three stages.  32-head tiles at D = 128 (one n-tile per warp, 128
 // registers) run three 16 KB stages and four CTAs per SM for either cache
 // type, measured against two 32 KB stages at three CTAs (ragged MQA batch:
-// 177 -> 157 us bf16, 165 -> 159 us E4M3).
-__host__ __device__ constexpr int stages_for(int D, int hpt, bool f8 = false) {
+// 177 -> 157 us bf16, 165 -> 159 us E4M3).  With 8 warps: the same rings,
+// half the CTAs (a third for the E4M3 8-head tile, whose registers allow it),
+// so about as many warps share an SM.
+__host__ __device__ constexpr int stages_for(int D, int hpt, bool f8, int nw) {
   return f8 ? (D == 256 || (D == 128 && hpt <= 16) ? 2 : 3) : (D == 64 || (D == 128 && hpt == 32) ? 3 : 2);
 }
-__host__ __device__ constexpr int ctas_per_sm_for(int D, int hpt, bool f8 = false) {
+__host__ __device__ constexpr int ctas_per_sm4(int D, int hpt, bool f8) {
   return f8 && D == 128 ? (hpt == 8 ? 5 : 4)
                         : D == 64 ? (hpt == 32 ? 3 : 4) : D == 128 ? (hpt == 32 ? 4 : 3) : (hpt == 16 ? 2 : 3);
+}
+__host__ __device__ constexpr int ctas_per_sm_for(int D, int hpt, bool f8, int nw) {
+  return nw == 4 ? ctas_per_sm4(D, hpt, f8)
+                 : (f8 && D == 128 && hpt == 8 ? 3 : (ctas_per_sm4(D, hpt, f8) + 1) / 2);
 }
 // Bytes of one K (or V) half-stage: bf16 rows of 2D bytes; E4M3 rows of D
 // bytes, in boxes padded to at least 128 bytes (only D = 64 with one-row boxes
 // needs it).
-__host__ __device__ constexpr int half_stage_bytes(int D, int hpt, bool f8) {
-  return stage_tokens_for(D, hpt, f8) * (f8 ? (D < 128 ? 128 : D) : 2 * D);
+__host__ __device__ constexpr int half_stage_bytes(int D, int hpt, bool f8, int nw) {
+  return stage_tokens_for(D, hpt, f8, nw) * (f8 ? (D < 128 ? 128 : D) : 2 * D);
+}
+
+// The same, for the warps each instantiation is built with.
+__host__ __device__ constexpr int stage_tokens_for(int D, int hpt, bool f8 = false) {
+  return stage_tokens_for(D, hpt, f8, warps_for(D, hpt, f8));
+}
+__host__ __device__ constexpr int stages_for(int D, int hpt, bool f8 = false) {
+  return stages_for(D, hpt, f8, warps_for(D, hpt, f8));
+}
+__host__ __device__ constexpr int ctas_per_sm_for(int D, int hpt, bool f8 = false) {
+  return ctas_per_sm_for(D, hpt, f8, warps_for(D, hpt, f8));
 }
 
 // Shared memory of one CTA (from a 1024-byte aligned base): the K/V ring,
@@ -90,13 +114,13 @@ struct SmemPlan {
   size_t stage_bytes, ring_bytes, warp_merge_bytes, split_merge_bytes, region_bytes, total;
 };
 
-__host__ __device__ constexpr SmemPlan smem_plan_for(int D, int hpt, bool f8 = false) {
+__host__ __device__ constexpr SmemPlan smem_plan_for(int D, int hpt, bool f8, int nw) {
   SmemPlan s{};
-  s.stages = stages_for(D, hpt, f8);
-  s.stage_tokens = stage_tokens_for(D, hpt, f8);
-  s.stage_bytes = (size_t)half_stage_bytes(D, hpt, f8) * 2;  // K and V rows of one stage
+  s.stages = stages_for(D, hpt, f8, nw);
+  s.stage_tokens = stage_tokens_for(D, hpt, f8, nw);
+  s.stage_bytes = (size_t)half_stage_bytes(D, hpt, f8, nw) * 2;  // K and V rows of one stage
   s.ring_bytes = (size_t)s.stages * s.stage_bytes;
-  s.warp_merge_bytes = (size_t)token_groups_for(D, hpt) * hpt * (D + 4 + 2) * 4;  // padded rows, m, l
+  s.warp_merge_bytes = (size_t)token_groups_for(D, hpt, nw) * hpt * (D + 4 + 2) * 4;  // padded rows, m, l
   s.split_merge_bytes = (size_t)hpt * (kMaxSplits + 1) * 4;
   size_t m = s.ring_bytes;
   if (s.warp_merge_bytes > m) m = s.warp_merge_bytes;
@@ -111,7 +135,7 @@ inline int max_heads_per_tile(int D) { return D <= 128 ? 32 : 16; }
 
 // What a launch records from inside the kernel (pad_last_launch).
 struct LaunchWitness {
-  int32_t kernel, head_dim, heads_per_tile, kv_dtype, stages, stage_tokens, num_splits, partition_tokens, ctas;
+  int32_t kernel, head_dim, heads_per_tile, kv_dtype, stages, stage_tokens, num_splits, partition_tokens, ctas, warps;
 };
 
 struct PartitionParams {
@@ -202,7 +226,7 @@ constexpr int kUmmaWarps = 6;
 
 // Rows of one TMA box: a page, or a stage's worth of rows of a larger page.
 inline int box_rows(int block_size, int D, int hpt, bool f8) {
-  const int st = stage_tokens_for(D, hpt, f8);
+  const int st = stage_tokens_for(D, hpt, f8, warps_for(D, hpt, f8));
   return block_size < st ? block_size : st;
 }
 int partition_stages(int D, int heads_per_tile, bool kv_fp8);

@@ -110,21 +110,22 @@ template <int D, int HPT, bool F8, int NST, int ST>
 __device__ __noinline__ void record_launch(const PartitionParams &p) {
   if (blockIdx.x == 0 && threadIdx.x == 0)
     *p.witness = LaunchWitness{1, D, HPT, F8 ? (int32_t)PAD_FP8_E4M3 : (int32_t)PAD_BF16, NST, ST, p.S, p.P,
-                               (int32_t)gridDim.x};
+                               (int32_t)gridDim.x, (int32_t)(blockDim.x / 32)};
 }
 
-template <int D, int HPT, bool F8>
-__global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
+template <int D, int HPT, bool F8, int NW>
+__global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
     partition_kernel(const __grid_constant__ PartitionParams p) {
-  constexpr SmemPlan SP = smem_plan_for(D, HPT, F8);
+  constexpr int NTH = NW * 32;             // threads of the CTA
+  constexpr SmemPlan SP = smem_plan_for(D, HPT, F8, NW);
   constexpr int NST = SP.stages;
   constexpr uint32_t STAGE_BYTES = (uint32_t)SP.stage_bytes;
   constexpr int ST = SP.stage_tokens;      // tokens per stage
   constexpr int ST_LOG2 = ST == 128 ? 7 : ST == 64 ? 6 : 5;
-  constexpr int DS = dsplit_for(D, HPT);   // warps sharing a token group's scores (head_dim split)
-  constexpr int HG = head_groups_for(D, HPT);  // warps splitting the tile's n-tiles
-  constexpr int TG = token_groups_for(D, HPT);  // token groups
-  constexpr int TPW = tiles_per_group(D, HPT, F8);  // 16-token tiles per warp per stage
+  constexpr int DS = dsplit_for(D, HPT, NW);   // warps sharing a token group's scores (head_dim split)
+  constexpr int HG = head_groups_for(D, HPT, NW);  // warps splitting the tile's n-tiles
+  constexpr int TG = token_groups_for(D, HPT, NW);  // token groups
+  constexpr int TPW = tiles_per_group(D, HPT, F8, NW);  // 16-token tiles per warp per stage
   constexpr int NT = HPT / 8;              // 8-head n-tiles of the head tile
   constexpr int NTW = NT / HG;             // n-tiles of one warp
   constexpr int KT = D / 16;               // QK k-steps
@@ -133,13 +134,13 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
   constexpr int RW = ROWB < 128 ? ROWB : 128;  // bytes of a row in one column block
   constexpr int CH = ROWB / 16;            // 16-byte chunks per K/V row
   constexpr int CPB = RW / 16;             // 16-byte chunks per column block
-  constexpr int HALF = half_stage_bytes(D, HPT, F8);  // K (or V) rows of one stage
+  constexpr int HALF = half_stage_bytes(D, HPT, F8, NW);  // K (or V) rows of one stage
   constexpr int IDW = (ST + 31) / 32;      // block ids per lane of warp 0 for one stage
   // independent QK accumulation chains per tile (four in all where registers allow)
   constexpr int NCH = NTW == 1 ? (TPW >= 4 ? 1 : 4 / TPW) : NTW == 2 && TPW == 1 ? 2 : 1;
   static_assert(KT % NCH == 0, "k-steps split evenly over the chains");
   static_assert(ST == 16 * TG * TPW && (1 << ST_LOG2) == ST, "stage shape");
-  static_assert(DS * HG * TG == kWarps && NTW * HG == NT, "warp roles");
+  static_assert(DS * HG * TG == NW && NTW * HG == NT, "warp roles");
   static_assert(!F8 || (KT % 2 == 0 && MT % 2 == 0), "E4M3 operands are loaded two k-steps / m-tiles at a time");
   static_assert(NST >= 2 && NST <= 8, "at least one stage in flight during the math; barrier area");
   static_assert(SP.total <= (size_t)kSmemBudget, "shared-memory plan over budget");
@@ -220,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
   const int tlo = max(t0, lo);
   if (tlo >= t1) {
     if (L == 0 && s == 0) {  // empty sequence: out = 0, lse = -inf (or the sink)
-      for (int i = tid; i < gl * D; i += kThreads)
+      for (int i = tid; i < gl * D; i += NTH)
         p.out[b * p.o_sb + (int64_t)(h0 + i / D) * p.o_sh + (i % D)] = 0;
       if (p.lse != nullptr && tid < gl)
         p.lse[b * p.lse_sb + (int64_t)(h0 + tid) * p.lse_sh] = p.sinks != nullptr ? p.sinks[h0 + tid] : -INFINITY;
@@ -632,7 +633,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
   __syncthreads();
 
   constexpr int D4 = D / 4;
-  for (int i = tid; i < gl * D4; i += kThreads) {
+  for (int i = tid; i < gl * D4; i += NTH) {
     const int hl = i / D4, d = (i % D4) * 4;
     float m = -INFINITY;
 #pragma unroll
@@ -677,7 +678,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm_for(D, HPT, F8))
   record_launch<D, HPT, F8, NST, ST>(p);
   if (ns == 1) return;
   if (claim_last_partition(p, b, kvh, ht, ns, flag))
-    merge_partials<D, kThreads>(p, b, h0, gl, s_first, ns, reinterpret_cast<float *>(smem));  // the ring is free
+    merge_partials<D, NTH>(p, b, h0, gl, s_first, ns, reinterpret_cast<float *>(smem));  // the ring is free
 }
 
 int partition_stages(int D, int hpt, bool kv_fp8) { return stages_for(D, hpt, kv_fp8); }
@@ -685,17 +686,19 @@ int partition_stages(int D, int hpt, bool kv_fp8) { return stages_for(D, hpt, kv
 template <int D, int HPT, bool F8>
 static cudaError_t launch_t(const PartitionParams &p, int grid, cudaStream_t stream) {
   static std::atomic<uint64_t> attr_done{0};
-  constexpr SmemPlan SP = smem_plan_for(D, HPT, F8);
+  constexpr int NW = warps_for(D, HPT, F8);
+  constexpr SmemPlan SP = smem_plan_for(D, HPT, F8, NW);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_done.load(std::memory_order_acquire) & bit)) {
-    e = cudaFuncSetAttribute(partition_kernel<D, HPT, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SP.total);
+    e = cudaFuncSetAttribute(partition_kernel<D, HPT, F8, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SP.total);
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(bit, std::memory_order_acq_rel);
   }
-  partition_kernel<D, HPT, F8><<<grid, kThreads, SP.total, stream>>>(p);
+  partition_kernel<D, HPT, F8, NW><<<grid, NW * 32, SP.total, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 2) umma_kernel(const __grid_cons
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (blockIdx.x == 0 && tid == 0)  // which kernel ran, and with what plan
-    *p.witness = LaunchWitness{2, kD, kHeads, (int32_t)PAD_BF16, 1, kChunk, p.S, p.P, (int32_t)gridDim.x};
+    *p.witness = LaunchWitness{2, kD, kHeads, (int32_t)PAD_BF16, 1, kChunk, p.S, p.P, (int32_t)gridDim.x, kUmmaWarps};
   uint32_t u = blockIdx.x;
   const int s = (int)(u % (uint32_t)p.S);
   u /= (uint32_t)p.S;

@@ -234,13 +234,13 @@ cudaError_t launch_partition(const PartitionParams &p, int D, int hpt, bool f8, 
   if (fake::launch_result != cudaSuccess) return fake::launch_result;
   fake::launches.push_back({p, D, hpt, grid, f8, false, s});
   fake::witness = LaunchWitness{1, D, hpt, f8 ? (int32_t)PAD_FP8_E4M3 : (int32_t)PAD_BF16, stages_for(D, hpt, f8),
-                                stage_tokens_for(D, hpt, f8), p.S, p.P, grid};
+                                stage_tokens_for(D, hpt, f8), p.S, p.P, grid, warps_for(D, hpt, f8)};
   return cudaSuccess;
 }
 cudaError_t launch_umma(const PartitionParams &p, int grid, cudaStream_t s) {
   if (fake::launch_result != cudaSuccess) return fake::launch_result;
   fake::launches.push_back({p, 128, 32, grid, false, true, s});
-  fake::witness = LaunchWitness{2, 128, 32, (int32_t)PAD_BF16, 1, kUmmaStageTokens, p.S, p.P, grid};
+  fake::witness = LaunchWitness{2, 128, 32, (int32_t)PAD_BF16, 1, kUmmaStageTokens, p.S, p.P, grid, kUmmaWarps};
   return cudaSuccess;
 }
 }  // namespace pad

@@ -40,6 +40,7 @@ def test_partition_kernel_runs_the_planned_shape(cuda_device, shape):
     assert got["kv_dtype"] == (pad.PAD_FP8_E4M3 if kv == "e4m3" else pad.PAD_BF16)
     for key in ("heads_per_tile", "stages", "stage_tokens", "num_splits", "partition_tokens", "ctas"):
         assert got[key] == plan[key], (key, got, plan)
+    assert got["warps"] == plan["warps_per_cta"], (got, plan)
 
 
 def test_tcgen05_entry_runs_the_tcgen05_kernel(cuda_device):
@@ -47,7 +48,7 @@ def test_tcgen05_entry_runs_the_tcgen05_kernel(cuda_device):
     DeviceWorkload(w, cuda_device).run(num_splits=4, entry=pad.pad_decode_tcgen05)
     got = pad.pad_last_launch()
     assert (got["kernel"], got["head_dim"], got["heads_per_tile"], got["kv_dtype"]) == (2, 128, 32, pad.PAD_BF16)
-    assert got["num_splits"] == 4 and got["ctas"] == 4 * 1 * 1 * 4
+    assert got["num_splits"] == 4 and got["ctas"] == 4 * 1 * 1 * 4 and got["warps"] == 6
 
 
 def test_static_scratch_and_caller_workspace_run_the_partition_kernel(cuda_device):
