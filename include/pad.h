@@ -384,14 +384,17 @@ pad_status pad_check_device_errors(void *stream, uint32_t *bits);
  * saved paged decode bindings once", section "Risk Assessment": focused tests
  * of failure recovery).  The next launch of the partition kernel made from the
  * calling thread (pad_decode, pad_decode_ex, the workspace and static-scratch
- * entry points; not pad_decode_tcgen05) runs with the CTAs of partition
- * `partition` waiting, after they issue their first copies, on a barrier that
- * nothing arrives on.  The wait gives up after a short limit (about 20 us),
- * sets bit 0x4 of the device error word, drains the CTA's own copies (bounded)
- * and returns, exactly as on a stage that never lands; the other partitions
- * count themselves and leave their merge counters set.  No GPU fault, trap or
- * hang is involved.  One-shot: the launch consumes it.  -1 disarms it; other
- * values outside [0, 256) are PAD_ERR_INVALID_ARG.
+ * entry points; not pad_decode_tcgen05) runs with every non-empty unit of
+ * partition `partition` giving up where it would count its partition for the
+ * merge: it waits on a barrier that nothing arrives on, the wait gives up after
+ * a short limit (about 20 us) and sets bit 0x4 of the device error word, as a
+ * stage that never lands would, and the unit returns uncounted.  The other
+ * partitions count themselves and leave their merge counters set, so no
+ * sequence with several partitions including that one is merged (its out and
+ * lse are left as they were); a sequence with one partition has already
+ * written its result.  No GPU fault, trap or hang is involved.  One-shot: the
+ * launch consumes it.  -1 disarms it; other values outside [0, 256) are
+ * PAD_ERR_INVALID_ARG.
  */
 pad_status pad_inject_stage_timeout(int32_t partition);
 

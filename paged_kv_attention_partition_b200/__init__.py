@@ -330,9 +330,10 @@ def pad_check_device_errors(stream=None, device=None) -> int:
 
 
 def pad_inject_stage_timeout(partition: int) -> None:
-    """Failure-path test hook (see include/pad.h): the next partition-kernel
-    launch from this thread makes the CTAs of ``partition`` give up on a bounded
-    wait, as on a stage that never lands (error bit 0x4).  -1 disarms it."""
+    """Failure-path test hook (see include/pad.h): in the next partition-kernel
+    launch from this thread the units of ``partition`` give up on a bounded wait
+    instead of counting themselves for the merge, as on a stage that never
+    lands (error bit 0x4).  -1 disarms it."""
     _raise(load_library().pad_inject_stage_timeout(int(partition)))
 
 

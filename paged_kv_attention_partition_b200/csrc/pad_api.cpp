@@ -744,7 +744,8 @@ pad_status pad_check_device_errors(void *stream_, uint32_t *bits) {
   if (v != 0)
     return fail(PAD_ERR_DEVICE_CHECK, "kernel saw %s%s%s", (v & pad::kErrBlockId) ? "an out-of-range block id; " : "",
                 (v & pad::kErrSeqLen) ? "an out-of-range sequence length; " : "",
-                (v & pad::kErrTimeout) ? "a stage whose copies never completed (internal error)" : "");
+                (v & pad::kErrTimeout) ? "a bounded wait that gave up (a stage whose copies never completed: an "
+                                         "internal error; or the failure-path test hook)" : "");
   return PAD_OK;
 }
 

@@ -179,9 +179,10 @@ struct PartitionParams {
   uint32_t *err;
   LaunchWitness *witness;  // written by block 0 of every launch
   // Failure-path test hook (pad_inject_stage_timeout): -1 normally; otherwise
-  // the partition kernel's CTAs of partition `stall_partition` wait, after
-  // issuing their first copies, on a barrier nothing arrives on, give up after
-  // a short bounded wait and take the timeout exit.
+  // the partition kernel's non-empty units of partition `stall_partition` wait,
+  // where they would count themselves for the merge, on a barrier nothing
+  // arrives on, give up after a short bounded wait (error bit 0x4) and return
+  // uncounted.
   int32_t stall_partition;
 };
 

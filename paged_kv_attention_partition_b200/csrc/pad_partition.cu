@@ -91,26 +91,33 @@ __device__ bool wait_stage(uint32_t bar, uint32_t parity, uint32_t *err, uint64_
   return true;
 }
 
-// Failure-path test hook: thread 0 of a CTA of the chosen partition waits on
-// `never` (initialised, never arrived on) until the short limit runs out, as a
-// stage whose copies never land would; true when it gave up.
-__device__ __noinline__ bool stall_for_test(uint32_t never, uint32_t *err) {
-  return !wait_stage(never, 0, err, kStallLimitNs);
-}
 }  // namespace
 
-// Which kernel ran, and with what plan: thread 0 of block 0 writes the record
-// when its unit is done (empty, or through the epilogue); a unit that gives up
-// on an internal error records nothing -- the error word reports that case.
-// Out of line and at the exits, the store leaves the main loop's code as it is:
-// inlined (at the start or at the exits) it changed the 32-head bf16
-// instance's schedule at its 128-register cap and cost ragged_mqa 6% on B200;
-// as a call it is within 1% of no record at all.
+// At a unit's exits.  (1) Which kernel ran, and with what plan: thread 0 of
+// block 0 writes the record when its unit is done (empty, or through the
+// epilogue); a unit that gives up on an internal error records nothing -- the
+// error word reports that case.  (2) The failure-path test hook, at the exit
+// after the unit's result is written (`spare`: an unused 8-byte barrier slot):
+// a unit of partition p.stall_partition gives up there instead of counting
+// its partition -- its thread 0 waits on a barrier nothing arrives on until the
+// short limit runs out, as on a stage whose copies never land (error bit 0x4)
+// -- and returns true in every thread.  Out of line, both leave the main
+// loop's code as it is: any code added to the kernel body (the record inlined
+// at the start or at the exits, or a hook of its own) changed the 32-head
+// instances' schedules at their 128-register cap and cost the ragged MQA batch
+// 6-10% on B200; as this one call it is within 1% of neither.
 template <int D, int HPT, bool F8, int NST, int ST>
-__device__ __noinline__ void record_launch(const PartitionParams &p) {
+__device__ __noinline__ bool unit_exit(const PartitionParams &p, int s, uint64_t *spare) {
   if (blockIdx.x == 0 && threadIdx.x == 0)
     *p.witness = LaunchWitness{1, D, HPT, F8 ? (int32_t)PAD_FP8_E4M3 : (int32_t)PAD_BF16, NST, ST, p.S, p.P,
                                (int32_t)gridDim.x, (int32_t)(blockDim.x / 32)};
+  if (s != p.stall_partition || spare == nullptr) return false;
+  if (threadIdx.x == 0) {
+    const uint32_t never = smem_addr(spare);
+    mbar_init(never, 1);
+    wait_stage(never, 0, p.err, kStallLimitNs);  // gives up: bit 0x4
+  }
+  return true;
 }
 
 template <int D, int HPT, bool F8, int NW>
@@ -148,7 +155,6 @@ __global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + SP.region_bytes);  // one per stage slot
   int *flag = reinterpret_cast<int *>(smem + SP.region_bytes + 64);
-  uint64_t *never = reinterpret_cast<uint64_t *>(smem + SP.region_bytes + 96);  // test hook only
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int dh = warp % DS, hg = (warp / DS) % HG, tg = warp / (DS * HG);  // head_dim part, head group, token group
@@ -203,7 +209,6 @@ __global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
   if (tid == 0) {
 #pragma unroll
     for (int i = 0; i < NST; ++i) mbar_init(smem_addr(full + i), 1);
-    if (p.stall_partition >= 0) mbar_init(smem_addr(never), 1);
     fence_mbar_init();
   }
 
@@ -226,7 +231,7 @@ __global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
       if (p.lse != nullptr && tid < gl)
         p.lse[b * p.lse_sb + (int64_t)(h0 + tid) * p.lse_sh] = p.sinks != nullptr ? p.sinks[h0 + tid] : -INFINITY;
     }
-    record_launch<D, HPT, F8, NST, ST>(p);
+    unit_exit<D, HPT, F8, NST, ST>(p, s, nullptr);
     return;  // pages wholly outside [lo, L) are never read
   }
   const int s_first = lo / p.P;                      // first non-empty partition of sequence b
@@ -272,18 +277,6 @@ __global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
       if (k < nstages) issue(ids[k], k);
   }
   int (&idn)[IDW] = ids[NST - 1];  // block ids of the next stage to issue
-  if (p.stall_partition >= 0) {
-    // failure-path test hook (uniform over the launch): the chosen partition's
-    // CTAs give up as on a stage that never lands, with the first stages'
-    // copies in flight, and drain them (bounded) before returning
-    const bool gave_up = tid == 0 && s == p.stall_partition && stall_for_test(smem_addr(never), p.err);
-    if (__syncthreads_or(gave_up)) {
-      if (tid == 0)
-        for (int j = 0; j < nstages && j < NST - 1; ++j) wait_stage(smem_addr(full + j), 0, p.err);
-      __syncthreads();
-      return;
-    }
-  }
 
   // Address of 16-byte chunk (column block h, chunk c of it) of row r in a K
   // or V half-stage: rows grouped in boxes of 2^bsb_log2 rows, each box laid out
@@ -675,8 +668,7 @@ __global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
       if (d == 0) p.lse_part[row] = lse_nat;
     }
   }
-  record_launch<D, HPT, F8, NST, ST>(p);
-  if (ns == 1) return;
+  if (unit_exit<D, HPT, F8, NST, ST>(p, s, full + 12) || ns == 1) return;
   if (claim_last_partition(p, b, kvh, ht, ns, flag))
     merge_partials<D, NTH>(p, b, h0, gl, s_first, ns, reinterpret_cast<float *>(smem));  // the ring is free
 }

@@ -239,9 +239,12 @@ __global__ void __launch_bounds__(kUmmaThreads, 2) umma_kernel(const __grid_cons
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (blockIdx.x == 0 && tid == 0)  // which kernel ran, and with what plan
     *p.witness = LaunchWitness{2, kD, kHeads, (int32_t)PAD_BF16, 1, kChunk, p.S, p.P, (int32_t)gridDim.x, kUmmaWarps};
+  // Grid order: partition index descending, outermost, as in partition_kernel:
+  // the longest sequences' work starts first and empty units exit early.
   uint32_t u = blockIdx.x;
-  const int s = (int)(u % (uint32_t)p.S);
-  u /= (uint32_t)p.S;
+  const uint32_t pairs = (uint32_t)p.B * p.Hkv * p.HT;
+  const int s = p.S - 1 - (int)(u / pairs);
+  u %= pairs;
   const int ht = (int)(u % (uint32_t)p.HT);
   u /= (uint32_t)p.HT;
   const int kvh = (int)(u % (uint32_t)p.Hkv);
@@ -302,11 +305,20 @@ __global__ void __launch_bounds__(kUmmaThreads, 2) umma_kernel(const __grid_cons
       mbar_arrive_expect_tx(q_full, kQBytes);
       tma_load_4d(smem_addr(smem + SM::q), &p.tmq, 0, h0, 0, b, q_full);
     }
+    // block id of lane l's box of chunk c (one chunk ahead, so the table's
+    // latency overlaps the waits for the buffers)
+    auto box_id = [&](int c) -> int {
+      const int tb = t0 + c * kChunk;
+      const int nbox = min(kChunk / kBoxRows, (t1 - tb + kBoxRows - 1) / kBoxRows);
+      return lane < nbox ? __ldg(trow + ((tb + kBoxRows * lane) >> p.bs_log2)) : 0;
+    };
+    int id_next = box_id(0);
     for (int c = 0; ok && c < nch; ++c) {
       const int tb = t0 + c * kChunk;
       const int nbox = min(kChunk / kBoxRows, (t1 - tb + kBoxRows - 1) / kBoxRows);
       const int tok = tb + kBoxRows * lane;
-      const int id = lane < nbox ? __ldg(trow + (tok >> p.bs_log2)) : 0;
+      const int id = id_next;
+      if (c + 1 < nch) id_next = box_id(c + 1);
       const int slot0 = tok & ((1 << p.bs_log2) - 1);
       if (lane < nbox && (unsigned)id >= (unsigned)p.num_blocks) atomicOr(p.err, kErrBlockId);  // reads as zeros
       // K(c) once S(c-1) has read the K buffer
@@ -550,6 +562,12 @@ cudaError_t launch_umma(const PartitionParams &p, int grid, cudaStream_t stream)
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_done.load(std::memory_order_acquire) & bit)) {
     e = cudaFuncSetAttribute(umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)UmmaSmem::total);
+    if (e != cudaSuccess) return e;
+    // all of the unified L1 / shared memory as shared memory: two CTAs of
+    // ~106 KB need more than the carveout the driver picks by itself, with
+    // which a timeline of the ragged MQA batch showed one CTA per SM
+    e = cudaFuncSetAttribute(umma_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(bit, std::memory_order_acq_rel);
   }
