@@ -179,7 +179,8 @@ void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan, b
   // one CTA per unit (both kernels)
   plan->ctas = (int32_t)(units > 0x7fffffffll ? 0x7fffffffll : units);
   plan->reduce = S > 1 ? 1 : 0;
-  plan->workspace_bytes = (int64_t)pad::workspace_layout(s.B, s.Hq, S, s.D).total;
+  plan->workspace_bytes =
+      (int64_t)pad::workspace_layout(s.B, s.Hq, S, s.D, units, pad::schedules_units(s.B, S, P, hpt)).total;
   plan->control_bytes = (int64_t)pad::control_layout(s.B, s.Hkv, HT, S).total;
   log_plan(s, num_splits, device, *plan, umma);
 }
@@ -362,6 +363,7 @@ struct Prepared {
   int D;
   int device;
   bool kv_fp8;
+  bool ordered;  // the launch orders its units (schedule pass first)
 };
 
 pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_tensor *v_cache,
@@ -446,7 +448,8 @@ pad_status prepare(const pad_tensor *q, const pad_tensor *k_cache, const pad_ten
   make_plan(s, num_splits, device, &pr->plan, tcgen05);
   const int64_t units = B * Hkv * pr->plan.head_tiles * (int64_t)pr->plan.num_splits;
   if (units > 0x7fffffffll) return fail(PAD_ERR_UNSUPPORTED, "too many work units (%lld) for one launch", (long long)units);
-  pr->ws = pad::workspace_layout(B, Hq, pr->plan.num_splits, D);
+  pr->ordered = pad::schedules_units(B, pr->plan.num_splits, pr->plan.partition_tokens, pr->plan.heads_per_tile);
+  pr->ws = pad::workspace_layout(B, Hq, pr->plan.num_splits, D, units, pr->ordered);
   pr->cl = pad::control_layout(B, Hkv, pr->plan.head_tiles, pr->plan.num_splits);
 
   uint32_t *err = nullptr;
@@ -520,6 +523,7 @@ void bind_buffers(Prepared &pr, void *partials, void *control) {
   char *base = static_cast<char *>(partials);
   pr.p.o_part = base != nullptr ? reinterpret_cast<float *>(base + pr.ws.o_part) : nullptr;
   pr.p.lse_part = base != nullptr ? reinterpret_cast<float *>(base + pr.ws.lse_part) : nullptr;
+  pr.p.order = base != nullptr && pr.ordered ? reinterpret_cast<const uint32_t *>(base + pr.ws.order) : nullptr;
   pr.p.counters = pr.cl.total > 0 ? reinterpret_cast<uint32_t *>(static_cast<char *>(control) + pr.cl.counters)
                                   : nullptr;
 }
@@ -533,9 +537,10 @@ pad_status check_caller_buffer(const Prepared &pr, void *buf, size_t bytes, size
 }
 
 pad_status run(const Prepared &pr, cudaStream_t stream) {
-  cudaError_t e = pr.umma ? pad::launch_umma(pr.p, pr.plan.ctas, stream)
-                          : pad::launch_partition(pr.p, pr.D, pr.plan.heads_per_tile, pr.kv_fp8, pr.plan.ctas,
-                                                  stream);
+  cudaError_t e = pr.p.order != nullptr ? pad::launch_schedule(pr.p, stream) : cudaSuccess;
+  if (e != cudaSuccess) return cuda_fail(e, "unit schedule launch");
+  e = pr.umma ? pad::launch_umma(pr.p, pr.plan.ctas, stream)
+              : pad::launch_partition(pr.p, pr.D, pr.plan.heads_per_tile, pr.kv_fp8, pr.plan.ctas, stream);
   if (!pr.umma) g_stall_partition = -1;  // the test hook is one-shot
   return e == cudaSuccess ? PAD_OK : cuda_fail(e, "partition kernel launch");
 }

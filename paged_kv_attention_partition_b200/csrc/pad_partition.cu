@@ -120,7 +120,7 @@ __device__ __noinline__ bool unit_exit(const PartitionParams &p, int s, uint64_t
   return true;
 }
 
-template <int D, int HPT, bool F8, int NW>
+template <int D, int HPT, bool F8, int NW, bool ORDERED>
 __global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
     partition_kernel(const __grid_constant__ PartitionParams p) {
   constexpr int NTH = NW * 32;             // threads of the CTA
@@ -158,14 +158,16 @@ __global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int dh = warp % DS, hg = (warp / DS) % HG, tg = warp / (DS * HG);  // head_dim part, head group, token group
-  // Grid order: partition index descending, outermost.  The highest partitions
+  // Unit order.  With several partitions per sequence, CTA i runs unit
+  // p.order[i], written just before the launch by schedule_kernel from the
+  // device-resident lengths: the longest units first, so the units dispatched
+  // last (after the first wave) are the shortest.  Otherwise, and as the unit
+  // numbering: partition index descending, outermost -- the highest partitions
   // exist only for the longest sequences, so their work starts first and the
-  // empty ones (short sequences) exit early; the last waves are every
-  // sequence's first partition, full for every sequence that reaches P tokens.
-  // Measured on B200: llama8b (lengths 512..4096) 59.4 -> 56.1 us against
-  // partition-innermost order; batches of uniform full lengths lose ~3% (every
-  // merge then falls in the last wave).
-  uint32_t u = blockIdx.x;
+  // empty ones (short sequences) exit early.
+  // (The instantiations without an order leave the code as it was: the order
+  // load, even untaken, cost the 8-head tiles ~2% on the Qwen3-14B-shaped batch.)
+  uint32_t u = ORDERED ? __ldg(p.order + blockIdx.x) : blockIdx.x;
   const uint32_t pairs = (uint32_t)p.B * p.Hkv * p.HT;
   const int s = p.S - 1 - (int)(u / pairs);
   u %= pairs;
@@ -675,8 +677,67 @@ __global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
 
 int partition_stages(int D, int hpt, bool kv_fp8) { return stages_for(D, hpt, kv_fp8); }
 
-template <int D, int HPT, bool F8>
-static cudaError_t launch_t(const PartitionParams &p, int grid, cudaStream_t stream) {
+// ---- the unit schedule -------------------------------------------------------
+//
+// One CTA orders the launch's units by the number of tokens they stream,
+// longest first (64 buckets of P/64 tokens; empty units last), and writes the
+// permutation to p.order.  A unit's tokens are those of partition s of
+// sequence b that take part: [max(s P, lo), min((s+1) P, L_b)), lo the first
+// token of a sliding window.  With more units than CTA slots, the block
+// scheduler dispatches the order's tail after the first wave; ordered this
+// way that tail is the partial last partitions rather than full ones, which is
+// what a ragged batch's time was waiting on (longest-processing-time-first
+// list scheduling).  Units of one (b, s) -- its KV heads and head tiles --
+// stay adjacent.  The order within a bucket follows shared-memory atomics and
+// may change from call to call; which CTA runs a unit changes no result.
+constexpr int kScheduleThreads = 1024;
+constexpr int kScheduleBuckets = 64;
+
+__global__ void __launch_bounds__(kScheduleThreads) schedule_kernel(const __grid_constant__ PartitionParams p) {
+  __shared__ uint32_t count[kScheduleBuckets], next[kScheduleBuckets];
+  const int tid = threadIdx.x;
+  if (tid < kScheduleBuckets) count[tid] = 0;
+  __syncthreads();
+  const int capacity = p.max_blocks << p.bs_log2;
+  const uint32_t per = (uint32_t)p.Hkv * p.HT;  // units of one (b, s)
+  const uint32_t pairs = (uint32_t)p.B * per;    // units of one partition index
+  const int npair = p.B * p.S;
+  auto bucket = [&](int i) -> int {  // 0: P tokens ... kScheduleBuckets - 1: none
+    const int b = i / p.S, s = i % p.S;
+    int L = __ldg(p.seq_lens + b);
+    L = L < 0 ? 0 : (L > capacity ? capacity : L);
+    const int lo = (p.window > 0 && L > p.window) ? L - p.window : 0;
+    const int t0 = s * p.P;
+    const int work = min(t0 + p.P, L) - max(t0, lo);
+    return work <= 0 ? kScheduleBuckets - 1
+                     : (int)((int64_t)(p.P - work) * (kScheduleBuckets - 1) / p.P);
+  };
+  for (int i = tid; i < npair; i += kScheduleThreads) atomicAdd(&count[bucket(i)], 1u);
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t acc = 0;
+    for (int k = 0; k < kScheduleBuckets; ++k) {
+      next[k] = acc;
+      acc += count[k];
+    }
+  }
+  __syncthreads();
+  uint32_t *order = const_cast<uint32_t *>(p.order);
+  for (int i = tid; i < npair; i += kScheduleThreads) {
+    const uint32_t slot = atomicAdd(&next[bucket(i)], 1u);
+    const int b = i / p.S, s = i % p.S;
+    const uint32_t first = (uint32_t)(p.S - 1 - s) * pairs + (uint32_t)b * per;  // unit (b, s, kv head 0, tile 0)
+    for (uint32_t j = 0; j < per; ++j) order[slot * per + j] = first + j;
+  }
+}
+
+cudaError_t launch_schedule(const PartitionParams &p, cudaStream_t stream) {
+  schedule_kernel<<<1, kScheduleThreads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D, int HPT, bool F8, bool ORDERED>
+static cudaError_t launch_o(const PartitionParams &p, int grid, cudaStream_t stream) {
   static std::atomic<uint64_t> attr_done{0};
   constexpr int NW = warps_for(D, HPT, F8);
   constexpr SmemPlan SP = smem_plan_for(D, HPT, F8, NW);
@@ -685,13 +746,18 @@ static cudaError_t launch_t(const PartitionParams &p, int grid, cudaStream_t str
   if (e != cudaSuccess) return e;
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_done.load(std::memory_order_acquire) & bit)) {
-    e = cudaFuncSetAttribute(partition_kernel<D, HPT, F8, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(partition_kernel<D, HPT, F8, NW, ORDERED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SP.total);
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(bit, std::memory_order_acq_rel);
   }
-  partition_kernel<D, HPT, F8, NW><<<grid, NW * 32, SP.total, stream>>>(p);
+  partition_kernel<D, HPT, F8, NW, ORDERED><<<grid, NW * 32, SP.total, stream>>>(p);
   return cudaGetLastError();
+}
+
+template <int D, int HPT, bool F8>
+static cudaError_t launch_t(const PartitionParams &p, int grid, cudaStream_t stream) {
+  return p.order != nullptr ? launch_o<D, HPT, F8, true>(p, grid, stream) : launch_o<D, HPT, F8, false>(p, grid, stream);
 }
 
 template <bool F8>

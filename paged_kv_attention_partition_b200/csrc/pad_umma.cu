@@ -212,7 +212,10 @@ static_assert(2 * kHalfBytes >= kHeads * kMaxSplits * 4, "merge weights fit the 
 
 // One CTA per work unit (sequence b, KV head, head tile, partition s), two
 // CTAs per SM: while one streams, the other's start, epilogue and split merge
-// proceed.  Roles: warps 0-3 softmax and epilogue (thread i = token i of a
+// proceed.  (Double-buffering the K and V chunks, ~171 KB of shared memory and
+// so one CTA per SM, was slower on the ragged MQA batch on B200: 200 against
+// 162 us -- a per-CTA timeline of this layout showed two CTAs resident on
+// every SM, 1.6 on average over the launch.)  Roles: warps 0-3 softmax and epilogue (thread i = token i of a
 // chunk, then head_dim row i of O^T), warp 4 copies (TMA), warp 5 issues the
 // MMAs (one thread).  Per chunk c of 128 tokens:
 //   K(c) lands -> S(c) = K(c).Q^T into S buffer c%2 -> K buffer refilled with K(c+1)
@@ -239,9 +242,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 2) umma_kernel(const __grid_cons
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (blockIdx.x == 0 && tid == 0)  // which kernel ran, and with what plan
     *p.witness = LaunchWitness{2, kD, kHeads, (int32_t)PAD_BF16, 1, kChunk, p.S, p.P, (int32_t)gridDim.x, kUmmaWarps};
-  // Grid order: partition index descending, outermost, as in partition_kernel:
-  // the longest sequences' work starts first and empty units exit early.
-  uint32_t u = blockIdx.x;
+  // Unit order as in partition_kernel: p.order (longest units first) when the
+  // launch schedules its units, else partition index descending, outermost.
+  uint32_t u = p.order != nullptr ? __ldg(p.order + blockIdx.x) : blockIdx.x;
   const uint32_t pairs = (uint32_t)p.B * p.Hkv * p.HT;
   const int s = p.S - 1 - (int)(u / pairs);
   u %= pairs;

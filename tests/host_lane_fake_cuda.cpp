@@ -54,6 +54,8 @@ struct Launch {
   cudaStream_t stream;
 };
 std::vector<Launch> launches;
+// schedule passes: the parameter block each was given and its stream
+std::vector<std::pair<pad::PartitionParams, cudaStream_t>> schedules;
 struct Encode {
   CUtensorMapDataType dt;
   cuuint32_t rank;
@@ -237,6 +239,11 @@ cudaError_t launch_partition(const PartitionParams &p, int D, int hpt, bool f8, 
                                 stage_tokens_for(D, hpt, f8), p.S, p.P, grid, warps_for(D, hpt, f8)};
   return cudaSuccess;
 }
+cudaError_t launch_schedule(const PartitionParams &p, cudaStream_t s) {
+  if (fake::launch_result != cudaSuccess) return fake::launch_result;
+  fake::schedules.push_back({p, s});
+  return cudaSuccess;
+}
 cudaError_t launch_umma(const PartitionParams &p, int grid, cudaStream_t s) {
   if (fake::launch_result != cudaSuccess) return fake::launch_result;
   fake::launches.push_back({p, 128, 32, grid, false, true, s});
@@ -338,6 +345,17 @@ static void check_launch(const Problem &pr, int32_t splits, const fake::Launch &
     const fake::Alloc *a = fake::find(p.o_part);
     CHECK(inside(p.o_part, ob, a) && inside(p.lse_part, lb, a), "%s: partials outside their buffer", what);
     CHECK((const char *)p.lse_part >= (const char *)p.o_part + ob, "%s: partial regions overlap", what);
+    // the unit order: after the partials, in the same buffer, written by a
+    // schedule pass launched just before on the same stream with the same order
+    const bool sched = pad::schedules_units(pr.B, p.S, p.P, pl.heads_per_tile);
+    CHECK((p.order != nullptr) == sched, "%s: unit order %s", what, sched ? "missing" : "unexpected");
+    if (sched) {
+      CHECK(inside(p.order, (size_t)p.n_units * 4, a) && (const char *)p.order >= (const char *)p.lse_part + lb,
+            "%s: unit order outside its place", what);
+      CHECK(!fake::schedules.empty() && fake::schedules.back().first.order == p.order &&
+                fake::schedules.back().second == L.stream && fake::schedules.back().first.n_units == p.n_units,
+            "%s: no schedule pass before the launch", what);
+    }
     const size_t cb = (size_t)(pr.B * pr.Hkv * p.HT * 4);
     const fake::Alloc *c = fake::find(p.counters);
     CHECK(inside(p.counters, cb, c) && c != a, "%s: counters outside their own buffer", what);
@@ -345,7 +363,8 @@ static void check_launch(const Problem &pr, int32_t splits, const fake::Launch &
     for (size_t i = 0; c && i < cb / 4; ++i) zero = zero && p.counters[i] == 0;
     CHECK(zero, "%s: merge counters not zero at launch", what);
   } else {
-    CHECK(p.o_part == nullptr && p.lse_part == nullptr && p.counters == nullptr, "%s: scratch with S == 1", what);
+    CHECK(p.o_part == nullptr && p.lse_part == nullptr && p.counters == nullptr && p.order == nullptr,
+          "%s: scratch with S == 1", what);
   }
 }
 
@@ -394,6 +413,16 @@ static void scenarios() {
   CHECK(a.decode(4, s1) == PAD_OK && fake::launches.size() == 2, "repeat decode");
   for (size_t i = ev; i < fake::events.size(); ++i)
     CHECK(fake::events[i].rfind("malloc", 0) != 0, "repeat decode allocated (%s)", fake::events[i].c_str());
+
+  // heavy units (2048-token partitions of a 32-head tile): a schedule pass on
+  // the same stream writes the unit order into the partials buffer first
+  Problem heavy(2, 32, 1, 128, 16, 256);
+  const size_t sched0 = fake::schedules.size();
+  CHECK(heavy.decode(2, s1) == PAD_OK && fake::schedules.size() == sched0 + 1, "scheduled decode: %s",
+        pad_last_error());
+  CHECK(heavy.plan(2).partition_tokens * heavy.plan(2).heads_per_tile >= 32768, "heavy units");
+  if (!fake::launches.empty()) check_launch(heavy, 2, fake::launches.back(), s1, "scheduled decode");
+  CHECK(a.decode(4, s1) == PAD_OK && fake::schedules.size() == sched0 + 1, "light units scheduled");
 
   // one partition: no scratch at all
   Problem one(2, 8, 2, 128, 16, 4);

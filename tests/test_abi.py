@@ -66,6 +66,22 @@ def test_every_declaration_cites_a_passage_or_says_it_has_none():
         assert cites or "no counterpart" in text, f"{name}: its comment names no page section: {text[:120]}"
 
 
+def test_unit_order_only_for_heavy_units(lib):
+    # heavy units (partition tokens x heads per tile >= 32 K) carry the launch's
+    # unit order after the partials: 4 bytes per CTA
+    r = lambda x: -(-x // 256) * 256
+    p = pad.pad_decode_plan(256, 32, 1, 128, 32, 1024, num_splits=0)  # the ragged MQA batch's shape
+    S = p["num_splits"]
+    assert p["partition_tokens"] * p["heads_per_tile"] >= 32768
+    assert p["workspace_bytes"] == r(256 * 32 * S * 128 * 4) + r(256 * 32 * S * 4) + r(p["ctas"] * 4)
+    for shape in ((32, 32, 8, 128, 16, 256), (64, 40, 8, 128, 16, 512)):  # llama8b- and qwen14b-shaped
+        p = pad.pad_decode_plan(*shape, num_splits=0)
+        B, Hq, _, D = shape[:4]
+        S = p["num_splits"]
+        assert p["partition_tokens"] * p["heads_per_tile"] < 32768
+        assert p["workspace_bytes"] == r(B * Hq * S * D * 4) + r(B * Hq * S * 4)
+
+
 def test_stage_timeout_hook_checks_its_argument(lib):
     assert lib.pad_inject_stage_timeout(-2) == pad.PAD_ERR_INVALID_ARG
     assert lib.pad_inject_stage_timeout(256) == pad.PAD_ERR_INVALID_ARG

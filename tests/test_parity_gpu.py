@@ -257,7 +257,7 @@ def test_partition_partials_match_oracle_on_subranges(cuda_device):
     ws = torch.full((plan["workspace_bytes"] // 4,), float("nan"), dtype=torch.float32, device=cuda_device)
     ref_out, ref_lse = oracle.decode_workload(w)
     lse_off = _round256(w.B * w.Hq * S * w.D * 4) // 4
-    assert (lse_off + _round256(w.B * w.Hq * S * 4) // 4) * 4 == plan["workspace_bytes"]
+    assert (lse_off + _round256(w.B * w.Hq * S * 4) // 4) * 4 == plan["workspace_bytes"]  # light units: no order
     assert plan["control_bytes"] == _round256(w.B * w.Hkv * HT * 4)
     for call in range(2):
         out = torch.full((w.B, w.Hq, w.D), float("nan"), dtype=torch.bfloat16, device=cuda_device)
