@@ -96,18 +96,29 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def workload_config(w, plan):
-    import synth  # noqa: F401
+def workload_config(w, args):
+    """The workload both arms run (the same keys in the GPU line and the
+    reference line): its shape, lengths, inputs and the options asked for.  The
+    GPU arm's launch plan and timing method ride beside it, not in it."""
     cfg = {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.D,
            "block_size": w.block_size, "max_blocks_per_seq": w.max_blocks_per_seq,
-           "kv_tokens": w.kv_tokens(), "seq_len_min": int(w.seq_lens.min()), "seq_len_max": int(w.seq_lens.max()),
-           "recipe": w.recipe, "lse": w.want_lse, "seed": w.seed, "pool_blocks": w.num_blocks - 1}
-    if plan is not None:
-        cfg.update({"num_splits": plan["num_splits"], "partition_tokens": plan["partition_tokens"],
-                    "heads_per_tile": plan["heads_per_tile"], "ctas": plan["ctas"]})
-    cfg["l2"] = (f"flushed between steps outside the timed events: {L2_FLUSH_BYTES >> 20} MiB write, "
-                 f"then {L2_FLUSH_BYTES >> 20} MiB read (cold, clean L2)")
+           "kv_tokens": w.kv_tokens(args.window), "seq_len_min": int(w.seq_lens.min()),
+           "seq_len_max": int(w.seq_lens.max()), "recipe": w.recipe, "lse": w.want_lse, "seed": w.seed,
+           "pool_blocks": w.num_blocks - 1, "num_splits_requested": w.num_splits}
+    if args.window:
+        cfg["window"] = args.window
+    if args.sinks:
+        cfg["sinks"] = "one N(0,1) logit per query head"
+    if args.kv_dtype == "e4m3":
+        cfg["kv_cache"] = f"e4m3, k_scale {w.k_scale:g}, v_scale {w.v_scale:g}"
     return cfg
+
+
+def plan_summary(w, plan):
+    return {"num_splits": plan["num_splits"], "partition_tokens": plan["partition_tokens"],
+            "heads_per_tile": plan["heads_per_tile"], "head_tiles": plan["head_tiles"], "ctas": plan["ctas"],
+            "warps_per_cta": plan["warps_per_cta"], "stages": plan["stages"], "stage_tokens": plan["stage_tokens"],
+            "launches_per_step": launches_per_step(w, plan)}
 
 
 def split_scratch_bytes(w, plan, window=0):
@@ -134,18 +145,23 @@ def launches_per_step(w, plan):
     return 2 if plan["workspace_bytes"] > partials else 1
 
 
-def cpu_baseline(w, budget_s, runs_max=50, prefix=None):
+def sink_logits(w, on):
+    """The per-head sink logits --sinks runs with (both arms): seeded N(0,1)."""
+    return np.random.default_rng(w.seed).standard_normal(w.Hq).astype(np.float32) if on else None
+
+
+def cpu_baseline(w, budget_s, runs_max=50, prefix=None, window=0, sinks=None):
     """Time the oracle as it stands on this host's cores on a bounded sample,
     plus a one-thread figure (on the whole batch, or on its first sequences
     when that would take more than a few seconds; `prefix(k)` builds that batch)."""
     import oracle
     threads = oracle.default_threads()
-    bytes_per = w.algorithmic_bytes()
+    bytes_per = w.algorithmic_bytes(window=window, sinks=sinks is not None)
     times = []
     t_all = time.perf_counter()
     while True:
         t0 = time.perf_counter()
-        oracle.decode_workload(w, nthreads=threads)
+        oracle.decode_workload(w, nthreads=threads, window=window, sinks=sinks)
         times.append(time.perf_counter() - t0)
         if time.perf_counter() - t_all > budget_s or len(times) >= runs_max:
             break
@@ -154,9 +170,10 @@ def cpu_baseline(w, budget_s, runs_max=50, prefix=None):
     est1 = med * threads  # rough one-thread time of the whole batch
     w1 = w if est1 <= 4.0 or prefix is None else prefix(max(1, int(w.B * 4.0 / est1)))
     t0 = time.perf_counter()
-    oracle.decode_workload(w1, nthreads=1)
+    oracle.decode_workload(w1, nthreads=1, window=window, sinks=sinks)
     t1 = time.perf_counter() - t0
-    one = {"value": round(w1.algorithmic_bytes() / t1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+    one = {"value": round(w1.algorithmic_bytes(window=window, sinks=sinks is not None) / t1 / 1e9, 4), "unit": "GB/s",
+           "cores": 1,
            "sample": (f"whole {w.name} batch" if w1 is w else f"first {w1.B} of {w.B} {w.name} sequences")
                      + f", one run, {t1 * 1e6:.0f} us"}
     return {"value": round(bytes_per / med / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
@@ -256,12 +273,13 @@ def run_reference(args, rank, world):
         return
     w = synth.config(args.workload, batch=args.batch, compact_pool=args.compact_pool, kv_dtype=args.kv_dtype)
     cb = cpu_baseline(w, args.cpu_seconds, prefix=lambda k: synth.config(
-        args.workload, batch=k, compact_pool=args.compact_pool, kv_dtype=args.kv_dtype))
+        args.workload, batch=k, compact_pool=args.compact_pool, kv_dtype=args.kv_dtype),
+        window=args.window, sinks=sink_logits(w, args.sinks))
     us = cb["us_per_call"]
     line = {"impl": "reference", "metric": metric, "value": cb["value"], "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1e3, 4), "us_per_call": us,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic (seeded generator, no dataset)", "config": workload_config(w, None),
+            "data": "synthetic (seeded generator, no dataset)", "config": workload_config(w, args),
             "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample", "one_thread")},
             "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
@@ -400,8 +418,7 @@ def main():
         flush.fill_(float(i))
         torch.sum(flush_rd, 0, out=flush_acc)
 
-    sinks_dev = (torch.from_numpy(np.random.default_rng(w.seed).standard_normal(w.Hq).astype(np.float32)).to(dev)
-                 if args.sinks else None)
+    sinks_dev = torch.from_numpy(sink_logits(w, True)).to(dev) if args.sinks else None
 
     def decode(q_, tables_, lens_, out_, lse_, stream_):
         # the public one-call API, with the decode options when asked for
@@ -564,11 +581,10 @@ def main():
             "value_mean": round(value_mean, 2), "us_per_call_mean": round(total_ms / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16",
             "data": "synthetic (seeded counter-based generator; no dataset)",
-            "config": {**workload_config(w, plan),
-                       **({"entry": "pad_decode_tcgen05"} if tc else {}),
-                       **({"window": args.window, "kv_tokens": w.kv_tokens(args.window)} if args.window else {}),
-                       **({"sinks": "one N(0,1) logit per query head"} if args.sinks else {}),
-                       **({"kv_cache": f"e4m3, k_scale {w.k_scale:g}, v_scale {w.v_scale:g}"} if fp8 else {})},
+            "config": workload_config(w, args),
+            "plan": {**plan_summary(w, plan), "api": api},
+            "l2": (f"flushed between steps outside the timed events: {L2_FLUSH_BYTES >> 20} MiB write, "
+                   f"then {L2_FLUSH_BYTES >> 20} MiB read (cold, clean L2)"),
             "hbm_frac_of_peak": round(value / peak, 4),
             "us_per_call_min_max": [round(min(step_ms) * 1e3, 2), round(max(step_ms) * 1e3, 2)],
             "roofline": {"kernel": kname, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
@@ -602,7 +618,8 @@ def main():
                                          "(tiny: launch latency only)", **table}
         if world == 1 and not args.no_cpu_baseline:
             cb = cpu_baseline(w, args.cpu_seconds, prefix=lambda k: synth.config(
-                args.workload, batch=k, compact_pool=args.compact_pool, kv_dtype=args.kv_dtype))
+                args.workload, batch=k, compact_pool=args.compact_pool, kv_dtype=args.kv_dtype),
+                window=args.window, sinks=sink_logits(w, args.sinks))
             line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample", "one_thread")}
         print(json.dumps(line), flush=True)
     if world > 1:
