@@ -523,7 +523,7 @@ void bind_buffers(Prepared &pr, void *partials, void *control) {
   char *base = static_cast<char *>(partials);
   pr.p.o_part = base != nullptr ? reinterpret_cast<float *>(base + pr.ws.o_part) : nullptr;
   pr.p.lse_part = base != nullptr ? reinterpret_cast<float *>(base + pr.ws.lse_part) : nullptr;
-  pr.p.order = base != nullptr && pr.ordered ? reinterpret_cast<const uint32_t *>(base + pr.ws.order) : nullptr;
+  pr.p.order = base != nullptr && pr.ordered ? reinterpret_cast<uint32_t *>(base + pr.ws.order) : nullptr;
   pr.p.counters = pr.cl.total > 0 ? reinterpret_cast<uint32_t *>(static_cast<char *>(control) + pr.cl.counters)
                                   : nullptr;
 }

@@ -177,7 +177,7 @@ struct PartitionParams {
   float *lse_part;     // [B, Hq, S] fp32 (natural log)
   // The launch's unit order, longest first (written by schedule_kernel just
   // before the launch): CTA i runs unit order[i].  Null: CTA i runs unit i.
-  const uint32_t *order;
+  uint32_t *order;
   uint32_t *counters;  // [B * Hkv * HT] partitions finished per (b, kv head, head tile)
   uint32_t *err;
   LaunchWitness *witness;  // written by block 0 of every launch

@@ -722,7 +722,7 @@ __global__ void __launch_bounds__(kScheduleThreads) schedule_kernel(const __grid
     }
   }
   __syncthreads();
-  uint32_t *order = const_cast<uint32_t *>(p.order);
+  uint32_t *order = p.order;
   for (int i = tid; i < npair; i += kScheduleThreads) {
     const uint32_t slot = atomicAdd(&next[bucket(i)], 1u);
     const int b = i / p.S, s = i % p.S;

@@ -3,11 +3,13 @@ allocate device memory (a runtime whose memory is planned up front, a thread
 that may not take the allocator's locks or absorb the synchronisation an
 allocation can cause).  Its split scratch is a fixed array inside the library.
 
-Checked through the C ABI against the CPU oracle, within the parity tolerances
-the other GPU tests use, on two calls in a row with different inputs (the shared
-array keeps the first call's partials; the second must not depend on them), and
-after a launch that left merge counters set in the array (the call must clear
-them itself).  This file is named so that pytest collects it last.
+Checked through the C ABI, on two calls in a row with different inputs (the
+shared array keeps the first call's partials; the second must not depend on
+them), against pad_decode's output on the same inputs and against the CPU oracle
+(a bug the two entry points shared would pass the first check only), within the
+parity tolerances the other GPU tests use; and after a launch that left merge
+counters set in the array (the call must clear them itself).  This file is named
+so that pytest collects it last.
 """
 import pytest
 import torch
@@ -15,7 +17,7 @@ import torch
 import oracle
 import synth
 import paged_kv_attention_partition_b200 as pad
-from pad_testing import DeviceWorkload, check_parity, to_f64
+from pad_testing import LSE_RTOL, OUT_ATOL, DeviceWorkload, check_parity, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -30,7 +32,7 @@ def _static(dw, w, splits):
     return out, lse
 
 
-def test_static_scratch_matches_the_oracle_twice(cuda_device):
+def test_static_scratch_matches_pad_decode_and_the_oracle_twice(cuda_device):
     # the first call has one partition per sequence (the array's address is
     # looked up all the same); the next two split and use the array
     w0 = synth.make_workload("na0", 3, 8, 2, 128, 16, [100, 1, 256], seed=60, max_blocks_per_seq=16)
@@ -47,6 +49,14 @@ def test_static_scratch_matches_the_oracle_twice(cuda_device):
         plan = pad.pad_decode_plan(w.B, w.Hq, w.Hkv, w.D, w.block_size, w.max_blocks_per_seq, num_splits=splits)
         assert plan["reduce"] == 1  # the split path, which needs scratch
         out, lse = _static(dw, w, splits)
+        # the existing entry point on the same inputs
+        dec_out, dec_lse = pad.pad_decode(dw.q, dw.k, dw.v, dw.tables, dw.lens, w.scale, num_splits=splits, lse=True)
+        torch.cuda.synchronize()
+        assert (out.float() - dec_out.float()).abs().max().item() <= OUT_ATOL
+        assert torch.equal(torch.isneginf(lse), torch.isneginf(dec_lse))
+        fin = ~torch.isneginf(dec_lse)
+        assert ((lse[fin] - dec_lse[fin]).abs() / dec_lse[fin].abs().clamp_min(1.0)).max().item() <= LSE_RTOL
+        # and the oracle
         ref_out, ref_lse = oracle.decode_workload(w)
         check_parity(to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, f"static {w.name}")
     assert pad.pad_check_device_errors() == 0
