@@ -27,7 +27,10 @@
  * group from that read, and keeps a running max/sum (online softmax) in fp32.
  * When a sequence has more than one non-empty partition, the unit that finishes
  * last merges the partial outputs weighted by their log-sum-exp (the split
- * reduce, folded into the same launch).
+ * reduce, folded into the same launch).  When units are heavy (partition tokens
+ * x heads per tile >= 32768), a one-CTA pass on the same stream first orders
+ * the launch's units longest first from the device-resident lengths, so the
+ * units the GPU dispatches last are the short ones (no host synchronisation).
  *
  * Conventions for every entry point:
  *  - All tensor data pointers are DEVICE pointers owned by the caller.  The
@@ -204,7 +207,11 @@ pad_status pad_decode_ex(const pad_tensor *q, const pad_tensor *k_cache, const p
  * bytes (may be NULL when that is 0, i.e. S == 1); its initial contents do not
  * matter.  It must not be shared by calls that may run concurrently.  Layout
  * (offsets rounded up to 256 bytes): fp32 partial outputs [B, Hq, S, D], each
- * normalised by its own softmax sum, then fp32 partial LSEs [B, Hq, S].  After
+ * normalised by its own softmax sum, then fp32 partial LSEs [B, Hq, S], then --
+ * when the launch orders its units longest first (a unit is heavy: partition
+ * tokens x heads per tile >= 32768, with B * S <= 65536) -- the unit order,
+ * one uint32 per CTA, written on the stream by a one-CTA pass just before the
+ * decode launch.  After
  * a call, the partials of every (b, head) whose sequence had more than one
  * non-empty partition are left in place; partitions past ceil(L_b / P) are
  * neither written nor read.  The small control block (merge counters,
