@@ -82,6 +82,17 @@ def test_unit_order_only_for_heavy_units(lib):
         assert p["workspace_bytes"] == r(B * Hq * S * D * 4) + r(B * Hq * S * 4)
 
 
+def test_unit_order_needs_the_pairs_to_fit_one_cta(lib):
+    # B * S <= 65536 (sequence, partition) pairs: the one-CTA pass handles them;
+    # one more pair and the launch keeps its default order
+    r = lambda x: -(-x // 256) * 256
+    for B, ordered in ((4096, True), (4097, False)):
+        p = pad.pad_decode_plan(B, 32, 1, 128, 16, 2048, num_splits=16)  # P = 2048 tokens x 32 heads
+        assert p["num_splits"] == 16 and B * 16 <= 65536 or not ordered
+        partials = r(B * 32 * 16 * 128 * 4) + r(B * 32 * 16 * 4)
+        assert p["workspace_bytes"] == partials + (r(p["ctas"] * 4) if ordered else 0), (B, ordered)
+
+
 def test_stage_timeout_hook_checks_its_argument(lib):
     assert lib.pad_inject_stage_timeout(-2) == pad.PAD_ERR_INVALID_ARG
     assert lib.pad_inject_stage_timeout(256) == pad.PAD_ERR_INVALID_ARG

@@ -91,3 +91,48 @@ def test_caller_workspace_holds_the_order_after_the_partials(cuda_device):
         work.append(max(0, min((s + 1) * P, L) - s * P))
     buckets = [63 if x <= 0 else (P - x) * 63 // P for x in work]
     assert buckets == sorted(buckets)
+
+
+def test_scheduled_launch_replays_in_a_cuda_graph(cuda_device):
+    # the schedule pass and the decode launch are both captured (scratch exists
+    # after one call outside capture); the replay reads the live lengths
+    w = _case(seed=95)
+    dw = DeviceWorkload(w, cuda_device)
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=cuda_device)
+    lse = torch.empty((w.B, w.Hq), device=cuda_device)
+    s = torch.cuda.Stream(cuda_device)
+    with torch.cuda.stream(s):
+        pad.pad_decode(dw.q, dw.k, dw.v, dw.tables, dw.lens, w.scale, num_splits=2, out=out, lse=lse)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        pad.pad_decode(dw.q, dw.k, dw.v, dw.tables, dw.lens, w.scale, num_splits=2, out=out, lse=lse)
+    # new lengths after capture: the replayed pass orders by them
+    lens2 = np.asarray([4096, 0, 17, 3000, 64, 2049, 1500, 2048], dtype=np.int32)
+    w2 = synth.make_workload("sched", len(lens2), 32, 1, 128, 16, lens2.tolist(), seed=95, max_blocks_per_seq=256)
+    dw.lens.copy_(torch.from_numpy(w2.seq_lens))
+    dw.tables.copy_(torch.from_numpy(w2.block_tables))
+    dw.q.copy_(torch.from_numpy(w2.q).view(torch.bfloat16))
+    dw.k.copy_(torch.from_numpy(w2.k_cache).view(torch.bfloat16))
+    dw.v.copy_(torch.from_numpy(w2.v_cache).view(torch.bfloat16))
+    out.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    ref_out, ref_lse = oracle.decode_workload(w2)
+    check_parity(to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, "scheduled graph replay")
+    assert pad.pad_check_device_errors() == 0
+    del g
+
+
+def test_stalled_scheduled_launch_then_a_clean_call(cuda_device):
+    # the failure-path hook in an ordered launch: partition 0's units give up
+    # uncounted, and the next ordinary call is the oracle's
+    w = _case(seed=96)
+    dw = DeviceWorkload(w, cuda_device)
+    pad.pad_inject_stage_timeout(0)
+    dw.run(num_splits=2)
+    assert pad.pad_check_device_errors() == 0x4
+    out, lse = dw.run(num_splits=2)
+    ref_out, ref_lse = oracle.decode_workload(w)
+    check_parity(to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, "after a stalled ordered launch")
+    assert pad.pad_check_device_errors() == 0
