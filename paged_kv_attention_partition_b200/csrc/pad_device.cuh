@@ -112,6 +112,18 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
   return h;
 }
 
+// The two code pairs of a 32-bit word, low and high half, widened the same way.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t four_codes, uint32_t &lo, uint32_t &hi) {
+  asm("{\n"
+      " .reg .b16 l, h;\n"
+      " mov.b32 {l, h}, %2;\n"
+      " cvt.rn.f16x2.e4m3x2 %0, l;\n"
+      " cvt.rn.f16x2.e4m3x2 %1, h;\n"
+      "}\n"
+      : "=r"(lo), "=r"(hi)
+      : "r"(four_codes));
+}
+
 // Bytes of x selected by `sel` (4 nibbles, byte indices 0-3 of x).
 __device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t sel) { return __byte_perm(x, 0, sel); }
 

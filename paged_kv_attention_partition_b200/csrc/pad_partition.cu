@@ -301,12 +301,38 @@ __global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
   // of V) of this warp's tiles: tile i of token group tg is stage rows
   // 16 (i TG + tg) .. +15.  (E4M3: both operands' matrices 0/1 are tokens
   // 0-7/8-15 of the first 16 bytes, matrices 2/3 the same tokens of the next 16.)
-  uint32_t kb[TPW], kk_key[TPW], vb[TPW], vkey[TPW];
+  // Each lane keeps, per tile and per column block it reads, the offset of its
+  // row's chunk c0 (lane/16 for K and E4M3 V, bit 3 of the lane for bf16 V).
+  // An operand x bytes into the column block is chunk c0 + x/16 with x/16
+  // even, i.e. c0 XOR x/16, and the swizzle XORs the chunk index, so its
+  // address is (stage address + offset) XOR x: one instruction per load,
+  // instead of the swizzle arithmetic (the stage address is a multiple of 128
+  // and an offset has c0's swizzled chunk in bits 4-6 only).  Written as
+  // (offset XOR x) + stage address, the same value, the bf16 32-head tile at
+  // D = 128 (at its 128-register cap) measured 1.5% faster on B200 and the
+  // other measured instances 1-4% slower, so only that tile takes that form.
+  constexpr int EB = F8 ? 1 : 2;                      // bytes per element
+  constexpr int NKB = ROWB / RW;                      // column blocks of a K row
+  constexpr int NVB = (MT * 16 * EB + RW - 1) / RW;   // column blocks of this warp's V rows
+  uint32_t kb[TPW][NKB], vb[TPW][NVB];
+  auto op_addr = [](uint32_t stage, uint32_t off, uint32_t x) -> uint32_t {
+    if constexpr (!F8 && D == 128 && HPT == 32) return (off ^ x) + stage;
+    else return (stage + off) ^ x;
+  };
+  {
+    const int vh0 = dh * MT * 16 * EB / RW;           // first of them
+    const int c0k = lane >> 4, c0v = F8 ? (lane >> 4) : ((lane >> 3) & 1);
 #pragma unroll
-  for (int i = 0; i < TPW; ++i) {
-    const int r0 = 16 * (i * TG + tg) + (lane & 7);
-    row_base(r0 + ((lane >> 3) & 1) * 8, kb[i], kk_key[i]);
-    row_base(r0 + ((F8 ? (lane >> 3) : (lane >> 4)) & 1) * 8, vb[i], vkey[i]);
+    for (int i = 0; i < TPW; ++i) {
+      const int r0 = 16 * (i * TG + tg) + (lane & 7);
+      uint32_t rb, rk;
+      row_base(r0 + ((lane >> 3) & 1) * 8, rb, rk);
+#pragma unroll
+      for (int h = 0; h < NKB; ++h) kb[i][h] = chunk(rb, rk, h, c0k);
+      row_base(r0 + ((F8 ? (lane >> 3) : (lane >> 4)) & 1) * 8, rb, rk);
+#pragma unroll
+      for (int h = 0; h < NVB; ++h) vb[i][h] = chunk(rb, rk, vh0 + h, c0v);
+    }
   }
 
   // Q^T fragments (B operand of S^T = K.Q^T): lane holds head nt*8 + lane/4,
@@ -390,6 +416,7 @@ __global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
 
     uint8_t *sK = smem + (st % NST) * STAGE_BYTES;
     uint8_t *sV = sK + HALF;
+    const uint32_t aK = smem_addr(sK), aV = aK + (uint32_t)HALF;
     const int tb = tu + st * ST;
     if (tb + ST > t1 || tb < tlo) {
       // the first and last stages: V rows outside [tlo, t1) (slots past L_b,
@@ -435,16 +462,13 @@ __global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
 #pragma unroll
           for (int kp = 0; kp < KT / 2; ++kp) {
             uint32_t r[4];
-            const int cb = kp * 32 + (lane >> 4) * 16;
-            ldsm_x4(r, smem_addr(sK + chunk(kb[i], kk_key[i], cb / RW, (cb % RW) >> 4)));
+            ldsm_x4(r, op_addr(aK, kb[i][kp * 32 / RW], kp * 32 % RW));
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
               const int kk = 2 * kp + hf;
               uint32_t a[4];
-              a[0] = e4m3x2_to_f16x2(r[2 * hf]);
-              a[1] = e4m3x2_to_f16x2(r[2 * hf + 1]);
-              a[2] = e4m3x2_to_f16x2(r[2 * hf] >> 16);
-              a[3] = e4m3x2_to_f16x2(r[2 * hf + 1] >> 16);
+              e4m3x4_to_f16x2x2(r[2 * hf], a[0], a[2]);
+              e4m3x4_to_f16x2x2(r[2 * hf + 1], a[1], a[3]);
 #pragma unroll
               for (int nt = 0; nt < NTW; ++nt) mma_16816_f16(sc[kk % NCH][i][nt], a, qf[kk][nt][0], qf[kk][nt][1]);
             }
@@ -453,7 +477,7 @@ __global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
 #pragma unroll
           for (int kk = 0; kk < KT; ++kk) {
             uint32_t a[4];
-            ldsm_x4(a, smem_addr(sK + chunk(kb[i], kk_key[i], kk >> 2, ((kk * 2) & 7) + (lane >> 4))));
+            ldsm_x4(a, op_addr(aK, kb[i][kk * 32 / RW], kk * 32 % RW));
 #pragma unroll
             for (int nt = 0; nt < NTW; ++nt) mma_16816(sc[kk % NCH][i][nt], a, qf[kk][nt][0], qf[kk][nt][1]);
           }
@@ -545,20 +569,16 @@ __global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
         // byte permute pairs the two tokens of each head_dim row.
 #pragma unroll
         for (int mp = 0; mp < MT / 2; ++mp) {
-          const int gm = dh * MT + 2 * mp;
-          const int cb = (gm + (lane >> 4)) * 16;
 #pragma unroll
           for (int i = 0; i < TPW; ++i) {
             uint32_t r[4];
-            ldsm_x4_t(r, smem_addr(sV + chunk(vb[i], vkey[i], cb / RW, (cb % RW) >> 4)));
+            ldsm_x4_t(r, op_addr(aV, vb[i][mp * 32 / RW], mp * 32 % RW));
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
               const uint32_t x0 = byte_perm(r[2 * hf], 0x3120), x1 = byte_perm(r[2 * hf + 1], 0x3120);
               uint32_t a[4];
-              a[0] = e4m3x2_to_f16x2(x0);
-              a[1] = e4m3x2_to_f16x2(x0 >> 16);
-              a[2] = e4m3x2_to_f16x2(x1);
-              a[3] = e4m3x2_to_f16x2(x1 >> 16);
+              e4m3x4_to_f16x2x2(x0, a[0], a[1]);
+              e4m3x4_to_f16x2x2(x1, a[2], a[3]);
 #pragma unroll
               for (int nt = 0; nt < NTW; ++nt) mma_16816_f16(oacc[2 * mp + hf][nt], a, pb[i][nt][0], pb[i][nt][1]);
             }
@@ -566,12 +586,11 @@ __global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
         }
       } else {
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          const int gm = dh * MT + mt;  // m-tile of head_dim rows
+        for (int mt = 0; mt < MT; ++mt) {  // m-tile dh MT + mt of head_dim rows
 #pragma unroll
           for (int i = 0; i < TPW; ++i) {
             uint32_t a[4];
-            ldsm_x4_t(a, smem_addr(sV + chunk(vb[i], vkey[i], gm >> 2, ((gm * 2) & 7) + ((lane >> 3) & 1))));
+            ldsm_x4_t(a, op_addr(aV, vb[i][mt * 32 / RW], mt * 32 % RW));
 #pragma unroll
             for (int nt = 0; nt < NTW; ++nt) mma_16816(oacc[mt][nt], a, pb[i][nt][0], pb[i][nt][1]);
           }
