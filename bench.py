@@ -117,7 +117,8 @@ def workload_config(w, args):
 def plan_summary(w, plan):
     return {"num_splits": plan["num_splits"], "partition_tokens": plan["partition_tokens"],
             "heads_per_tile": plan["heads_per_tile"], "head_tiles": plan["head_tiles"], "ctas": plan["ctas"],
-            "warps_per_cta": plan["warps_per_cta"], "stages": plan["stages"], "stage_tokens": plan["stage_tokens"],
+            "warps_per_cta": plan["warps_per_cta"], "ctas_per_sm": plan["ctas_per_sm"], "stages": plan["stages"],
+            "stage_tokens": plan["stage_tokens"],
             "launches_per_step": launches_per_step(w, plan)}
 
 

@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define PAD_ABI_VERSION 2
+#define PAD_ABI_VERSION 3
 
 typedef enum pad_status {
   PAD_OK = 0,
@@ -96,6 +96,11 @@ typedef struct pad_plan {
   int32_t stage_tokens;      /* tokens per shared-memory pipeline stage */
   int32_t stages;            /* pipeline depth */
   int32_t ctas;              /* CTAs launched: one per unit (B * Hkv * head_tiles * num_splits) */
+  int32_t ctas_per_sm;       /* resident CTAs per SM the launched kernel instance is built for
+                                (its launch bound): fixed per head_dim, heads per tile and
+                                cache type, except the E4M3 8-head tile at D = 128, which
+                                takes its six-per-SM build for launches of at least four
+                                full waves at five per SM (2 for the tcgen05 kernel) */
   int32_t reduce;            /* 1 when partitions may need merging (S > 1) */
   int64_t workspace_bytes;   /* partial-output scratch (0 when S == 1) */
   int64_t control_bytes;     /* merge counters, 0 when S == 1 (library-owned except
@@ -349,6 +354,7 @@ typedef struct pad_launch_witness {
   int32_t partition_tokens;  /* P it was launched with */
   int32_t ctas;              /* grid size */
   int32_t warps;             /* warps per CTA it was compiled for */
+  int32_t ctas_per_sm;       /* resident CTAs per SM it was compiled for (its launch bound) */
 } pad_launch_witness;
 
 pad_status pad_last_launch(pad_launch_witness *witness);

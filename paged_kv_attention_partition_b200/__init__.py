@@ -39,7 +39,8 @@ class PadPlan(ctypes.Structure):
     _fields_ = [("num_splits", ctypes.c_int32), ("partition_tokens", ctypes.c_int32),
                 ("heads_per_tile", ctypes.c_int32), ("head_tiles", ctypes.c_int32),
                 ("warps_per_cta", ctypes.c_int32), ("stage_tokens", ctypes.c_int32),
-                ("stages", ctypes.c_int32), ("ctas", ctypes.c_int32), ("reduce", ctypes.c_int32),
+                ("stages", ctypes.c_int32), ("ctas", ctypes.c_int32), ("ctas_per_sm", ctypes.c_int32),
+                ("reduce", ctypes.c_int32),
                 ("workspace_bytes", ctypes.c_int64), ("control_bytes", ctypes.c_int64)]
 
     def as_dict(self) -> dict:
@@ -56,7 +57,7 @@ class PadLaunchWitness(ctypes.Structure):
     """pad_launch_witness: what the most recent launch recorded from inside the kernel."""
     _fields_ = [(n, ctypes.c_int32) for n in ("kernel", "head_dim", "heads_per_tile", "kv_dtype", "stages",
                                                   "stage_tokens", "num_splits", "partition_tokens", "ctas",
-                                                  "warps")]
+                                                  "warps", "ctas_per_sm")]
 
 
 class PadError(RuntimeError):

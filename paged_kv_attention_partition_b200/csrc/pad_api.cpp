@@ -133,12 +133,12 @@ void log_plan(const Shape &s, int32_t requested, int device, const pad_plan &p, 
   char line[512];
   snprintf(line, sizeof line,
            "pad: plan B=%lld Hq=%lld Hkv=%lld D=%lld bs=%lld capacity=%lld kv=%s num_splits=%d device=%d -> "
-           "kernel=%s S=%d P=%d heads_per_tile=%d head_tiles=%d stages=%dx%d warps=%d ctas=%d "
+           "kernel=%s S=%d P=%d heads_per_tile=%d head_tiles=%d stages=%dx%d warps=%d ctas=%d ctas_per_sm=%d "
            "workspace_bytes=%lld control_bytes=%lld\n",
            (long long)s.B, (long long)s.Hq, (long long)s.Hkv, (long long)s.D, (long long)s.bs,
            (long long)(s.W * s.bs), s.fp8 ? "e4m3" : "bf16", requested, device, umma ? "tcgen05" : "partition",
            p.num_splits, p.partition_tokens, p.heads_per_tile, p.head_tiles, p.stages, p.stage_tokens,
-           p.warps_per_cta, p.ctas, (long long)p.workspace_bytes, (long long)p.control_bytes);
+           p.warps_per_cta, p.ctas, p.ctas_per_sm, (long long)p.workspace_bytes, (long long)p.control_bytes);
   static std::mutex mu;
   static std::set<std::string> seen;
   std::lock_guard<std::mutex> lock(mu);
@@ -178,6 +178,8 @@ void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan, b
   plan->stages = umma ? pad::umma_stages() : pad::partition_stages((int)s.D, hpt, s.fp8);
   // one CTA per unit (both kernels)
   plan->ctas = (int32_t)(units > 0x7fffffffll ? 0x7fffffffll : units);
+  plan->ctas_per_sm = umma ? pad::kUmmaCtasPerSm
+                           : pad::ctas_per_sm_choice((int)s.D, hpt, s.fp8, units, sm_count(device < 0 ? 0 : device));
   plan->reduce = S > 1 ? 1 : 0;
   plan->workspace_bytes =
       (int64_t)pad::workspace_layout(s.B, s.Hq, S, s.D, units, pad::schedules_units(s.B, S, P, hpt)).total;
@@ -540,7 +542,8 @@ pad_status run(const Prepared &pr, cudaStream_t stream) {
   cudaError_t e = pr.p.order != nullptr ? pad::launch_schedule(pr.p, stream) : cudaSuccess;
   if (e != cudaSuccess) return cuda_fail(e, "unit schedule launch");
   e = pr.umma ? pad::launch_umma(pr.p, pr.plan.ctas, stream)
-              : pad::launch_partition(pr.p, pr.D, pr.plan.heads_per_tile, pr.kv_fp8, pr.plan.ctas, stream);
+              : pad::launch_partition(pr.p, pr.D, pr.plan.heads_per_tile, pr.kv_fp8, pr.plan.ctas,
+                                      pr.plan.ctas_per_sm, stream);
   if (!pr.umma) g_stall_partition = -1;  // the test hook is one-shot
   return e == cudaSuccess ? PAD_OK : cuda_fail(e, "partition kernel launch");
 }
@@ -722,6 +725,7 @@ pad_status pad_last_launch(pad_launch_witness *w) {
   w->partition_tokens = h.partition_tokens;
   w->ctas = h.ctas;
   w->warps = h.warps;
+  w->ctas_per_sm = h.ctas_per_sm;
   return PAD_OK;
 }
 

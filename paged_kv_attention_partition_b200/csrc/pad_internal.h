@@ -105,6 +105,21 @@ __host__ __device__ constexpr int ctas_per_sm_for(int D, int hpt, bool f8 = fals
   return ctas_per_sm_for(D, hpt, f8, warps_for(D, hpt, f8));
 }
 
+// Resident CTAs per SM a launch is built for (the kernel's launch bound).
+// One instantiation has a second, denser build: the E4M3 8-head tile at
+// D = 128 also runs at six CTAs per SM (80 registers instead of 88).  On B200
+// that build measured 2.5-3.5% faster on launches of at least four full waves
+// at five CTAs per SM and 4-13% slower on shorter ones (GQA batches of
+// 1024-16384 units: there the CTAs' own start and finish latency weighs more
+// than the extra resident warps), so the host picks it by the unit count.
+__host__ __device__ constexpr bool has_dense_build(int D, int hpt, bool f8) { return f8 && D == 128 && hpt == 8; }
+constexpr int kDenseCtasPerSm = 6;
+constexpr int kDenseMinWaves = 4;
+inline int ctas_per_sm_choice(int D, int hpt, bool f8, int64_t units, int sms) {
+  const int base = ctas_per_sm_for(D, hpt, f8);
+  return has_dense_build(D, hpt, f8) && units >= (int64_t)kDenseMinWaves * base * sms ? kDenseCtasPerSm : base;
+}
+
 // Shared memory of one CTA (from a 1024-byte aligned base): the K/V ring,
 // reused after the last stage for the token groups' merge (O^T, m, l) and then
 // for the split merge's weight table; then one mbarrier per stage and two flag
@@ -135,7 +150,8 @@ inline int max_heads_per_tile(int D) { return D <= 128 ? 32 : 16; }
 
 // What a launch records from inside the kernel (pad_last_launch).
 struct LaunchWitness {
-  int32_t kernel, head_dim, heads_per_tile, kv_dtype, stages, stage_tokens, num_splits, partition_tokens, ctas, warps;
+  int32_t kernel, head_dim, heads_per_tile, kv_dtype, stages, stage_tokens, num_splits, partition_tokens, ctas, warps,
+      ctas_per_sm;
 };
 
 struct PartitionParams {
@@ -237,8 +253,11 @@ inline ControlLayout control_layout(int64_t B, int64_t Hkv, int64_t HT, int64_t 
   return c;
 }
 
+// Launches the partition kernel instance for (D, heads_per_tile, cache type)
+// built for `ctas_per_sm` resident CTAs per SM (ctas_per_sm_choice); an
+// instance that does not exist is cudaErrorInvalidValue.
 cudaError_t launch_partition(const PartitionParams &p, int D, int heads_per_tile, bool kv_fp8, int grid,
-                             cudaStream_t s);
+                             int ctas_per_sm, cudaStream_t s);
 // The tcgen05 kernel (pad_umma.cu) takes 32-head tiles at head_dim 128 with
 // pages of at least 8 tokens (its K/V boxes are 8 rows of one page).
 inline bool umma_eligible(int D, int hpt, int block_size) { return D == 128 && hpt == 32 && block_size >= 8; }
@@ -246,6 +265,7 @@ cudaError_t launch_umma(const PartitionParams &p, int grid, cudaStream_t s);
 int umma_stages();
 constexpr int kUmmaStageTokens = 128;
 constexpr int kUmmaWarps = 6;
+constexpr int kUmmaCtasPerSm = 2;
 
 // Rows of one TMA box: a page, or a stage's worth of rows of a larger page.
 inline int box_rows(int block_size, int D, int hpt, bool f8) {

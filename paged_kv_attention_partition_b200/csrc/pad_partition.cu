@@ -106,11 +106,11 @@ __device__ bool wait_stage(uint32_t bar, uint32_t parity, uint32_t *err, uint64_
 // at the start or at the exits, or a hook of its own) changed the 32-head
 // instances' schedules at their 128-register cap and cost the ragged MQA batch
 // 6-10% on B200; as this one call it is within 1% of neither.
-template <int D, int HPT, bool F8, int NST, int ST>
+template <int D, int HPT, bool F8, int NST, int ST, int CPS>
 __device__ __noinline__ bool unit_exit(const PartitionParams &p, int s, uint64_t *spare) {
   if (blockIdx.x == 0 && threadIdx.x == 0)
     *p.witness = LaunchWitness{1, D, HPT, F8 ? (int32_t)PAD_FP8_E4M3 : (int32_t)PAD_BF16, NST, ST, p.S, p.P,
-                               (int32_t)gridDim.x, (int32_t)(blockDim.x / 32)};
+                               (int32_t)gridDim.x, (int32_t)(blockDim.x / 32), CPS};
   if (s != p.stall_partition || spare == nullptr) return false;
   if (threadIdx.x == 0) {
     const uint32_t never = smem_addr(spare);
@@ -120,9 +120,8 @@ __device__ __noinline__ bool unit_exit(const PartitionParams &p, int s, uint64_t
   return true;
 }
 
-template <int D, int HPT, bool F8, int NW, bool ORDERED>
-__global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
-    partition_kernel(const __grid_constant__ PartitionParams p) {
+template <int D, int HPT, bool F8, int NW, bool ORDERED, int CPS>
+__global__ void __launch_bounds__(NW * 32, CPS) partition_kernel(const __grid_constant__ PartitionParams p) {
   constexpr int NTH = NW * 32;             // threads of the CTA
   constexpr SmemPlan SP = smem_plan_for(D, HPT, F8, NW);
   constexpr int NST = SP.stages;
@@ -233,7 +232,7 @@ __global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
       if (p.lse != nullptr && tid < gl)
         p.lse[b * p.lse_sb + (int64_t)(h0 + tid) * p.lse_sh] = p.sinks != nullptr ? p.sinks[h0 + tid] : -INFINITY;
     }
-    unit_exit<D, HPT, F8, NST, ST>(p, s, nullptr);
+    unit_exit<D, HPT, F8, NST, ST, CPS>(p, s, nullptr);
     return;  // pages wholly outside [lo, L) are never read
   }
   const int s_first = lo / p.P;                      // first non-empty partition of sequence b
@@ -689,7 +688,7 @@ __global__ void __launch_bounds__(NW * 32, ctas_per_sm_for(D, HPT, F8, NW))
       if (d == 0) p.lse_part[row] = lse_nat;
     }
   }
-  if (unit_exit<D, HPT, F8, NST, ST>(p, s, full + 12) || ns == 1) return;
+  if (unit_exit<D, HPT, F8, NST, ST, CPS>(p, s, full + 12) || ns == 1) return;
   if (claim_last_partition(p, b, kvh, ht, ns, flag))
     merge_partials<D, NTH>(p, b, h0, gl, s_first, ns, reinterpret_cast<float *>(smem));  // the ring is free
 }
@@ -755,7 +754,7 @@ cudaError_t launch_schedule(const PartitionParams &p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-template <int D, int HPT, bool F8, bool ORDERED>
+template <int D, int HPT, bool F8, bool ORDERED, int CPS>
 static cudaError_t launch_o(const PartitionParams &p, int grid, cudaStream_t stream) {
   static std::atomic<uint64_t> attr_done{0};
   constexpr int NW = warps_for(D, HPT, F8);
@@ -765,39 +764,51 @@ static cudaError_t launch_o(const PartitionParams &p, int grid, cudaStream_t str
   if (e != cudaSuccess) return e;
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_done.load(std::memory_order_acquire) & bit)) {
-    e = cudaFuncSetAttribute(partition_kernel<D, HPT, F8, NW, ORDERED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)SP.total);
+    e = cudaFuncSetAttribute(partition_kernel<D, HPT, F8, NW, ORDERED, CPS>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SP.total);
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(bit, std::memory_order_acq_rel);
   }
-  partition_kernel<D, HPT, F8, NW, ORDERED><<<grid, NW * 32, SP.total, stream>>>(p);
+  partition_kernel<D, HPT, F8, NW, ORDERED, CPS><<<grid, NW * 32, SP.total, stream>>>(p);
   return cudaGetLastError();
 }
 
+template <int D, int HPT, bool F8, int CPS>
+static cudaError_t launch_c(const PartitionParams &p, int grid, cudaStream_t stream) {
+  return p.order != nullptr ? launch_o<D, HPT, F8, true, CPS>(p, grid, stream)
+                            : launch_o<D, HPT, F8, false, CPS>(p, grid, stream);
+}
+
 template <int D, int HPT, bool F8>
-static cudaError_t launch_t(const PartitionParams &p, int grid, cudaStream_t stream) {
-  return p.order != nullptr ? launch_o<D, HPT, F8, true>(p, grid, stream) : launch_o<D, HPT, F8, false>(p, grid, stream);
+static cudaError_t launch_t(const PartitionParams &p, int grid, int ctas_per_sm, cudaStream_t stream) {
+  if constexpr (has_dense_build(D, HPT, F8)) {
+    if (ctas_per_sm == kDenseCtasPerSm) return launch_c<D, HPT, F8, kDenseCtasPerSm>(p, grid, stream);
+  }
+  constexpr int base = ctas_per_sm_for(D, HPT, F8);
+  if (ctas_per_sm != base) return cudaErrorInvalidValue;
+  return launch_c<D, HPT, F8, base>(p, grid, stream);
 }
 
 template <bool F8>
-static cudaError_t launch_f(const PartitionParams &p, int D, int heads_per_tile, int grid, cudaStream_t s) {
+static cudaError_t launch_f(const PartitionParams &p, int D, int heads_per_tile, int grid, int cps, cudaStream_t s) {
   switch (D * 64 + heads_per_tile) {
-    case 64 * 64 + 8: return launch_t<64, 8, F8>(p, grid, s);
-    case 64 * 64 + 16: return launch_t<64, 16, F8>(p, grid, s);
-    case 64 * 64 + 32: return launch_t<64, 32, F8>(p, grid, s);
-    case 128 * 64 + 8: return launch_t<128, 8, F8>(p, grid, s);
-    case 128 * 64 + 16: return launch_t<128, 16, F8>(p, grid, s);
-    case 128 * 64 + 32: return launch_t<128, 32, F8>(p, grid, s);
-    case 256 * 64 + 8: return launch_t<256, 8, F8>(p, grid, s);
-    case 256 * 64 + 16: return launch_t<256, 16, F8>(p, grid, s);
+    case 64 * 64 + 8: return launch_t<64, 8, F8>(p, grid, cps, s);
+    case 64 * 64 + 16: return launch_t<64, 16, F8>(p, grid, cps, s);
+    case 64 * 64 + 32: return launch_t<64, 32, F8>(p, grid, cps, s);
+    case 128 * 64 + 8: return launch_t<128, 8, F8>(p, grid, cps, s);
+    case 128 * 64 + 16: return launch_t<128, 16, F8>(p, grid, cps, s);
+    case 128 * 64 + 32: return launch_t<128, 32, F8>(p, grid, cps, s);
+    case 256 * 64 + 8: return launch_t<256, 8, F8>(p, grid, cps, s);
+    case 256 * 64 + 16: return launch_t<256, 16, F8>(p, grid, cps, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_partition(const PartitionParams &p, int D, int heads_per_tile, bool kv_fp8, int grid,
-                             cudaStream_t s) {
+                             int ctas_per_sm, cudaStream_t s) {
   if (heads_per_tile > max_heads_per_tile(D)) return cudaErrorInvalidValue;
-  return kv_fp8 ? launch_f<true>(p, D, heads_per_tile, grid, s) : launch_f<false>(p, D, heads_per_tile, grid, s);
+  return kv_fp8 ? launch_f<true>(p, D, heads_per_tile, grid, ctas_per_sm, s)
+                : launch_f<false>(p, D, heads_per_tile, grid, ctas_per_sm, s);
 }
 
 cudaError_t device_witness(int device, LaunchWitness **ptr) {

@@ -223,7 +223,7 @@ static_assert(2 * kHalfBytes >= kHeads * kMaxSplits * 4, "merge weights fit the 
 //   -> V buffer refilled with V(c+1)
 // The MMA thread issues S(0), then PV(c), S(c+1) for each c, so K(c+1) and
 // V(c+1) stream while the softmax works on chunk c.
-__global__ void __launch_bounds__(kUmmaThreads, 2) umma_kernel(const __grid_constant__ PartitionParams p) {
+__global__ void __launch_bounds__(kUmmaThreads, kUmmaCtasPerSm) umma_kernel(const __grid_constant__ PartitionParams p) {
   using SM = UmmaSmem;
   static_assert(SM::total <= (uint32_t)kSmemBudget, "shared-memory plan over budget");
   extern __shared__ uint8_t smem_raw[];
@@ -241,7 +241,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 2) umma_kernel(const __grid_cons
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (blockIdx.x == 0 && tid == 0)  // which kernel ran, and with what plan
-    *p.witness = LaunchWitness{2, kD, kHeads, (int32_t)PAD_BF16, 1, kChunk, p.S, p.P, (int32_t)gridDim.x, kUmmaWarps};
+    *p.witness = LaunchWitness{2, kD, kHeads, (int32_t)PAD_BF16, 1, kChunk, p.S, p.P, (int32_t)gridDim.x, kUmmaWarps,
+                               kUmmaCtasPerSm};
   // Unit order as in partition_kernel: p.order (longest units first) when the
   // launch schedules its units, else partition index descending, outermost.
   uint32_t u = p.order != nullptr ? __ldg(p.order + blockIdx.x) : blockIdx.x;

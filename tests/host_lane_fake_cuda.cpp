@@ -49,7 +49,7 @@ cudaError_t launch_result = cudaSuccess;
 std::vector<std::string> events;  // "malloc N", "free", "sync", "devsync", "memset N"
 struct Launch {
   pad::PartitionParams p;
-  int D, hpt, grid;
+  int D, hpt, grid, ctas_per_sm;
   bool fp8, umma;
   cudaStream_t stream;
 };
@@ -232,11 +232,15 @@ cudaError_t device_witness(int, LaunchWitness **ptr) {
   *ptr = &fake::witness;
   return cudaSuccess;
 }
-cudaError_t launch_partition(const PartitionParams &p, int D, int hpt, bool f8, int grid, cudaStream_t s) {
+cudaError_t launch_partition(const PartitionParams &p, int D, int hpt, bool f8, int grid, int cps, cudaStream_t s) {
   if (fake::launch_result != cudaSuccess) return fake::launch_result;
-  fake::launches.push_back({p, D, hpt, grid, f8, false, s});
+  // the instances the kernel module has: the fixed residency, and the dense
+  // build of the E4M3 8-head tile at D = 128
+  if (cps != ctas_per_sm_for(D, hpt, f8) && !(has_dense_build(D, hpt, f8) && cps == kDenseCtasPerSm))
+    return cudaErrorInvalidValue;
+  fake::launches.push_back({p, D, hpt, grid, cps, f8, false, s});
   fake::witness = LaunchWitness{1, D, hpt, f8 ? (int32_t)PAD_FP8_E4M3 : (int32_t)PAD_BF16, stages_for(D, hpt, f8),
-                                stage_tokens_for(D, hpt, f8), p.S, p.P, grid, warps_for(D, hpt, f8)};
+                                stage_tokens_for(D, hpt, f8), p.S, p.P, grid, warps_for(D, hpt, f8), cps};
   return cudaSuccess;
 }
 cudaError_t launch_schedule(const PartitionParams &p, cudaStream_t s) {
@@ -246,8 +250,9 @@ cudaError_t launch_schedule(const PartitionParams &p, cudaStream_t s) {
 }
 cudaError_t launch_umma(const PartitionParams &p, int grid, cudaStream_t s) {
   if (fake::launch_result != cudaSuccess) return fake::launch_result;
-  fake::launches.push_back({p, 128, 32, grid, false, true, s});
-  fake::witness = LaunchWitness{2, 128, 32, (int32_t)PAD_BF16, 1, kUmmaStageTokens, p.S, p.P, grid, kUmmaWarps};
+  fake::launches.push_back({p, 128, 32, grid, kUmmaCtasPerSm, false, true, s});
+  fake::witness = LaunchWitness{2, 128, 32, (int32_t)PAD_BF16, 1, kUmmaStageTokens, p.S, p.P, grid, kUmmaWarps,
+                                kUmmaCtasPerSm};
   return cudaSuccess;
 }
 }  // namespace pad
@@ -329,7 +334,8 @@ static void check_launch(const Problem &pr, int32_t splits, const fake::Launch &
   const pad::PartitionParams &p = L.p;
   CHECK(L.grid == pl.ctas && (uint32_t)pl.ctas == p.n_units, "%s: grid %d, plan %d", what, L.grid, pl.ctas);
   CHECK(L.stream == s, "%s: launched on another stream", what);
-  CHECK(L.D == pr.D && L.hpt == pl.heads_per_tile && L.fp8 == pr.fp8, "%s: kernel instance", what);
+  CHECK(L.D == pr.D && L.hpt == pl.heads_per_tile && L.fp8 == pr.fp8 && L.ctas_per_sm == pl.ctas_per_sm,
+        "%s: kernel instance", what);
   CHECK(p.S == pl.num_splits && p.P == pl.partition_tokens && p.HT == pl.head_tiles, "%s: plan fields", what);
   CHECK(p.B == pr.B && p.Hq == pr.Hq && p.Hkv == pr.Hkv && p.g == pr.Hq / pr.Hkv, "%s: sizes", what);
   CHECK((1 << p.bs_log2) == pr.bs && p.max_blocks == pr.W && p.num_blocks == pr.NB, "%s: table sizes", what);
@@ -405,8 +411,9 @@ static void scenarios() {
   CHECK(fake::library_live() == 2, "partials and control buffers: %d live", fake::library_live());
   pad_launch_witness w;
   CHECK(pad_last_launch(&w) == PAD_OK && w.kernel == 1 && w.num_splits == a.plan(4).num_splits &&
-            w.ctas == a.plan(4).ctas,
+            w.ctas == a.plan(4).ctas && w.ctas_per_sm == a.plan(4).ctas_per_sm && w.ctas_per_sm == 3,
         "witness read back");
+
 
   // the same shape again: no new allocation
   size_t ev = fake::events.size();
@@ -582,6 +589,21 @@ static void scenarios() {
   CHECK(pad_release_workspace(-1) == PAD_OK && fake::library_live() == 0, "release left %d buffers",
         fake::library_live());
   CHECK(a.decode(4, s1) == PAD_OK && fake::library_live() == 2, "decode after release");
+
+  // the E4M3 8-head tile at D = 128: its six-per-SM build from four full
+  // waves at five per SM (4 * 5 * 148 = 2960 units) on, the five-per-SM one below
+  pad_launch_witness w2;
+  Problem e_few(23, 8, 8, 128, 16, 16, true), e_many(24, 8, 8, 128, 16, 16, true);  // 2944 / 3072 units at S = 16
+  CHECK(e_few.plan(16).ctas == 2944 && e_few.plan(16).ctas_per_sm == 5, "E4M3 8-head, 2944 units: %d per SM",
+        e_few.plan(16).ctas_per_sm);
+  CHECK(e_many.plan(16).ctas == 3072 && e_many.plan(16).ctas_per_sm == 6, "E4M3 8-head, 3072 units: %d per SM",
+        e_many.plan(16).ctas_per_sm);
+  CHECK(Problem(24, 8, 8, 128, 16, 16).plan(16).ctas_per_sm == 3, "bf16 8-head: one residency");
+  CHECK(e_many.decode(16, s1) == PAD_OK, "dense E4M3 decode: %s", pad_last_error());
+  if (!fake::launches.empty()) check_launch(e_many, 16, fake::launches.back(), s1, "dense E4M3 decode");
+  CHECK(pad_last_launch(&w2) == PAD_OK && w2.ctas_per_sm == 6, "dense build witnessed");
+  CHECK(e_few.decode(16, s1) == PAD_OK, "E4M3 decode: %s", pad_last_error());
+  if (!fake::launches.empty()) check_launch(e_few, 16, fake::launches.back(), s1, "E4M3 decode");
   CHECK(fake::encoder_violations.empty(), "encoder rule broken: %s",
         fake::encoder_violations.empty() ? "" : fake::encoder_violations[0].c_str());
 }

@@ -108,7 +108,7 @@ def test_library_is_built_for_sm100a():
 def test_status_strings(lib):
     assert pad.pad_status_string(0) == "PAD_OK"
     assert pad.pad_status_string(5) == "PAD_ERR_DEVICE_CHECK"
-    assert pad.pad_abi_version() == 2
+    assert pad.pad_abi_version() == 3
 
 
 def test_plan_follows_the_partition_rule(lib):

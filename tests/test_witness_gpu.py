@@ -10,9 +10,10 @@ path on both targets", opening summary) would show here.
 import pytest
 import torch
 
+import oracle
 import synth
 import paged_kv_attention_partition_b200 as pad
-from pad_testing import DeviceWorkload
+from pad_testing import DeviceWorkload, check_parity, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -38,7 +39,7 @@ def test_partition_kernel_runs_the_planned_shape(cuda_device, shape):
     assert got["kernel"] == 1
     assert got["head_dim"] == D
     assert got["kv_dtype"] == (pad.PAD_FP8_E4M3 if kv == "e4m3" else pad.PAD_BF16)
-    for key in ("heads_per_tile", "stages", "stage_tokens", "num_splits", "partition_tokens", "ctas"):
+    for key in ("heads_per_tile", "stages", "stage_tokens", "num_splits", "partition_tokens", "ctas", "ctas_per_sm"):
         assert got[key] == plan[key], (key, got, plan)
     assert got["warps"] == plan["warps_per_cta"], (got, plan)
 
@@ -48,7 +49,7 @@ def test_tcgen05_entry_runs_the_tcgen05_kernel(cuda_device):
     DeviceWorkload(w, cuda_device).run(num_splits=4, entry=pad.pad_decode_tcgen05)
     got = pad.pad_last_launch()
     assert (got["kernel"], got["head_dim"], got["heads_per_tile"], got["kv_dtype"]) == (2, 128, 32, pad.PAD_BF16)
-    assert got["num_splits"] == 4 and got["ctas"] == 4 * 1 * 1 * 4 and got["warps"] == 6
+    assert got["num_splits"] == 4 and got["ctas"] == 4 * 1 * 1 * 4 and got["warps"] == 6 and got["ctas_per_sm"] == 2
 
 
 def test_static_scratch_and_caller_workspace_run_the_partition_kernel(cuda_device):
@@ -62,3 +63,22 @@ def test_static_scratch_and_caller_workspace_run_the_partition_kernel(cuda_devic
     pad.pad_decode_with_workspace(dw.q, dw.k, dw.v, dw.tables, dw.lens, w.scale, 4, out, None, ws)
     got = pad.pad_last_launch()
     assert got["kernel"] == 1 and got["num_splits"] == plan["num_splits"]
+
+
+@pytest.mark.parametrize("dense", [False, True], ids=["below", "at"])
+def test_e4m3_8_head_tile_takes_its_dense_build_from_four_waves(cuda_device, dense):
+    # Qwen3-14B-shaped heads (40 / 8, one 8-head tile per KV head) at S = 16:
+    # 128 units per sequence.  From four full waves at five CTAs per SM on,
+    # the plan takes the six-per-SM build; one sequence fewer stays at five.
+    # Either way the result is the oracle's.
+    sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
+    B = -(-4 * 5 * sms // 128) - (0 if dense else 1)
+    lens = [int(x) for x in synth.uniform_int(B, 1, 256, 90, synth.S_LENS)]
+    w = synth.make_workload("wit_dense", B, 40, 8, 128, 16, lens, seed=91, max_blocks_per_seq=16, kv_dtype="e4m3")
+    plan = pad.pad_decode_plan(B, 40, 8, 128, 16, 16, num_splits=16, kv_dtype="e4m3")
+    assert plan["ctas"] == B * 128 and (plan["ctas"] >= 4 * 5 * sms) == dense
+    out, lse = DeviceWorkload(w, cuda_device).run(num_splits=16)
+    got = pad.pad_last_launch()
+    assert got["ctas_per_sm"] == plan["ctas_per_sm"] == (6 if dense else 5), (got, plan)
+    ref_out, ref_lse = oracle.decode_workload(w)
+    check_parity(to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, f"e4m3 8-head, {plan['ctas_per_sm']} per SM")
