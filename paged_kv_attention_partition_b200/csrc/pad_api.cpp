@@ -107,9 +107,13 @@ int sm_count(int device) {
 // grows with the head group, so larger groups get longer partitions), and is
 // halved, down to max(64, 16 g) (the split scratch a partition writes, g * D *
 // 4 bytes, stays under 1/16 of the K/V bytes it streams, 4 * D * P), while the
-// batch would give fewer than two waves of CTAs on this device: a small batch
-// still fills every SM.  Measured on B200 this picks the best of 64..8192-token
-// partitions for the llama8b (512) and ragged_mqa (2048) batches.  At most
+// batch would give fewer than three units per SM of this device: a small batch
+// still spreads over every SM.  Measured on B200 this picks the best of
+// 64..8192-token partitions for the llama8b (512) and ragged_mqa (2048)
+// batches, and for GQA batches of 1-16 sequences of 4096-8192 tokens the best
+// or within 8% of it (fewer, longer units win there: each unit's start, the
+// merge of its warps and its partial are fixed costs, and about three units
+// per SM keep the SMs busy while leaving them few).  At most
 // kMaxSplits partitions per sequence.  One CTA per unit; units past a
 // sequence's length exit at once.
 // PAD_LOG=1: one line on stderr for each distinct (shape, request, device,
@@ -145,6 +149,8 @@ void log_plan(const Shape &s, int32_t requested, int device, const pad_plan &p, 
   if (seen.insert(line).second) fputs(line, stderr);
 }
 
+constexpr int kSplitUnitsPerSm = 3;  // the automatic split halves P until the launch has this many units per SM
+
 void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan, bool tcgen05 = false) {
   const int64_t C = s.W * s.bs;
   int hpt = s.g <= 8 ? 8 : (s.g <= 16 ? 16 : 32);
@@ -157,10 +163,9 @@ void make_plan(const Shape &s, int32_t num_splits, int device, pad_plan *plan, b
     const int64_t p_floor = round_up(16 * s.g > 64 ? 16 * s.g : 64, 64);
     P = 512;
     while (P < 64 * s.g) P *= 2;
-    const int64_t slots = (int64_t)sm_count(device < 0 ? 0 : device) *
-                          pad::ctas_per_sm_for((int)s.D, hpt, false);
+    const int64_t min_units = (int64_t)kSplitUnitsPerSm * sm_count(device < 0 ? 0 : device);
     const int64_t pairs = s.B * s.Hkv * HT;
-    while (P / 2 >= p_floor && P / 2 >= s.bs && pairs * ((C + P - 1) / P) < 2 * slots) P /= 2;
+    while (P / 2 >= p_floor && P / 2 >= s.bs && pairs * ((C + P - 1) / P) < min_units) P /= 2;
     P = round_up(P, s.bs);
   }
   if (P > round_up(C, s.bs)) P = round_up(C, s.bs);

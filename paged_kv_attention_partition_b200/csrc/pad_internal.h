@@ -24,8 +24,9 @@ enum : uint32_t {
 //     stage for it (a quarter or half of the accumulator a warp holding the whole
 //     tile would need, and each head's softmax stays inside one warp);
 //   - head_dim parts split O^T's rows between the two warps of a pair that
-//     compute the same scores (D = 256, and 8-head tiles at D = 128 with 8
-//     warps: where a stage and the accumulator would otherwise limit residency);
+//     compute the same scores (D = 256, bf16 8-head tiles at D = 128, and E4M3
+//     8-head tiles at D = 128 with 8 warps: where a stage and the accumulator
+//     would otherwise limit residency);
 //   - the remaining warps form token groups: group tg computes 16-token tiles
 //     tg, tg + TG, ... of every stage, and the groups merge at the end.
 constexpr int kSmemBudget = 232448;  // 227 KiB per CTA
@@ -37,28 +38,28 @@ __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + 
 // the measured choice (4 and 8 were timed on every named workload on B200).
 __host__ __device__ constexpr int warps_for(int D, int hpt, bool f8) { return 4; }
 
-__host__ __device__ constexpr int dsplit_for(int D, int hpt, int nw) {
-  return D == 256 ? 2 : (nw == 8 && D == 128 && hpt == 8 ? 2 : 1);
+__host__ __device__ constexpr int dsplit_for(int D, int hpt, bool f8, int nw) {
+  return D == 256 ? 2 : (D == 128 && hpt == 8 && (nw == 8 || !f8) ? 2 : 1);
 }
-__host__ __device__ constexpr int head_groups_for(int D, int hpt, int nw) {
-  return (hpt / 8) * dsplit_for(D, hpt, nw) <= nw ? hpt / 8 : nw / dsplit_for(D, hpt, nw);
+__host__ __device__ constexpr int head_groups_for(int D, int hpt, bool f8, int nw) {
+  return (hpt / 8) * dsplit_for(D, hpt, f8, nw) <= nw ? hpt / 8 : nw / dsplit_for(D, hpt, f8, nw);
 }
-__host__ __device__ constexpr int token_groups_for(int D, int hpt, int nw) {
-  return nw / (dsplit_for(D, hpt, nw) * head_groups_for(D, hpt, nw));
+__host__ __device__ constexpr int token_groups_for(int D, int hpt, bool f8, int nw) {
+  return nw / (dsplit_for(D, hpt, f8, nw) * head_groups_for(D, hpt, f8, nw));
 }
 // Tokens of one pipeline stage: 64; 32 at D = 256, whose rows are twice as
-// long, and for bf16 32-head tiles at D = 128, whose 16 KB stages let four CTAs
-// share an SM; an E4M3 cache at D = 256 with 8 or 16 heads per tile doubles
-// them, so its stage carries as many bytes as a bf16 one.  At least one
-// 16-token tile per token group.
+// long, and for bf16 8- and 32-head tiles at D = 128, whose 16 KB stages let
+// five and four CTAs share an SM; an E4M3 cache at D = 256 with 8 or 16 heads
+// per tile doubles them, so its stage carries as many bytes as a bf16 one.  At
+// least one 16-token tile per token group.
 __host__ __device__ constexpr int stage_tokens_for(int D, int hpt, bool f8, int nw) {
-  int st = (D == 256 || (D == 128 && hpt == 32 && !f8) ? 32 : 64) * (f8 && D == 256 && hpt <= 16 ? 2 : 1);
-  while (st < 16 * token_groups_for(D, hpt, nw)) st *= 2;
+  int st = (D == 256 || (D == 128 && (hpt == 32 || hpt == 8) && !f8) ? 32 : 64) * (f8 && D == 256 && hpt <= 16 ? 2 : 1);
+  while (st < 16 * token_groups_for(D, hpt, f8, nw)) st *= 2;
   return st;
 }
 // 16-token tiles a warp computes per stage.
 __host__ __device__ constexpr int tiles_per_group(int D, int hpt, bool f8, int nw) {
-  return stage_tokens_for(D, hpt, f8, nw) / (16 * token_groups_for(D, hpt, nw));
+  return stage_tokens_for(D, hpt, f8, nw) / (16 * token_groups_for(D, hpt, f8, nw));
 }
 
 // Pipeline depth and resident CTAs per SM of one (head_dim, heads-per-tile,
@@ -73,7 +74,13 @@ __host__ __device__ constexpr int tiles_per_group(int D, int hpt, bool f8, int n
 // it at three stages.  32-head tiles at D = 128 (one n-tile per warp, 128
 // registers) run three 16 KB stages and four CTAs per SM for either cache
 // type, measured against two 32 KB stages at three CTAs (ragged MQA batch:
-// 177 -> 157 us bf16, 165 -> 159 us E4M3).  With 8 warps: the same rings,
+// 177 -> 157 us bf16, 165 -> 159 us E4M3).  The bf16 8-head tile at D = 128
+// splits head_dim over warp pairs (two token groups of two head_dim halves),
+// which halves its accumulator (93 registers) and its stage (32 tokens, 16 KB):
+// two stages and five CTAs per SM, measured against two 32 KB stages of four
+// token groups at three CTAs (Qwen3-14B-shaped batch 349 -> 338 us, Llama-8B-
+// shaped unchanged) and against three or four 16 KB stages at three or four
+// CTAs (339-373 us).  With 8 warps: the same rings,
 // half the CTAs (a third for the E4M3 8-head tile, whose registers allow it),
 // so about as many warps share an SM.
 __host__ __device__ constexpr int stages_for(int D, int hpt, bool f8, int nw) {
@@ -81,7 +88,8 @@ __host__ __device__ constexpr int stages_for(int D, int hpt, bool f8, int nw) {
 }
 __host__ __device__ constexpr int ctas_per_sm4(int D, int hpt, bool f8) {
   return f8 && D == 128 ? (hpt == 8 ? 5 : 4)
-                        : D == 64 ? (hpt == 32 ? 3 : 4) : D == 128 ? (hpt == 32 ? 4 : 3) : (hpt == 16 ? 2 : 3);
+                        : D == 64 ? (hpt == 32 ? 3 : 4) : D == 128 ? (hpt == 32 ? 4 : hpt == 8 ? 5 : 3)
+                        : (hpt == 16 ? 2 : 3);
 }
 __host__ __device__ constexpr int ctas_per_sm_for(int D, int hpt, bool f8, int nw) {
   return nw == 4 ? ctas_per_sm4(D, hpt, f8)
@@ -135,7 +143,7 @@ __host__ __device__ constexpr SmemPlan smem_plan_for(int D, int hpt, bool f8, in
   s.stage_tokens = stage_tokens_for(D, hpt, f8, nw);
   s.stage_bytes = (size_t)half_stage_bytes(D, hpt, f8, nw) * 2;  // K and V rows of one stage
   s.ring_bytes = (size_t)s.stages * s.stage_bytes;
-  s.warp_merge_bytes = (size_t)token_groups_for(D, hpt, nw) * hpt * (D + 4 + 2) * 4;  // padded rows, m, l
+  s.warp_merge_bytes = (size_t)token_groups_for(D, hpt, f8, nw) * hpt * (D + 4 + 2) * 4;  // padded rows, m, l
   s.split_merge_bytes = (size_t)hpt * (kMaxSplits + 1) * 4;
   size_t m = s.ring_bytes;
   if (s.warp_merge_bytes > m) m = s.warp_merge_bytes;

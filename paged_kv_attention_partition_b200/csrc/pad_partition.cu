@@ -128,9 +128,9 @@ __global__ void __launch_bounds__(NW * 32, CPS) partition_kernel(const __grid_co
   constexpr uint32_t STAGE_BYTES = (uint32_t)SP.stage_bytes;
   constexpr int ST = SP.stage_tokens;      // tokens per stage
   constexpr int ST_LOG2 = ST == 128 ? 7 : ST == 64 ? 6 : 5;
-  constexpr int DS = dsplit_for(D, HPT, NW);   // warps sharing a token group's scores (head_dim split)
-  constexpr int HG = head_groups_for(D, HPT, NW);  // warps splitting the tile's n-tiles
-  constexpr int TG = token_groups_for(D, HPT, NW);  // token groups
+  constexpr int DS = dsplit_for(D, HPT, F8, NW);       // warps sharing a token group's scores (head_dim split)
+  constexpr int HG = head_groups_for(D, HPT, F8, NW);  // warps splitting the tile's n-tiles
+  constexpr int TG = token_groups_for(D, HPT, F8, NW);  // token groups
   constexpr int TPW = tiles_per_group(D, HPT, F8, NW);  // 16-token tiles per warp per stage
   constexpr int NT = HPT / 8;              // 8-head n-tiles of the head tile
   constexpr int NTW = NT / HG;             // n-tiles of one warp

@@ -411,7 +411,7 @@ static void scenarios() {
   CHECK(fake::library_live() == 2, "partials and control buffers: %d live", fake::library_live());
   pad_launch_witness w;
   CHECK(pad_last_launch(&w) == PAD_OK && w.kernel == 1 && w.num_splits == a.plan(4).num_splits &&
-            w.ctas == a.plan(4).ctas && w.ctas_per_sm == a.plan(4).ctas_per_sm && w.ctas_per_sm == 3,
+            w.ctas == a.plan(4).ctas && w.ctas_per_sm == a.plan(4).ctas_per_sm && w.ctas_per_sm == 5,
         "witness read back");
 
 
@@ -598,7 +598,7 @@ static void scenarios() {
         e_few.plan(16).ctas_per_sm);
   CHECK(e_many.plan(16).ctas == 3072 && e_many.plan(16).ctas_per_sm == 6, "E4M3 8-head, 3072 units: %d per SM",
         e_many.plan(16).ctas_per_sm);
-  CHECK(Problem(24, 8, 8, 128, 16, 16).plan(16).ctas_per_sm == 3, "bf16 8-head: one residency");
+  CHECK(Problem(24, 8, 8, 128, 16, 16).plan(16).ctas_per_sm == 5, "bf16 8-head: one residency");
   CHECK(e_many.decode(16, s1) == PAD_OK, "dense E4M3 decode: %s", pad_last_error());
   if (!fake::launches.empty()) check_launch(e_many, 16, fake::launches.back(), s1, "dense E4M3 decode");
   CHECK(pad_last_launch(&w2) == PAD_OK && w2.ctas_per_sm == 6, "dense build witnessed");

@@ -117,7 +117,8 @@ def test_plan_follows_the_partition_rule(lib):
     assert (p["num_splits"], p["partition_tokens"], p["reduce"]) == (16, 512, 1)
     # one CTA per (sequence, KV head, head tile, partition)
     assert p["ctas"] == 64 * 8 * 16 and p["head_tiles"] == 1 and p["heads_per_tile"] == 8
-    assert p["warps_per_cta"] == 4 and p["stage_tokens"] == 64 and p["stages"] == 2
+    # bf16 8-head tile at D = 128: head_dim split over warp pairs, 32-token stages, five per SM
+    assert p["warps_per_cta"] == 4 and p["stage_tokens"] == 32 and p["stages"] == 2 and p["ctas_per_sm"] == 5
     assert p["workspace_bytes"] >= 64 * 40 * 16 * (128 + 1) * 4 and p["control_bytes"] >= 64 * 8 * 4
     p = pad.pad_decode_plan(16, 16, 4, 256, 16, 2048, num_splits=32, device=0)
     assert (p["num_splits"], p["partition_tokens"]) == (32, 1024)
@@ -148,12 +149,14 @@ def test_heuristic_plans(lib):
         if p["num_splits"] > 1:
             assert p["partition_tokens"] >= 64 and g / p["partition_tokens"] <= 1 / 16 + 1e-9
     # a large batch gets max(512, 64 g) tokens per partition (a power of two); a
-    # small batch is cut finer (down to 64 tokens) until it fills about two
-    # waves of CTAs on 148 SMs
+    # small batch is cut finer (down to 64 tokens) until the launch has three
+    # units per SM (444 on 148 SMs)
     assert pad.pad_decode_plan(32, 32, 8, 128, 16, 256, num_splits=0, device=0)["partition_tokens"] == 512
     assert pad.pad_decode_plan(256, 32, 1, 128, 32, 1024, num_splits=0, device=0)["partition_tokens"] == 2048
     assert pad.pad_decode_plan(1, 32, 8, 128, 16, 256, num_splits=0, device=0)["partition_tokens"] == 64
-    assert pad.pad_decode_plan(4, 32, 8, 128, 16, 256, num_splits=0, device=0)["partition_tokens"] == 128
+    assert pad.pad_decode_plan(4, 32, 8, 128, 16, 256, num_splits=0, device=0)["partition_tokens"] == 256
+    assert pad.pad_decode_plan(8, 32, 8, 128, 16, 256, num_splits=0, device=0)["partition_tokens"] == 512
+    assert pad.pad_decode_plan(2, 40, 8, 128, 16, 512, num_splits=0, device=0)["partition_tokens"] == 256
     # group 20: one 32-head tile at D=128, two 16-head tiles at D=256; group 64: two tiles
     p = pad.pad_decode_plan(2, 20, 1, 128, 16, 10, num_splits=1, device=0)
     assert (p["heads_per_tile"], p["head_tiles"]) == (32, 1)
