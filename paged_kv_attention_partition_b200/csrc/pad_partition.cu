@@ -313,6 +313,7 @@ __global__ void __launch_bounds__(NW * 32, CPS) partition_kernel(const __grid_co
   constexpr int EB = F8 ? 1 : 2;                      // bytes per element
   constexpr int NKB = ROWB / RW;                      // column blocks of a K row
   constexpr int NVB = (MT * 16 * EB + RW - 1) / RW;   // column blocks of this warp's V rows
+  static_assert(DS == 1 || (MT * 16 * EB) % RW == 0, "a warp's head_dim rows start on a column block");
   uint32_t kb[TPW][NKB], vb[TPW][NVB];
   auto op_addr = [](uint32_t stage, uint32_t off, uint32_t x) -> uint32_t {
     if constexpr (!F8 && D == 128 && HPT == 32) return (off ^ x) + stage;
