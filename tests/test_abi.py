@@ -66,6 +66,19 @@ def test_every_declaration_cites_a_passage_or_says_it_has_none():
         assert cites or "no counterpart" in text, f"{name}: its comment names no page section: {text[:120]}"
 
 
+def test_resident_ctas_per_sm_in_the_plan(lib):
+    # each instantiation's launch bound, and the E4M3 8-head tile's six-per-SM
+    # build from four full waves at five per SM (4 * 5 * 148 = 2960 units; the
+    # plan counts 148 SMs without a device)
+    plan = lambda B, Hq, kv, splits=16: pad.pad_decode_plan(B, Hq, 8, 128, 16, 16, num_splits=splits, kv_dtype=kv)
+    assert plan(23, 40, "e4m3")["ctas"] == 2944 and plan(23, 40, "e4m3")["ctas_per_sm"] == 5
+    assert plan(24, 40, "e4m3")["ctas"] == 3072 and plan(24, 40, "e4m3")["ctas_per_sm"] == 6
+    assert plan(64, 40, "bf16")["ctas_per_sm"] == 5  # bf16 8-head tile: head_dim split, one build
+    assert plan(64, 128, "bf16")["ctas_per_sm"] == 3 and plan(64, 128, "e4m3")["ctas_per_sm"] == 4  # 16-head tiles
+    assert plan(4, 256, "bf16")["ctas_per_sm"] == 4 and plan(4, 256, "e4m3")["ctas_per_sm"] == 4  # 32-head tiles
+    assert pad.pad_decode_plan(16, 16, 4, 256, 16, 2048, num_splits=32)["ctas_per_sm"] == 3  # D = 256
+
+
 def test_unit_order_only_for_heavy_units(lib):
     # heavy units (partition tokens x heads per tile >= 32 K) carry the launch's
     # unit order after the partials: 4 bytes per CTA
