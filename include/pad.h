@@ -98,8 +98,8 @@ typedef struct pad_plan {
   int32_t ctas;              /* CTAs launched: one per unit (B * Hkv * head_tiles * num_splits) */
   int32_t ctas_per_sm;       /* resident CTAs per SM the launched kernel instance is built for
                                 (its launch bound): fixed per head_dim, heads per tile and
-                                cache type, except the E4M3 8-head tile at D = 128, which
-                                takes its six-per-SM build for launches of at least four
+                                cache type, except the 8-head tiles at D = 128, which
+                                take their six-per-SM build for launches of at least four
                                 full waves at five per SM (2 for the tcgen05 kernel) */
   int32_t reduce;            /* 1 when partitions may need merging (S > 1) */
   int64_t workspace_bytes;   /* partial-output scratch (0 when S == 1) */

@@ -114,13 +114,13 @@ __host__ __device__ constexpr int ctas_per_sm_for(int D, int hpt, bool f8 = fals
 }
 
 // Resident CTAs per SM a launch is built for (the kernel's launch bound).
-// One instantiation has a second, denser build: the E4M3 8-head tile at
-// D = 128 also runs at six CTAs per SM (80 registers instead of 88).  On B200
-// that build measured 2.5-3.5% faster on launches of at least four full waves
-// at five CTAs per SM and 4-13% slower on shorter ones (GQA batches of
-// 1024-16384 units: there the CTAs' own start and finish latency weighs more
-// than the extra resident warps), so the host picks it by the unit count.
-__host__ __device__ constexpr bool has_dense_build(int D, int hpt, bool f8) { return f8 && D == 128 && hpt == 8; }
+// The 8-head tiles at D = 128 have a second, denser build at six CTAs per SM
+// (80 registers instead of 88 for E4M3 and 93 for bf16).  On B200 the E4M3
+// one measured 2.5-3.5% faster on launches of at least four full waves at five
+// CTAs per SM and 4-13% slower on shorter ones (GQA batches of 1024-16384
+// units: there the CTAs' own start and finish latency weighs more than the
+// extra resident warps), so the host picks it by the unit count.
+__host__ __device__ constexpr bool has_dense_build(int D, int hpt, bool f8) { return D == 128 && hpt == 8; }
 constexpr int kDenseCtasPerSm = 6;
 constexpr int kDenseMinWaves = 4;
 inline int ctas_per_sm_choice(int D, int hpt, bool f8, int64_t units, int sms) {

@@ -590,15 +590,16 @@ static void scenarios() {
         fake::library_live());
   CHECK(a.decode(4, s1) == PAD_OK && fake::library_live() == 2, "decode after release");
 
-  // the E4M3 8-head tile at D = 128: its six-per-SM build from four full
-  // waves at five per SM (4 * 5 * 148 = 2960 units) on, the five-per-SM one below
+  // the 8-head tiles at D = 128: the six-per-SM build from four full waves
+  // at five per SM (4 * 5 * 148 = 2960 units) on, the five-per-SM one below
   pad_launch_witness w2;
   Problem e_few(23, 8, 8, 128, 16, 16, true), e_many(24, 8, 8, 128, 16, 16, true);  // 2944 / 3072 units at S = 16
   CHECK(e_few.plan(16).ctas == 2944 && e_few.plan(16).ctas_per_sm == 5, "E4M3 8-head, 2944 units: %d per SM",
         e_few.plan(16).ctas_per_sm);
   CHECK(e_many.plan(16).ctas == 3072 && e_many.plan(16).ctas_per_sm == 6, "E4M3 8-head, 3072 units: %d per SM",
         e_many.plan(16).ctas_per_sm);
-  CHECK(Problem(24, 8, 8, 128, 16, 16).plan(16).ctas_per_sm == 5, "bf16 8-head: one residency");
+  CHECK(Problem(23, 8, 8, 128, 16, 16).plan(16).ctas_per_sm == 5 && Problem(24, 8, 8, 128, 16, 16).plan(16).ctas_per_sm == 6,
+        "bf16 8-head: the same two builds");
   CHECK(e_many.decode(16, s1) == PAD_OK, "dense E4M3 decode: %s", pad_last_error());
   if (!fake::launches.empty()) check_launch(e_many, 16, fake::launches.back(), s1, "dense E4M3 decode");
   CHECK(pad_last_launch(&w2) == PAD_OK && w2.ctas_per_sm == 6, "dense build witnessed");

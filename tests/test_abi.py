@@ -67,13 +67,13 @@ def test_every_declaration_cites_a_passage_or_says_it_has_none():
 
 
 def test_resident_ctas_per_sm_in_the_plan(lib):
-    # each instantiation's launch bound, and the E4M3 8-head tile's six-per-SM
+    # each instantiation's launch bound, and the 8-head tiles' six-per-SM
     # build from four full waves at five per SM (4 * 5 * 148 = 2960 units; the
     # plan counts 148 SMs without a device)
     plan = lambda B, Hq, kv, splits=16: pad.pad_decode_plan(B, Hq, 8, 128, 16, 16, num_splits=splits, kv_dtype=kv)
-    assert plan(23, 40, "e4m3")["ctas"] == 2944 and plan(23, 40, "e4m3")["ctas_per_sm"] == 5
-    assert plan(24, 40, "e4m3")["ctas"] == 3072 and plan(24, 40, "e4m3")["ctas_per_sm"] == 6
-    assert plan(64, 40, "bf16")["ctas_per_sm"] == 5  # bf16 8-head tile: head_dim split, one build
+    for kv in ("e4m3", "bf16"):
+        assert plan(23, 40, kv)["ctas"] == 2944 and plan(23, 40, kv)["ctas_per_sm"] == 5
+        assert plan(24, 40, kv)["ctas"] == 3072 and plan(24, 40, kv)["ctas_per_sm"] == 6
     assert plan(64, 128, "bf16")["ctas_per_sm"] == 3 and plan(64, 128, "e4m3")["ctas_per_sm"] == 4  # 16-head tiles
     assert plan(4, 256, "bf16")["ctas_per_sm"] == 4 and plan(4, 256, "e4m3")["ctas_per_sm"] == 4  # 32-head tiles
     assert pad.pad_decode_plan(16, 16, 4, 256, 16, 2048, num_splits=32)["ctas_per_sm"] == 3  # D = 256
@@ -131,7 +131,8 @@ def test_plan_follows_the_partition_rule(lib):
     # one CTA per (sequence, KV head, head tile, partition)
     assert p["ctas"] == 64 * 8 * 16 and p["head_tiles"] == 1 and p["heads_per_tile"] == 8
     # bf16 8-head tile at D = 128: head_dim split over warp pairs, 32-token stages, five per SM
-    assert p["warps_per_cta"] == 4 and p["stage_tokens"] == 32 and p["stages"] == 2 and p["ctas_per_sm"] == 5
+    # (8192 units: the six-per-SM build)
+    assert p["warps_per_cta"] == 4 and p["stage_tokens"] == 32 and p["stages"] == 2 and p["ctas_per_sm"] == 6
     assert p["workspace_bytes"] >= 64 * 40 * 16 * (128 + 1) * 4 and p["control_bytes"] >= 64 * 8 * 4
     p = pad.pad_decode_plan(16, 16, 4, 256, 16, 2048, num_splits=32, device=0)
     assert (p["num_splits"], p["partition_tokens"]) == (32, 1024)

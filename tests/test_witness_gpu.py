@@ -65,8 +65,9 @@ def test_static_scratch_and_caller_workspace_run_the_partition_kernel(cuda_devic
     assert got["kernel"] == 1 and got["num_splits"] == plan["num_splits"]
 
 
+@pytest.mark.parametrize("kv", ["e4m3", "bf16"])
 @pytest.mark.parametrize("dense", [False, True], ids=["below", "at"])
-def test_e4m3_8_head_tile_takes_its_dense_build_from_four_waves(cuda_device, dense):
+def test_8_head_tile_takes_its_dense_build_from_four_waves(cuda_device, dense, kv):
     # Qwen3-14B-shaped heads (40 / 8, one 8-head tile per KV head) at S = 16:
     # 128 units per sequence.  From four full waves at five CTAs per SM on,
     # the plan takes the six-per-SM build; one sequence fewer stays at five.
@@ -74,11 +75,11 @@ def test_e4m3_8_head_tile_takes_its_dense_build_from_four_waves(cuda_device, den
     sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
     B = -(-4 * 5 * sms // 128) - (0 if dense else 1)
     lens = [int(x) for x in synth.uniform_int(B, 1, 256, 90, synth.S_LENS)]
-    w = synth.make_workload("wit_dense", B, 40, 8, 128, 16, lens, seed=91, max_blocks_per_seq=16, kv_dtype="e4m3")
-    plan = pad.pad_decode_plan(B, 40, 8, 128, 16, 16, num_splits=16, kv_dtype="e4m3")
+    w = synth.make_workload("wit_dense", B, 40, 8, 128, 16, lens, seed=91, max_blocks_per_seq=16, kv_dtype=kv)
+    plan = pad.pad_decode_plan(B, 40, 8, 128, 16, 16, num_splits=16, kv_dtype=kv)
     assert plan["ctas"] == B * 128 and (plan["ctas"] >= 4 * 5 * sms) == dense
     out, lse = DeviceWorkload(w, cuda_device).run(num_splits=16)
     got = pad.pad_last_launch()
     assert got["ctas_per_sm"] == plan["ctas_per_sm"] == (6 if dense else 5), (got, plan)
     ref_out, ref_lse = oracle.decode_workload(w)
-    check_parity(to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, f"e4m3 8-head, {plan['ctas_per_sm']} per SM")
+    check_parity(to_f64(out), lse.cpu().numpy(), ref_out, ref_lse, f"{kv} 8-head, {plan['ctas_per_sm']} per SM")
